@@ -1,0 +1,344 @@
+#!/usr/bin/env python
+"""Benchmark of one fused RNN-T joint + transducer-loss forward+backward call
+per batch (lattice-vocab cells/s = B*T*(U+1)*V / step time, and peak GB).
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload medium] [--mode tiled|untiled]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
+
+A step is one frnnt_fwd_bwd call over one synthetic batch (all steps of the
+path: projections, forward joint, lattice DP, backward joint, projection
+backward).  With N > 1 (torchrun, one process per GPU) every rank runs its
+own batch of the same shape (weak scaling) and the step time is the max over
+ranks.  Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rnn_joint_network_02_b200 import frnnt, synth  # noqa: E402
+
+METRIC = "RNN-T joint+loss fwd+bwd lattice-vocab cells/sec (B·T·(U+1)·V) and peak GB"
+UNIT = "cells/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="medium", choices=list(synth.WORKLOADS))
+    p.add_argument("--mode", default="tiled", choices=["tiled", "untiled"])
+    p.add_argument("--path", default="auto", choices=["auto", "simt"])
+    p.add_argument("--chunk-cells", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=d["hbm_gbs"], tensor=d["bf16_tflops"], tensor_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
+
+
+def config_of(batch, args, n_gpus):
+    d = batch.dims
+    return {"workload": args.workload, "B": d["B"], "T": d["T"], "U": d["U"], "D_enc": d["D_enc"],
+            "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": args.mode, "path": args.path,
+            "valid_cells": batch.valid_cells(), "padded_cells": batch.padded_cells(),
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{n_gpus}",
+            "global_batch": d["B"] * n_gpus}
+
+
+# ------------------------------------------------------------------ algorithmic work per stage
+
+def stage_work(batch, stage, mode):
+    """(kind, amount per call): tensor flops or HBM bytes that the stage must
+    do by definition (recomputation excluded)."""
+    d = batch.dims
+    H, V = d["H"], d["V"]
+    cells = batch.valid_cells()
+    if stage == "joint_fwd":
+        return "tensor", 2.0 * H * V * cells
+    if stage in ("joint_bwd",):
+        return "tensor", 4.0 * H * V * cells
+    if stage == "lattice_dp":
+        return "hbm", (8 + 4 + 8 + 4) * cells
+    if stage == "projection":
+        return "tensor", 2.0 * (d["B"] * d["T"] * d["D_enc"] * H + d["B"] * (d["U"] + 1) * d["D_pred"] * H)
+    if stage == "projection_bwd":
+        return "tensor", 4.0 * (d["B"] * d["T"] * d["D_enc"] * H + d["B"] * (d["U"] + 1) * d["D_pred"] * H)
+    return None, 0.0
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-i", str(index), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        for r in rows:
+            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
+                              ("sw_power_cap", 8)):
+                if r[col].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) leg
+
+def oracle_sample(batch, utterance=0):
+    """Times the fp64 oracle on one utterance; returns (seconds, metric units)."""
+    import numpy as np
+
+    import oracle
+    f, g, W_f, W_g, W_o, b_o = (t.numpy() for t in batch.float64())
+    w = np.zeros(batch.f.shape[0])
+    w[utterance] = 1.0
+    t0 = time.perf_counter()
+    oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                   grad_loss=w, utterances=[utterance])
+    dt = time.perf_counter() - t0
+    d = batch.dims
+    units = d["T"] * (d["U"] + 1) * d["V"]      # this utterance's share of B*T*(U+1)*V
+    return dt, units
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    batch = synth.workload(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(batch)
+    times = []
+    units = 0
+    for _ in range(args.steps):
+        dt, units = oracle_sample(batch)
+        times.append(dt)
+    sec = sum(times) / len(times)
+    value = units / sec
+    Tb, Ub = int(batch.T_len[0]), int(batch.U_len[0])
+    sample = (f"utterance 0 of {args.workload} (T_len={Tb}, U_len={Ub}) per step; "
+              f"units = T*(U+1)*V of one utterance")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(batch, args, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    idx = synth.WORKLOADS[args.workload]["index"]
+    batch = synth.workload(args.workload, seed=1000 + idx + 7919 * rank)
+    d = {k: getattr(batch, k).to(dev).contiguous()
+         for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+    dtype = "bf16" if batch.dtype == "bf16" else "f32"
+    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, args.mode, args.path, args.chunk_cells, batch.blank)
+    out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(check=False):
+        return frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                             d["U_len"], mode=args.mode, path=args.path, chunk_cells=args.chunk_cells,
+                             blank=batch.blank, out=out, check=check, stream=stream)
+
+    # peak device memory of one call: every buffer is caller-owned, so the
+    # peak is inputs + outputs + workspace (no flush buffer allocated yet)
+    call(check=True)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    call(check=True)
+    torch.cuda.synchronize()
+    peak_bytes = torch.cuda.max_memory_allocated(dev)
+    elt = 2 if dtype == "bf16" else 4
+    footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
+                 4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
+
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    frnnt.profile_read()
+    frnnt.profile(True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        call()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    frnnt.profile(False)
+    stages = frnnt.profile_read()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    units = batch.padded_cells() * batch.dims["V"]
+    value = world * units / (ms / 1e3)
+
+    # end to end through the public API with host buffers: pinned H2D of
+    # the step's inputs, the call, D2H of the loss and status word
+    host = {k: v.cpu().pin_memory() for k, v in d.items()}
+    loss_h = torch.empty(batch.f.shape[0], dtype=torch.float32).pin_memory()
+    status_h = torch.empty(4, dtype=torch.int32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = loss_h.numel() * 4 + status_h.numel() * 4
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        call()
+        loss_h.copy_(out.loss, non_blocking=True)
+        status_h.copy_(out.status, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if int(status_h[0]) != 0:
+            raise RuntimeError(f"device status {int(status_h[0])}")
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = sum(e2e_ms) / len(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    launches = sum(s["launches"] for s in stages)
+    roofline = None
+    pk = peaks()
+    if stages:
+        dom = max(stages, key=lambda k: stages[k]["ms"])
+        kind, work = stage_work(batch, dom, args.mode)
+        per_launch_ms = stages[dom]["ms"] / max(stages[dom]["calls"], 1)
+        work_per_call = work / max(stages[dom]["calls"] / args.steps, 1)
+        if kind == "tensor":
+            achieved = work_per_call / (per_launch_ms / 1e3) / 1e12
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor_sustained"], "unit": "TFLOP/s",
+                        "frac": achieved / pk["tensor_sustained"], "traffic": None, "stage": dom,
+                        "peak_source": pk["source"] + " sustained bf16"}
+        elif kind == "hbm":
+            achieved = work_per_call / (per_launch_ms / 1e3) / 1e9
+            roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                        "frac": achieved / pk["hbm"], "traffic": None, "stage": dom, "peak_source": pk["source"]}
+        else:
+            roofline = {"bound": None, "stage": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
+                        "traffic": None}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, u = oracle_sample(batch)
+        Tb, Ub = int(batch.T_len[0]), int(batch.U_len[0])
+        cpu = {"value": u / dt, "unit": UNIT, "cores": cores(), "kind": "oracle",
+               "sample": f"utterance 0 of {args.workload} (T_len={Tb}, U_len={Ub}); units = T*(U+1)*V of one "
+                         f"utterance; numpy fp64, BLAS threads = all cores"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes of the workload)",
+                "config": config_of(batch, args, world),
+                "peak_gb": peak_bytes / 1e9, "footprint_gb": footprint / 1e9,
+                "peak_over_footprint": peak_bytes / footprint,
+                "valid_cells_per_s": world * batch.valid_cells() * batch.dims["V"] / (ms / 1e3),
+                "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+                "gpu_launches": launches,
+                "stages": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps}
+                           for k, v in stages.items()},
+                "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * frnnt -- fused RNN-T joint network + transducer loss, forward and backward,
+ * for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * What one call computes ("Flash RNN-T: Memory-Efficient Joint Network and
+ * Transducer Loss Computation", abstract: a joint and loss implementation with
+ * optional tiled recomputation over the full alignment space and vocabulary;
+ * the transducer of "Sequence Transduction with Recurrent Neural Networks",
+ * abstract; the feed-forward joint of "Transformer Transducer", abstract):
+ *
+ *   h[b,t,u,:] = tanh(f[b,t,:] W_f + g[b,u,:] W_g)          (H)
+ *   z[b,t,u,:] = W_o h[b,t,u,:] + b_o                        (V)
+ *   blank_lp = z_blank - logsumexp(z), label_lp = z_{y_u} - logsumexp(z)
+ *   loss[b]  = -log sum over all alignments of the (T_len, U_len+1) lattice
+ *   and the gradients of sum_b w_b loss[b] for f, g, W_f, W_g, W_o and b_o.
+ *
+ * Shapes (all row-major, contiguous, element strides only):
+ *   f [B, T, D_enc]      g [B, U+1, D_pred]     (g[b,u] = prediction output
+ *                                                after u labels)
+ *   W_f [D_enc, H]       W_g [D_pred, H]
+ *   W_o [V, H]           b_o [V]
+ *   labels [B, U] int32  T_len [B] int32        U_len [B] int32
+ * Valid lattice cells of utterance b: 0 <= t < T_len[b], 0 <= u <= U_len[b].
+ * Frames t >= T_len[b], positions u > U_len[b] and labels[b, u >= U_len[b]]
+ * are padding: never read into the result; their gradient rows are 0.
+ *
+ * Modes:
+ *   FRNNT_UNTILED  the logits z are materialised (bf16 for FRNNT_BF16, fp32
+ *                  for FRNNT_F32) in the workspace by the forward joint and
+ *                  re-read by the backward -- fastest, memory ~ cells * V.
+ *   FRNNT_TILED    only per-cell log-sum-exp / blank / label log-probs are
+ *                  kept; the backward recomputes z tile by tile, and the
+ *                  logit gradient lives in a bounded chunk of the workspace
+ *                  (chunk_cells) -- memory independent of the batch's cells*V.
+ * Both modes return the same result up to floating-point rounding.
+ *
+ * Precision: FRNNT_BF16 takes bf16 inputs/weights (raw uint16 bit patterns),
+ * multiplies in bf16 on the tensor cores with fp32 accumulation, keeps every
+ * reduction, log-sum-exp and lattice value in fp32, and returns bf16
+ * gradients (round-to-nearest-even).  FRNNT_F32 computes in fp32 throughout
+ * (CUDA-core FMA) and returns fp32 gradients.
+ */
+#ifndef FRNNT_H
+#define FRNNT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FRNNT_API __attribute__((visibility("default")))
+#else
+#define FRNNT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FRNNT_UNTILED = 0, FRNNT_TILED = 1 } frnnt_mode;
+typedef enum { FRNNT_F32 = 0, FRNNT_BF16 = 1 } frnnt_dtype;
+/* Kernel family.  AUTO picks the tcgen05 tensor-core kernels for FRNNT_BF16
+ * when the shape allows them (H, D_enc, D_pred multiples of 64 and V a
+ * multiple of 128) and the CUDA-core kernels otherwise; SIMT forces the
+ * CUDA-core kernels (fp32 arithmetic on bf16 or fp32 inputs). */
+typedef enum { FRNNT_PATH_AUTO = 0, FRNNT_PATH_SIMT = 1 } frnnt_path;
+
+typedef struct {
+  int B, T, U;            /* batch, max frames, max labels (g has U+1 rows) */
+  int D_enc, D_pred;      /* encoder / prediction feature sizes              */
+  int H, V;               /* joint hidden size, vocabulary size (incl. blank)*/
+  int blank;              /* blank id, 0 <= blank < V                         */
+  frnnt_dtype dtype;
+  frnnt_mode mode;
+  frnnt_path path;
+  int chunk_cells;        /* FRNNT_TILED: lattice cells per backward chunk;
+                             0 = default (65536).  Rounded up to whole tiles. */
+} frnnt_dims;
+
+/* Host return codes. */
+enum {
+  FRNNT_OK = 0,
+  FRNNT_ERR_NULL = 1,          /* a required pointer is NULL                  */
+  FRNNT_ERR_DIMS = 2,          /* a size <= 0, blank outside [0,V), U+1 > 1024 */
+  FRNNT_ERR_WORKSPACE = 3,     /* workspace_bytes smaller than required       */
+  FRNNT_ERR_UNSUPPORTED = 4,   /* unknown dtype / mode / path value            */
+  FRNNT_ERR_CUDA = 5,          /* a CUDA launch or query failed                */
+  FRNNT_ERR_ALIGN = 6          /* a pointer is not 16-byte aligned             */
+};
+
+/* Device status bits written to *status (0 = all inputs valid). */
+enum {
+  FRNNT_STATUS_LENGTH = 1,     /* T_len[b] outside [1,T] or U_len[b] outside [0,U] */
+  FRNNT_STATUS_LABEL = 2,      /* labels[b,u] (u < U_len[b]) outside [0,V) or == blank */
+  FRNNT_STATUS_TIMEOUT = 4     /* a bounded device-side wait gave up           */
+};
+
+/* Bytes of device workspace frnnt_fwd_bwd needs for these dims.  Host-only:
+ * makes no CUDA call.  Returns FRNNT_OK or FRNNT_ERR_NULL / _DIMS / _UNSUPPORTED. */
+FRNNT_API int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes);
+
+/* One forward + backward pass over one batch (one call per batch).
+ *
+ * All pointers are DEVICE pointers on the current device, 16-byte aligned,
+ * owned by the caller; the library allocates nothing and keeps no state
+ * between calls.  Float tensors are fp32 (FRNNT_F32) or bf16 bit patterns
+ * (FRNNT_BF16); b_o and all gradients have that same element type.
+ *   grad_loss   [B] fp32 weights w_b of d(sum_b w_b loss_b), or NULL (= 1)
+ *   loss        [B] fp32 output, -log P(y_b | x_b) per utterance
+ *   df, dg, dW_f, dW_g, dW_o, db_o   outputs, overwritten (not accumulated),
+ *               same shapes as f, g, W_f, W_g, W_o, b_o
+ *   workspace   >= frnnt_workspace_size bytes, contents undefined on entry
+ *   status      [1] int32 output: 0, or an OR of FRNNT_STATUS_* bits found by
+ *               the device-side validation; when non-zero every other output
+ *               is unspecified (no out-of-bounds access happens either way:
+ *               lengths and labels are clamped before use)
+ *   stream      cudaStream_t the work is queued on (NULL = legacy stream)
+ * The call is stream-ordered and returns without synchronising.  Host-side
+ * errors (return value != FRNNT_OK) are detected before any launch. */
+FRNNT_API int frnnt_fwd_bwd(const frnnt_dims* d,
+                  const void* f, const void* g, const void* W_f, const void* W_g,
+                  const void* W_o, const void* b_o,
+                  const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                  const float* grad_loss, float* loss,
+                  void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream);
+
+/* Static description of a return code or status bit set. */
+FRNNT_API const char* frnnt_error_string(int code);
+
+/* Per-stage statistics (tracing).  A stage is one step of the path (for
+ * example the forward joint) and may be one or several kernel launches. */
+typedef struct {
+  char name[32];
+  int launches;       /* kernel launches issued by this stage since the last read */
+  int calls;          /* times the stage ran since the last read                  */
+  double ms;          /* summed device time between the stage's CUDA events, or 0
+                         when timing was off                                       */
+} frnnt_stage_stat;
+
+/* Turns per-stage device timing on (1) or off (0) for subsequent calls.
+ * When on, each stage is bracketed by two CUDA events on the call's stream
+ * (events are created on first use and reused).  Launch counting is always
+ * on.  Host-only; not thread-safe.  Returns FRNNT_OK. */
+FRNNT_API int frnnt_profile(int enable);
+
+/* Copies up to `capacity` stage statistics accumulated since the previous
+ * read into `out`, sets *count to the number of stages, then resets them.
+ * Waits for the recorded events to complete.  Returns FRNNT_OK, or
+ * FRNNT_ERR_CUDA if an event query failed. */
+FRNNT_API int frnnt_profile_read(frnnt_stage_stat* out, int capacity, int* count);
+
+/* Library version, "MAJOR.MINOR.PATCH". */
+FRNNT_API const char* frnnt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FRNNT_H */

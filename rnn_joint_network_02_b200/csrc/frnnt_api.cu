@@ -1,0 +1,224 @@
+// C ABI of the frnnt library: argument checks, workspace planning and the
+// launch sequence of one forward + backward call.
+//
+// One call per batch ("Flash RNN-T", abstract: comparisons use one backward
+// call per batch).  Every launch goes on the caller's stream; nothing is
+// allocated and nothing is synchronised.
+#include <string.h>
+
+#include "frnnt_common.cuh"
+#include "frnnt_internal.h"
+
+namespace frnnt {
+namespace {
+
+constexpr int kDefaultChunkCells = 65536;
+
+// Bump allocator over the caller's workspace (256-byte aligned slices).
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* p) : base((char*)p) {}
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~(size_t)255;
+    T* p = base ? (T*)(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+bool dims_ok(const frnnt_dims* d) {
+  if (d->B <= 0 || d->T <= 0 || d->U < 0 || d->D_enc <= 0 || d->D_pred <= 0 || d->H <= 0 || d->V <= 0) return false;
+  if (d->blank < 0 || d->blank >= d->V) return false;
+  if (d->U + 1 > 1024) return false;
+  if (d->chunk_cells < 0) return false;
+  return true;
+}
+
+bool enums_ok(const frnnt_dims* d) {
+  if (d->dtype != FRNNT_F32 && d->dtype != FRNNT_BF16) return false;
+  if (d->mode != FRNNT_UNTILED && d->mode != FRNNT_TILED) return false;
+  if (d->path != FRNNT_PATH_AUTO && d->path != FRNNT_PATH_SIMT) return false;
+  return true;
+}
+
+Shape shape_of(const frnnt_dims* d) {
+  Shape s;
+  s.B = d->B; s.T = d->T; s.U = d->U; s.Dx = d->D_enc; s.Dy = d->D_pred; s.H = d->H; s.V = d->V;
+  s.blank = d->blank;
+  s.Up1 = d->U + 1;
+  s.BT = (long long)d->B * d->T;
+  s.BU = (long long)d->B * (d->U + 1);
+  s.Np = s.BT * s.Up1;
+  s.bf16 = d->dtype == FRNNT_BF16;
+  return s;
+}
+
+// ------------------------------------------------------------------ SIMT plan
+struct SimtPlan {
+  float *F, *G, *dF, *dG;
+  Lattice L;
+  float *accWf, *accWg, *accWo, *accbo;
+  float *df_tmp, *dg_tmp;
+  float *h, *dh, *z;
+  long long rows_per_chunk;
+  size_t bytes;
+};
+
+SimtPlan plan_simt(const frnnt_dims* d, const Shape& s, void* ws) {
+  SimtPlan p;
+  Carver c(ws);
+  long long cells = d->chunk_cells > 0 ? d->chunk_cells : kDefaultChunkCells;
+  p.rows_per_chunk = cells / s.Up1;
+  if (p.rows_per_chunk < 1) p.rows_per_chunk = 1;
+  if (p.rows_per_chunk > s.BT) p.rows_per_chunk = s.BT;
+  const long long C = p.rows_per_chunk * s.Up1;
+  p.F = c.take<float>(s.BT * s.H);
+  p.G = c.take<float>(s.BU * s.H);
+  p.dF = c.take<float>(s.BT * s.H);
+  p.dG = c.take<float>(s.BU * s.H);
+  p.L.lse = c.take<float>(s.Np);
+  p.L.blank_lp = c.take<float>(s.Np);
+  p.L.label_lp = c.take<float>(s.Np);
+  p.L.alpha = c.take<float>(s.Np);
+  p.L.beta = c.take<float>(s.Np);
+  p.accWf = c.take<float>((size_t)s.Dx * s.H);
+  p.accWg = c.take<float>((size_t)s.Dy * s.H);
+  p.accWo = c.take<float>((size_t)s.V * s.H);
+  p.accbo = c.take<float>(s.V);
+  p.df_tmp = s.bf16 ? c.take<float>(s.BT * s.Dx) : nullptr;
+  p.dg_tmp = s.bf16 ? c.take<float>(s.BU * s.Dy) : nullptr;
+  p.h = c.take<float>(C * s.H);
+  p.dh = c.take<float>(C * s.H);
+  p.z = c.take<float>((d->mode == FRNNT_UNTILED ? s.Np : C) * s.V);
+  p.bytes = c.off + 256;
+  return p;
+}
+
+int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, const void* W_f, const void* W_g,
+             const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+             const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g, void* dW_o,
+             void* db_o, void* ws, int32_t* status, cudaStream_t st) {
+  SimtPlan p = plan_simt(d, s, ws);
+  const bool bf = s.bf16;
+  const bool untiled = d->mode == FRNNT_UNTILED;
+  {
+    StageScope sc("validate", st);
+    launch_validate(s, labels, T_len, U_len, status, st);
+    cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.accWo, 0, (size_t)s.V * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.accbo, 0, (size_t)s.V * sizeof(float), st);
+  }
+  {  // projections F = f W_f, G = g W_g
+    StageScope sc("projection", st);
+    launch_gemm_simt((int)s.BT, s.H, s.Dx, f, s.Dx, bf, false, W_f, s.H, bf, false, p.F, s.H, false, st);
+    launch_gemm_simt((int)s.BU, s.H, s.Dy, g, s.Dy, bf, false, W_g, s.H, bf, false, p.G, s.H, false, st);
+  }
+
+  // forward joint: per-cell log-sum-exp, blank and label log-probs
+  for (long long r0 = 0; r0 < s.BT; r0 += p.rows_per_chunk) {
+    StageScope sc("joint_fwd", st);
+    const long long nr = (r0 + p.rows_per_chunk <= s.BT) ? p.rows_per_chunk : s.BT - r0;
+    const long long c0 = r0 * s.Up1, C = nr * s.Up1;
+    float* zc = untiled ? p.z + (size_t)c0 * s.V : p.z;
+    launch_hidden_simt(s, p.F, p.G, T_len, U_len, c0, C, p.h, st);
+    launch_gemm_simt((int)C, s.V, s.H, p.h, s.H, false, false, W_o, s.H, bf, true, zc, s.V, false, st);
+    launch_lse_simt(s, zc, b_o, labels, T_len, U_len, c0, C, p.L, st);
+  }
+
+  {  // transducer forward-backward
+    StageScope sc("lattice_dp", st);
+    launch_dp(s, p.L, T_len, U_len, loss, st);
+  }
+
+  // backward through the joint
+  for (long long r0 = 0; r0 < s.BT; r0 += p.rows_per_chunk) {
+    StageScope sc("joint_bwd", st);
+    const long long nr = (r0 + p.rows_per_chunk <= s.BT) ? p.rows_per_chunk : s.BT - r0;
+    const long long c0 = r0 * s.Up1, C = nr * s.Up1;
+    float* zc = untiled ? p.z + (size_t)c0 * s.V : p.z;
+    launch_hidden_simt(s, p.F, p.G, T_len, U_len, c0, C, p.h, st);
+    if (!untiled) launch_gemm_simt((int)C, s.V, s.H, p.h, s.H, false, false, W_o, s.H, bf, true, zc, s.V, false, st);
+    launch_dz_simt(s, zc, !untiled, b_o, labels, T_len, U_len, grad_loss, c0, C, p.L, p.accbo, st);
+    launch_gemm_simt((int)C, s.H, s.V, zc, s.V, false, false, W_o, s.H, bf, false, p.dh, s.H, false, st);
+    launch_dtanh_reduce_simt(s, p.dh, p.h, c0, C, p.dF, p.dG, st);
+    launch_gemm_simt(s.V, s.H, (int)C, zc, s.V, false, true, p.h, s.H, false, false, p.accWo, s.H, true, st);
+  }
+
+  StageScope sc("projection_bwd", st);
+  float* dfo = bf ? p.df_tmp : (float*)df;
+  float* dgo = bf ? p.dg_tmp : (float*)dg;
+  launch_gemm_simt((int)s.BT, s.Dx, s.H, p.dF, s.H, false, false, W_f, s.H, bf, true, dfo, s.Dx, false, st);
+  launch_gemm_simt(s.Dx, s.H, (int)s.BT, f, s.Dx, bf, true, p.dF, s.H, false, false, p.accWf, s.H, false, st);
+  launch_gemm_simt((int)s.BU, s.Dy, s.H, p.dG, s.H, false, false, W_g, s.H, bf, true, dgo, s.Dy, false, st);
+  launch_gemm_simt(s.Dy, s.H, (int)s.BU, g, s.Dy, bf, true, p.dG, s.H, false, false, p.accWg, s.H, false, st);
+  if (bf) {
+    launch_convert(p.df_tmp, df, s.BT * s.Dx, true, st);
+    launch_convert(p.dg_tmp, dg, s.BU * s.Dy, true, st);
+  }
+  launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, bf, st);
+  launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, bf, st);
+  launch_convert(p.accWo, dW_o, (long long)s.V * s.H, bf, st);
+  launch_convert(p.accbo, db_o, s.V, bf, st);
+  return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+}  // namespace frnnt
+
+using namespace frnnt;
+
+extern "C" int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes) {
+  if (!d || !bytes) return FRNNT_ERR_NULL;
+  if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
+  if (!dims_ok(d)) return FRNNT_ERR_DIMS;
+  Shape s = shape_of(d);
+  *bytes = plan_simt(d, s, nullptr).bytes;
+  return FRNNT_OK;
+}
+
+extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g,
+                             const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len,
+                             const int32_t* U_len, const float* grad_loss, float* loss, void* df, void* dg,
+                             void* dW_f, void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes,
+                             int32_t* status, void* stream) {
+  if (!d) return FRNNT_ERR_NULL;
+  if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
+  if (!dims_ok(d)) return FRNNT_ERR_DIMS;
+  const void* req[] = {f, g, W_f, W_g, W_o, b_o, T_len, U_len, loss, df, dg, dW_f, dW_g, dW_o, db_o, workspace, status};
+  for (const void* p : req)
+    if (!p) return FRNNT_ERR_NULL;
+  if (!labels && d->U > 0) return FRNNT_ERR_NULL;
+  const void* al[] = {f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
+                      db_o, workspace, status};
+  for (const void* p : al)
+    if (p && !aligned16(p)) return FRNNT_ERR_ALIGN;
+  size_t need = 0;
+  frnnt_workspace_size(d, &need);
+  if (workspace_bytes < need) return FRNNT_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  Shape s = shape_of(d);
+  cudaGetLastError();   // clear a stale error so it is not reported as ours
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return FRNNT_ERR_CUDA;
+  return run_simt(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
+                  db_o, workspace, status, st);
+}
+
+extern "C" const char* frnnt_error_string(int code) {
+  switch (code) {
+    case FRNNT_OK: return "ok";
+    case FRNNT_ERR_NULL: return "a required pointer is NULL";
+    case FRNNT_ERR_DIMS: return "invalid dimensions (size <= 0, blank outside [0,V), or U+1 > 1024)";
+    case FRNNT_ERR_WORKSPACE: return "workspace smaller than frnnt_workspace_size";
+    case FRNNT_ERR_UNSUPPORTED: return "unsupported dtype, mode or path";
+    case FRNNT_ERR_CUDA: return "a CUDA launch failed";
+    case FRNNT_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    default: break;
+  }
+  return "unknown frnnt code";
+}
+
+extern "C" const char* frnnt_version(void) { return "0.1.0"; }

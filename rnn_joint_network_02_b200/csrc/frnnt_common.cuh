@@ -1,0 +1,45 @@
+// Shared device helpers of the frnnt library (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "frnnt.h"
+
+namespace frnnt {
+
+__host__ __device__ inline int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+// Lengths as every kernel sees them: clamped into range so that invalid
+// inputs (already flagged in the status word by the validation kernel) can
+// never turn into out-of-bounds accesses.
+struct Lengths {
+  int Tb, Ub;
+};
+__device__ inline Lengths lengths_of(const int32_t* T_len, const int32_t* U_len, int b, int T, int U) {
+  Lengths l;
+  l.Tb = clampi(T_len[b], 1, T);
+  l.Ub = clampi(U_len[b], 0, U);
+  return l;
+}
+__device__ inline int label_of(const int32_t* labels, int b, int u, int U, int V) {
+  return clampi(labels[(size_t)b * U + u], 0, V - 1);
+}
+
+// log(exp(a) + exp(b)) in fp32, exact for -inf operands.
+__device__ __forceinline__ float log_add_exp(float a, float b) {
+  float m = fmaxf(a, b);
+  if (m == -INFINITY) return -INFINITY;
+  return m + log1pf(__expf(-fabsf(a - b)));
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+}  // namespace frnnt

@@ -1,0 +1,118 @@
+// Validation of lengths / labels and the transducer forward-backward over the
+// (T_len, U_len+1) lattice.
+//
+// The lattice recursion is the transducer's ("Sequence Transduction with
+// Recurrent Neural Networks", abstract: the loss sums over every alignment):
+//   alpha(t,u) = lae(alpha(t-1,u) + blank_lp(t-1,u), alpha(t,u-1) + label_lp(t,u-1))
+//   beta(t,u)  = lae(beta(t+1,u)  + blank_lp(t,u),   beta(t,u+1)  + label_lp(t,u))
+// with alpha(0,0) = 0, beta(T-1,U) = blank_lp(T-1,U) and log P = beta(0,0).
+//
+// Schedule: an anti-diagonal wavefront.  Cells with the same d = t + u depend
+// only on diagonal d-1 (alpha) or d+1 (beta), so one thread owns one label
+// position u and walks the diagonals; the value it needs from its neighbour
+// u-1 (alpha) or u+1 (beta) is the neighbour's result on the previous
+// diagonal, passed by a warp shuffle, and across a warp boundary by a
+// parity-double-buffered shared-memory slot.  One block per (utterance,
+// direction): alpha and beta run concurrently.
+#include "frnnt_common.cuh"
+#include "frnnt_internal.h"
+
+namespace frnnt {
+
+__global__ void validate_kernel(int B, int T, int U, int V, int blank, const int32_t* __restrict__ labels,
+                                const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
+                                int32_t* __restrict__ status) {
+  int bits = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int tl = T_len[b], ul = U_len[b];
+    if (tl < 1 || tl > T || ul < 0 || ul > U) bits |= FRNNT_STATUS_LENGTH;
+  }
+  long long n = (long long)B * U;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+    int b = (int)(i / U), u = (int)(i % U);
+    int tl = T_len[b], ul = U_len[b];
+    if (tl < 1 || tl > T || ul < 0 || ul > U) continue;   // length already flagged
+    if (u >= ul) continue;                                // padding label
+    int y = labels[i];
+    if (y < 0 || y >= V || y == blank) bits |= FRNNT_STATUS_LABEL;
+  }
+  bits = __reduce_or_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0 && bits) atomicOr(status, bits);
+}
+
+void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                     int32_t* status, cudaStream_t st) {
+  validate_kernel<<<1, 256, 0, st>>>(s.B, s.T, s.U, s.V, s.blank, labels, T_len, U_len, status);
+  note_launch();
+}
+
+__global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
+                          float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
+                          const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  __shared__ float xs[2][32];
+  const int b = blockIdx.x;
+  const bool is_beta = blockIdx.y == 1;
+  const int u = threadIdx.x;
+  const int lane = u & 31, warp = u >> 5, nwarps = blockDim.x >> 5;
+  const Lengths l = lengths_of(T_len, U_len, b, T, U);
+  const int Tb = l.Tb, Ub = l.Ub;
+  const int Up1 = U + 1;
+  const size_t base = (size_t)b * T * Up1;
+  const int ndiag = Tb + Ub;        // diagonals d = 0 .. Tb-1+Ub
+
+  float cur = -INFINITY;            // this thread's value on the previous diagonal
+  for (int step = 0; step < ndiag; ++step) {
+    const int d = is_beta ? (ndiag - 1 - step) : step;
+    const int t = d - u;
+    const bool active = (u <= Ub) && (t >= 0) && (t < Tb);
+    float nb;                       // neighbour's value on the previous diagonal
+    if (!is_beta) {
+      nb = __shfl_up_sync(0xffffffffu, cur, 1);
+      if (lane == 0) nb = warp > 0 ? xs[(step + 1) & 1][warp - 1] : -INFINITY;
+    } else {
+      nb = __shfl_down_sync(0xffffffffu, cur, 1);
+      if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1] : -INFINITY;
+    }
+    float v = -INFINITY;
+    if (active) {
+      const size_t c = base + (size_t)t * Up1 + u;
+      if (!is_beta) {
+        if (t == 0 && u == 0) {
+          v = 0.f;
+        } else {
+          float fb = t > 0 ? cur + blank_lp[c - Up1] : -INFINITY;   // from (t-1, u)
+          float fl = u > 0 ? nb + label_lp[c - 1] : -INFINITY;      // from (t, u-1)
+          v = log_add_exp(fb, fl);
+        }
+        alpha[c] = v;
+      } else {
+        if (t == Tb - 1 && u == Ub) {
+          v = blank_lp[c];
+        } else {
+          float bb = t + 1 < Tb ? cur + blank_lp[c] : -INFINITY;    // to (t+1, u)
+          float bl = u < Ub ? nb + label_lp[c] : -INFINITY;         // to (t, u+1)
+          v = log_add_exp(bb, bl);
+        }
+        beta[c] = v;
+        if (t == 0 && u == 0) loss[b] = -v;
+      }
+    }
+    cur = v;
+    if (!is_beta) {
+      if (lane == 31) xs[step & 1][warp] = cur;
+    } else {
+      if (lane == 0) xs[step & 1][warp] = cur;
+    }
+    __syncthreads();
+  }
+}
+
+void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
+               cudaStream_t st) {
+  int threads = ((s.Up1 + 31) / 32) * 32;
+  dim3 grid(s.B, 2);
+  dp_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
+  note_launch();
+}
+
+}  // namespace frnnt

@@ -1,0 +1,83 @@
+// Internal launcher interface of the frnnt library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "frnnt.h"
+
+namespace frnnt {
+
+// ---------------------------------------------------------------- tracing
+// Every launcher calls note_launch() once per kernel it launches; a StageScope
+// names the step of the path those launches belong to and, when timing is
+// on, brackets it with CUDA events on the stream.
+void note_launch(int n = 1);
+class StageScope {
+ public:
+  StageScope(const char* name, cudaStream_t st);
+  ~StageScope();
+  StageScope(const StageScope&) = delete;
+  StageScope& operator=(const StageScope&) = delete;
+
+ private:
+  cudaStream_t st_;
+  long long launches0_;
+  int stage_ = 0;
+  cudaEvent_t start_ = nullptr;
+};
+
+// Problem sizes as the launchers see them.
+struct Shape {
+  int B, T, U, Dx, Dy, H, V, blank;
+  int Up1;            // U + 1
+  long long BT;       // B * T        (rows of f, F, dF, df)
+  long long BU;       // B * (U + 1)  (rows of g, G, dG, dg)
+  long long Np;       // B * T * (U + 1) padded lattice cells
+  bool bf16;
+};
+
+// Lattice arrays, fp32, padded layout [b][t][u] with u fastest.
+struct Lattice {
+  float* lse;
+  float* blank_lp;
+  float* label_lp;
+  float* alpha;
+  float* beta;
+};
+
+// ---------------------------------------------------------------- validation / DP
+void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                     int32_t* status, cudaStream_t st);
+void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
+               cudaStream_t st);
+
+// ---------------------------------------------------------------- CUDA-core kernels
+// C[M,N] (fp32, row stride ldc) = op(A)[M,K] * op(B)[K,N]  (+ C when accumulate)
+// op(A)(m,k) = transA ? A[k*lda+m] : A[m*lda+k]; op(B)(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n]
+// a_bf16 / b_bf16 select the element type of A / B (bf16 or fp32).
+void launch_gemm_simt(int M, int N, int K, const void* A, int lda, bool a_bf16, bool transA, const void* B,
+                      int ldb, bool b_bf16, bool transB, float* C, int ldc, bool accumulate, cudaStream_t st);
+
+// h[c,:] = tanh(F[b,t,:] + G[b,u,:]) for padded cells c in [c0, c0+C); 0 outside the valid lattice.
+void launch_hidden_simt(const Shape& s, const float* F, const float* G, const int32_t* T_len,
+                        const int32_t* U_len, long long c0, long long C, float* h, cudaStream_t st);
+
+// z rows of cells [c0, c0+C): z += b_o, then per-cell lse / blank_lp / label_lp into the lattice.
+void launch_lse_simt(const Shape& s, float* z, const void* b_o, const int32_t* labels, const int32_t* T_len,
+                     const int32_t* U_len, long long c0, long long C, const Lattice& L, cudaStream_t st);
+
+// In place z -> dz for cells [c0, c0+C) (adding b_o first when add_bias); accumulates db_o.
+void launch_dz_simt(const Shape& s, float* z, bool add_bias, const void* b_o, const int32_t* labels,
+                    const int32_t* T_len, const int32_t* U_len, const float* grad_loss, long long c0,
+                    long long C, const Lattice& L, float* db_o_acc, cudaStream_t st);
+
+// dpre = dh * (1 - h^2); dF[b,t] = sum_u dpre (rows of the chunk), dG[b,u] += sum_t dpre.
+void launch_dtanh_reduce_simt(const Shape& s, const float* dh, const float* h, long long c0, long long C,
+                              float* dF, float* dG, cudaStream_t st);
+
+// out[i] = (dtype) in[i]
+void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaStream_t st);
+
+}  // namespace frnnt

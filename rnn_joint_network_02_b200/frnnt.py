@@ -1,0 +1,184 @@
+"""Thin Python binding of libfrnnt.so (ctypes).
+
+Argument marshalling only: every step of the forward and backward pass runs
+in the library's CUDA kernels.  PyTorch supplies device memory and the
+stream.  If the shared library is missing the first call raises; there is no
+other implementation behind these names.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfrnnt.so")
+
+UNTILED, TILED = 0, 1
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_SIMT = 0, 1
+
+OK = 0
+STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT = 1, 2, 4
+
+EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
+            "frnnt_profile_read")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("U", ctypes.c_int), ("D_enc", ctypes.c_int),
+                ("D_pred", ctypes.c_int), ("H", ctypes.c_int), ("V", ctypes.c_int), ("blank", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("path", ctypes.c_int),
+                ("chunk_cells", ctypes.c_int)]
+
+
+class StageStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int), ("calls", ctypes.c_int),
+                ("ms", ctypes.c_double)]
+
+
+class FrnntError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"frnnt error {code}: {msg}")
+        self.code = code
+
+
+class FrnntStatusError(RuntimeError):
+    def __init__(self, bits: int):
+        names = [n for n, v in (("length", STATUS_LENGTH), ("label", STATUS_LABEL), ("timeout", STATUS_TIMEOUT))
+                 if bits & v]
+        super().__init__(f"frnnt device status {bits}: invalid {', '.join(names)}")
+        self.bits = bits
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m rnn_joint_network_02_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32p, f32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+        L.frnnt_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(ctypes.c_size_t)]
+        L.frnnt_workspace_size.restype = ctypes.c_int
+        L.frnnt_fwd_bwd.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] + [vp] * 6 +
+                                    [vp, ctypes.c_size_t, i32p, vp])
+        L.frnnt_fwd_bwd.restype = ctypes.c_int
+        L.frnnt_error_string.argtypes = [ctypes.c_int]
+        L.frnnt_error_string.restype = ctypes.c_char_p
+        L.frnnt_version.argtypes = []
+        L.frnnt_version.restype = ctypes.c_char_p
+        L.frnnt_profile.argtypes = [ctypes.c_int]
+        L.frnnt_profile.restype = ctypes.c_int
+        L.frnnt_profile_read.argtypes = [ctypes.POINTER(StageStat), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        L.frnnt_profile_read.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return lib().frnnt_error_string(code).decode()
+
+
+def version() -> str:
+    return lib().frnnt_version().decode()
+
+
+def profile(enable: bool) -> None:
+    """Per-stage CUDA-event timing on/off for later calls (launch counts are always kept)."""
+    lib().frnnt_profile(1 if enable else 0)
+
+
+def profile_read() -> dict:
+    """{stage: dict(launches, calls, ms)} accumulated since the previous read (then reset)."""
+    cap = 64
+    arr = (StageStat * cap)()
+    n = ctypes.c_int(0)
+    rc = lib().frnnt_profile_read(arr, cap, ctypes.byref(n))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    out = {}
+    for i in range(min(n.value, cap)):
+        st = arr[i]
+        if st.calls or st.launches:
+            out[st.name.decode()] = dict(launches=st.launches, calls=st.calls, ms=st.ms)
+    return out
+
+
+def make_dims(B, T, U, D_enc, D_pred, H, V, dtype="bf16", mode="tiled", path="auto", chunk_cells=0,
+              blank=0) -> Dims:
+    return Dims(B, T, U, D_enc, D_pred, H, V, blank, BF16 if dtype == "bf16" else F32,
+                TILED if mode == "tiled" else UNTILED, PATH_SIMT if path == "simt" else PATH_AUTO,
+                chunk_cells)
+
+
+def workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    rc = lib().frnnt_workspace_size(ctypes.byref(dims), ctypes.byref(n))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    return n.value
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank) -> Dims:
+    B, T, D_enc = f.shape
+    U = g.shape[1] - 1
+    V, H = W_o.shape
+    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank)
+
+
+class Outputs:
+    """Preallocated outputs and workspace of one call shape."""
+
+    def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims):
+        dev = f.device
+        self.loss = torch.empty(f.shape[0], dtype=torch.float32, device=dev)
+        self.df = torch.empty_like(f)
+        self.dg = torch.empty_like(g)
+        self.dW_f = torch.empty_like(W_f)
+        self.dW_g = torch.empty_like(W_g)
+        self.dW_o = torch.empty_like(W_o)
+        self.db_o = torch.empty_like(b_o)
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.workspace = torch.empty(max(workspace_size(dims), 16), dtype=torch.uint8, device=dev)
+
+    def grads(self):
+        return dict(df=self.df, dg=self.dg, dW_f=self.dW_f, dW_g=self.dW_g, dW_o=self.dW_o, db_o=self.db_o)
+
+
+def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
+            chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+    """One call of frnnt_fwd_bwd on CUDA tensors.
+
+    Float tensors are all float32 or all bfloat16; labels/T_len/U_len int32.
+    Returns (loss [B] fp32, dict of gradients).  With ``check`` the device
+    status word is read back (one 4-byte device-to-host copy, which
+    synchronises the stream) and a non-zero status raises FrnntStatusError.
+    """
+    dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank)
+    if out is None:
+        out = Outputs(f, g, W_f, W_g, W_o, b_o, dims)
+    if stream is None:
+        stream = torch.cuda.current_stream(f.device)
+    rc = lib().frnnt_fwd_bwd(ctypes.byref(dims), _ptr(f), _ptr(g), _ptr(W_f), _ptr(W_g), _ptr(W_o), _ptr(b_o),
+                             _ptr(labels), _ptr(T_len), _ptr(U_len), _ptr(grad_loss), _ptr(out.loss),
+                             _ptr(out.df), _ptr(out.dg), _ptr(out.dW_f), _ptr(out.dW_g), _ptr(out.dW_o),
+                             _ptr(out.db_o), _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
+                             ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    if check:
+        bits = int(out.status[0].item())
+        if bits:
+            raise FrnntStatusError(bits)
+    return out.loss, out.grads()

@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every symbol its header declares, and the
+host-only entry points (workspace sizing, argument checks) behave as
+documented.  No compute call is made here, so these run without a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from rnn_joint_network_02_b200 import frnnt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            names |= set(re.findall(r"FRNNT_API\s+[\w\s\*]*?\b(frnnt_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert {"frnnt_fwd_bwd", "frnnt_workspace_size", "frnnt_error_string", "frnnt_version"} <= declared
+    lib = frnnt.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(frnnt.EXPORTED) <= declared
+
+
+def test_version_and_error_strings():
+    assert re.match(r"^\d+\.\d+\.\d+$", frnnt.version())
+    for code in range(7):
+        assert frnnt.error_string(code)
+    assert "unknown" in frnnt.error_string(99)
+
+
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_workspace_size_is_host_only_and_positive(mode, dtype):
+    d = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype=dtype, mode=mode)
+    n = frnnt.workspace_size(d)
+    assert n > 0
+
+
+def test_tiled_workspace_bounded_by_chunk():
+    big = frnnt.make_dims(8, 1500, 300, 512, 640, 640, 1024, mode="untiled")
+    small = frnnt.make_dims(8, 1500, 300, 512, 640, 640, 1024, mode="tiled", chunk_cells=65536)
+    assert frnnt.workspace_size(small) < frnnt.workspace_size(big) / 10
+
+
+@pytest.mark.parametrize("field,value,code", [("B", 0, 2), ("H", -1, 2), ("blank", 8, 2), ("U", 1024, 2),
+                                              ("dtype", 7, 4), ("mode", 3, 4), ("path", 9, 4)])
+def test_bad_dims_rejected(field, value, code):
+    d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
+    setattr(d, field, value)
+    n = ctypes.c_size_t(0)
+    assert frnnt.lib().frnnt_workspace_size(ctypes.byref(d), ctypes.byref(n)) == code
+
+
+def test_null_arguments_rejected_before_any_launch():
+    lib = frnnt.lib()
+    d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
+    nul = [None] * 17
+    args = [ctypes.byref(d)] + nul[:6] + [None] * 3 + [None, None] + [None] * 6 + [None, 0, None, None]
+    assert lib.frnnt_fwd_bwd(*args) == frnnt.FrnntError(1, "").code
+    assert lib.frnnt_fwd_bwd(None, *args[1:]) == 1
+
+
+def test_misaligned_pointer_rejected_before_any_launch():
+    lib = frnnt.lib()
+    d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
+    fake = [ctypes.c_void_p(4096 * (i + 1)) for i in range(20)]
+    fake[0] = ctypes.c_void_p(4096 + 4)            # f misaligned
+    args = ([ctypes.byref(d)] + fake[:6] + fake[6:9] + [None, fake[9]] + fake[10:16] +
+            [fake[16], 1 << 40, fake[17], None])
+    assert lib.frnnt_fwd_bwd(*args) == 6
+
+
+def test_small_workspace_rejected_before_any_launch():
+    lib = frnnt.lib()
+    d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
+    fake = [ctypes.c_void_p(4096 * (i + 1)) for i in range(20)]
+    args = ([ctypes.byref(d)] + fake[:6] + fake[6:9] + [None, fake[9]] + fake[10:16] +
+            [fake[16], 16, fake[17], None])
+    assert lib.frnnt_fwd_bwd(*args) == 3

@@ -1,0 +1,133 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+the same seeded inputs, at the contract's tolerances."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from rnn_joint_network_02_b200 import frnnt, synth
+from tests.helpers import GRADS, TOL, compare, rel_l2, run_oracle, to_device, weights_for
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _call(batch, mode="tiled", path="auto", grad_loss=None, chunk_cells=0, check=True):
+    d = to_device(batch)
+    w = None if grad_loss is None else torch.as_tensor(grad_loss, dtype=torch.float32).cuda()
+    loss, grads = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                                d["U_len"], grad_loss=w, mode=mode, path=path, chunk_cells=chunk_cells,
+                                blank=batch.blank, check=check)
+    torch.cuda.synchronize()
+    return loss, grads
+
+
+# ---------------------------------------------------------------- fp32 (tiny)
+
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
+def test_tiny_fp32_against_golden_and_oracle(cuda_ok, mode):
+    batch = synth.workload("tiny")
+    loss, grads = _call(batch, mode=mode)
+    ref = run_oracle(batch)
+    compare(loss, grads, ref, "f32", extra_note=f"tiny/{mode}")
+    gold = json.load(open(os.path.join(HERE, "golden", "tiny_oracle.json")))
+    np.testing.assert_allclose(loss.cpu().numpy(), gold["loss"], rtol=TOL["f32"]["loss"])
+    for name in GRADS:
+        assert rel_l2(grads[name].cpu().numpy(), np.array(gold[name])) <= TOL["f32"]["grad"]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_small_fp32_ragged(cuda_ok, seed):
+    """Ragged lengths, a bias, U_len = 0 and T_len = 1 utterances, fp32."""
+    batch = synth.make(B=5, T=9, U=6, D_enc=12, D_pred=10, H=24, V=11, dtype="f32", seed=200 + seed,
+                       T_range=(1, 9), U_range=(0, 6), bias_std=0.5)
+    batch.T_len[0] = 1
+    batch.U_len[1] = 0
+    w = np.linspace(-1.0, 2.0, 5)
+    for mode in ("tiled", "untiled"):
+        loss, grads = _call(batch, mode=mode, grad_loss=w, chunk_cells=20)
+        compare(loss, grads, run_oracle(batch, grad_loss=w), "f32", extra_note=f"ragged/{mode}")
+
+
+# ---------------------------------------------------------------- bf16 (short)
+
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
+@pytest.mark.parametrize("path", ["auto", "simt"])
+def test_short_bf16(cuda_ok, mode, path):
+    batch = synth.workload("short")
+    loss, grads = _call(batch, mode=mode, path=path)
+    compare(loss, grads, run_oracle(batch), "bf16", extra_note=f"short/{mode}/{path}")
+
+
+def test_padding_does_not_leak(cuda_ok):
+    batch = synth.workload("short")
+    other = synth.redraw_padding(batch, seed=9)
+    l1, g1 = _call(batch)
+    l2, g2 = _call(other)
+    assert torch.equal(l1, l2)
+    for name in ("dW_f", "dW_g", "dW_o", "db_o"):
+        assert torch.equal(g1[name], g2[name]), name
+    for b in range(batch.f.shape[0]):
+        Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
+        assert torch.equal(g1["df"][b, :Tb], g2["df"][b, :Tb])
+        assert torch.equal(g1["dg"][b, :Ub + 1], g2["dg"][b, :Ub + 1])
+        assert int(torch.count_nonzero(g1["df"][b, Tb:])) == 0
+        assert int(torch.count_nonzero(g1["dg"][b, Ub + 1:])) == 0
+
+
+# ---------------------------------------------------------------- status word (bit-exact)
+
+@pytest.mark.parametrize("case,bits", [("T0", 1), ("Tbig", 1), ("Uneg", 1), ("Ubig", 1), ("blank", 2),
+                                       ("label_hi", 2), ("label_neg", 2), ("both", 3)])
+def test_status_bits(cuda_ok, case, bits):
+    batch = synth.workload("tiny")
+    if case == "T0":
+        batch.T_len[0] = 0
+    elif case == "Tbig":
+        batch.T_len[1] = 13
+    elif case == "Uneg":
+        batch.U_len[0] = -1
+    elif case == "Ubig":
+        batch.U_len[1] = 6
+    elif case == "blank":
+        batch.labels[0, 2] = 0
+    elif case == "label_hi":
+        batch.labels[1, 4] = 8
+    elif case == "label_neg":
+        batch.labels[1, 0] = -2
+    elif case == "both":
+        batch.T_len[0] = 99
+        batch.labels[1, 1] = 0
+    import oracle
+    expect = oracle.validate(12, 5, 8, 0, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy())
+    assert expect == bits
+    with pytest.raises(frnnt.FrnntStatusError) as ei:
+        _call(batch)
+    assert ei.value.bits == bits
+
+
+def test_padding_labels_are_not_validated(cuda_ok):
+    batch = synth.workload("tiny")
+    batch.U_len[0] = 3
+    batch.labels[0, 3] = -7          # padding: u >= U_len
+    batch.labels[0, 4] = 0
+    _call(batch)                     # must not raise
+
+
+# ---------------------------------------------------------------- full-size, sampled utterances
+
+@pytest.mark.parametrize("name", ["medium", "large", "long"])
+def test_full_size_sampled_utterances(cuda_ok, name):
+    """Full-size workloads in the bench's launch configuration: the gradient
+    weights select two utterances, so every output is the oracle's on those two."""
+    batch = synth.workload(name)
+    B = batch.f.shape[0]
+    pick = [0, B - 1]
+    w = weights_for(B, pick, device="cpu").numpy()
+    loss, grads = _call(batch, mode="tiled", grad_loss=w)
+    ref = run_oracle(batch, grad_loss=w, utterances=pick)
+    compare(loss, grads, ref, "bf16", utterances=pick, extra_note=name)
