@@ -283,7 +283,7 @@ def run_ours(args):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e = float(t.item())
 
-    launches = sum(s["launches"] for s in stages)
+    launches = sum(v["launches"] for v in stages.values())
     roofline = None
     pk = peaks()
     if stages:
