@@ -125,6 +125,36 @@ FRNNT_API int frnnt_fwd_bwd(const frnnt_dims* d,
                   void* workspace, size_t workspace_bytes,
                   int32_t* status, void* stream);
 
+/* Size of the library-owned scratch array used by frnnt_fwd_bwd_noalloc. */
+#define FRNNT_NOALLOC_MAX_BYTES (64u * 1024u * 1024u)
+
+/* frnnt_fwd_bwd without caller-provided workspace, for callers that cannot
+ * allocate device memory when they run the loss (their framework's allocator
+ * owns all device memory, or an allocation could synchronise the device).
+ * Not from the pages: the paper has no counterpart; this is a deployment
+ * convenience of this library.
+ *
+ * Same arguments, semantics and return codes as frnnt_fwd_bwd, minus the
+ * workspace.  The scratch is one FRNNT_NOALLOC_MAX_BYTES __device__ array in
+ * the library, reserved on every GPU that loads the library until the process
+ * exits; dims whose frnnt_workspace_size exceeds it return FRNNT_ERR_WORKSPACE
+ * before any launch (a smaller chunk_cells lowers the need in tiled mode).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    outside any stream capture.
+ *  - All calls share the one array, which keeps the previous call's
+ *    contents; each call clears on its stream what must start at zero.
+ *    Calls that can overlap on the GPU (different streams, or different
+ *    host threads on one device) race on the array: serialise them. */
+FRNNT_API int frnnt_fwd_bwd_noalloc(const frnnt_dims* d,
+                  const void* f, const void* g, const void* W_f, const void* W_g,
+                  const void* W_o, const void* b_o,
+                  const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                  const float* grad_loss, float* loss,
+                  void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+                  int32_t* status, void* stream);
+
 /* Static description of a return code or status bit set. */
 FRNNT_API const char* frnnt_error_string(int code);
 

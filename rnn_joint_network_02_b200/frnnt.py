@@ -24,7 +24,8 @@ OK = 0
 STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT = 1, 2, 4
 
 EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
-            "frnnt_profile_read")
+            "frnnt_profile_read", "frnnt_fwd_bwd_noalloc")
+NOALLOC_MAX_BYTES = 64 * 1024 * 1024
 
 
 class Dims(ctypes.Structure):
@@ -69,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.frnnt_fwd_bwd.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] + [vp] * 6 +
                                     [vp, ctypes.c_size_t, i32p, vp])
         L.frnnt_fwd_bwd.restype = ctypes.c_int
+        L.frnnt_fwd_bwd_noalloc.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] +
+                                            [vp] * 6 + [i32p, vp])
+        L.frnnt_fwd_bwd_noalloc.restype = ctypes.c_int
         L.frnnt_error_string.argtypes = [ctypes.c_int]
         L.frnnt_error_string.restype = ctypes.c_char_p
         L.frnnt_version.argtypes = []
@@ -139,7 +143,7 @@ def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank) -> Dims:
 class Outputs:
     """Preallocated outputs and workspace of one call shape."""
 
-    def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims):
+    def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims, with_workspace: bool = True):
         dev = f.device
         self.loss = torch.empty(f.shape[0], dtype=torch.float32, device=dev)
         self.df = torch.empty_like(f)
@@ -149,7 +153,8 @@ class Outputs:
         self.dW_o = torch.empty_like(W_o)
         self.db_o = torch.empty_like(b_o)
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
-        self.workspace = torch.empty(max(workspace_size(dims), 16), dtype=torch.uint8, device=dev)
+        n = max(workspace_size(dims), 16) if with_workspace else 16
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def grads(self):
         return dict(df=self.df, dg=self.dg, dW_f=self.dW_f, dW_g=self.dW_g, dW_o=self.dW_o, db_o=self.db_o)
@@ -177,6 +182,35 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode
                              ctypes.c_void_p(stream.cuda_stream))
     if rc != OK:
         raise FrnntError(rc, error_string(rc))
+    if check:
+        bits = int(out.status[0].item())
+        if bits:
+            raise FrnntStatusError(bits)
+    return out.loss, out.grads()
+
+
+def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
+                    chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+    """frnnt_fwd_bwd_noalloc: like fwd_bwd, but the library's fixed scratch
+    array replaces the workspace (``out.workspace`` is not used).  Raises
+    FrnntError(FRNNT_ERR_WORKSPACE) when these dims need more than
+    NOALLOC_MAX_BYTES of scratch."""
+    dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank)
+    if out is None:
+        out = Outputs(f, g, W_f, W_g, W_o, b_o, dims, with_workspace=False)
+    if stream is None:
+        stream = torch.cuda.current_stream(f.device)
+    rc = lib().frnnt_fwd_bwd_noalloc(ctypes.byref(dims), _ptr(f), _ptr(g), _ptr(W_f), _ptr(W_g), _ptr(W_o),
+                                     _ptr(b_o), _ptr(labels), _ptr(T_len), _ptr(U_len), _ptr(grad_loss),
+                                     _ptr(out.loss), _ptr(out.df), _ptr(out.dg), _ptr(out.dW_f), _ptr(out.dW_g),
+                                     _ptr(out.dW_o), _ptr(out.db_o), _ptr(out.status),
+                                     ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        msg = error_string(rc)
+        if rc == 3:
+            msg += f" (these dims need {workspace_size(dims)} bytes; the fixed scratch holds {NOALLOC_MAX_BYTES})"
+        raise FrnntError(rc, msg)
     if check:
         bits = int(out.status[0].item())
         if bits:
