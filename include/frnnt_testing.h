@@ -1,0 +1,31 @@
+/*
+ * frnnt test hooks -- building blocks of frnnt_fwd_bwd exposed so the test
+ * suite can check each kernel family on its own.  Not needed to use the
+ * library; same ownership rules as frnnt.h (device pointers, caller-owned,
+ * stream-ordered, nothing allocated).
+ */
+#ifndef FRNNT_TESTING_H
+#define FRNNT_TESTING_H
+
+#include "frnnt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The tensor-core (tcgen05 + TMA) bf16 GEMM used for the joint's
+ * contractions and the projections:  D[M,N] = A[M,K] * B[K,N], fp32
+ * accumulation.  A is K-major ([M][lda], a_mn = 0) or MN-major ([K][lda],
+ * a_mn = 1); B is K-major ([N][ldb], b_mn = 0) or MN-major ([K][ldb]).
+ * epi: 0 = store fp32 to out[M][ldo]; 1 = store bf16; 2 = fp32 atomic add
+ * into out (k_splits >= 1 K slices); 3 = out (bf16, holding h on entry)
+ * becomes D * (1 - h*h).  Requires lda, ldb multiples of 8, N a multiple of
+ * 32, 16-byte aligned pointers.  Returns FRNNT_OK or an FRNNT_ERR_* code. */
+FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn, long long lda,
+                                   const void* B, int b_mn, long long ldb, int epi, int k_splits,
+                                   void* out, long long ldo, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FRNNT_TESTING_H */

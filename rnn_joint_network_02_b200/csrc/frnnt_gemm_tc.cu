@@ -1,0 +1,365 @@
+// Persistent, warp-specialised bf16 GEMM on the 5th-generation tensor cores:
+//   D[M,N] (fp32, TMEM) = A[M,K] * B[K,N]   with a fused epilogue.
+//
+// Roles (192 threads, one CTA per SM):
+//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), then store / reduce
+//   warp 4     producer: TMA tile loads of A and B into a STAGES-deep ring
+//   warp 5     MMA issuer: one thread issues tcgen05.mma, commits to mbarriers
+// The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
+// of one output tile overlaps the main loop of the next.  Work units are
+// (m tile, n tile, k slice) triples handed out round-robin; split-K slices
+// reduce into fp32 with vector atomics.
+//
+// Operand layouts: A is K-major ([M][lda], K contiguous) or MN-major
+// ([K][lda], M contiguous); B is K-major ([N][ldb]) or MN-major ([K][ldb]).
+// All tiles use the 128-byte swizzle; K blocks are 64 elements wide.
+#include <stdio.h>
+
+#include "frnnt_common.cuh"
+#include "frnnt_internal.h"
+#include "sm100.cuh"
+
+namespace frnnt {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+struct GemmParams {
+  int M, N, K;
+  int m_tiles, n_tiles, k_splits, kblocks;
+  int epi;
+  float* out_f32;
+  __nv_bfloat16* out_bf16;
+  long long ldo;
+  int32_t* status;
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TILES_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int TOTAL = TILES_BYTES + BAR_BYTES + 1024;   // + alignment slack
+};
+
+__device__ __forceinline__ void unit_coords(int unit, const GemmParams& p, int& m0, int& n0, int& kb0, int& kb1) {
+  const int mt = unit % p.m_tiles;
+  const int rest = unit / p.m_tiles;
+  const int nt = rest % p.n_tiles;
+  const int ks = rest / p.n_tiles;
+  m0 = mt * BM;
+  n0 = nt;                          // n tile index; the caller scales it by BN
+  const int per = (p.kblocks + p.k_splits - 1) / p.k_splits;
+  kb0 = ks * per;
+  kb1 = min(p.kblocks, kb0 + per);
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  using S = GemmSmem<BN, STAGES>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + S::TILES_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_base_p = (uint32_t*)(tempty + 2);
+  volatile int* abort_flag = (volatile int*)(tmem_base_p + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = p.m_tiles * p.n_tiles * p.k_splits;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_base_p, 2 * BN);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_base_p;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int unit = blockIdx.x; unit < units && !*abort_flag; unit += gridDim.x) {
+        int m0, nt, kb0, kb1;
+        unit_coords(unit, p, m0, nt, kb0, kb1);
+        const int n0 = nt * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
+          uint8_t* sa = smem + s * S::STAGE_BYTES;
+          uint8_t* sb = sa + S::A_BYTES;
+          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+          if (!A_MN) {
+            tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
+          } else {
+            tma_load_2d(sa, &tmA, &full[s], m0, kb * BK);
+            tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, kb * BK);
+          }
+          if (!B_MN) {
+            tma_load_2d(sb, &tmB, &full[s], kb * BK, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, &full[s], n0 + 64 * j, kb * BK);
+          }
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc_i = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x, ++acc_i) {
+        int m0, nt, kb0, kb1;
+        unit_coords(unit, p, m0, nt, kb0, kb1);
+        const int a = acc_i & 1;
+        const uint32_t aph = (acc_i >> 1) & 1;
+        if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dt = tbase + a * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
+          const uint32_t sb = sa + S::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
+            mma_bf16_ss(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) mma_commit(&tfull[a]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 0-3)
+    int acc_i = 0;
+    for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++acc_i) {
+      int m0, nt, kb0, kb1;
+      unit_coords(unit, p, m0, nt, kb0, kb1);
+      const int n0 = nt * BN;
+      const int a = acc_i & 1;
+      const uint32_t aph = (acc_i >> 1) & 1;
+      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      tc_fence_after();
+      const int row = m0 + warp * 32 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
+        tmem_wait_ld();
+        const int col0 = n0 + c * 32;
+        if (!row_ok || col0 >= p.N) continue;
+        if (p.epi == 0) {          // store fp32
+          float4* dst = (float4*)(p.out_f32 + (size_t)row * p.ldo + col0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        } else if (p.epi == 1) {   // store bf16
+          uint4* dst = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+            v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+            v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+            v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+            dst[j] = v;
+          }
+        } else if (p.epi == 2) {   // fp32 reduce (split-K / accumulate)
+          float* dst = p.out_f32 + (size_t)row * p.ldo + col0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                       __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        } else {                   // dtanh: out = acc * (1 - h^2), h read from and result written to out_bf16
+          uint4* hp = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 hv = hp[j];
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[q]);
+              float2 hf = __bfloat1622float2(h2);
+              float d0 = __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x);
+              float d1 = __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y);
+              o[q] = pack_bf16x2(d0, d1);
+            }
+            hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 2 * BN);
+  }
+  if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, FRNNT_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN>
+bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
+  using S = GemmSmem<BN, STAGES>;
+  auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) != cudaSuccess)
+      return false;
+    attr = true;
+  }
+  kern<<<grid, kThreads, S::TOTAL, st>>>(ta, tb, p);
+  note_launch();
+  return cudaPeekAtLastError() == cudaSuccess;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
+                       uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
+  // shape rules of the tensor-core GEMM: 16-byte aligned rows and N a multiple of 32
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return FRNNT_OK;
+  if ((g.lda % 8) || (g.ldb % 8) || (g.N % 32)) return FRNNT_ERR_DIMS;
+  if ((g.epi == GEMM_EPI_STORE_F32 || g.epi == GEMM_EPI_RED_F32) && (g.ldo % 4 || !g.out_f32)) return FRNNT_ERR_DIMS;
+  if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH) && (g.ldo % 8 || !g.out_bf16)) return FRNNT_ERR_DIMS;
+  if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
+  const int BN = (g.N % 256 == 0 && g.N >= 256) ? 256 : 128;
+  CUtensorMap ta, tb;
+  bool ok;
+  if (!g.a_mn) ok = make_tmap_bf16_2d(&ta, g.A, g.K, g.M, (uint64_t)g.lda, 64, 128);
+  else ok = make_tmap_bf16_2d(&ta, g.A, g.M, g.K, (uint64_t)g.lda, 64, 64);
+  if (!ok) return FRNNT_ERR_CUDA;
+  if (!g.b_mn) ok = make_tmap_bf16_2d(&tb, g.B, g.K, g.N, (uint64_t)g.ldb, 64, BN);
+  else ok = make_tmap_bf16_2d(&tb, g.B, g.N, g.K, (uint64_t)g.ldb, 64, 64);
+  if (!ok) return FRNNT_ERR_CUDA;
+  GemmParams p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.m_tiles = (g.M + BM - 1) / BM;
+  p.n_tiles = (g.N + BN - 1) / BN;
+  p.kblocks = (g.K + BK - 1) / BK;
+  int splits = g.k_splits < 1 ? 1 : g.k_splits;
+  if (splits > p.kblocks) splits = p.kblocks;
+  if (splits > 1 && g.epi != GEMM_EPI_RED_F32) return FRNNT_ERR_UNSUPPORTED;
+  // every split must own at least one k block
+  const int per = (p.kblocks + splits - 1) / splits;
+  splits = (p.kblocks + per - 1) / per;
+  p.k_splits = splits;
+  p.epi = g.epi;
+  p.out_f32 = g.out_f32;
+  p.out_bf16 = (__nv_bfloat16*)g.out_bf16;
+  p.ldo = g.ldo;
+  p.status = g.status;
+  const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  const int grid = units < sm_count() ? units : sm_count();
+  bool launched;
+  if (BN == 256) {
+    if (!g.a_mn && !g.b_mn) launched = launch_t<256, 4, false, false>(ta, tb, p, grid, st);
+    else if (!g.a_mn && g.b_mn) launched = launch_t<256, 4, false, true>(ta, tb, p, grid, st);
+    else if (g.a_mn && !g.b_mn) launched = launch_t<256, 4, true, false>(ta, tb, p, grid, st);
+    else launched = launch_t<256, 4, true, true>(ta, tb, p, grid, st);
+  } else {
+    if (!g.a_mn && !g.b_mn) launched = launch_t<128, 6, false, false>(ta, tb, p, grid, st);
+    else if (!g.a_mn && g.b_mn) launched = launch_t<128, 6, false, true>(ta, tb, p, grid, st);
+    else if (g.a_mn && !g.b_mn) launched = launch_t<128, 6, true, false>(ta, tb, p, grid, st);
+    else launched = launch_t<128, 6, true, true>(ta, tb, p, grid, st);
+  }
+  return launched ? FRNNT_OK : FRNNT_ERR_CUDA;
+}
+
+}  // namespace frnnt

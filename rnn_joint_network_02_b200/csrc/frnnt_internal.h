@@ -77,6 +77,27 @@ void launch_dz_simt(const Shape& s, float* z, bool add_bias, const void* b_o, co
 void launch_dtanh_reduce_simt(const Shape& s, const float* dh, const float* h, long long c0, long long C,
                               float* dF, float* dG, cudaStream_t st);
 
+// ---------------------------------------------------------------- tensor-core GEMM
+// D[M,N] = A[M,K] * B[K,N] in bf16 with fp32 accumulation (tcgen05, TMA).
+// A: K-major [M][lda] or MN-major [K][lda]; B: K-major [N][ldb] or MN-major [K][ldb].
+enum GemmEpilogue { GEMM_EPI_STORE_F32 = 0, GEMM_EPI_STORE_BF16 = 1, GEMM_EPI_RED_F32 = 2, GEMM_EPI_DTANH = 3 };
+struct GemmTcArgs {
+  int M, N, K;
+  const void* A;
+  bool a_mn;
+  long long lda;
+  const void* B;
+  bool b_mn;
+  long long ldb;
+  int epi;             // GemmEpilogue
+  int k_splits;        // > 1 only with GEMM_EPI_RED_F32
+  float* out_f32;      // STORE_F32 / RED_F32 output [M][ldo]
+  void* out_bf16;      // STORE_BF16 output, or DTANH h-in / dpre-out [M][ldo]
+  long long ldo;
+  int32_t* status;     // device status word (timeout bit), may be NULL
+};
+int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
+
 // out[i] = (dtype) in[i]
 void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaStream_t st);
 

@@ -26,6 +26,7 @@ STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
             "frnnt_profile_read", "frnnt_fwd_bwd_noalloc")
 NOALLOC_MAX_BYTES = 64 * 1024 * 1024
+TEST_HOOKS = ("frnnt_test_gemm_bf16",)
 
 
 class Dims(ctypes.Structure):
@@ -81,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.frnnt_profile.restype = ctypes.c_int
         L.frnnt_profile_read.argtypes = [ctypes.POINTER(StageStat), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         L.frnnt_profile_read.restype = ctypes.c_int
+        L.frnnt_test_gemm_bf16.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int,
+                                           ctypes.c_longlong, vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_int,
+                                           ctypes.c_int, vp, ctypes.c_longlong, vp, vp]
+        L.frnnt_test_gemm_bf16.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -216,3 +221,18 @@ def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=No
         if bits:
             raise FrnntStatusError(bits)
     return out.loss, out.grads()
+
+
+def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: int = 0, k_splits: int = 1,
+                   out=None, stream=None):
+    """Test hook: the tensor-core GEMM D = A * B (see include/frnnt_testing.h).
+    A is [M][K] (a_mn False) or [K][M]; B is [N][K] (b_mn False) or [K][N]."""
+    if out is None:
+        out = torch.zeros(M, N, dtype=torch.bfloat16 if epi in (1, 3) else torch.float32, device=A.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(A.device)
+    rc = lib().frnnt_test_gemm_bf16(M, N, K, _ptr(A), int(a_mn), A.stride(0), _ptr(B), int(b_mn), B.stride(0), epi,
+                                    k_splits, _ptr(out), out.stride(0), None, ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    return out
