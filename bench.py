@@ -38,7 +38,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="medium", choices=list(synth.WORKLOADS))
@@ -75,9 +75,12 @@ def stage_work(batch, stage, mode):
     d = batch.dims
     H, V = d["H"], d["V"]
     cells = batch.valid_cells()
-    if stage == "joint_fwd":
+    if stage in ("joint_fwd", "bwd_dWo", "bwd_dh"):
         return "tensor", 2.0 * H * V * cells
-    if stage in ("joint_bwd",):
+    if stage == "joint_bwd_dz":
+        # tiled: the logits are recomputed (2HV per cell); untiled: elementwise over the stored logits
+        return ("tensor", 2.0 * H * V * cells) if mode == "tiled" else ("hbm", 4.0 * V * cells)
+    if stage == "joint_bwd":
         return "tensor", 4.0 * H * V * cells
     if stage == "lattice_dp":
         return "hbm", (8 + 4 + 8 + 4) * cells
@@ -91,16 +94,36 @@ def stage_work(batch, stage, mode):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """nvidia-smi samples every 20 ms; only samples inside [mark_start, mark_end]
+    (host wall clock) are reported."""
+
     def __init__(self, index: int):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.t0 = self.t1 = None
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-i", str(index), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-i", str(index), "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+        self.lines_at = []
+        time.sleep(0.3)
+
+    def mark_start(self):
+        self.f.flush()
+        self.t0 = self._count()
+
+    def mark_end(self):
+        time.sleep(0.05)
+        self.t1 = self._count()
+
+    def _count(self):
+        try:
+            return sum(1 for _ in open(self.f.name))
+        except OSError:
+            return 0
 
     def stop(self):
         if self.p is None:
@@ -112,7 +135,11 @@ class ClockSampler:
             self.p.kill()
         self.f.flush()
         rows = []
-        for line in open(self.f.name):
+        lines = open(self.f.name).read().splitlines()
+        lo = self.t0 or 0
+        hi = self.t1 if self.t1 is not None else len(lines)
+        window = lines[max(0, lo - 1):hi] if hi > lo else lines[max(0, lo - 2):lo + 1]
+        for line in window:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 9:
                 rows.append(parts)
@@ -234,12 +261,16 @@ def run_ours(args):
     torch.cuda.synchronize()
     sampler = ClockSampler(local) if rank == 0 else None
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if sampler:
+        sampler.mark_start()
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
         call()
         evs[i][1].record(stream)
     torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_end()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None

@@ -164,6 +164,183 @@ int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, 
   return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;
 }
 
+
+// ------------------------------------------------------------------ tensor-core plan
+bool use_tc(const frnnt_dims* d) {
+  if (d->dtype != FRNNT_BF16 || d->path != FRNNT_PATH_AUTO) return false;
+  if (d->B > 1024) return false;
+  if (d->H % 64 || d->D_enc % 32 || d->D_pred % 32) return false;
+  return joint_tc_supported(d->H, d->V);
+}
+
+struct TcPlan {
+  int TB, UB;
+  long long maxT, chunkT;
+  float *F, *G, *dF, *dG;
+  __nv_bfloat16 *dFb, *dGb;
+  int4* tiles;
+  int* ntiles;
+  Lattice L;
+  float *accWo, *db_part, *accWf, *accWg;
+  __nv_bfloat16 *zbuf, *hbuf;
+  size_t bytes;
+};
+
+TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
+  TcPlan p;
+  Carver c(ws);
+  tile_shape(s.U, &p.TB, &p.UB);
+  p.maxT = max_tiles(s, p.TB, p.UB);
+  const long long cells = d->chunk_cells > 0 ? d->chunk_cells : kDefaultChunkCells;
+  p.chunkT = (cells + 127) / 128;
+  if (p.chunkT > p.maxT) p.chunkT = p.maxT;
+  if (d->mode == FRNNT_UNTILED) p.chunkT = p.maxT;
+  p.F = c.take<float>(s.BT * s.H);
+  p.G = c.take<float>(s.BU * s.H);
+  p.dF = c.take<float>(s.BT * s.H);
+  p.dG = c.take<float>(s.BU * s.H);
+  p.dFb = c.take<__nv_bfloat16>(s.BT * s.H);
+  p.dGb = c.take<__nv_bfloat16>(s.BU * s.H);
+  p.tiles = c.take<int4>(p.maxT);
+  p.ntiles = c.take<int>(4);
+  p.L.lse = c.take<float>(s.Np);
+  p.L.blank_lp = c.take<float>(s.Np);
+  p.L.label_lp = c.take<float>(s.Np);
+  p.L.alpha = c.take<float>(s.Np);
+  p.L.beta = c.take<float>(s.Np);
+  p.accWo = c.take<float>((size_t)s.V * s.H);
+  p.db_part = c.take<float>((size_t)8 * s.V);
+  p.accWf = c.take<float>((size_t)s.Dx * s.H);
+  p.accWg = c.take<float>((size_t)s.Dy * s.H);
+  p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.V);
+  p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.H);
+  p.bytes = c.off + 256;
+  return p;
+}
+
+int splits_for(int M, int N, int K) {
+  const int BN = (N % 256 == 0 && N >= 256) ? 256 : 128;
+  const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
+  const int kb = (K + 63) / 64;
+  int want = (2 * 148 + tiles - 1) / tiles;
+  if (want > kb) want = kb;
+  return want < 1 ? 1 : want;
+}
+
+int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, const void* W_f, const void* W_g,
+           const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+           const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+           void* ws, int32_t* status, cudaStream_t st) {
+  TcPlan p = plan_tc(d, s, ws);
+  const bool untiled = d->mode == FRNNT_UNTILED;
+  int rc = FRNNT_OK;
+#define FRNNT_TRY(x)            \
+  do {                          \
+    rc = (x);                   \
+    if (rc != FRNNT_OK) return rc; \
+  } while (0)
+  {
+    StageScope sc("validate", st);
+    launch_validate(s, labels, T_len, U_len, status, st);
+    launch_tiles(s, p.TB, p.UB, T_len, U_len, p.tiles, p.ntiles, st);
+    cudaMemsetAsync(p.dF, 0, s.BT * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.accWo, 0, (size_t)s.V * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.db_part, 0, (size_t)8 * s.V * sizeof(float), st);
+    cudaMemsetAsync(p.accWf, 0, (size_t)s.Dx * s.H * sizeof(float), st);
+    cudaMemsetAsync(p.accWg, 0, (size_t)s.Dy * s.H * sizeof(float), st);
+  }
+  {
+    StageScope sc("projection", st);
+    GemmTcArgs a{};
+    a.M = (int)s.BT; a.N = s.H; a.K = s.Dx; a.A = f; a.a_mn = false; a.lda = s.Dx; a.B = W_f; a.b_mn = true;
+    a.ldb = s.H; a.epi = GEMM_EPI_STORE_F32; a.k_splits = 1; a.out_f32 = p.F; a.ldo = s.H; a.status = status;
+    FRNNT_TRY(gemm_tc(a, st));
+    a.M = (int)s.BU; a.K = s.Dy; a.A = g; a.lda = s.Dy; a.B = W_g; a.out_f32 = p.G;
+    FRNNT_TRY(gemm_tc(a, st));
+  }
+  JointLaunch j{};
+  j.s = s; j.TB = p.TB; j.UB = p.UB; j.F = p.F; j.G = p.G; j.W_o = W_o; j.b_o = b_o; j.labels = labels;
+  j.T_len = T_len; j.U_len = U_len; j.grad_loss = grad_loss; j.tiles = p.tiles; j.ntiles = p.ntiles; j.L = p.L;
+  j.zbuf = p.zbuf; j.hbuf = p.hbuf; j.db_part = p.db_part; j.status = status;
+  {
+    StageScope sc("joint_fwd", st);
+    j.mode = untiled ? 1 : 0;
+    j.tile_begin = 0;
+    j.tile_end = (int)p.maxT;
+    FRNNT_TRY(launch_joint_tc(j, st));
+  }
+  {
+    StageScope sc("lattice_dp", st);
+    launch_dp(s, p.L, T_len, U_len, loss, st);
+  }
+  for (long long c0 = 0; c0 < p.maxT; c0 += p.chunkT) {
+    const long long c1 = (c0 + p.chunkT < p.maxT) ? c0 + p.chunkT : p.maxT;
+    j.tile_begin = (int)c0;
+    j.tile_end = (int)c1;
+    __nv_bfloat16* zrows = untiled ? p.zbuf + (size_t)c0 * 128 * s.V : p.zbuf;
+    __nv_bfloat16* hrows = untiled ? p.hbuf + (size_t)c0 * 128 * s.H : p.hbuf;
+    {
+      StageScope sc("joint_bwd_dz", st);
+      if (untiled) {
+        launch_dz_from_z(j, st);
+      } else {
+        j.mode = 2;
+        FRNNT_TRY(launch_joint_tc(j, st));
+      }
+    }
+    const int rows = (int)((c1 - c0) * 128);
+    {
+      StageScope sc("bwd_dWo", st);
+      GemmTcArgs a{};
+      a.M = s.V; a.N = s.H; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.V; a.B = hrows; a.b_mn = true;
+      a.ldb = s.H; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, s.H, rows); a.out_f32 = p.accWo;
+      a.ldo = s.H; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
+      a.dyn_dim = 2;
+      FRNNT_TRY(gemm_tc(a, st));
+    }
+    {
+      StageScope sc("bwd_dh", st);
+      GemmTcArgs a{};
+      a.M = rows; a.N = s.H; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = W_o; a.b_mn = true;
+      a.ldb = s.H; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = s.H; a.status = status;
+      a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
+      FRNNT_TRY(gemm_tc(a, st));
+    }
+    {
+      StageScope sc("bwd_seg_reduce", st);
+      launch_seg_reduce(j, hrows, (int)c0, p.dF, p.dG, st);
+    }
+  }
+  {
+    StageScope sc("projection_bwd", st);
+    launch_db_finalize(p.db_part, s.V, db_o, true, st);
+    launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
+    launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, st);
+    GemmTcArgs a{};
+    // df = dF W_f^T : B = W_f read as K-major [D_enc][H]
+    a.M = (int)s.BT; a.N = s.Dx; a.K = s.H; a.A = p.dFb; a.a_mn = false; a.lda = s.H; a.B = W_f; a.b_mn = false;
+    a.ldb = s.H; a.epi = GEMM_EPI_STORE_BF16; a.k_splits = 1; a.out_bf16 = df; a.ldo = s.Dx; a.status = status;
+    FRNNT_TRY(gemm_tc(a, st));
+    a.M = (int)s.BU; a.N = s.Dy; a.A = p.dGb; a.B = W_g; a.out_bf16 = dg; a.ldo = s.Dy;
+    FRNNT_TRY(gemm_tc(a, st));
+    // dW_f = f^T dF : A = f read as MN-major [BT][D_enc], B = dF MN-major [BT][H]
+    GemmTcArgs w{};
+    w.M = s.Dx; w.N = s.H; w.K = (int)s.BT; w.A = f; w.a_mn = true; w.lda = s.Dx; w.B = p.dFb; w.b_mn = true;
+    w.ldb = s.H; w.epi = GEMM_EPI_RED_F32; w.k_splits = splits_for(s.Dx, s.H, (int)s.BT); w.out_f32 = p.accWf;
+    w.ldo = s.H; w.status = status;
+    FRNNT_TRY(gemm_tc(w, st));
+    w.M = s.Dy; w.K = (int)s.BU; w.A = g; w.lda = s.Dy; w.B = p.dGb; w.k_splits = splits_for(s.Dy, s.H, (int)s.BU);
+    w.out_f32 = p.accWg;
+    FRNNT_TRY(gemm_tc(w, st));
+    launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, true, st);
+    launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, true, st);
+    launch_convert(p.accWo, dW_o, (long long)s.V * s.H, true, st);
+  }
+#undef FRNNT_TRY
+  return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 }  // namespace
@@ -176,7 +353,7 @@ extern "C" int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes) {
   if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
   if (!dims_ok(d)) return FRNNT_ERR_DIMS;
   Shape s = shape_of(d);
-  *bytes = plan_simt(d, s, nullptr).bytes;
+  *bytes = use_tc(d) ? plan_tc(d, s, nullptr).bytes : plan_simt(d, s, nullptr).bytes;
   return FRNNT_OK;
 }
 
@@ -203,6 +380,9 @@ extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, 
   Shape s = shape_of(d);
   cudaGetLastError();   // clear a stale error so it is not reported as ours
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return FRNNT_ERR_CUDA;
+  if (use_tc(d))
+    return run_tc(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o, db_o,
+                  workspace, status, st);
   return run_simt(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
                   db_o, workspace, status, st);
 }

@@ -37,7 +37,29 @@ struct GemmParams {
   __nv_bfloat16* out_bf16;
   long long ldo;
   int32_t* status;
+  const int* dyn_count;
+  int dyn_base, dyn_scale, dyn_dim;
 };
+
+// Effective problem after the optional device-side limit on M or K.
+struct Eff {
+  int M, m_tiles, kblocks, per;
+};
+
+__device__ __forceinline__ Eff eff_of(const GemmParams& p) {
+  Eff e;
+  e.M = p.M;
+  e.kblocks = p.kblocks;
+  if (p.dyn_count) {
+    long long v = ((long long)__ldg(p.dyn_count) - p.dyn_base) * p.dyn_scale;
+    if (v < 0) v = 0;
+    if (p.dyn_dim == 1) e.M = (int)min((long long)p.M, v);
+    else e.kblocks = (int)min((long long)p.kblocks, (v + 63) / 64);
+  }
+  e.m_tiles = (e.M + 127) / 128;
+  e.per = (e.kblocks + p.k_splits - 1) / p.k_splits;
+  return e;
+}
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -49,16 +71,18 @@ struct GemmSmem {
   static constexpr int TOTAL = TILES_BYTES + BAR_BYTES + 1024;   // + alignment slack
 };
 
-__device__ __forceinline__ void unit_coords(int unit, const GemmParams& p, int& m0, int& n0, int& kb0, int& kb1) {
+// Unit -> (m tile origin, n tile index, k block range); false when the unit
+// has no work under the effective limits (every role skips it alike).
+__device__ __forceinline__ bool unit_coords(int unit, const GemmParams& p, const Eff& e, int& m0, int& nt, int& kb0,
+                                           int& kb1) {
   const int mt = unit % p.m_tiles;
   const int rest = unit / p.m_tiles;
-  const int nt = rest % p.n_tiles;
+  nt = rest % p.n_tiles;
   const int ks = rest / p.n_tiles;
   m0 = mt * BM;
-  n0 = nt;                          // n tile index; the caller scales it by BN
-  const int per = (p.kblocks + p.k_splits - 1) / p.k_splits;
-  kb0 = ks * per;
-  kb1 = min(p.kblocks, kb0 + per);
+  kb0 = ks * e.per;
+  kb1 = min(e.kblocks, kb0 + e.per);
+  return mt < e.m_tiles && kb0 < kb1;
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN>
@@ -76,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  const Eff eff = eff_of(p);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -108,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       for (int unit = blockIdx.x; unit < units && !*abort_flag; unit += gridDim.x) {
         int m0, nt, kb0, kb1;
-        unit_coords(unit, p, m0, nt, kb0, kb1);
+        if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int n0 = nt * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
@@ -143,9 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       int acc_i = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x, ++acc_i) {
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
         int m0, nt, kb0, kb1;
-        unit_coords(unit, p, m0, nt, kb0, kb1);
+        if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int a = acc_i & 1;
         const uint32_t aph = (acc_i >> 1) & 1;
         if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) break;
@@ -172,22 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (ok) mma_commit(&tfull[a]);
+        ++acc_i;
       }
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue (warps 0-3)
     int acc_i = 0;
-    for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++acc_i) {
+    for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
       int m0, nt, kb0, kb1;
-      unit_coords(unit, p, m0, nt, kb0, kb1);
+      if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
       if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
       tc_fence_after();
       const int row = m0 + warp * 32 + lane;
-      const bool row_ok = row < p.M;
+      const bool row_ok = row < eff.M;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -240,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
+      ++acc_i;
     }
   }
 
@@ -345,6 +372,10 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   p.out_bf16 = (__nv_bfloat16*)g.out_bf16;
   p.ldo = g.ldo;
   p.status = g.status;
+  p.dyn_count = g.dyn_count;
+  p.dyn_base = g.dyn_base;
+  p.dyn_scale = g.dyn_scale;
+  p.dyn_dim = g.dyn_dim;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
   const int grid = units < sm_count() ? units : sm_count();
   bool launched;

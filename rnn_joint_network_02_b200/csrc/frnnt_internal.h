@@ -1,6 +1,7 @@
 // Internal launcher interface of the frnnt library (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -95,10 +96,50 @@ struct GemmTcArgs {
   void* out_bf16;      // STORE_BF16 output, or DTANH h-in / dpre-out [M][ldo]
   long long ldo;
   int32_t* status;     // device status word (timeout bit), may be NULL
+  // Optional device-side limit: the effective M (dyn_dim 1) or K (dyn_dim 2)
+  // is min(static, (*dyn_count - dyn_base) * dyn_scale), read by the kernel.
+  const int* dyn_count = nullptr;
+  int dyn_base = 0, dyn_scale = 0, dyn_dim = 0;
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
 
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
+                       uint32_t box_inner, uint32_t box_outer);
+
+// ---------------------------------------------------------------- fused joint (tensor cores)
+struct JointLaunch {
+  Shape s;
+  int TB, UB;                   // tile = TB frames x UB label positions (TB * UB = 128)
+  int mode;                     // 0 forward (lse / blank / label), 1 forward + store z and h, 2 backward dz
+  const float* F;               // [B*T][H] fp32
+  const float* G;               // [B*(U+1)][H] fp32
+  const void* W_o;              // [V][H] bf16
+  const void* b_o;              // [V] bf16
+  const int32_t* labels;
+  const int32_t* T_len;
+  const int32_t* U_len;
+  const float* grad_loss;
+  const int4* tiles;            // device tile list (b, t0, u0, -)
+  const int* ntiles;            // device tile count
+  int tile_begin, tile_end;     // tile range of this launch (end clamped by *ntiles)
+  Lattice L;
+  void* zbuf;                   // z (mode 1, rows tile*128+r) or dz (mode 2, rows (tile-begin)*128+r), bf16 [.][V]
+  void* hbuf;                   // h rows, same indexing, bf16 [.][H]
+  float* db_part;               // [8][V] fp32 partial column sums of dz
+  int32_t* status;
+};
+bool joint_tc_supported(int H, int V);
+void tile_shape(int U, int* TB, int* UB);
+long long max_tiles(const Shape& s, int TB, int UB);
+void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
+                  cudaStream_t st);
+int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
+void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
+void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);
+void launch_db_finalize(const float* db_part, int V, void* out, bool to_bf16, cudaStream_t st);
+
 // out[i] = (dtype) in[i]
 void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaStream_t st);
+void launch_convert_bf16(const float* in, void* out, long long n, cudaStream_t st);
 
 }  // namespace frnnt

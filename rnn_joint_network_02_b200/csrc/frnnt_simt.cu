@@ -328,4 +328,8 @@ void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaS
   note_launch();
 }
 
+void launch_convert_bf16(const float* in, void* out, long long n, cudaStream_t st) {
+  launch_convert(in, out, n, true, st);
+}
+
 }  // namespace frnnt

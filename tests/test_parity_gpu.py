@@ -64,19 +64,24 @@ def test_short_bf16(cuda_ok, mode, path):
 
 
 def test_padding_does_not_leak(cuda_ok):
+    """Redrawing every padding value (frames past T_len, positions past U_len,
+    labels past U_len, here with large and out-of-range values) changes
+    nothing beyond the floating-point reassociation of the fp32 atomics:
+    losses are bit-exact, gradients agree to 1e-3 relative L2 (a leak would be
+    O(1)), and padded gradient rows are exactly zero."""
     batch = synth.workload("short")
     other = synth.redraw_padding(batch, seed=9)
-    l1, g1 = _call(batch)
-    l2, g2 = _call(other)
-    assert torch.equal(l1, l2)
-    for name in ("dW_f", "dW_g", "dW_o", "db_o"):
-        assert torch.equal(g1[name], g2[name]), name
-    for b in range(batch.f.shape[0]):
-        Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
-        assert torch.equal(g1["df"][b, :Tb], g2["df"][b, :Tb])
-        assert torch.equal(g1["dg"][b, :Ub + 1], g2["dg"][b, :Ub + 1])
-        assert int(torch.count_nonzero(g1["df"][b, Tb:])) == 0
-        assert int(torch.count_nonzero(g1["dg"][b, Ub + 1:])) == 0
+    for mode in ("tiled", "untiled"):
+        l1, g1 = _call(batch, mode=mode)
+        l2, g2 = _call(other, mode=mode)
+        assert torch.equal(l1, l2)
+        for name in GRADS:
+            assert rel_l2(g1[name].float().cpu().numpy(), g2[name].float().cpu().numpy()) <= 1e-3, name
+        for b in range(batch.f.shape[0]):
+            Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
+            assert int(torch.count_nonzero(g1["df"][b, Tb:])) == 0
+            assert int(torch.count_nonzero(g1["dg"][b, Ub + 1:])) == 0
+            assert int(torch.count_nonzero(g2["df"][b, Tb:])) == 0
 
 
 # ---------------------------------------------------------------- status word (bit-exact)
