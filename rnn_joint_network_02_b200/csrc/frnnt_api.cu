@@ -170,13 +170,14 @@ bool use_tc(const frnnt_dims* d) {
   if (d->dtype != FRNNT_BF16 || d->path != FRNNT_PATH_AUTO) return false;
   if (d->B > 1024) return false;
   if (d->H % 64 || d->D_enc % 32 || d->D_pred % 32) return false;
-  return joint_tc_supported(d->H, d->V);
+  return joint_tc_supported(d->H, d->V, d->U);
 }
 
 struct TcPlan {
   int TB, UB;
   long long maxT, chunkT;
-  float *F, *G, *dF, *dG;
+  __nv_bfloat16 *F, *G;
+  float *dF, *dG;
   __nv_bfloat16 *dFb, *dGb;
   int4* tiles;
   int* ntiles;
@@ -195,8 +196,8 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.chunkT = (cells + 127) / 128;
   if (p.chunkT > p.maxT) p.chunkT = p.maxT;
   if (d->mode == FRNNT_UNTILED) p.chunkT = p.maxT;
-  p.F = c.take<float>(s.BT * s.H);
-  p.G = c.take<float>(s.BU * s.H);
+  p.F = c.take<__nv_bfloat16>(s.BT * s.H);
+  p.G = c.take<__nv_bfloat16>(s.BU * s.H);
   p.dF = c.take<float>(s.BT * s.H);
   p.dG = c.take<float>(s.BU * s.H);
   p.dFb = c.take<__nv_bfloat16>(s.BT * s.H);
@@ -208,12 +209,12 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.label_lp = c.take<float>(s.Np);
   p.L.alpha = c.take<float>(s.Np);
   p.L.beta = c.take<float>(s.Np);
-  p.accWo = c.take<float>((size_t)s.V * s.H);
-  p.db_part = c.take<float>((size_t)8 * s.V);
+  p.accWo = c.take<float>((size_t)s.V * (s.H + 64));
+  p.db_part = nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.V);
-  p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.H);
+  p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * (s.H + 64));
   p.bytes = c.off + 256;
   return p;
 }
@@ -245,8 +246,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     launch_tiles(s, p.TB, p.UB, T_len, U_len, p.tiles, p.ntiles, st);
     cudaMemsetAsync(p.dF, 0, s.BT * s.H * sizeof(float), st);
     cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
-    cudaMemsetAsync(p.accWo, 0, (size_t)s.V * s.H * sizeof(float), st);
-    cudaMemsetAsync(p.db_part, 0, (size_t)8 * s.V * sizeof(float), st);
+    cudaMemsetAsync(p.accWo, 0, (size_t)s.V * (s.H + 64) * sizeof(float), st);
     cudaMemsetAsync(p.accWf, 0, (size_t)s.Dx * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accWg, 0, (size_t)s.Dy * s.H * sizeof(float), st);
   }
@@ -254,9 +254,9 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     StageScope sc("projection", st);
     GemmTcArgs a{};
     a.M = (int)s.BT; a.N = s.H; a.K = s.Dx; a.A = f; a.a_mn = false; a.lda = s.Dx; a.B = W_f; a.b_mn = true;
-    a.ldb = s.H; a.epi = GEMM_EPI_STORE_F32; a.k_splits = 1; a.out_f32 = p.F; a.ldo = s.H; a.status = status;
+    a.ldb = s.H; a.epi = GEMM_EPI_STORE_BF16; a.k_splits = 1; a.out_bf16 = p.F; a.ldo = s.H; a.status = status;
     FRNNT_TRY(gemm_tc(a, st));
-    a.M = (int)s.BU; a.K = s.Dy; a.A = g; a.lda = s.Dy; a.B = W_g; a.out_f32 = p.G;
+    a.M = (int)s.BU; a.K = s.Dy; a.A = g; a.lda = s.Dy; a.B = W_g; a.out_bf16 = p.G;
     FRNNT_TRY(gemm_tc(a, st));
   }
   JointLaunch j{};
@@ -279,7 +279,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     j.tile_begin = (int)c0;
     j.tile_end = (int)c1;
     __nv_bfloat16* zrows = untiled ? p.zbuf + (size_t)c0 * 128 * s.V : p.zbuf;
-    __nv_bfloat16* hrows = untiled ? p.hbuf + (size_t)c0 * 128 * s.H : p.hbuf;
+    const int HS = s.H + 64;
+    __nv_bfloat16* hrows = untiled ? p.hbuf + (size_t)c0 * 128 * HS : p.hbuf;
     {
       StageScope sc("joint_bwd_dz", st);
       if (untiled) {
@@ -293,9 +294,10 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     {
       StageScope sc("bwd_dWo", st);
       GemmTcArgs a{};
-      a.M = s.V; a.N = s.H; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.V; a.B = hrows; a.b_mn = true;
-      a.ldb = s.H; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, s.H, rows); a.out_f32 = p.accWo;
-      a.ldo = s.H; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
+      // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias gradient
+      a.M = s.V; a.N = HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.V; a.B = hrows; a.b_mn = true;
+      a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, HS, rows); a.out_f32 = p.accWo;
+      a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;
       FRNNT_TRY(gemm_tc(a, st));
     }
@@ -303,7 +305,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       StageScope sc("bwd_dh", st);
       GemmTcArgs a{};
       a.M = rows; a.N = s.H; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = W_o; a.b_mn = true;
-      a.ldb = s.H; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = s.H; a.status = status;
+      a.ldb = s.H; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
       a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
       FRNNT_TRY(gemm_tc(a, st));
     }
@@ -314,7 +316,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   }
   {
     StageScope sc("projection_bwd", st);
-    launch_db_finalize(p.db_part, s.V, db_o, true, st);
+    launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st);
     launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
     launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, st);
     GemmTcArgs a{};
@@ -335,7 +337,6 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     FRNNT_TRY(gemm_tc(w, st));
     launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, true, st);
     launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, true, st);
-    launch_convert(p.accWo, dW_o, (long long)s.V * s.H, true, st);
   }
 #undef FRNNT_TRY
   return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;

@@ -46,6 +46,31 @@ void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len
   note_launch();
 }
 
+// Operands of step `step` for thread u: alpha needs blank_lp(t-1,u) and
+// label_lp(t,u-1); beta needs blank_lp(t,u) and label_lp(t,u) (t = d - u).
+// They do not depend on the recursion, so they are fetched kPrefetch steps
+// ahead into a register ring to hide the global-memory latency.
+constexpr int kPrefetch = 4;
+
+__device__ __forceinline__ void dp_operands(bool is_beta, int step, int ndiag, int u, int Tb, int Ub, int Up1,
+                                            size_t base, const float* __restrict__ blank_lp,
+                                            const float* __restrict__ label_lp, float& ob, float& ol) {
+  ob = 0.f;
+  ol = 0.f;
+  if (step >= ndiag) return;
+  const int d = is_beta ? (ndiag - 1 - step) : step;
+  const int t = d - u;
+  if (u > Ub || t < 0 || t >= Tb) return;
+  const size_t c = base + (size_t)t * Up1 + u;
+  if (!is_beta) {
+    if (t > 0) ob = __ldg(blank_lp + c - Up1);
+    if (u > 0) ol = __ldg(label_lp + c - 1);
+  } else {
+    ob = __ldg(blank_lp + c);
+    if (u < Ub) ol = __ldg(label_lp + c);
+  }
+}
+
 __global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
                           float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
                           const int32_t* __restrict__ U_len, float* __restrict__ loss) {
@@ -60,50 +85,62 @@ __global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, cons
   const size_t base = (size_t)b * T * Up1;
   const int ndiag = Tb + Ub;        // diagonals d = 0 .. Tb-1+Ub
 
+  float qb[kPrefetch], ql[kPrefetch];
+#pragma unroll
+  for (int i = 0; i < kPrefetch; ++i)
+    dp_operands(is_beta, i, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
+
   float cur = -INFINITY;            // this thread's value on the previous diagonal
-  for (int step = 0; step < ndiag; ++step) {
-    const int d = is_beta ? (ndiag - 1 - step) : step;
-    const int t = d - u;
-    const bool active = (u <= Ub) && (t >= 0) && (t < Tb);
-    float nb;                       // neighbour's value on the previous diagonal
-    if (!is_beta) {
-      nb = __shfl_up_sync(0xffffffffu, cur, 1);
-      if (lane == 0) nb = warp > 0 ? xs[(step + 1) & 1][warp - 1] : -INFINITY;
-    } else {
-      nb = __shfl_down_sync(0xffffffffu, cur, 1);
-      if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1] : -INFINITY;
-    }
-    float v = -INFINITY;
-    if (active) {
-      const size_t c = base + (size_t)t * Up1 + u;
+  for (int step0 = 0; step0 < ndiag; step0 += kPrefetch) {
+#pragma unroll
+    for (int i = 0; i < kPrefetch; ++i) {
+      const int step = step0 + i;
+      if (step >= ndiag) break;     // uniform across the block
+      const float ob = qb[i], ol = ql[i];
+      dp_operands(is_beta, step + kPrefetch, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
+      const int d = is_beta ? (ndiag - 1 - step) : step;
+      const int t = d - u;
+      const bool active = (u <= Ub) && (t >= 0) && (t < Tb);
+      float nb;                     // neighbour's value on the previous diagonal
       if (!is_beta) {
-        if (t == 0 && u == 0) {
-          v = 0.f;
-        } else {
-          float fb = t > 0 ? cur + blank_lp[c - Up1] : -INFINITY;   // from (t-1, u)
-          float fl = u > 0 ? nb + label_lp[c - 1] : -INFINITY;      // from (t, u-1)
-          v = log_add_exp(fb, fl);
-        }
-        alpha[c] = v;
+        nb = __shfl_up_sync(0xffffffffu, cur, 1);
+        if (lane == 0) nb = warp > 0 ? xs[(step + 1) & 1][warp - 1] : -INFINITY;
       } else {
-        if (t == Tb - 1 && u == Ub) {
-          v = blank_lp[c];
-        } else {
-          float bb = t + 1 < Tb ? cur + blank_lp[c] : -INFINITY;    // to (t+1, u)
-          float bl = u < Ub ? nb + label_lp[c] : -INFINITY;         // to (t, u+1)
-          v = log_add_exp(bb, bl);
-        }
-        beta[c] = v;
-        if (t == 0 && u == 0) loss[b] = -v;
+        nb = __shfl_down_sync(0xffffffffu, cur, 1);
+        if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1] : -INFINITY;
       }
+      float v = -INFINITY;
+      if (active) {
+        const size_t c = base + (size_t)t * Up1 + u;
+        if (!is_beta) {
+          if (t == 0 && u == 0) {
+            v = 0.f;
+          } else {
+            const float fb = t > 0 ? cur + ob : -INFINITY;   // from (t-1, u)
+            const float fl = u > 0 ? nb + ol : -INFINITY;    // from (t, u-1)
+            v = log_add_exp(fb, fl);
+          }
+          alpha[c] = v;
+        } else {
+          if (t == Tb - 1 && u == Ub) {
+            v = ob;
+          } else {
+            const float bb = t + 1 < Tb ? cur + ob : -INFINITY;    // to (t+1, u)
+            const float bl = u < Ub ? nb + ol : -INFINITY;         // to (t, u+1)
+            v = log_add_exp(bb, bl);
+          }
+          beta[c] = v;
+          if (t == 0 && u == 0) loss[b] = -v;
+        }
+      }
+      cur = v;
+      if (!is_beta) {
+        if (lane == 31) xs[step & 1][warp] = cur;
+      } else {
+        if (lane == 0) xs[step & 1][warp] = cur;
+      }
+      __syncthreads();
     }
-    cur = v;
-    if (!is_beta) {
-      if (lane == 31) xs[step & 1][warp] = cur;
-    } else {
-      if (lane == 0) xs[step & 1][warp] = cur;
-    }
-    __syncthreads();
   }
 }
 

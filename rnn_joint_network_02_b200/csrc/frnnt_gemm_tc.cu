@@ -181,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
           const uint32_t sb = sa + S::A_BYTES;
 #pragma unroll

@@ -111,8 +111,8 @@ struct JointLaunch {
   Shape s;
   int TB, UB;                   // tile = TB frames x UB label positions (TB * UB = 128)
   int mode;                     // 0 forward (lse / blank / label), 1 forward + store z and h, 2 backward dz
-  const float* F;               // [B*T][H] fp32
-  const float* G;               // [B*(U+1)][H] fp32
+  const void* F;                // [B*T][H] bf16
+  const void* G;                // [B*(U+1)][H] bf16
   const void* W_o;              // [V][H] bf16
   const void* b_o;              // [V] bf16
   const int32_t* labels;
@@ -124,11 +124,11 @@ struct JointLaunch {
   int tile_begin, tile_end;     // tile range of this launch (end clamped by *ntiles)
   Lattice L;
   void* zbuf;                   // z (mode 1, rows tile*128+r) or dz (mode 2, rows (tile-begin)*128+r), bf16 [.][V]
-  void* hbuf;                   // h rows, same indexing, bf16 [.][H]
-  float* db_part;               // [8][V] fp32 partial column sums of dz
+  void* hbuf;                   // h rows, same indexing, bf16 [.][H + 64]; column H is 1 (cell count column)
+  float* db_part;               // unused
   int32_t* status;
 };
-bool joint_tc_supported(int H, int V);
+bool joint_tc_supported(int H, int V, int U);
 void tile_shape(int U, int* TB, int* UB);
 long long max_tiles(const Shape& s, int TB, int UB);
 void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
@@ -136,7 +136,7 @@ void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const in
 int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
 void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);
-void launch_db_finalize(const float* db_part, int V, void* out, bool to_bf16, cudaStream_t st);
+void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st);
 
 // out[i] = (dtype) in[i]
 void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaStream_t st);

@@ -35,12 +35,26 @@ namespace frnnt {
 
 using namespace sm100;
 
+void tile_shape(int U, int* TB, int* UB);
+
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+// warps 0-7 epilogue (two per TMEM lane quadrant, each half of a V tile's
+// columns), warp 8 TMA, warp 9 MMA, warps 10-17 h generators (two per quadrant,
+// each half of every K block)
+constexpr int kThreads = 576;
+constexpr int kEpiWarps = 8, kGenWarps = 8;
+constexpr int kTmaWarp = 8, kMmaWarp = 9, kGen0 = 10;
+constexpr int BN = 128;             // V tile (MMA N)
+constexpr int kStageBytes = BN * 128;
+constexpr int kMaxStages = 16;
 constexpr int kMaxKB = 16;          // H <= 1024
+constexpr int kTmemKB = 8;          // the first 8 K blocks (512 columns of h) live in TMEM
+constexpr int kHCol = 256;          // TMEM columns: [0,128) and [128,256) accumulators, [256,512) h
 constexpr int kDbSlots = 8;
+
+// Shared memory of the staged F / G rows: TB + UB rows of 2H + 16 bytes, 1 KB aligned.
+__host__ __device__ constexpr int fg_bytes(int TB, int UB, int H) { return (((TB + UB) * (2 * H + 16)) + 1023) & ~1023; }
 
 enum JointMode { MODE_FWD = 0, MODE_FWD_STORE = 1, MODE_BWD_DZ = 2 };
 
@@ -49,8 +63,8 @@ struct JointParams {
   int KB;                 // H / 64
   int nV;                 // V / BN
   int stages;
-  const float* F;         // [B*T][H] fp32
-  const float* G;         // [B*(U+1)][H] fp32
+  const __nv_bfloat16* F;   // [B*T][H] bf16
+  const __nv_bfloat16* G;   // [B*(U+1)][H] bf16
   const __nv_bfloat16* b_o;
   const int32_t* labels;
   const int32_t* T_len;
@@ -61,7 +75,8 @@ struct JointParams {
   int tile_begin, tile_end;   // this launch's tile range (clamped by *ntiles)
   Lattice L;
   __nv_bfloat16* zbuf;    // FWD_STORE: z [tile*128 + r][V]; BWD_DZ: dz [(tile-tile_begin)*128 + r][V]
-  __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows, same row indexing as zbuf
+  __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
+  int HS;                 // row stride of hbuf (H + 64)
   float* db_part;         // BWD_DZ: [kDbSlots][V]
   int32_t* status;
 };
@@ -97,40 +112,39 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Sum over the 32 lanes of v[j] for every j; lane l ends up with column l's
-// total in v[0] (reduce-scatter by halving exchanges).
-__device__ __forceinline__ float warp_column_sums(float (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int k = 16; k >= 1; k >>= 1) {
-    const bool upper = (lane & k) != 0;
-#pragma unroll
-    for (int j = 0; j < k; ++j) {
-      const float send = upper ? v[j] : v[j + k];
-      const float keep = upper ? v[j + k] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, k);
-    }
-  }
-  return v[0];
+__device__ __forceinline__ uint32_t tanh_bf16x2(uint32_t x) {
+  uint32_t y;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hadd2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
-template <int BN, int MODE>
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_constant__ CUtensorMap tmW, JointParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int STAGE_BYTES = BN * 128;
-  uint8_t* hs = smem;                                   // KB x 16 KB
-  uint8_t* ring = smem + p.KB * 16384;                  // stages x STAGE_BYTES
-  uint64_t* full = (uint64_t*)(ring + p.stages * STAGE_BYTES);
+  const int KB_hi = p.KB > kTmemKB ? p.KB - kTmemKB : 0;
+  uint8_t* hhi = smem;                                            // K blocks >= kTmemKB of h, 16 KB each
+  uint8_t* ring = hhi + KB_hi * 16384;                            // stages x 16 KB of W_o
+  const int fg_stride = 2 * p.H + 16;                             // padded bf16 row (bank spread)
+  uint8_t* fgs = ring + p.stages * kStageBytes;                   // TB F rows then UB G rows of this tile
+  float* bias_s = (float*)(fgs + fg_bytes(p.TB, p.UB, p.H));      // b_o as fp32
+  uint64_t* full = (uint64_t*)(bias_s + ((p.V + 255) & ~255));
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* hfull = tempty + 2;
   uint64_t* hempty = hfull + kMaxKB;
-  uint32_t* tmem_base_p = (uint32_t*)(hempty + kMaxKB);
+  uint64_t* fg_full = hempty + kMaxKB;
+  uint64_t* fg_empty = fg_full + 1;
+  uint32_t* tmem_base_p = (uint32_t*)(fg_empty + 1);
   volatile int* abort_flag = (volatile int*)(tmem_base_p + 1);
+  float* lse_x = (float*)(tmem_base_p + 4);       // [128][4] half-1 epilogue state for the combine
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = min(p.tile_end, *p.ntiles);
@@ -142,25 +156,28 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     for (int i = 0; i < kMaxKB; ++i) {
-      mbar_init(&hfull[i], 4);
+      mbar_init(&hfull[i], kGenWarps);
       mbar_init(&hempty[i], 1);
     }
+    mbar_init(fg_full, 1);
+    mbar_init(fg_empty, kGenWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
-    tmem_alloc(tmem_base_p, 2 * BN);
+  for (int k = threadIdx.x; k < p.V; k += blockDim.x) bias_s[k] = __bfloat162float(p.b_o[k]);
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_base_p, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) tma_prefetch_desc(&tmW);
+  if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmW);
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
 
-  if (warp == 4) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer: W_o tiles
     if (lane == 0) {
       int s = 0;
@@ -173,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(ring + s * STAGE_BYTES, &tmW, &full[s], kb * 64, n * BN);
+            mbar_arrive_expect_tx(&full[s], kStageBytes);
+            tma_load_2d(ring + s * kStageBytes, &tmW, &full[s], kb * 64, n * BN);
             if (++s == p.stages) {
               s = 0;
               ph ^= 1;
@@ -184,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
@@ -193,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       int acc_i = 0;
       uint32_t hph = 0;
       bool ok = true;
-      const uint32_t hs_addr = smem_u32(hs);
+      const uint32_t hhi_addr = smem_u32(hhi);
       for (int tile = p.tile_begin + blockIdx.x; tile < ntiles && ok; tile += gridDim.x, hph ^= 1) {
         for (int n = 0; n < p.nV && ok; ++n, ++acc_i) {
           const int a = acc_i & 1;
@@ -205,21 +222,31 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           tc_fence_after();
           const uint32_t dt = tbase + a * BN;
           for (int kb = 0; kb < p.KB; ++kb) {
-            if (n == 0 && !mbar_wait(&hfull[kb], hph, abort_flag)) {
-              ok = false;
-              break;
+            if (n == 0) {
+              // h block kb written by the generators (TMEM stores / shared stores)
+              if (!mbar_wait(&hfull[kb], hph, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
+            // W_o stage landed (TMA completion is ordered by the mbarrier itself)
             if (!mbar_wait(&full[s], ph, abort_flag)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            const uint32_t sa = hs_addr + kb * 16384;
-            const uint32_t sb = smem_u32(ring + s * STAGE_BYTES);
+            const uint32_t sb = smem_u32(ring + s * kStageBytes);
+            if (kb < kTmemKB) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16_ss(dt, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024), idesc,
-                          (kb > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts(dt, tbase + kHCol + kb * 32 + k * 8, sdesc_sw128(sb + k * 32, 16, 1024), idesc,
+                            (kb > 0 || k > 0) ? 1u : 0u);
+            } else {
+              const uint32_t sa = hhi_addr + (kb - kTmemKB) * 16384;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ss(dt, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024), idesc, 1u);
+            }
             mma_commit(&empty[s]);
             if (n == p.nV - 1) mma_commit(&hempty[kb]);   // h block kb is free once these MMAs finish
             if (++s == p.stages) {
@@ -232,59 +259,123 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ h generation + epilogue (warps 0-3)
-    const int tid = threadIdx.x;            // 0..127
-    const int r = warp * 32 + lane;         // tile row owned in the epilogue
-    const int H = p.H, V = p.V;
-    const int Up1 = p.U + 1;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    int acc_i = 0;
+  } else if (warp >= kGen0) {
+    // ------------------------------------------------------------ h generators (warps 10-17)
+    // The tile's TB rows of F and UB rows of G are bulk-copied into shared
+    // memory (by warp kGen0, one tile ahead), then every thread builds its row
+    // h[r, :] = tanh(F[t] + G[u]) 16 columns at a time (half of each 64-wide
+    // K block per warp), into TMEM (first 512 columns of h) or the swizzled
+    // shared-memory operand (the rest).
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    const int half = (warp - kGen0) >> 2;    // which two of the four 16-column segments of each K block
+    const int r = q * 32 + lane;             // tile row generated by this thread
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const int H = p.H, Up1 = p.U + 1;
+    const int nseg = H / 16;
     uint32_t hph = 0;
-    for (int tile = p.tile_begin + blockIdx.x; tile < ntiles; tile += gridDim.x, hph ^= 1) {
+    uint32_t fph = 0;
+    // warp kGen0 only: wait until the generator warps are done with the buffer
+    // (empty_parity 1 on the first call passes at once), then copy
+    auto issue_fg = [&](int tile, uint32_t empty_parity) {
+      const int4 td = p.tiles[tile];
+      const int nF = min(p.TB, p.T - td.y), nG = min(p.UB, Up1 - td.z);
+      if (!mbar_wait(fg_empty, empty_parity, abort_flag)) return false;
+      if (lane == 0) mbar_arrive_expect_tx(fg_full, (uint32_t)(nF + nG) * H * 2);
+      __syncwarp();
+      if (lane < nF)
+        bulk_load(fgs + lane * fg_stride, p.F + ((size_t)td.x * p.T + td.y + lane) * H, H * 2, fg_full);
+      else if (lane >= 16 && lane - 16 < nG)
+        bulk_load(fgs + (p.TB + lane - 16) * fg_stride, p.G + ((size_t)td.x * Up1 + td.z + lane - 16) * H, H * 2,
+                  fg_full);
+      return true;
+    };
+    int tile = p.tile_begin + blockIdx.x;
+    bool ok = true;
+    if (warp == kGen0 && tile < ntiles) ok = issue_fg(tile, 1u);
+    for (; tile < ntiles && ok; tile += gridDim.x, hph ^= 1, fph ^= 1) {
+      const int4 td = p.tiles[tile];
+      const RowInfo ri = row_info(p, td, r);
+      const size_t row_base = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
+      __nv_bfloat16* hrow = (MODE != MODE_FWD) ? p.hbuf + (row_base + r) * p.HS : nullptr;
+      if (MODE != MODE_FWD && half == 0) {
+        // the extra column block of the hidden row: 1 at column H (so the dW_o GEMM also yields
+        // db_o = sum over cells of dz), zeros after it
+        uint4* e = (uint4*)(hrow + H);
+        e[0] = make_uint4(ri.valid ? 0x3F80u : 0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int j = 1; j < 8; ++j) e[j] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
+      const uint8_t* grow = fgs + (p.TB + r % p.UB) * fg_stride;
+      if (!mbar_wait(fg_full, fph, abort_flag)) break;
+      for (int si = 0; si < nseg / 2; ++si) {
+        const int kb = si >> 1, sub = 2 * half + (si & 1);
+        const int seg = kb * 4 + sub;
+        uint32_t pk[8];
+        if (ri.valid) {
+          // h = tanh(F + G) in packed bf16 pairs (F, G already bf16; h is consumed as bf16)
+          const uint4 f0 = *(const uint4*)(frow + seg * 32), f1 = *(const uint4*)(frow + seg * 32 + 16);
+          const uint4 g0 = *(const uint4*)(grow + seg * 32), g1 = *(const uint4*)(grow + seg * 32 + 16);
+          pk[0] = tanh_bf16x2(add_bf16x2(f0.x, g0.x));
+          pk[1] = tanh_bf16x2(add_bf16x2(f0.y, g0.y));
+          pk[2] = tanh_bf16x2(add_bf16x2(f0.z, g0.z));
+          pk[3] = tanh_bf16x2(add_bf16x2(f0.w, g0.w));
+          pk[4] = tanh_bf16x2(add_bf16x2(f1.x, g1.x));
+          pk[5] = tanh_bf16x2(add_bf16x2(f1.y, g1.y));
+          pk[6] = tanh_bf16x2(add_bf16x2(f1.z, g1.z));
+          pk[7] = tanh_bf16x2(add_bf16x2(f1.w, g1.w));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) pk[j] = 0u;
+        }
+        if ((si & 1) == 0 && !mbar_wait(&hempty[kb], hph ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (kb < kTmemKB) {
+          tmem_st8(tbase + lane_base + kHCol + kb * 32 + sub * 8, pk);
+        } else {
+          uint8_t* blk = hhi + (kb - kTmemKB) * 16384;
+          *(uint4*)(blk + sw128_offset(r, sub * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *(uint4*)(blk + sw128_offset(r, sub * 16 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        if (MODE != MODE_FWD) {
+          uint4* dst = (uint4*)(hrow + seg * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        if ((si & 1) == 1) {
+          if (kb < kTmemKB) {
+            tmem_wait_st();
+            tc_fence_before();
+          } else {
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hfull[kb]);
+        }
+      }
+      if (!ok) break;
+      // this warp is done reading the tile's F/G rows
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fg_empty);
+      if (warp == kGen0 && tile + (int)gridDim.x < ntiles) ok = issue_fg(tile + gridDim.x, fph);
+      if (*abort_flag) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-7)
+    const int q = warp & 3;                   // TMEM lane quadrant
+    const int half = warp >> 2;               // columns [64 half, 64 half + 64) of each V tile
+    const int r = q * 32 + lane;
+    const int V = p.V, Up1 = p.U + 1;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    int acc_i = 0;
+    for (int tile = p.tile_begin + blockIdx.x; tile < ntiles; tile += gridDim.x) {
       const int4 td = p.tiles[tile];
       const size_t row_base = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
-      // rows this thread generates: (tid >> 3) + 16 i, i = 0..7; -1 marks a cell outside the lattice
-      int frow[8], grow[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const RowInfo gi = row_info(p, td, (tid >> 3) + 16 * i);
-        frow[i] = gi.valid ? gi.b * p.T + gi.t : -1;
-        grow[i] = gi.b * Up1 + gi.u;
-      }
-      const int c8 = tid & 7;
-      // ---- generate h, one 64-wide K block at a time
-      for (int kb = 0; kb < p.KB; ++kb) {
-        if (!mbar_wait(&hempty[kb], hph ^ 1, abort_flag)) break;
-        uint8_t* blk = hs + kb * 16384;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = (tid >> 3) + 16 * i;
-          uint4 packed = make_uint4(0, 0, 0, 0);
-          if (frow[i] >= 0) {
-            const float* Fr = p.F + (size_t)frow[i] * H + kb * 64 + c8 * 8;
-            const float* Gr = p.G + (size_t)grow[i] * H + kb * 64 + c8 * 8;
-            const float4 f0 = __ldg((const float4*)Fr), f1 = __ldg((const float4*)Fr + 1);
-            const float4 g0 = __ldg((const float4*)Gr), g1 = __ldg((const float4*)Gr + 1);
-            packed.x = pack_bf16x2(tanh_approx(f0.x + g0.x), tanh_approx(f0.y + g0.y));
-            packed.y = pack_bf16x2(tanh_approx(f0.z + g0.z), tanh_approx(f0.w + g0.w));
-            packed.z = pack_bf16x2(tanh_approx(f1.x + g1.x), tanh_approx(f1.y + g1.y));
-            packed.w = pack_bf16x2(tanh_approx(f1.z + g1.z), tanh_approx(f1.w + g1.w));
-          }
-          *(uint4*)(blk + sw128_offset(row, c8 * 8)) = packed;
-          if (MODE != MODE_FWD)
-            *(uint4*)(p.hbuf + (row_base + row) * H + kb * 64 + c8 * 8) = packed;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&hfull[kb]);
-      }
-      if (*abort_flag) break;
-
-      // ---- per-row state
       const RowInfo ri = row_info(p, td, r);
       float m = -INFINITY, ssum = 0.f, zb = 0.f, zy = 0.f;
-      float lse = 0.f, bpost = 0.f, lpost = 0.f, occ = 0.f, w = 0.f;
+      float lk = 0.f, bpost = 0.f, lpost = 0.f, occ = 0.f;
       if (MODE == MODE_BWD_DZ && ri.valid) {
         const size_t c = ri.cell;
         const float logp = p.L.beta[(size_t)ri.b * p.T * Up1];
@@ -292,53 +383,65 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
         float beta_t1;
         if (ri.t + 1 < ri.Tb) beta_t1 = p.L.beta[c + Up1];
         else beta_t1 = (ri.u == ri.Ub) ? 0.f : -INFINITY;
-        lse = p.L.lse[c];
-        bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp);
-        lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) : 0.f;
+        lk = p.L.lse[c] * kLog2e;
+        const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
+        bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp) * w;
+        lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) * w : 0.f;
         occ = bpost + lpost;
-        w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
       }
-
-      // ---- epilogue over the V tiles
+      bool ok = true;
       for (int n = 0; n < p.nV; ++n, ++acc_i) {
         const int a = acc_i & 1;
         const uint32_t aph = (acc_i >> 1) & 1;
-        if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+        if (!mbar_wait(&tfull[a], aph, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tbase + lane_base + a * BN + c * 32, rr);
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
+          uint32_t buf[32];
+          tmem_ld32(tbase + lane_base + a * BN + c * 32, buf);
           tmem_wait_ld();
           const int col0 = n * BN + c * 32;
           float v[32];
-          const uint4* bp = (const uint4*)(p.b_o + col0);
+          const float4* b4 = (const float4*)(bias_s + col0);
 #pragma unroll
-          for (int j8 = 0; j8 < 4; ++j8) {
-            const uint4 bw = __ldg(bp + j8);
-            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb[q]));
-              v[8 * j8 + 2 * q] = __uint_as_float(rr[8 * j8 + 2 * q]) + bf.x;
-              v[8 * j8 + 2 * q + 1] = __uint_as_float(rr[8 * j8 + 2 * q + 1]) + bf.y;
-            }
+          for (int j = 0; j < 8; ++j) {
+            const float4 bb = b4[j];
+            v[4 * j] = __uint_as_float(buf[4 * j]) + bb.x;
+            v[4 * j + 1] = __uint_as_float(buf[4 * j + 1]) + bb.y;
+            v[4 * j + 2] = __uint_as_float(buf[4 * j + 2]) + bb.z;
+            v[4 * j + 3] = __uint_as_float(buf[4 * j + 3]) + bb.w;
           }
           if (MODE != MODE_BWD_DZ) {
-            float cm = v[0];
+            float t0 = fmaxf(v[0], v[1]), t1 = fmaxf(v[2], v[3]);
 #pragma unroll
-            for (int j = 1; j < 32; ++j) cm = fmaxf(cm, v[j]);
-            const float mn = fmaxf(m, cm);
-            float acc = ssum * ex2((m - mn) * kLog2e);
+            for (int j = 4; j < 32; j += 4) {
+              t0 = fmaxf(t0, fmaxf(v[j], v[j + 1]));
+              t1 = fmaxf(t1, fmaxf(v[j + 2], v[j + 3]));
+            }
+            const float mn = fmaxf(m, fmaxf(t0, t1));
             const float mk = mn * kLog2e;
+            float s0 = ssum * ex2((m - mn) * kLog2e), s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc += ex2(fmaf(v[j], kLog2e, -mk));
-            ssum = acc;
+            for (int j = 0; j < 32; j += 4) {
+              s0 += ex2(fmaf(v[j], kLog2e, -mk));
+              s1 += ex2(fmaf(v[j + 1], kLog2e, -mk));
+              s2 += ex2(fmaf(v[j + 2], kLog2e, -mk));
+              s3 += ex2(fmaf(v[j + 3], kLog2e, -mk));
+            }
+            ssum = (s0 + s1) + (s2 + s3);
             m = mn;
+            if (p.blank >= col0 && p.blank < col0 + 32) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (col0 + j == p.blank) zb = v[j];
-              if (col0 + j == ri.y) zy = v[j];
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j == p.blank) zb = v[j];
+            }
+            if (ri.y >= col0 && ri.y < col0 + 32) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j == ri.y) zy = v[j];
             }
             if (MODE == MODE_FWD_STORE) {
               uint4* dst = (uint4*)(p.zbuf + (row_base + r) * V + col0);
@@ -349,41 +452,53 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
                                     pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
             }
           } else {
-            const float lk = lse * kLog2e;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               float d = occ * ex2(fmaf(v[j], kLog2e, -lk));
               if (col0 + j == p.blank) d -= bpost;
               if (col0 + j == ri.y) d -= lpost;
-              v[j] = ri.valid ? d * w : 0.f;
+              v[j] = ri.valid ? d : 0.f;
             }
             uint4* dst = (uint4*)(p.zbuf + (row_base + r) * V + col0);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                                   pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-            const float colsum = warp_column_sums(v);
-            atomicAdd(p.db_part + (size_t)(blockIdx.x % kDbSlots) * V + col0 + lane, colsum);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[a]);
       }
-      if (*abort_flag) break;
-      if (MODE != MODE_BWD_DZ && ri.valid) {
-        const float l = m + __logf(ssum);
-        p.L.lse[ri.cell] = l;
-        p.L.blank_lp[ri.cell] = zb - l;
-        p.L.label_lp[ri.cell] = ri.u < ri.Ub ? zy - l : -INFINITY;
+      if (!ok || *abort_flag) break;
+      if (MODE != MODE_BWD_DZ) {
+        // combine the two column halves of this row: half 1 hands its state to half 0
+        if (half == 1) {
+          lse_x[r * 4 + 0] = m;
+          lse_x[r * 4 + 1] = ssum;
+          lse_x[r * 4 + 2] = zb;
+          lse_x[r * 4 + 3] = zy;
+        }
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+        if (half == 0 && ri.valid) {
+          const float m1 = lse_x[r * 4 + 0], s1 = lse_x[r * 4 + 1];
+          const float mm = fmaxf(m, m1);
+          const float st = ssum * ex2((m - mm) * kLog2e) + s1 * ex2((m1 - mm) * kLog2e);
+          const float l = mm + __logf(st);
+          const float zbb = zb + lse_x[r * 4 + 2], zyy = zy + lse_x[r * 4 + 3];
+          p.L.lse[ri.cell] = l;
+          p.L.blank_lp[ri.cell] = zbb - l;
+          p.L.label_lp[ri.cell] = ri.u < ri.Ub ? zyy - l : -INFINITY;
+        }
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
       }
     }
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tbase, 2 * BN);
+    tmem_dealloc(tbase, 512);
   }
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, FRNNT_STATUS_TIMEOUT);
 }
@@ -426,9 +541,6 @@ __global__ void dz_from_z_kernel(JointParams p) {
   const int V = p.V, Up1 = p.U + 1;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
-  extern __shared__ float dbs[];   // [V] block partial sums
-  for (int k = threadIdx.x; k < V; k += blockDim.x) dbs[k] = 0.f;
-  __syncthreads();
   for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows;
        row += (long long)gridDim.x * (blockDim.x >> 5)) {
     const int tile = p.tile_begin + (int)(row >> 7);
@@ -445,10 +557,10 @@ __global__ void dz_from_z_kernel(JointParams p) {
     if (ri.t + 1 < ri.Tb) beta_t1 = p.L.beta[c + Up1];
     else beta_t1 = (ri.u == ri.Ub) ? 0.f : -INFINITY;
     const float lse = p.L.lse[c];
-    const float bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp);
-    const float lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) : 0.f;
-    const float occ = bpost + lpost;
     const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
+    const float bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp) * w;
+    const float lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) * w : 0.f;
+    const float occ = bpost + lpost;
     const float lk = lse * kLog2e;
     for (int k = lane * 8; k < V; k += 256) {
       uint4 zv = *(const uint4*)(zr + k);
@@ -464,18 +576,11 @@ __global__ void dz_from_z_kernel(JointParams p) {
         if (k0 + 1 == p.blank) d1 -= bpost;
         if (k0 == ri.y) d0 -= lpost;
         if (k0 + 1 == ri.y) d1 -= lpost;
-        d0 *= w;
-        d1 *= w;
-        atomicAdd(&dbs[k0], d0);
-        atomicAdd(&dbs[k0 + 1], d1);
         o[q] = pack_bf16x2(d0, d1);
       }
       *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
-  __syncthreads();
-  for (int k = threadIdx.x; k < V; k += blockDim.x)
-    atomicAdd(p.db_part + (size_t)(blockIdx.x % kDbSlots) * V + k, dbs[k]);
 }
 
 // ------------------------------------------------------------------ dtanh'd hidden gradient -> dF, dG
@@ -489,16 +594,19 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
   const int4 td = p.tiles[tile];
   const int H = p.H, TB = p.TB, UB = p.UB, Up1 = p.U + 1;
   const Lengths l = lengths_of(p.T_len, p.U_len, td.x, p.T, p.U);
-  const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * H;
-  // each thread owns 8 consecutive columns; dF rows first, then dG rows
+  const int HS = p.HS;
+  const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * HS;
+  // thread (c8, g): 8 consecutive columns, frame rows tl = g (mod 4) for dF and
+  // label rows ul = g (mod 4) for dG
+  const int g = threadIdx.y;
   for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
-    for (int tl = 0; tl < TB; ++tl) {
+    for (int tl = g; tl < TB; tl += 4) {
       const int t = td.y + tl;
       if (t >= l.Tb) break;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int ul = 0; ul < UB; ++ul) {
         if (td.z + ul > l.Ub) break;
-        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * H + c8 * 8);
+        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * HS + c8 * 8);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -511,13 +619,13 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
       red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
       red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
     }
-    for (int ul = 0; ul < UB; ++ul) {
+    for (int ul = g; ul < UB; ul += 4) {
       const int u = td.z + ul;
       if (u > l.Ub) break;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int tl = 0; tl < TB; ++tl) {
         if (td.y + tl >= l.Tb) break;
-        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * H + c8 * 8);
+        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * HS + c8 * 8);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -533,12 +641,15 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
   }
 }
 
-__global__ void db_finalize_kernel(const float* __restrict__ db_part, int V, void* out, int to_bf16) {
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < V; k += gridDim.x * blockDim.x) {
-    float s = 0.f;
-    for (int i = 0; i < kDbSlots; ++i) s += db_part[(size_t)i * V + k];
-    if (to_bf16) ((__nv_bfloat16*)out)[k] = __float2bfloat16_rn(s);
-    else ((float*)out)[k] = s;
+// dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][H + 64]
+// whose column H is the sum of dz over cells.
+__global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, __nv_bfloat16* __restrict__ dW_o,
+                                   __nv_bfloat16* __restrict__ db_o) {
+  const long long n = (long long)V * H;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long k = i / H, j = i % H;
+    dW_o[i] = __float2bfloat16_rn(acc[k * HS + j]);
+    if (j == 0) db_o[k] = __float2bfloat16_rn(acc[k * HS + H]);
   }
 }
 
@@ -554,26 +665,29 @@ int sms() {
 }
 
 constexpr int kSmemLimit = 232448;   // max dynamic shared memory per block on sm_100
-constexpr int kBarBytes = 1024;
+constexpr int kBarBytes = 4096;   // mbarriers + TMEM address + abort flag + 2 KB epilogue combine area
 
-template <int BN>
-int stages_for(int KB) {
-  const int avail = kSmemLimit - 1024 - kBarBytes - KB * 16384;
-  int st = avail / (BN * 128);
+int smem_fixed(int KB, int V, int TB, int UB) {
+  const int KB_hi = KB > kTmemKB ? KB - kTmemKB : 0;
+  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 255) & ~255) * 4 + kBarBytes;
+}
+
+int stages_for(int KB, int V, int TB, int UB) {
+  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB)) / kStageBytes;
   return st > kMaxStages ? kMaxStages : st;
 }
 
-template <int BN, int MODE>
+template <int MODE>
 int launch_joint_t(const CUtensorMap& tm, JointParams p, cudaStream_t st) {
-  p.stages = stages_for<BN>(p.KB);
+  p.stages = stages_for(p.KB, p.V, p.TB, p.UB);
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
-  const int smem = 1024 + p.KB * 16384 + p.stages * BN * 128 + kBarBytes;
-  auto kern = joint_tc_kernel<BN, MODE>;
-  static int attr_set = 0;
-  if (attr_set < smem) {
+  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB) + p.stages * kStageBytes;
+  auto kern = joint_tc_kernel<MODE>;
+  static bool attr_set = false;
+  if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return FRNNT_ERR_CUDA;
-    attr_set = kSmemLimit;
+    attr_set = true;
   }
   kern<<<sms(), kThreads, smem, st>>>(tm, p);
   note_launch();
@@ -583,10 +697,11 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, cudaStream_t st) {
 }  // namespace
 
 // ------------------------------------------------------------------ host entry points
-bool joint_tc_supported(int H, int V) {
+bool joint_tc_supported(int H, int V, int U) {
   if (H % 64 || H > 1024 || V % 128) return false;
-  const int KB = H / 64;
-  return (V % 256 == 0) ? stages_for<256>(KB) >= 2 : stages_for<128>(KB) >= 2;
+  int TB, UB;
+  tile_shape(U, &TB, &UB);
+  return stages_for(H / 64, V, TB, UB) >= 2;
 }
 
 void tile_shape(int U, int* TB, int* UB) {
@@ -620,8 +735,8 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.TB = j.TB;
   p.UB = j.UB;
   p.KB = j.s.H / 64;
-  p.F = j.F;
-  p.G = j.G;
+  p.F = (const __nv_bfloat16*)j.F;
+  p.G = (const __nv_bfloat16*)j.G;
   p.b_o = (const __nv_bfloat16*)j.b_o;
   p.labels = j.labels;
   p.T_len = j.T_len;
@@ -634,21 +749,15 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
+  p.HS = j.s.H + 64;
   p.db_part = j.db_part;
   p.status = j.status;
-  const int BN = (p.V % 256 == 0) ? 256 : 128;
   p.nV = p.V / BN;
   CUtensorMap tm;
   if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.V, p.H, 64, BN)) return FRNNT_ERR_CUDA;
-  const int mode = j.mode;
-  if (BN == 256) {
-    if (mode == MODE_FWD) return launch_joint_t<256, MODE_FWD>(tm, p, st);
-    if (mode == MODE_FWD_STORE) return launch_joint_t<256, MODE_FWD_STORE>(tm, p, st);
-    return launch_joint_t<256, MODE_BWD_DZ>(tm, p, st);
-  }
-  if (mode == MODE_FWD) return launch_joint_t<128, MODE_FWD>(tm, p, st);
-  if (mode == MODE_FWD_STORE) return launch_joint_t<128, MODE_FWD_STORE>(tm, p, st);
-  return launch_joint_t<128, MODE_BWD_DZ>(tm, p, st);
+  if (j.mode == MODE_FWD) return launch_joint_t<MODE_FWD>(tm, p, st);
+  if (j.mode == MODE_FWD_STORE) return launch_joint_t<MODE_FWD_STORE>(tm, p, st);
+  return launch_joint_t<MODE_BWD_DZ>(tm, p, st);
 }
 
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
@@ -670,8 +779,7 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.tile_end = j.tile_end;
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
-  p.db_part = j.db_part;
-  dz_from_z_kernel<<<sms() * 4, 256, (size_t)p.V * sizeof(float), st>>>(p);
+  dz_from_z_kernel<<<sms() * 4, 256, 0, st>>>(p);
   note_launch();
 }
 
@@ -688,16 +796,20 @@ void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, fl
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
+  p.HS = j.s.H + 64;
   const int n = j.tile_end - j.tile_begin;
   if (n <= 0) return;
   int threads = (p.H / 8 + 31) / 32 * 32;
   if (threads > 128) threads = 128;
-  seg_reduce_kernel<<<n, threads, 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
+  seg_reduce_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
   note_launch();
 }
 
-void launch_db_finalize(const float* db_part, int V, void* out, bool to_bf16, cudaStream_t st) {
-  db_finalize_kernel<<<(V + 255) / 256, 256, 0, st>>>(db_part, V, out, to_bf16);
+void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st) {
+  long long n = (long long)V * H;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, H + 64, (__nv_bfloat16*)dW_o, (__nv_bfloat16*)db_o);
   note_launch();
 }
 
