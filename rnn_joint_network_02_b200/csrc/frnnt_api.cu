@@ -290,6 +290,10 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
         FRNNT_TRY(launch_joint_tc(j, st));
       }
     }
+    {
+      StageScope sc("bwd_hidden", st);
+      launch_hidden_rows(j, untiled ? 0 : (int)c0, st);
+    }
     const int rows = (int)((c1 - c0) * 128);
     {
       StageScope sc("bwd_dWo", st);

@@ -135,6 +135,7 @@ void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const in
                   cudaStream_t st);
 int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
+void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st);
 void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);
 void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st);
 

@@ -133,8 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   uint8_t* ring = hhi + KB_hi * 16384;                            // stages x 16 KB of W_o
   const int fg_stride = 2 * p.H + 16;                             // padded bf16 row (bank spread)
   uint8_t* fgs = ring + p.stages * kStageBytes;                   // TB F rows then UB G rows of this tile
-  float* bias_s = (float*)(fgs + fg_bytes(p.TB, p.UB, p.H));      // b_o as fp32
-  uint64_t* full = (uint64_t*)(bias_s + ((p.V + 255) & ~255));
+  __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + fg_bytes(p.TB, p.UB, p.H));   // b_o (bf16)
+  uint64_t* full = (uint64_t*)(bias_s + ((p.V + 511) & ~511));
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int k = threadIdx.x; k < p.V; k += blockDim.x) bias_s[k] = __bfloat162float(p.b_o[k]);
+  for (int k = threadIdx.x; k < p.V; k += blockDim.x) bias_s[k] = p.b_o[k];
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_base_p, 512);
     tmem_relinquish();
@@ -295,16 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     for (; tile < ntiles && ok; tile += gridDim.x, hph ^= 1, fph ^= 1) {
       const int4 td = p.tiles[tile];
       const RowInfo ri = row_info(p, td, r);
-      const size_t row_base = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
-      __nv_bfloat16* hrow = (MODE != MODE_FWD) ? p.hbuf + (row_base + r) * p.HS : nullptr;
-      if (MODE != MODE_FWD && half == 0) {
-        // the extra column block of the hidden row: 1 at column H (so the dW_o GEMM also yields
-        // db_o = sum over cells of dz), zeros after it
-        uint4* e = (uint4*)(hrow + H);
-        e[0] = make_uint4(ri.valid ? 0x3F80u : 0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int j = 1; j < 8; ++j) e[j] = make_uint4(0u, 0u, 0u, 0u);
-      }
       const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
       const uint8_t* grow = fgs + (p.TB + r % p.UB) * fg_stride;
       if (!mbar_wait(fg_full, fph, abort_flag)) break;
@@ -338,11 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           uint8_t* blk = hhi + (kb - kTmemKB) * 16384;
           *(uint4*)(blk + sw128_offset(r, sub * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *(uint4*)(blk + sw128_offset(r, sub * 16 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-        if (MODE != MODE_FWD) {
-          uint4* dst = (uint4*)(hrow + seg * 16);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
         if ((si & 1) == 1) {
           if (kb < kTmemKB) {
@@ -405,14 +390,17 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           tmem_wait_ld();
           const int col0 = n * BN + c * 32;
           float v[32];
-          const float4* b4 = (const float4*)(bias_s + col0);
+          const uint4* b8 = (const uint4*)(bias_s + col0);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 bb = b4[j];
-            v[4 * j] = __uint_as_float(buf[4 * j]) + bb.x;
-            v[4 * j + 1] = __uint_as_float(buf[4 * j + 1]) + bb.y;
-            v[4 * j + 2] = __uint_as_float(buf[4 * j + 2]) + bb.z;
-            v[4 * j + 3] = __uint_as_float(buf[4 * j + 3]) + bb.w;
+          for (int j = 0; j < 4; ++j) {
+            const uint4 bw = b8[j];
+            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb[q]));
+              v[8 * j + 2 * q] = __uint_as_float(buf[8 * j + 2 * q]) + bf.x;
+              v[8 * j + 2 * q + 1] = __uint_as_float(buf[8 * j + 2 * q + 1]) + bf.y;
+            }
           }
           if (MODE != MODE_BWD_DZ) {
             float t0 = fmaxf(v[0], v[1]), t1 = fmaxf(v[2], v[3]);
@@ -583,6 +571,38 @@ __global__ void dz_from_z_kernel(JointParams p) {
   }
 }
 
+// ------------------------------------------------------------------ hidden rows for the backward GEMMs
+// h rows (bf16, stride HS = H + 64) of tiles [tile_begin, ntiles) into hbuf rows
+// (tile - row_tile0) * 128 + r: the same packed-bf16 tanh(F + G) as the joint
+// kernel, plus the extra column block [1, 0, ..., 0] (0 for cells outside the
+// lattice) whose dz-weighted sum is db_o.  One warp per row, coalesced.
+__global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int H = p.H, HS = p.HS, Up1 = p.U + 1;
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows;
+       row += (long long)gridDim.x * (blockDim.x >> 5)) {
+    const int tile = p.tile_begin + (int)(row >> 7);
+    const RowInfo ri = row_info(p, p.tiles[tile], (int)(row & 127));
+    __nv_bfloat16* hr = p.hbuf + ((size_t)(tile - row_tile0) * 128 + (row & 127)) * HS;
+    const __nv_bfloat16* Fr = p.F + ((size_t)ri.b * p.T + (ri.valid ? ri.t : 0)) * H;
+    const __nv_bfloat16* Gr = p.G + ((size_t)ri.b * Up1 + (ri.valid ? ri.u : 0)) * H;
+    for (int k = lane * 8; k < H; k += 256) {
+      uint4 o = make_uint4(0u, 0u, 0u, 0u);
+      if (ri.valid) {
+        const uint4 f = *(const uint4*)(Fr + k), g = *(const uint4*)(Gr + k);
+        o.x = tanh_bf16x2(add_bf16x2(f.x, g.x));
+        o.y = tanh_bf16x2(add_bf16x2(f.y, g.y));
+        o.z = tanh_bf16x2(add_bf16x2(f.z, g.z));
+        o.w = tanh_bf16x2(add_bf16x2(f.w, g.w));
+      }
+      *(uint4*)(hr + k) = o;
+    }
+    if (lane < 8) *(uint4*)(hr + H + lane * 8) = make_uint4((lane == 0 && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
+  }
+}
+
 // ------------------------------------------------------------------ dtanh'd hidden gradient -> dF, dG
 // dpre rows of the tiles in [tile_begin, ntiles) (bf16, rows (tile - row_tile0) * 128 + r):
 // dF[b, t] += sum over the tile's u of dpre, dG[b, u] += sum over the tile's t.
@@ -665,11 +685,11 @@ int sms() {
 }
 
 constexpr int kSmemLimit = 232448;   // max dynamic shared memory per block on sm_100
-constexpr int kBarBytes = 4096;   // mbarriers + TMEM address + abort flag + 2 KB epilogue combine area
+constexpr int kBarBytes = 3072;   // mbarriers + TMEM address + abort flag + 2 KB epilogue combine area
 
 int smem_fixed(int KB, int V, int TB, int UB) {
   const int KB_hi = KB > kTmemKB ? KB - kTmemKB : 0;
-  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 255) & ~255) * 4 + kBarBytes;
+  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 511) & ~511) * 2 + kBarBytes;
 }
 
 int stages_for(int KB, int V, int TB, int UB) {
@@ -780,6 +800,29 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   dz_from_z_kernel<<<sms() * 4, 256, 0, st>>>(p);
+  note_launch();
+}
+
+void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st) {
+  JointParams p{};
+  p.T = j.s.T;
+  p.U = j.s.U;
+  p.H = j.s.H;
+  p.V = j.s.V;
+  p.TB = j.TB;
+  p.UB = j.UB;
+  p.HS = j.s.H + 64;
+  p.F = (const __nv_bfloat16*)j.F;
+  p.G = (const __nv_bfloat16*)j.G;
+  p.labels = j.labels;
+  p.T_len = j.T_len;
+  p.U_len = j.U_len;
+  p.tiles = j.tiles;
+  p.ntiles = j.ntiles;
+  p.tile_begin = j.tile_begin;
+  p.tile_end = j.tile_end;
+  p.hbuf = (__nv_bfloat16*)j.hbuf;
+  hidden_rows_kernel<<<sms() * 8, 256, 0, st>>>(p, row_tile0);
   note_launch();
 }
 
