@@ -28,6 +28,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from rnn_joint_network_02_b200 import dist as rdist  # noqa: E402
 from rnn_joint_network_02_b200 import frnnt, synth  # noqa: E402
 
 METRIC = "RNN-T joint+loss fwd+bwd lattice-vocab cells/sec (B·T·(U+1)·V) and peak GB"
@@ -234,9 +235,13 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def call(check=False):
-        return frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
-                             d["U_len"], mode=args.mode, path=args.path, chunk_cells=args.chunk_cells,
-                             blank=batch.blank, out=out, check=check, stream=stream)
+        res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                            d["U_len"], mode=args.mode, path=args.path, chunk_cells=args.chunk_cells,
+                            blank=batch.blank, out=out, check=check, stream=stream)
+        if world > 1:
+            # the data-parallel exchange: weight gradients summed over ranks
+            rdist.allreduce_weight_grads(res[1])
+        return res
 
     # peak device memory of one call: every buffer is caller-owned, so the
     # peak is inputs + outputs + workspace (no flush buffer allocated yet)
