@@ -43,7 +43,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="medium", choices=list(synth.WORKLOADS))
-    p.add_argument("--mode", default="tiled", choices=["tiled", "untiled"])
+    p.add_argument("--mode", default="both", choices=["both", "tiled", "untiled"],
+                   help="both: untiled is the headline value, tiled is reported alongside")
     p.add_argument("--path", default="auto", choices=["auto", "simt"])
     p.add_argument("--chunk-cells", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -213,49 +214,33 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    idx = synth.WORKLOADS[args.workload]["index"]
-    batch = synth.workload(args.workload, seed=1000 + idx + 7919 * rank)
-    d = {k: getattr(batch, k).to(dev).contiguous()
-         for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
+    """Times one mode: warm-up, K timed steps (each after an L2 flush), the
+    end-to-end variant with host buffers, per-stage device times."""
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
-    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, args.mode, args.path, args.chunk_cells, batch.blank)
+    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank)
     out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims)
     stream = torch.cuda.current_stream(dev)
 
     def call(check=False):
         res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
-                            d["U_len"], mode=args.mode, path=args.path, chunk_cells=args.chunk_cells,
+                            d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells,
                             blank=batch.blank, out=out, check=check, stream=stream)
         if world > 1:
             # the data-parallel exchange: weight gradients summed over ranks
             rdist.allreduce_weight_grads(res[1])
         return res
 
-    # peak device memory of one call: every buffer is caller-owned, so the
-    # peak is inputs + outputs + workspace (no flush buffer allocated yet)
+    # peak device memory of one call: the library allocates nothing, so the
+    # peak is inputs + outputs + workspace (measured before other buffers exist)
     call(check=True)
     torch.cuda.synchronize()
+    flush_bytes = flush.numel()           # the L2-flush buffer is the bench's, not the call's
     torch.cuda.reset_peak_memory_stats(dev)
     call(check=True)
     torch.cuda.synchronize()
-    peak_bytes = torch.cuda.max_memory_allocated(dev)
-    elt = 2 if dtype == "bf16" else 4
-    footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
-                 4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
+    peak_bytes = torch.cuda.max_memory_allocated(dev) - flush_bytes
 
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
@@ -286,11 +271,9 @@ def run_ours(args):
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    units = batch.padded_cells() * batch.dims["V"]
-    value = world * units / (ms / 1e3)
 
-    # end to end through the public API with host buffers: pinned H2D of
-    # the step's inputs, the call, D2H of the loss and status word
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the call, D2H of the loss and status word
     host = {k: v.cpu().pin_memory() for k, v in d.items()}
     loss_h = torch.empty(batch.f.shape[0], dtype=torch.float32).pin_memory()
     status_h = torch.empty(4, dtype=torch.int32).pin_memory()
@@ -319,26 +302,60 @@ def run_ours(args):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e = float(t.item())
 
+    units = batch.padded_cells() * batch.dims["V"]
     launches = sum(v["launches"] for v in stages.values())
     roofline = None
     pk = peaks()
     if stages:
         dom = max(stages, key=lambda k: stages[k]["ms"])
-        kind, work = stage_work(batch, dom, args.mode)
-        per_launch_ms = stages[dom]["ms"] / max(stages[dom]["calls"], 1)
-        work_per_call = work / max(stages[dom]["calls"] / args.steps, 1)
+        kind, work = stage_work(batch, dom, mode)
+        per_call_ms = stages[dom]["ms"] / args.steps
         if kind == "tensor":
-            achieved = work_per_call / (per_launch_ms / 1e3) / 1e12
+            achieved = work / (per_call_ms / 1e3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor_sustained"], "unit": "TFLOP/s",
                         "frac": achieved / pk["tensor_sustained"], "traffic": None, "stage": dom,
-                        "peak_source": pk["source"] + " sustained bf16"}
+                        "launches_per_step": stages[dom]["launches"] / args.steps,
+                        "peak_source": pk["source"] + " sustained dense bf16 (the stage runs inside a long step)"}
         elif kind == "hbm":
-            achieved = work_per_call / (per_launch_ms / 1e3) / 1e9
+            achieved = work / (per_call_ms / 1e3) / 1e9
             roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                         "frac": achieved / pk["hbm"], "traffic": None, "stage": dom, "peak_source": pk["source"]}
-        else:
-            roofline = {"bound": None, "stage": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
-                        "traffic": None}
+    return {"ms": ms, "value": world * units / (ms / 1e3), "peak_bytes": peak_bytes,
+            "valid_cells_per_s": world * batch.valid_cells() * batch.dims["V"] / (ms / 1e3),
+            "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+            "launches": launches, "roofline": roofline, "clocks": clocks,
+            "stages": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps}
+                       for k, v in stages.items()}}
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    idx = synth.WORKLOADS[args.workload]["index"]
+    batch = synth.workload(args.workload, seed=1000 + idx + 7919 * rank)
+    d = {k: getattr(batch, k).to(dev).contiguous()
+         for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+    dtype = "bf16" if batch.dtype == "bf16" else "f32"
+    elt = 2 if dtype == "bf16" else 4
+    footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
+                 4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
+
+    modes = ["untiled", "tiled"] if args.mode == "both" else [args.mode]
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    results = {}
+    for m in modes:
+        results[m] = measure_mode(args, m, batch, d, dev, world, rank, local, flush)
+    head = results[modes[0]]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -349,19 +366,21 @@ def run_ours(args):
                          f"utterance; numpy fp64, BLAS threads = all cores"}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        cfg = config_of(batch, args, world)
+        cfg["mode"] = modes[0]
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes of the workload)",
-                "config": config_of(batch, args, world),
-                "peak_gb": peak_bytes / 1e9, "footprint_gb": footprint / 1e9,
-                "peak_over_footprint": peak_bytes / footprint,
-                "valid_cells_per_s": world * batch.valid_cells() * batch.dims["V"] / (ms / 1e3),
-                "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
-                "gpu_launches": launches,
-                "stages": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps}
-                           for k, v in stages.items()},
-                "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks}
+                "config": cfg,
+                "peak_gb": head["peak_bytes"] / 1e9, "footprint_gb": footprint / 1e9,
+                "peak_over_footprint": head["peak_bytes"] / footprint,
+                "valid_cells_per_s": head["valid_cells_per_s"], "e2e": head["e2e"], "gpu_launches": head["launches"],
+                "stages": head["stages"], "roofline": head["roofline"], "cpu_baseline": cpu,
+                "clocks": head["clocks"],
+                "modes": {m: {"value": r["value"], "ms_per_step": r["ms"], "peak_gb": r["peak_bytes"] / 1e9,
+                              "peak_over_footprint": r["peak_bytes"] / footprint, "e2e_value": r["e2e"]["value"],
+                              "roofline": r["roofline"], "stages": r["stages"], "clocks": r["clocks"]}
+                          for m, r in results.items()}}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()
