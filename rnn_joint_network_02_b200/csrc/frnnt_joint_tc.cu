@@ -76,7 +76,7 @@ struct JointParams {
   Lattice L;
   __nv_bfloat16* zbuf;    // FWD_STORE: z [tile*128 + r][V]; BWD_DZ: dz [(tile-tile_begin)*128 + r][V]
   __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
-  int HS;                 // row stride of hbuf (H + 64)
+  int HS;                 // row stride of hbuf (hidden_stride(H))
   float* db_part;         // BWD_DZ: [kDbSlots][V]
   int32_t* status;
 };
@@ -572,7 +572,7 @@ __global__ void dz_from_z_kernel(JointParams p) {
 }
 
 // ------------------------------------------------------------------ hidden rows for the backward GEMMs
-// h rows (bf16, stride HS = H + 64) of tiles [tile_begin, ntiles) into hbuf rows
+// h rows (bf16, stride HS = hidden_stride(H)) of tiles [tile_begin, ntiles) into hbuf rows
 // (tile - row_tile0) * 128 + r: the same packed-bf16 tanh(F + G) as the joint
 // kernel, plus the extra column block [1, 0, ..., 0] (0 for cells outside the
 // lattice) whose dz-weighted sum is db_o.  One warp per row, coalesced.
@@ -599,7 +599,8 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
       }
       *(uint4*)(hr + k) = o;
     }
-    if (lane < 8) *(uint4*)(hr + H + lane * 8) = make_uint4((lane == 0 && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
+    for (int k = H + lane * 8; k < HS; k += 256)
+      *(uint4*)(hr + k) = make_uint4((k == H && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
   }
 }
 
@@ -661,7 +662,7 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
   }
 }
 
-// dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][H + 64]
+// dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
 // whose column H is the sum of dz over cells.
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, __nv_bfloat16* __restrict__ dW_o,
                                    __nv_bfloat16* __restrict__ db_o) {
@@ -769,7 +770,7 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
-  p.HS = j.s.H + 64;
+  p.HS = hidden_stride(j.s.H);
   p.db_part = j.db_part;
   p.status = j.status;
   p.nV = p.V / BN;
@@ -811,7 +812,7 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st) {
   p.V = j.s.V;
   p.TB = j.TB;
   p.UB = j.UB;
-  p.HS = j.s.H + 64;
+  p.HS = hidden_stride(j.s.H);
   p.F = (const __nv_bfloat16*)j.F;
   p.G = (const __nv_bfloat16*)j.G;
   p.labels = j.labels;
@@ -839,7 +840,7 @@ void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, fl
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
-  p.HS = j.s.H + 64;
+  p.HS = hidden_stride(j.s.H);
   const int n = j.tile_end - j.tile_begin;
   if (n <= 0) return;
   int threads = (p.H / 8 + 31) / 32 * 32;
@@ -852,7 +853,27 @@ void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, 
   long long n = (long long)V * H;
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, H + 64, (__nv_bfloat16*)dW_o, (__nv_bfloat16*)db_o);
+  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), (__nv_bfloat16*)dW_o,
+                                                       (__nv_bfloat16*)db_o);
+  note_launch();
+}
+
+// dst[r][0, cols) = src[r][0, cols), dst[r][cols, dcols) = 0 (bf16)
+__global__ void pad_cols_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
+                                __nv_bfloat16* __restrict__ dst, int dcols) {
+  const long long n = (long long)rows * dcols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / dcols, c = i % dcols;
+    dst[i] = c < cols ? src[r * cols + c] : __float2bfloat16_rn(0.f);
+  }
+}
+
+void launch_pad_cols(const void* src, int rows, int cols, void* dst, int dcols, cudaStream_t st) {
+  long long n = (long long)rows * dcols;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  pad_cols_kernel<<<(unsigned)blocks, 256, 0, st>>>((const __nv_bfloat16*)src, rows, cols, (__nv_bfloat16*)dst,
+                                                    dcols);
   note_launch();
 }
 
