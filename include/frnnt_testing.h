@@ -20,10 +20,12 @@ extern "C" {
  * epi: 0 = store fp32 to out[M][ldo]; 1 = store bf16; 2 = fp32 atomic add
  * into out (k_splits >= 1 K slices); 3 = out (bf16, holding h on entry)
  * becomes D * (1 - h*h).  Requires lda, ldb multiples of 8, N a multiple of
- * 32, 16-byte aligned pointers.  Returns FRNNT_OK or an FRNNT_ERR_* code. */
+ * 32, 16-byte aligned pointers.  variant: -1 automatic, 0 one CTA per 128-row
+ * tile, 1 CTA pairs sharing 256-row tiles (cta_group::2).  Returns FRNNT_OK or
+ * an FRNNT_ERR_* code. */
 FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn, long long lda,
                                    const void* B, int b_mn, long long ldb, int epi, int k_splits,
-                                   void* out, long long ldo, int32_t* status, void* stream);
+                                   void* out, long long ldo, int variant, int32_t* status, void* stream);
 
 #ifdef __cplusplus
 }

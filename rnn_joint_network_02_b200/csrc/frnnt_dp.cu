@@ -50,7 +50,7 @@ void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len
 // label_lp(t,u-1); beta needs blank_lp(t,u) and label_lp(t,u) (t = d - u).
 // They do not depend on the recursion, so they are fetched kPrefetch steps
 // ahead into a register ring to hide the global-memory latency.
-constexpr int kPrefetch = 4;
+constexpr int kPrefetch = 8;
 
 __device__ __forceinline__ void dp_operands(bool is_beta, int step, int ndiag, int u, int Tb, int Ub, int Up1,
                                             size_t base, const float* __restrict__ blank_lp,

@@ -75,14 +75,66 @@ struct GemmSmem {
 // has no work under the effective limits (every role skips it alike).
 __device__ __forceinline__ bool unit_coords(int unit, const GemmParams& p, const Eff& e, int& m0, int& nt, int& kb0,
                                            int& kb1) {
-  const int mt = unit % p.m_tiles;
-  const int rest = unit / p.m_tiles;
-  nt = rest % p.n_tiles;
-  const int ks = rest / p.n_tiles;
+  // raster: the n tiles of one m tile run back to back when m tiles dominate, so
+  // the A panel is fetched from DRAM once and re-read from L2 (k slices outermost)
+  int mt;
+  const int mn = unit % (p.m_tiles * p.n_tiles);
+  const int ks = unit / (p.m_tiles * p.n_tiles);
+  if (p.m_tiles >= p.n_tiles) {
+    nt = mn % p.n_tiles;
+    mt = mn / p.n_tiles;
+  } else {
+    mt = mn % p.m_tiles;
+    nt = mn / p.m_tiles;
+  }
   m0 = mt * BM;
   kb0 = ks * e.per;
   kb1 = min(e.kblocks, kb0 + e.per);
   return mt < e.m_tiles && kb0 < kb1;
+}
+
+__device__ __forceinline__ void epilogue_store(const GemmParams& p, int row, int col0, const uint32_t (&r)[32]) {
+  if (p.epi == 0) {          // store fp32
+    float4* dst = (float4*)(p.out_f32 + (size_t)row * p.ldo + col0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                           __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  } else if (p.epi == 1) {   // store bf16
+    uint4* dst = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 v;
+      v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+      v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+      v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+      v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+      dst[j] = v;
+    }
+  } else if (p.epi == 2) {   // fp32 reduce (split-K / accumulate)
+    float* dst = p.out_f32 + (size_t)row * p.ldo + col0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  } else {                   // dtanh: out = acc * (1 - h^2), h read from and result written to out_bf16
+    uint4* hp = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 hv = hp[j];
+      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[q]);
+        float2 hf = __bfloat1622float2(h2);
+        float d0 = __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x);
+        float d1 = __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y);
+        o[q] = pack_bf16x2(d0, d1);
+      }
+      hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN>
@@ -220,47 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const int col0 = n0 + c * 32;
         if (!row_ok || col0 >= p.N) continue;
-        if (p.epi == 0) {          // store fp32
-          float4* dst = (float4*)(p.out_f32 + (size_t)row * p.ldo + col0);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        } else if (p.epi == 1) {   // store bf16
-          uint4* dst = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-            v.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-            v.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-            v.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-            dst[j] = v;
-          }
-        } else if (p.epi == 2) {   // fp32 reduce (split-K / accumulate)
-          float* dst = p.out_f32 + (size_t)row * p.ldo + col0;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                       __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        } else {                   // dtanh: out = acc * (1 - h^2), h read from and result written to out_bf16
-          uint4* hp = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 hv = hp[j];
-            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[q]);
-              float2 hf = __bfloat1622float2(h2);
-              float d0 = __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x);
-              float d1 = __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y);
-              o[q] = pack_bf16x2(d0, d1);
-            }
-            hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
+        epilogue_store(p, row, col0, r);
       }
       tc_fence_before();
       __syncwarp();
@@ -273,6 +285,197 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tbase, 2 * BN);
+  }
+  if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, FRNNT_STATUS_TIMEOUT);
+}
+
+
+// ------------------------------------------------------------------ CTA-pair variant
+// Two CTAs of a cluster share one M = 256 output tile: each stages its own 128
+// rows of A and half of the B tile, the leader (rank 0) issues cta_group::2 MMAs
+// that read both CTAs' shared memory, and each CTA's TMEM receives its 128 rows.
+// Per CTA this halves the B-operand traffic of shared memory and of the L2.
+template <int BN, int STAGES>
+struct Gemm2Smem {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TILES_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = TILES_BYTES + 256 + 1024;
+};
+
+__device__ __forceinline__ bool unit_coords2(int unit, const GemmParams& p, const Eff& e, int& m0, int& nt, int& kb0,
+                                            int& kb1) {
+  int mt;                                   // m tiles of 256 rows here
+  const int mn = unit % (p.m_tiles * p.n_tiles);
+  const int ks = unit / (p.m_tiles * p.n_tiles);
+  if (p.m_tiles >= p.n_tiles) {
+    nt = mn % p.n_tiles;
+    mt = mn / p.n_tiles;
+  } else {
+    mt = mn % p.m_tiles;
+    nt = mn / p.m_tiles;
+  }
+  m0 = mt * 256;
+  kb0 = ks * e.per;
+  kb1 = min(e.kblocks, kb0 + e.per);
+  return m0 < e.M && kb0 < kb1;
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  using S = Gemm2Smem<BN, STAGES>;
+  constexpr int HB = BN / 2;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + S::TILES_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_base_p = (uint32_t*)(tempty + 2);
+  volatile int* abort_flag = (volatile int*)(tmem_base_p + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  const Eff eff = eff_of(p);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);         // 4 epilogue warps in each CTA of the pair
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(tmem_base_p, 2 * BN);
+    tmem_relinquish_pair();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_base_p;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int unit = pair; unit < units && !*abort_flag; unit += npairs) {
+        int m0, nt, kb0, kb1;
+        if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
+        const int ma = m0 + (int)rank * 128;
+        const int nb = nt * BN + (int)rank * HB;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
+          uint8_t* sa = smem + s * S::STAGE_BYTES;
+          uint8_t* sb = sa + S::A_BYTES;
+          const uint32_t fl = mapa_shared(smem_u32(&full[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * S::STAGE_BYTES);
+          if (!A_MN) {
+            tma_load_2d_pair(sa, &tmA, fl, kb * BK, ma);
+          } else {
+            tma_load_2d_pair(sa, &tmA, fl, ma, kb * BK);
+            tma_load_2d_pair(sa + 8192, &tmA, fl, ma + 64, kb * BK);
+          }
+          if (!B_MN) {
+            tma_load_2d_pair(sb, &tmB, fl, kb * BK, nb);
+          } else {
+#pragma unroll
+            for (int j = 0; j < HB / 64; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fl, nb + 64 * j, kb * BK);
+          }
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer (leader CTA only)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(256, BN, A_MN, B_MN);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc_i = 0;
+      bool ok = true;
+      for (int unit = pair; unit < units && ok; unit += npairs) {
+        int m0, nt, kb0, kb1;
+        if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
+        const int a = acc_i & 1;
+        const uint32_t aph = (acc_i >> 1) & 1;
+        if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dt = tbase + a * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
+          const uint32_t sb = sa + S::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
+            mma_bf16_ss_pair(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[s], 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) mma_commit_pair(&tfull[a], 0x3);
+        ++acc_i;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 0-3, both CTAs)
+    int acc_i = 0;
+    for (int unit = pair; unit < units; unit += npairs) {
+      int m0, nt, kb0, kb1;
+      if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
+      const int n0 = nt * BN;
+      const int a = acc_i & 1;
+      const uint32_t aph = (acc_i >> 1) & 1;
+      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      tc_fence_after();
+      const int row = m0 + (int)rank * 128 + warp * 32 + lane;
+      const bool row_ok = row < eff.M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
+        tmem_wait_ld();
+        const int col0 = n0 + c * 32;
+        if (!row_ok || col0 >= p.N) continue;
+        epilogue_store(p, row, col0, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
+      ++acc_i;
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tbase, 2 * BN);
   }
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, FRNNT_STATUS_TIMEOUT);
 }
@@ -320,6 +523,33 @@ bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
   return cudaPeekAtLastError() == cudaSuccess;
 }
 
+template <int BN, int STAGES, bool A_MN, bool B_MN>
+bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
+  using S = Gemm2Smem<BN, STAGES>;
+  auto kern = gemm2_tc_kernel<BN, STAGES, A_MN, B_MN>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) != cudaSuccess)
+      return false;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 2;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  const bool ok = cudaLaunchKernelEx(&cfg, kern, ta, tb, p) == cudaSuccess;
+  note_launch();
+  return ok && cudaPeekAtLastError() == cudaSuccess;
+}
+
 }  // namespace
 
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
@@ -344,19 +574,22 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH) && (g.ldo % 8 || !g.out_bf16)) return FRNNT_ERR_DIMS;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
   const int BN = (g.N % 256 == 0 && g.N >= 256) ? 256 : 128;
+  // CTA pairs (M = 256 per MMA) unless the problem has too few rows to fill them
+  const bool pair = g.variant == 1 || (g.variant < 0 && g.M >= 512);
   CUtensorMap ta, tb;
   bool ok;
   if (!g.a_mn) ok = make_tmap_bf16_2d(&ta, g.A, g.K, g.M, (uint64_t)g.lda, 64, 128);
   else ok = make_tmap_bf16_2d(&ta, g.A, g.M, g.K, (uint64_t)g.lda, 64, 64);
   if (!ok) return FRNNT_ERR_CUDA;
-  if (!g.b_mn) ok = make_tmap_bf16_2d(&tb, g.B, g.K, g.N, (uint64_t)g.ldb, 64, BN);
+  const int b_rows = pair ? BN / 2 : BN;
+  if (!g.b_mn) ok = make_tmap_bf16_2d(&tb, g.B, g.K, g.N, (uint64_t)g.ldb, 64, b_rows);
   else ok = make_tmap_bf16_2d(&tb, g.B, g.N, g.K, (uint64_t)g.ldb, 64, 64);
   if (!ok) return FRNNT_ERR_CUDA;
   GemmParams p;
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
-  p.m_tiles = (g.M + BM - 1) / BM;
+  p.m_tiles = (g.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
   p.n_tiles = (g.N + BN - 1) / BN;
   p.kblocks = (g.K + BK - 1) / BK;
   int splits = g.k_splits < 1 ? 1 : g.k_splits;
@@ -376,8 +609,24 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   p.dyn_scale = g.dyn_scale;
   p.dyn_dim = g.dyn_dim;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
-  const int grid = units < sm_count() ? units : sm_count();
   bool launched;
+  if (pair) {
+    const int npairs = units < sm_count() / 2 ? units : sm_count() / 2;
+    const int grid = 2 * npairs;
+    if (BN == 256) {
+      if (!g.a_mn && !g.b_mn) launched = launch2_t<256, 6, false, false>(ta, tb, p, grid, st);
+      else if (!g.a_mn && g.b_mn) launched = launch2_t<256, 6, false, true>(ta, tb, p, grid, st);
+      else if (g.a_mn && !g.b_mn) launched = launch2_t<256, 6, true, false>(ta, tb, p, grid, st);
+      else launched = launch2_t<256, 6, true, true>(ta, tb, p, grid, st);
+    } else {
+      if (!g.a_mn && !g.b_mn) launched = launch2_t<128, 8, false, false>(ta, tb, p, grid, st);
+      else if (!g.a_mn && g.b_mn) launched = launch2_t<128, 8, false, true>(ta, tb, p, grid, st);
+      else if (g.a_mn && !g.b_mn) launched = launch2_t<128, 8, true, false>(ta, tb, p, grid, st);
+      else launched = launch2_t<128, 8, true, true>(ta, tb, p, grid, st);
+    }
+    return launched ? FRNNT_OK : FRNNT_ERR_CUDA;
+  }
+  const int grid = units < sm_count() ? units : sm_count();
   if (BN == 256) {
     if (!g.a_mn && !g.b_mn) launched = launch_t<256, 4, false, false>(ta, tb, p, grid, st);
     else if (!g.a_mn && g.b_mn) launched = launch_t<256, 4, false, true>(ta, tb, p, grid, st);

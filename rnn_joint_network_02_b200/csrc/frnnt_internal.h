@@ -100,6 +100,7 @@ struct GemmTcArgs {
   // is min(static, (*dyn_count - dyn_base) * dyn_scale), read by the kernel.
   const int* dyn_count = nullptr;
   int dyn_base = 0, dyn_scale = 0, dyn_dim = 0;
+  int variant = -1;    // -1 auto, 0 one CTA per tile (M = 128), 1 CTA pairs (M = 256, cta_group::2)
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
 

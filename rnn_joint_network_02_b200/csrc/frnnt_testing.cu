@@ -4,7 +4,8 @@
 
 extern "C" FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn, long long lda,
                                               const void* B, int b_mn, long long ldb, int epi, int k_splits,
-                                              void* out, long long ldo, int32_t* status, void* stream) {
+                                              void* out, long long ldo, int variant, int32_t* status,
+                                              void* stream) {
   if (!A || !B || !out) return FRNNT_ERR_NULL;
   if (epi < 0 || epi > 3) return FRNNT_ERR_UNSUPPORTED;
   frnnt::GemmTcArgs g{};
@@ -23,6 +24,7 @@ extern "C" FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A
   g.out_bf16 = (epi == 1 || epi == 3) ? out : nullptr;
   g.ldo = ldo;
   g.status = status;
+  g.variant = variant < -1 || variant > 1 ? -1 : variant;
   cudaGetLastError();
   return frnnt::gemm_tc(g, (cudaStream_t)stream);
 }

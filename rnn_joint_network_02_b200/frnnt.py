@@ -84,7 +84,7 @@ def lib() -> ctypes.CDLL:
         L.frnnt_profile_read.restype = ctypes.c_int
         L.frnnt_test_gemm_bf16.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int,
                                            ctypes.c_longlong, vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_int,
-                                           ctypes.c_int, vp, ctypes.c_longlong, vp, vp]
+                                           ctypes.c_int, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
         L.frnnt_test_gemm_bf16.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -224,7 +224,7 @@ def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=No
 
 
 def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: int = 0, k_splits: int = 1,
-                   out=None, stream=None):
+                   out=None, stream=None, variant: int = -1):
     """Test hook: the tensor-core GEMM D = A * B (see include/frnnt_testing.h).
     A is [M][K] (a_mn False) or [K][M]; B is [N][K] (b_mn False) or [K][N]."""
     if out is None:
@@ -232,7 +232,8 @@ def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: in
     if stream is None:
         stream = torch.cuda.current_stream(A.device)
     rc = lib().frnnt_test_gemm_bf16(M, N, K, _ptr(A), int(a_mn), A.stride(0), _ptr(B), int(b_mn), B.stride(0), epi,
-                                    k_splits, _ptr(out), out.stride(0), None, ctypes.c_void_p(stream.cuda_stream))
+                                    k_splits, _ptr(out), out.stride(0), variant, None,
+                                    ctypes.c_void_p(stream.cuda_stream))
     if rc != OK:
         raise FrnntError(rc, error_string(rc))
     return out

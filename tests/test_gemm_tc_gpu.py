@@ -24,50 +24,56 @@ def _check(out, ref, tol=2e-3):
     assert err.item() <= tol, err.item()
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("a_mn", [False, True])
 @pytest.mark.parametrize("b_mn", [False, True])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 256, 128), (296, 640, 520), (1000, 512, 256)])
-def test_store_f32(cuda_ok, a_mn, b_mn, M, N, K):
+def test_store_f32(cuda_ok, a_mn, b_mn, M, N, K, variant):
+    """variant 0: one CTA per 128-row tile; 1: CTA pairs on 256-row tiles (cta_group::2)."""
     A, B, ref = _operands(M, N, K, a_mn, b_mn)
-    out = frnnt.test_gemm_bf16(A, B, a_mn, b_mn, M, N, K, epi=0)
+    out = frnnt.test_gemm_bf16(A, B, a_mn, b_mn, M, N, K, epi=0, variant=variant)
     torch.cuda.synchronize()
     _check(out, ref, 1e-5)
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("a_mn,b_mn", [(False, True), (True, True), (False, False)])
-def test_store_bf16(cuda_ok, a_mn, b_mn):
+def test_store_bf16(cuda_ok, a_mn, b_mn, variant):
     M, N, K = 384, 256, 640
     A, B, ref = _operands(M, N, K, a_mn, b_mn, seed=1)
-    out = frnnt.test_gemm_bf16(A, B, a_mn, b_mn, M, N, K, epi=1)
+    out = frnnt.test_gemm_bf16(A, B, a_mn, b_mn, M, N, K, epi=1, variant=variant)
     torch.cuda.synchronize()
     _check(out, ref, 8e-3)
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("splits", [1, 3, 7])
-def test_split_k_reduce(cuda_ok, splits):
+def test_split_k_reduce(cuda_ok, splits, variant):
     M, N, K = 1024, 640, 4096 + 64
     A, B, ref = _operands(M, N, K, True, True, seed=2)
     out = torch.full((M, N), 0.5, device="cuda")
-    frnnt.test_gemm_bf16(A, B, True, True, M, N, K, epi=2, k_splits=splits, out=out)
+    frnnt.test_gemm_bf16(A, B, True, True, M, N, K, epi=2, k_splits=splits, out=out, variant=variant)
     torch.cuda.synchronize()
     _check(out - 0.5, ref, 1e-5)
 
 
-def test_dtanh_epilogue(cuda_ok):
+@pytest.mark.parametrize("variant", [0, 1])
+def test_dtanh_epilogue(cuda_ok, variant):
     M, N, K = 512, 640, 1024
     A, B, ref = _operands(M, N, K, False, True, seed=3)
     h = torch.tanh(torch.randn(M, N, device="cuda")).bfloat16()
     out = h.clone()
-    frnnt.test_gemm_bf16(A, B, False, True, M, N, K, epi=3, out=out)
+    frnnt.test_gemm_bf16(A, B, False, True, M, N, K, epi=3, out=out, variant=variant)
     torch.cuda.synchronize()
     expect = ref * (1 - h.float() ** 2)
     _check(out, expect, 8e-3)
 
 
-def test_many_tiles_persistent(cuda_ok):
+@pytest.mark.parametrize("variant", [0, 1])
+def test_many_tiles_persistent(cuda_ok, variant):
     """More output tiles than SMs: every CTA walks several tiles and both TMEM buffers."""
     M, N, K = 6400, 640, 512
     A, B, ref = _operands(M, N, K, False, True, seed=4)
-    out = frnnt.test_gemm_bf16(A, B, False, True, M, N, K, epi=0)
+    out = frnnt.test_gemm_bf16(A, B, False, True, M, N, K, epi=0, variant=variant)
     torch.cuda.synchronize()
     _check(out, ref, 1e-5)
