@@ -27,11 +27,13 @@ __device__ inline int label_of(const int32_t* labels, int b, int u, int U, int V
   return clampi(labels[(size_t)b * U + u], 0, V - 1);
 }
 
-// log(exp(a) + exp(b)) in fp32, exact for -inf operands.
+// log(exp(a) + exp(b)) in fp32, exact for -inf operands: max + ln(1 + e^-|a-b|),
+// with the 1 + e^-d in [1, 2] taken by the hardware exp2 / log2 (absolute error
+// of the correction term ~1e-7, far below fp32 rounding of the running sums).
 __device__ __forceinline__ float log_add_exp(float a, float b) {
   float m = fmaxf(a, b);
   if (m == -INFINITY) return -INFINITY;
-  return m + log1pf(__expf(-fabsf(a - b)));
+  return m + __logf(1.f + __expf(-fabsf(a - b)));
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

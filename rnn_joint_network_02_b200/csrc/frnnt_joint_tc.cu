@@ -77,6 +77,7 @@ struct JointParams {
   __nv_bfloat16* zbuf;    // FWD_STORE: z [tile*128 + r][V]; BWD_DZ: dz [(tile-tile_begin)*128 + r][V]
   __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
   int HS;                 // row stride of hbuf (hidden_stride(H))
+  int srows;              // rows per epilogue store-staging pass (8 or 32)
   float* db_part;         // BWD_DZ: [kDbSlots][V]
   int32_t* status;
 };
@@ -124,6 +125,31 @@ __device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Store this warp's 32 rows x 32 bf16 (each lane holds its row's 64 bytes in
+// w[16]) to global rows grow0 + i, columns col0.., through a shared staging
+// block of srows rows (80-byte padded rows, bank-conflict-free on both sides),
+// so every global store instruction writes 8 rows x 64 contiguous bytes.
+__device__ __forceinline__ void staged_store_rows(uint8_t* stage, int srows, const uint32_t (&w)[16],
+                                                  __nv_bfloat16* gbase, size_t grow0, size_t ld, int col0) {
+  const int lane = threadIdx.x & 31;
+  for (int pass = 0; pass < 32 / srows; ++pass) {
+    if (lane / srows == pass) {
+      uint4* d = (uint4*)(stage + (lane % srows) * 80);
+      d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      d[2] = make_uint4(w[8], w[9], w[10], w[11]);
+      d[3] = make_uint4(w[12], w[13], w[14], w[15]);
+    }
+    __syncwarp();
+    for (int k = 0; k < srows / 8; ++k) {
+      const int rr = 8 * k + lane / 4, ch = lane % 4;
+      const uint4 v = *(const uint4*)(stage + rr * 80 + ch * 16);
+      *(uint4*)(gbase + (grow0 + pass * srows + rr) * ld + col0 + ch * 8) = v;
+    }
+    __syncwarp();
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_constant__ CUtensorMap tmW, JointParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -134,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   const int fg_stride = 2 * p.H + 16;                             // padded bf16 row (bank spread)
   uint8_t* fgs = ring + p.stages * kStageBytes;                   // TB F rows then UB G rows of this tile
   __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + fg_bytes(p.TB, p.UB, p.H));   // b_o (bf16)
-  uint64_t* full = (uint64_t*)(bias_s + ((p.V + 511) & ~511));
+  uint8_t* stage_s = (uint8_t*)(bias_s + ((p.V + 511) & ~511));   // per epilogue warp: srows x 80 B
+  uint64_t* full = (uint64_t*)(stage_s + kEpiWarps * p.srows * 80);
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
@@ -432,12 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
                 if (col0 + j == ri.y) zy = v[j];
             }
             if (MODE == MODE_FWD_STORE) {
-              uint4* dst = (uint4*)(p.zbuf + (row_base + r) * V + col0);
+              uint32_t w[16];
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                    pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                                    pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+              for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+              staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
             }
           } else {
 #pragma unroll
@@ -447,11 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               if (col0 + j == ri.y) d -= lpost;
               v[j] = ri.valid ? d : 0.f;
             }
-            uint4* dst = (uint4*)(p.zbuf + (row_base + r) * V + col0);
+            uint32_t w[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+            staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
           }
         }
         tc_fence_before();
@@ -688,21 +712,28 @@ int sms() {
 constexpr int kSmemLimit = 232448;   // max dynamic shared memory per block on sm_100
 constexpr int kBarBytes = 3072;   // mbarriers + TMEM address + abort flag + 2 KB epilogue combine area
 
-int smem_fixed(int KB, int V, int TB, int UB) {
+int smem_fixed(int KB, int V, int TB, int UB, int srows) {
   const int KB_hi = KB > kTmemKB ? KB - kTmemKB : 0;
-  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 511) & ~511) * 2 + kBarBytes;
+  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 511) & ~511) * 2 + kEpiWarps * srows * 80 +
+         kBarBytes;
+}
+
+// Staging rows: 32 when that still leaves at least 6 W_o stages, else 8.
+int staging_rows(int KB, int V, int TB, int UB) {
+  return (kSmemLimit - smem_fixed(KB, V, TB, UB, 32)) / kStageBytes >= 6 ? 32 : 8;
 }
 
 int stages_for(int KB, int V, int TB, int UB) {
-  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB)) / kStageBytes;
+  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB, staging_rows(KB, V, TB, UB))) / kStageBytes;
   return st > kMaxStages ? kMaxStages : st;
 }
 
 template <int MODE>
 int launch_joint_t(const CUtensorMap& tm, JointParams p, cudaStream_t st) {
+  p.srows = staging_rows(p.KB, p.V, p.TB, p.UB);
   p.stages = stages_for(p.KB, p.V, p.TB, p.UB);
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
-  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB) + p.stages * kStageBytes;
+  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB, p.srows) + p.stages * kStageBytes;
   auto kern = joint_tc_kernel<MODE>;
   static bool attr_set = false;
   if (!attr_set) {
