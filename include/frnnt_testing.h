@@ -27,6 +27,15 @@ FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn,
                                    const void* B, int b_mn, long long ldb, int epi, int k_splits,
                                    void* out, long long ldo, int variant, int32_t* status, void* stream);
 
+/* Selects the fused joint kernel's variant for the frnnt_fwd_bwd calls that
+ * follow (process-wide, not thread-safe; set it between calls): -1 automatic
+ * (the default), 0 one CTA per 128-cell tile, 1 CTA pairs (a 2-CTA cluster,
+ * each CTA its own cell tile and half of every W_o tile, M = 256 cta_group::2
+ * MMAs).  Out-of-range values clamp to the nearest.  Returns the previous
+ * setting.  Results of the two variants agree up to the order of fp32 atomic
+ * additions. */
+FRNNT_API int frnnt_test_joint_variant(int variant);
+
 #ifdef __cplusplus
 }
 #endif

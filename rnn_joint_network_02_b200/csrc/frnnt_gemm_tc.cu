@@ -179,31 +179,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_base_p;
 
   if (warp == 4) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+    // ---------------------------------------------------------------- producer (warp polls, one lane issues)
+    {
       int s = 0;
       uint32_t ph = 0;
-      for (int unit = blockIdx.x; unit < units && !*abort_flag; unit += gridDim.x) {
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
         int m0, nt, kb0, kb1;
         if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int n0 = nt * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
-          uint8_t* sa = smem + s * S::STAGE_BYTES;
-          uint8_t* sb = sa + S::A_BYTES;
-          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-          if (!A_MN) {
-            tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
-          } else {
-            tma_load_2d(sa, &tmA, &full[s], m0, kb * BK);
-            tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, kb * BK);
+          if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
           }
-          if (!B_MN) {
-            tma_load_2d(sb, &tmB, &full[s], kb * BK, n0);
-          } else {
+          if (elect_one()) {
+            uint8_t* sa = smem + s * S::STAGE_BYTES;
+            uint8_t* sb = sa + S::A_BYTES;
+            mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+            if (!A_MN) {
+              tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
+            } else {
+              tma_load_2d(sa, &tmA, &full[s], m0, kb * BK);
+              tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, kb * BK);
+            }
+            if (!B_MN) {
+              tma_load_2d(sb, &tmB, &full[s], kb * BK, n0);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, &full[s], n0 + 64 * j, kb * BK);
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, &full[s], n0 + 64 * j, kb * BK);
+            }
           }
+          __syncwarp();
           if (++s == STAGES) {
             s = 0;
             ph ^= 1;
@@ -213,8 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer (warp polls, one lane issues)
+    {
       constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
       int s = 0;
       uint32_t ph = 0;
@@ -225,29 +232,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int a = acc_i & 1;
         const uint32_t aph = (acc_i >> 1) & 1;
-        if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) break;
+        if (!warp_wait(&tempty[a], aph ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t dt = tbase + a * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
+          if (!warp_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
+            const uint32_t sb = sa + S::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
-            mma_bf16_ss(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
+              mma_bf16_ss(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
           }
-          mma_commit(&empty[s]);
+          __syncwarp();
           if (++s == STAGES) {
             s = 0;
             ph ^= 1;
           }
         }
-        if (ok) mma_commit(&tfull[a]);
+        if (ok && elect_one()) mma_commit(&tfull[a]);
+        __syncwarp();
         ++acc_i;
       }
     }
@@ -367,33 +378,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_base_p;
 
   if (warp == 4) {
-    // ---------------------------------------------------------------- producer (both CTAs)
-    if (lane == 0) {
+    // ---------------------------------------------------------------- producer (both CTAs; warp polls, one lane issues)
+    {
       int s = 0;
       uint32_t ph = 0;
-      for (int unit = pair; unit < units && !*abort_flag; unit += npairs) {
+      bool ok = true;
+      for (int unit = pair; unit < units && ok; unit += npairs) {
         int m0, nt, kb0, kb1;
         if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int ma = m0 + (int)rank * 128;
         const int nb = nt * BN + (int)rank * HB;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
-          uint8_t* sa = smem + s * S::STAGE_BYTES;
-          uint8_t* sb = sa + S::A_BYTES;
-          const uint32_t fl = mapa_shared(smem_u32(&full[s]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * S::STAGE_BYTES);
-          if (!A_MN) {
-            tma_load_2d_pair(sa, &tmA, fl, kb * BK, ma);
-          } else {
-            tma_load_2d_pair(sa, &tmA, fl, ma, kb * BK);
-            tma_load_2d_pair(sa + 8192, &tmA, fl, ma + 64, kb * BK);
+          if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) {
+            ok = false;
+            break;
           }
-          if (!B_MN) {
-            tma_load_2d_pair(sb, &tmB, fl, kb * BK, nb);
-          } else {
+          if (elect_one()) {
+            uint8_t* sa = smem + s * S::STAGE_BYTES;
+            uint8_t* sb = sa + S::A_BYTES;
+            const uint32_t fl = mapa_shared(smem_u32(&full[s]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * S::STAGE_BYTES);
+            if (!A_MN) {
+              tma_load_2d_pair(sa, &tmA, fl, kb * BK, ma);
+            } else {
+              tma_load_2d_pair(sa, &tmA, fl, ma, kb * BK);
+              tma_load_2d_pair(sa + 8192, &tmA, fl, ma + 64, kb * BK);
+            }
+            if (!B_MN) {
+              tma_load_2d_pair(sb, &tmB, fl, kb * BK, nb);
+            } else {
 #pragma unroll
-            for (int j = 0; j < HB / 64; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fl, nb + 64 * j, kb * BK);
+              for (int j = 0; j < HB / 64; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fl, nb + 64 * j, kb * BK);
+            }
           }
+          __syncwarp();
           if (++s == STAGES) {
             s = 0;
             ph ^= 1;
@@ -403,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer (leader CTA only)
-    if (lane == 0 && rank == 0) {
+    // ---------------------------------------------------------------- MMA issuer (leader CTA only; warp polls, one lane issues)
+    if (rank == 0) {
       constexpr uint32_t idesc = idesc_bf16(256, BN, A_MN, B_MN);
       int s = 0;
       uint32_t ph = 0;
@@ -415,29 +433,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
         const int a = acc_i & 1;
         const uint32_t aph = (acc_i >> 1) & 1;
-        if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) break;
+        if (!warp_wait(&tempty[a], aph ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t dt = tbase + a * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
+          if (!warp_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
+            const uint32_t sb = sa + S::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
-            mma_bf16_ss_pair(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = A_MN ? sdesc_sw128(sa + k * 2048, 8192, 1024) : sdesc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bd = B_MN ? sdesc_sw128(sb + k * 2048, 8192, 1024) : sdesc_sw128(sb + k * 32, 16, 1024);
+              mma_bf16_ss_pair(dt, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit_pair(&empty[s], 0x3);
           }
-          mma_commit_pair(&empty[s], 0x3);
+          __syncwarp();
           if (++s == STAGES) {
             s = 0;
             ph ^= 1;
           }
         }
-        if (ok) mma_commit_pair(&tfull[a], 0x3);
+        if (ok && elect_one()) mma_commit_pair(&tfull[a], 0x3);
+        __syncwarp();
         ++acc_i;
       }
     }

@@ -140,6 +140,8 @@ long long max_tiles(const Shape& s, int TB, int UB);
 void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
                   cudaStream_t st);
 int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
+// Joint kernel variant for later calls: -1 automatic, 0 one CTA per cell tile, 1 CTA pairs; returns the previous one.
+int set_joint_variant(int variant);
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st);
 void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);

@@ -27,6 +27,8 @@
 // Roles: warps 0-3 generate h and run the epilogue (warp w owns TMEM lanes
 // 32w..32w+31 = tile rows), warp 4 issues TMA loads of W_o, warp 5 issues the
 // MMAs.  Persistent: one CTA per SM walks the tile list.
+#include <algorithm>
+
 #include "frnnt_common.cuh"
 #include "frnnt_internal.h"
 #include "sm100.cuh"
@@ -51,7 +53,6 @@ constexpr int kMaxStages = 16;
 constexpr int kMaxKB = 16;          // H <= 1024
 constexpr int kTmemKB = 8;          // the first 8 K blocks (512 columns of h) live in TMEM
 constexpr int kHCol = 256;          // TMEM columns: [0,128) and [128,256) accumulators, [256,512) h
-constexpr int kDbSlots = 8;
 
 // Shared memory of the staged F / G rows: TB + UB rows of 2H + 16 bytes, 1 KB aligned.
 __host__ __device__ constexpr int fg_bytes(int TB, int UB, int H) { return (((TB + UB) * (2 * H + 16)) + 1023) & ~1023; }
@@ -63,6 +64,7 @@ struct JointParams {
   int KB;                 // H / 64
   int nV;                 // V / BN
   int stages;
+  int ks;                 // 64-wide K blocks per ring stage and per h signal (1 or 2)
   const __nv_bfloat16* F;   // [B*T][H] bf16
   const __nv_bfloat16* G;   // [B*(U+1)][H] bf16
   const __nv_bfloat16* b_o;
@@ -78,7 +80,7 @@ struct JointParams {
   __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
   int HS;                 // row stride of hbuf (hidden_stride(H))
   int srows;              // rows per epilogue store-staging pass (8 or 32)
-  float* db_part;         // BWD_DZ: [kDbSlots][V]
+  float* db_part;         // unused
   int32_t* status;
 };
 
@@ -105,11 +107,6 @@ __device__ __forceinline__ RowInfo row_info(const JointParams& p, int4 tile, int
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -150,15 +147,23 @@ __device__ __forceinline__ void staged_store_rows(uint8_t* stage, int srows, con
   }
 }
 
-template <int MODE>
+// PAIR: the CTAs of a 2-CTA cluster each own a cell tile (h, epilogue, F/G
+// staging) and stage half of every W_o tile; the leader issues M = 256
+// cta_group::2 MMAs over both, halving the W_o traffic per CTA.  Generator and
+// epilogue signals go to the leader's barriers (cluster-scope release/acquire);
+// the leader's commits reach both CTAs.
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_constant__ CUtensorMap tmW, JointParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int KB_hi = p.KB > kTmemKB ? p.KB - kTmemKB : 0;
   uint8_t* hhi = smem;                                            // K blocks >= kTmemKB of h, 16 KB each
-  uint8_t* ring = hhi + KB_hi * 16384;                            // stages x 16 KB of W_o
+  uint8_t* ring = hhi + KB_hi * 16384;                            // stages x ks K blocks of W_o
   const int fg_stride = 2 * p.H + 16;                             // padded bf16 row (bank spread)
-  uint8_t* fgs = ring + p.stages * kStageBytes;                   // TB F rows then UB G rows of this tile
+  constexpr int KBB = PAIR ? kStageBytes / 2 : kStageBytes;      // this CTA's rows of one K block of a W_o tile
+  const int STAGE = p.ks * KBB;
+  const int ngrp = (p.KB + p.ks - 1) / p.ks;                      // K-block groups (one ring stage each)
+  uint8_t* fgs = ring + p.stages * STAGE;                         // TB F rows then UB G rows of this tile
   __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + fg_bytes(p.TB, p.UB, p.H));   // b_o (bf16)
   uint8_t* stage_s = (uint8_t*)(bias_s + ((p.V + 511) & ~511));   // per epilogue warp: srows x 80 B
   uint64_t* full = (uint64_t*)(stage_s + kEpiWarps * p.srows * 80);
@@ -175,6 +180,23 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = min(p.tile_end, *p.ntiles);
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  // iteration i of the persistent loop covers tile tile_begin + i (one CTA) or
+  // tiles tile_begin + 2i and 2i + 1 (a pair; a missing odd tile is a dummy)
+  const int slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nslots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int span = ntiles - p.tile_begin;
+  const int niter = span <= 0 ? 0 : (PAIR ? (span + 1) / 2 : span);
+  auto tile_of = [&](int i) { return p.tile_begin + (PAIR ? 2 * i + (int)rank : i); };
+  // arrivals on barriers the (leader's) MMA thread waits for
+  auto arrive_leader = [&](uint64_t* bar) {
+    if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
+    else mbar_arrive(bar);
+  };
+  auto commit_all = [&](uint64_t* bar) {
+    if (PAIR) mma_commit_pair(bar, 0x3);
+    else mma_commit(bar);
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxStages; ++i) {
@@ -183,10 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kEpiWarps);
+      mbar_init(&tempty[i], PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     for (int i = 0; i < kMaxKB; ++i) {
-      mbar_init(&hfull[i], kGenWarps);
+      mbar_init(&hfull[i], PAIR ? 2 * kGenWarps : kGenWarps);
       mbar_init(&hempty[i], 1);
     }
     mbar_init(fg_full, 1);
@@ -196,29 +218,49 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   }
   for (int k = threadIdx.x; k < p.V; k += blockDim.x) bias_s[k] = p.b_o[k];
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_base_p, 512);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_base_p, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_base_p, 512);
+      tmem_relinquish();
+    }
   }
   if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmW);
-  __syncthreads();
+  if (PAIR) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer: W_o tiles
-    if (lane == 0) {
+    // (the whole warp polls, one elected lane issues)
+    {
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = p.tile_begin + blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int it = slot; it < niter && ok; it += nslots) {
         for (int n = 0; n < p.nV && ok; ++n) {
-          for (int kb = 0; kb < p.KB; ++kb) {
-            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+          for (int g = 0; g < ngrp; ++g) {
+            if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[s], kStageBytes);
-            tma_load_2d(ring + s * kStageBytes, &tmW, &full[s], kb * 64, n * BN);
+            const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
+            if (!elect_one()) {
+              // other lanes: nothing to issue
+            } else if (PAIR) {
+              // both halves credit the leader's barrier, which expects both
+              if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * nk * KBB);
+              const uint32_t fl = mapa_shared(smem_u32(&full[s]), 0);
+              for (int kk = 0; kk < nk; ++kk)
+                tma_load_2d_pair(ring + s * STAGE + kk * KBB, &tmW, fl, (kb0 + kk) * 64, n * BN + (int)rank * (BN / 2));
+            } else {
+              mbar_arrive_expect_tx(&full[s], nk * KBB);
+              for (int kk = 0; kk < nk; ++kk)
+                tma_load_2d(ring + s * STAGE + kk * KBB, &tmW, &full[s], (kb0 + kk) * 64, n * BN);
+            }
+            __syncwarp();
             if (++s == p.stages) {
               s = 0;
               ph ^= 1;
@@ -229,59 +271,74 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
+    // ------------------------------------------------------------ MMA issuer (the leader's warp; one elected lane issues)
+    if (rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, BN, false, false);
       int s = 0;
       uint32_t ph = 0;
       int acc_i = 0;
       uint32_t hph = 0;
       bool ok = true;
       const uint32_t hhi_addr = smem_u32(hhi);
-      for (int tile = p.tile_begin + blockIdx.x; tile < ntiles && ok; tile += gridDim.x, hph ^= 1) {
+      for (int it = slot; it < niter && ok; it += nslots, hph ^= 1) {
         for (int n = 0; n < p.nV && ok; ++n, ++acc_i) {
           const int a = acc_i & 1;
           const uint32_t aph = (acc_i >> 1) & 1;
-          if (!mbar_wait(&tempty[a], aph ^ 1, abort_flag)) {
+          if (!(PAIR ? warp_wait_cluster(&tempty[a], aph ^ 1, abort_flag) : warp_wait(&tempty[a], aph ^ 1, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t dt = tbase + a * BN;
-          for (int kb = 0; kb < p.KB; ++kb) {
+          for (int g = 0; g < ngrp; ++g) {
             if (n == 0) {
-              // h block kb written by the generators (TMEM stores / shared stores)
-              if (!mbar_wait(&hfull[kb], hph, abort_flag)) {
+              // h blocks of group g written by the generators (TMEM stores / shared stores)
+              if (!(PAIR ? warp_wait_cluster(&hfull[g], hph, abort_flag) : warp_wait(&hfull[g], hph, abort_flag))) {
                 ok = false;
                 break;
               }
               tc_fence_after();
             }
             // W_o stage landed (TMA completion is ordered by the mbarrier itself)
-            if (!mbar_wait(&full[s], ph, abort_flag)) {
+            if (!warp_wait(&full[s], ph, abort_flag)) {
               ok = false;
               break;
             }
-            const uint32_t sb = smem_u32(ring + s * kStageBytes);
-            if (kb < kTmemKB) {
+            const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
+            if (elect_one()) {
+              for (int kk = 0; kk < nk; ++kk) {
+                const int kb = kb0 + kk;
+                const uint32_t sb = smem_u32(ring + s * STAGE + kk * KBB);
+                if (kb < kTmemKB) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(dt, tbase + kHCol + kb * 32 + k * 8, sdesc_sw128(sb + k * 32, 16, 1024), idesc,
-                            (kb > 0 || k > 0) ? 1u : 0u);
-            } else {
-              const uint32_t sa = hhi_addr + (kb - kTmemKB) * 16384;
+                  for (int k = 0; k < 4; ++k) {
+                    const uint32_t at = tbase + kHCol + kb * 32 + k * 8;
+                    const uint64_t bd = sdesc_sw128(sb + k * 32, 16, 1024);
+                    const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                    if (PAIR) mma_bf16_ts_pair(dt, at, bd, idesc, acc);
+                    else mma_bf16_ts(dt, at, bd, idesc, acc);
+                  }
+                } else {
+                  const uint32_t sa = hhi_addr + (kb - kTmemKB) * 16384;
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ss(dt, sdesc_sw128(sa + k * 32, 16, 1024), sdesc_sw128(sb + k * 32, 16, 1024), idesc, 1u);
+                  for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = sdesc_sw128(sa + k * 32, 16, 1024), bd = sdesc_sw128(sb + k * 32, 16, 1024);
+                    if (PAIR) mma_bf16_ss_pair(dt, ad, bd, idesc, 1u);
+                    else mma_bf16_ss(dt, ad, bd, idesc, 1u);
+                  }
+                }
+              }
+              commit_all(&empty[s]);
+              if (n == p.nV - 1) commit_all(&hempty[g]);   // h group g is free once these MMAs finish
             }
-            mma_commit(&empty[s]);
-            if (n == p.nV - 1) mma_commit(&hempty[kb]);   // h block kb is free once these MMAs finish
+            __syncwarp();
             if (++s == p.stages) {
               s = 0;
               ph ^= 1;
             }
           }
-          if (ok) mma_commit(&tfull[a]);
+          if (ok && elect_one()) commit_all(&tfull[a]);
+          __syncwarp();
         }
       }
     }
@@ -304,8 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     // warp kGen0 only: wait until the generator warps are done with the buffer
     // (empty_parity 1 on the first call passes at once), then copy
     auto issue_fg = [&](int tile, uint32_t empty_parity) {
-      const int4 td = p.tiles[tile];
-      const int nF = min(p.TB, p.T - td.y), nG = min(p.UB, Up1 - td.z);
+      const bool dummy = tile >= ntiles;
+      const int4 td = dummy ? make_int4(0, p.T, 0, 0) : p.tiles[tile];
+      const int nF = dummy ? 0 : min(p.TB, p.T - td.y), nG = dummy ? 0 : min(p.UB, Up1 - td.z);
       if (!mbar_wait(fg_empty, empty_parity, abort_flag)) return false;
       if (lane == 0) mbar_arrive_expect_tx(fg_full, (uint32_t)(nF + nG) * H * 2);
       __syncwarp();
@@ -316,11 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
                   fg_full);
       return true;
     };
-    int tile = p.tile_begin + blockIdx.x;
     bool ok = true;
-    if (warp == kGen0 && tile < ntiles) ok = issue_fg(tile, 1u);
-    for (; tile < ntiles && ok; tile += gridDim.x, hph ^= 1, fph ^= 1) {
-      const int4 td = p.tiles[tile];
+    if (warp == kGen0 && slot < niter) ok = issue_fg(tile_of(slot), 1u);
+    for (int it = slot; it < niter && ok; it += nslots, hph ^= 1, fph ^= 1) {
+      const int tile = tile_of(it);
+      // a dummy tile (the odd one out of a pair) has no valid row: its h is zero
+      const int4 td = tile < ntiles ? p.tiles[tile] : make_int4(0, p.T, 0, 0);
       const RowInfo ri = row_info(p, td, r);
       const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
       const uint8_t* grow = fgs + (p.TB + r % p.UB) * fg_stride;
@@ -345,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
 #pragma unroll
           for (int j = 0; j < 8; ++j) pk[j] = 0u;
         }
-        if ((si & 1) == 0 && !mbar_wait(&hempty[kb], hph ^ 1, abort_flag)) {
+        const int grp = kb / p.ks;
+        if ((si & 1) == 0 && kb % p.ks == 0 && !mbar_wait(&hempty[grp], hph ^ 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -356,7 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           *(uint4*)(blk + sw128_offset(r, sub * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *(uint4*)(blk + sw128_offset(r, sub * 16 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
-        if ((si & 1) == 1) {
+        if ((si & 1) == 1 && (kb % p.ks == p.ks - 1 || kb == p.KB - 1)) {
+          // last K block of the group (a group lies wholly in TMEM or wholly in shared memory)
           if (kb < kTmemKB) {
             tmem_wait_st();
             tc_fence_before();
@@ -364,14 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
             fence_proxy_async_smem();
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&hfull[kb]);
+          if (lane == 0) arrive_leader(&hfull[grp]);
         }
       }
       if (!ok) break;
       // this warp is done reading the tile's F/G rows
       __syncwarp();
       if (lane == 0) mbar_arrive(fg_empty);
-      if (warp == kGen0 && tile + (int)gridDim.x < ntiles) ok = issue_fg(tile + gridDim.x, fph);
+      if (warp == kGen0 && it + nslots < niter) ok = issue_fg(tile_of(it + nslots), fph);
       if (*abort_flag) break;
     }
   } else {
@@ -382,8 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     const int V = p.V, Up1 = p.U + 1;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     int acc_i = 0;
-    for (int tile = p.tile_begin + blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      const int4 td = p.tiles[tile];
+    for (int it = slot; it < niter; it += nslots) {
+      const int tile = tile_of(it);
+      const bool real = tile < ntiles;   // else the dummy of a pair: consume the accumulators, store nothing
+      const int4 td = real ? p.tiles[tile] : make_int4(0, p.T, 0, 0);
       const size_t row_base = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
       const RowInfo ri = row_info(p, td, r);
       float m = -INFINITY, ssum = 0.f, zb = 0.f, zy = 0.f;
@@ -458,13 +521,13 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               for (int j = 0; j < 32; ++j)
                 if (col0 + j == ri.y) zy = v[j];
             }
-            if (MODE == MODE_FWD_STORE) {
+            if (MODE == MODE_FWD_STORE && real) {
               uint32_t w[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
               staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
             }
-          } else {
+          } else if (real) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               float d = occ * ex2(fmaf(v[j], kLog2e, -lk));
@@ -480,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[a]);
+        if (lane == 0) arrive_leader(&tempty[a]);
       }
       if (!ok || *abort_flag) break;
       if (MODE != MODE_BWD_DZ) {
@@ -508,9 +571,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   }
 
   __syncthreads();
+  if (PAIR) cluster_sync();   // no CTA leaves while its peer may still signal its barriers
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tbase, 512);
+    if (PAIR) tmem_dealloc_pair(tbase, 512);
+    else tmem_dealloc(tbase, 512);
   }
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, FRNNT_STATUS_TIMEOUT);
 }
@@ -718,30 +783,73 @@ int smem_fixed(int KB, int V, int TB, int UB, int srows) {
          kBarBytes;
 }
 
-// Staging rows: 32 when that still leaves at least 6 W_o stages, else 8.
+// Staging rows: 32 when that still leaves at least 6 full W_o tiles of ring, else 8.
 int staging_rows(int KB, int V, int TB, int UB) {
   return (kSmemLimit - smem_fixed(KB, V, TB, UB, 32)) / kStageBytes >= 6 ? 32 : 8;
 }
 
-int stages_for(int KB, int V, int TB, int UB) {
-  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB, staging_rows(KB, V, TB, UB))) / kStageBytes;
+// Ring stages of stage_bytes each (a full W_o tile, or half of one per CTA of a pair).
+int stages_for(int KB, int V, int TB, int UB, int stage_bytes = kStageBytes) {
+  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB, staging_rows(KB, V, TB, UB))) / stage_bytes;
   return st > kMaxStages ? kMaxStages : st;
 }
 
-template <int MODE>
-int launch_joint_t(const CUtensorMap& tm, JointParams p, cudaStream_t st) {
+int g_joint_variant = -1;   // -1 automatic, 0 one CTA per tile, 1 CTA pairs
+
+template <int MODE, bool PAIR>
+int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStream_t st) {
+  constexpr int kb_bytes = PAIR ? kStageBytes / 2 : kStageBytes;
   p.srows = staging_rows(p.KB, p.V, p.TB, p.UB);
-  p.stages = stages_for(p.KB, p.V, p.TB, p.UB);
+  // two K blocks per ring stage (half as many barrier polls in the MMA issuer)
+  // while that still leaves at least three stages
+  p.ks = stages_for(p.KB, p.V, p.TB, p.UB, 2 * kb_bytes) >= 3 ? 2 : 1;
+  const int stage_bytes = p.ks * kb_bytes;
+  p.stages = stages_for(p.KB, p.V, p.TB, p.UB, stage_bytes);
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
-  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB, p.srows) + p.stages * kStageBytes;
-  auto kern = joint_tc_kernel<MODE>;
+  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB, p.srows) + p.stages * stage_bytes;
+  auto kern = joint_tc_kernel<MODE, PAIR>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return FRNNT_ERR_CUDA;
     attr_set = true;
   }
-  kern<<<sms(), kThreads, smem, st>>>(tm, p);
+  if (!PAIR) {
+    kern<<<sms(), kThreads, smem, st>>>(tm, p);
+  } else {
+    // one cluster of two CTAs per pair of tiles; persistent, so no more
+    // clusters than can be resident at once (an SM left without a partner in
+    // its GPC stays idle)
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = 2;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    static int resident = 0, resident_smem = -1;
+    if (resident_smem != smem) {
+      cfg.gridDim = dim3(sms(), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sms() / 2;
+      }
+      resident = n < sms() / 2 ? n : sms() / 2;
+      resident_smem = smem;
+    }
+    const int pairs = (ntiles_max + 1) / 2;
+    const int npairs = pairs < resident ? (pairs > 0 ? pairs : 1) : resident;
+    cfg.gridDim = dim3(2 * npairs, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, tm, p) != cudaSuccess) {
+      note_launch();
+      return FRNNT_ERR_CUDA;
+    }
+  }
   note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;
 }
@@ -805,11 +913,30 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.db_part = j.db_part;
   p.status = j.status;
   p.nV = p.V / BN;
+  // upper bound of this launch's tile count (the exact count is on the device)
+  const long long span = (long long)std::min<long long>(j.tile_end, max_tiles(j.s, j.TB, j.UB)) - j.tile_begin;
+  const int ntiles_max = (int)std::max<long long>(0, span);
+  // CTA pairs pay off when W_o is large (each CTA then streams half of it);
+  // for small W_o the coupling of the two CTAs' h generation costs more
+  const bool pair = g_joint_variant == 1 ||
+                    (g_joint_variant < 0 && ntiles_max >= sms() && (long long)p.V * p.H >= (1LL << 21));
   CUtensorMap tm;
-  if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.V, p.H, 64, BN)) return FRNNT_ERR_CUDA;
-  if (j.mode == MODE_FWD) return launch_joint_t<MODE_FWD>(tm, p, st);
-  if (j.mode == MODE_FWD_STORE) return launch_joint_t<MODE_FWD_STORE>(tm, p, st);
-  return launch_joint_t<MODE_BWD_DZ>(tm, p, st);
+  // a pair CTA stages 64 of the BN rows of every W_o tile
+  if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.V, p.H, 64, pair ? BN / 2 : BN)) return FRNNT_ERR_CUDA;
+  if (pair) {
+    if (j.mode == MODE_FWD) return launch_joint_t<MODE_FWD, true>(tm, p, ntiles_max, st);
+    if (j.mode == MODE_FWD_STORE) return launch_joint_t<MODE_FWD_STORE, true>(tm, p, ntiles_max, st);
+    return launch_joint_t<MODE_BWD_DZ, true>(tm, p, ntiles_max, st);
+  }
+  if (j.mode == MODE_FWD) return launch_joint_t<MODE_FWD, false>(tm, p, ntiles_max, st);
+  if (j.mode == MODE_FWD_STORE) return launch_joint_t<MODE_FWD_STORE, false>(tm, p, ntiles_max, st);
+  return launch_joint_t<MODE_BWD_DZ, false>(tm, p, ntiles_max, st);
+}
+
+int set_joint_variant(int variant) {
+  const int prev = g_joint_variant;
+  g_joint_variant = variant < 0 ? -1 : (variant > 1 ? 1 : variant);
+  return prev;
 }
 
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {

@@ -28,3 +28,5 @@ extern "C" FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A
   cudaGetLastError();
   return frnnt::gemm_tc(g, (cudaStream_t)stream);
 }
+
+extern "C" FRNNT_API int frnnt_test_joint_variant(int variant) { return frnnt::set_joint_variant(variant); }

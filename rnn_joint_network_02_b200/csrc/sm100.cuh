@@ -42,6 +42,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
   return ok != 0;
 }
 
+// Cluster-scope acquire: for barriers that other CTAs of the cluster arrive on.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Every wait is bounded: after kMaxTries polls of up to kSuspendNs each (about
 // two seconds) the waiter raises the CTA's abort flag and gives up, so a lost
 // arrival ends the kernel with an error status instead of a hang.  Waiters
@@ -49,14 +62,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
 constexpr uint32_t kSuspendNs = 100000;
 constexpr uint32_t kMaxTries = 20000;
 
+// The first poll carries no suspend hint: for a phase that has already
+// completed it returns sooner, which matters in the MMA-issuing thread where
+// every poll delays the next tcgen05.mma.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity, kSuspendNs)) return true;
+  if (mbar_try_wait(bar, parity, 0)) return true;
   for (uint32_t i = 1; i < kMaxTries; ++i) {
     if (*abort_flag) return false;
     if (mbar_try_wait(bar, parity, kSuspendNs)) return true;
   }
   *abort_flag = 1;
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity, 0)) return true;
+  for (uint32_t i = 1; i < kMaxTries; ++i) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait_cluster(bar, parity, kSuspendNs)) return true;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// Warp-wide forms for the roles that issue tcgen05 / TMA work: the whole warp
+// polls (so the decision is uniform) and one elected lane issues.  Issuing
+// from a lone lane of an otherwise parked warp makes every barrier poll stall
+// the MMA stream; a converged warp with elect.sync does not.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity, abort_flag));
 }
 
 // ------------------------------------------------------------------ clusters (CTA pairs)
@@ -201,6 +247,15 @@ __device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive on the mbarrier at this shared offset in every CTA of `cta_mask` once

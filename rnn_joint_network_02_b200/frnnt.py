@@ -26,7 +26,7 @@ STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
             "frnnt_profile_read", "frnnt_fwd_bwd_noalloc")
 NOALLOC_MAX_BYTES = 64 * 1024 * 1024
-TEST_HOOKS = ("frnnt_test_gemm_bf16",)
+TEST_HOOKS = ("frnnt_test_gemm_bf16", "frnnt_test_joint_variant")
 
 
 class Dims(ctypes.Structure):
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
                                            ctypes.c_longlong, vp, ctypes.c_int, ctypes.c_longlong, ctypes.c_int,
                                            ctypes.c_int, vp, ctypes.c_longlong, ctypes.c_int, vp, vp]
         L.frnnt_test_gemm_bf16.restype = ctypes.c_int
+        L.frnnt_test_joint_variant.argtypes = [ctypes.c_int]
+        L.frnnt_test_joint_variant.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -237,3 +239,9 @@ def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: in
     if rc != OK:
         raise FrnntError(rc, error_string(rc))
     return out
+
+
+def set_joint_variant(variant: int) -> int:
+    """Test hook: fused joint kernel variant for later calls (-1 automatic,
+    0 one CTA per cell tile, 1 CTA pairs); returns the previous setting."""
+    return int(lib().frnnt_test_joint_variant(int(variant)))

@@ -125,14 +125,60 @@ def test_padding_labels_are_not_validated(cuda_ok):
 
 # ---------------------------------------------------------------- full-size, sampled utterances
 
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
 @pytest.mark.parametrize("name", ["medium", "large", "long"])
-def test_full_size_sampled_utterances(cuda_ok, name):
+def test_full_size_sampled_utterances(cuda_ok, name, mode):
     """Full-size workloads in the bench's launch configuration: the gradient
-    weights select two utterances, so every output is the oracle's on those two."""
+    weights select two utterances, so every output is the oracle's on those two
+    (the other utterances still run through every kernel)."""
     batch = synth.workload(name)
     B = batch.f.shape[0]
     pick = [0, B - 1]
     w = weights_for(B, pick, device="cpu").numpy()
-    loss, grads = _call(batch, mode="tiled", grad_loss=w)
+    loss, grads = _call(batch, mode=mode, grad_loss=w)
     ref = run_oracle(batch, grad_loss=w, utterances=pick)
-    compare(loss, grads, ref, "bf16", utterances=pick, extra_note=name)
+    compare(loss, grads, ref, "bf16", utterances=pick, extra_note=f"{name}/{mode}")
+
+
+def test_tiled_small_chunks_match_untiled(cuda_ok):
+    """Many backward chunks (one per 4 tiles), including empty trailing chunks,
+    give the untiled result up to floating-point reassociation."""
+    batch = synth.workload("short")
+    lt, gt = _call(batch, mode="tiled", chunk_cells=512)
+    lt, gt = lt.clone(), {k: v.clone() for k, v in gt.items()}
+    lu, gu = _call(batch, mode="untiled")
+    assert torch.allclose(lt, lu, rtol=1e-4)
+    for k in GRADS:
+        assert rel_l2(gt[k].float().cpu().numpy(), gu[k].float().cpu().numpy()) <= 1e-2, k
+
+
+# ---------------------------------------------------------------- joint kernel variants
+
+@pytest.fixture
+def joint_variant():
+    prev = frnnt.set_joint_variant(-1)
+    yield frnnt.set_joint_variant
+    frnnt.set_joint_variant(prev)
+
+
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
+@pytest.mark.parametrize("variant", [0, 1])
+def test_joint_variants_odd_tile_count(cuda_ok, joint_variant, mode, variant):
+    """Both joint kernel variants on the tensor-core path, forced, on a batch
+    with an odd number of cell tiles (5: the last CTA pair holds one real tile
+    and one empty one) and ragged lengths."""
+    batch = synth.make(B=3, T=20, U=5, D_enc=64, D_pred=32, H=128, V=256, dtype="bf16", seed=31,
+                       T_range=(13, 20), U_range=(0, 5), bias_std=0.2)
+    batch.T_len[:] = torch.tensor([20, 13, 17], dtype=batch.T_len.dtype)
+    joint_variant(variant)
+    loss, grads = _call(batch, mode=mode, chunk_cells=256)
+    compare(loss, grads, run_oracle(batch), "bf16", extra_note=f"odd/{mode}/v{variant}")
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+def test_joint_variants_short(cuda_ok, joint_variant, variant):
+    batch = synth.workload("short")
+    joint_variant(variant)
+    for mode in ("tiled", "untiled"):
+        loss, grads = _call(batch, mode=mode)
+        compare(loss, grads, run_oracle(batch), "bf16", extra_note=f"short/{mode}/v{variant}")
