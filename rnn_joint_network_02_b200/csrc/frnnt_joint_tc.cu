@@ -355,7 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     const int r = q * 32 + lane;             // tile row generated by this thread
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const int H = p.H, Up1 = p.U + 1;
-    const int nseg = H / 16;
     uint32_t hph = 0;
     uint32_t fph = 0;
     // warp kGen0 only: wait until the generator warps are done with the buffer
@@ -384,49 +383,64 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
       const uint8_t* grow = fgs + (p.TB + r % p.UB) * fg_stride;
       if (!mbar_wait(fg_full, fph, abort_flag)) break;
-      for (int si = 0; si < nseg / 2; ++si) {
-        const int kb = si >> 1, sub = 2 * half + (si & 1);
-        const int seg = kb * 4 + sub;
-        uint32_t pk[8];
-        if (ri.valid) {
-          // h = tanh(F + G) in packed bf16 pairs (F, G already bf16; h is consumed as bf16)
-          const uint4 f0 = *(const uint4*)(frow + seg * 32), f1 = *(const uint4*)(frow + seg * 32 + 16);
-          const uint4 g0 = *(const uint4*)(grow + seg * 32), g1 = *(const uint4*)(grow + seg * 32 + 16);
-          pk[0] = tanh_bf16x2(add_bf16x2(f0.x, g0.x));
-          pk[1] = tanh_bf16x2(add_bf16x2(f0.y, g0.y));
-          pk[2] = tanh_bf16x2(add_bf16x2(f0.z, g0.z));
-          pk[3] = tanh_bf16x2(add_bf16x2(f0.w, g0.w));
-          pk[4] = tanh_bf16x2(add_bf16x2(f1.x, g1.x));
-          pk[5] = tanh_bf16x2(add_bf16x2(f1.y, g1.y));
-          pk[6] = tanh_bf16x2(add_bf16x2(f1.z, g1.z));
-          pk[7] = tanh_bf16x2(add_bf16x2(f1.w, g1.w));
-        } else {
+      for (int g = 0; g < ngrp; ++g) {
+        const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
+        // the whole group's values first (loads and MUFU work overlap the
+        // wait for the MMAs to release the group), then the stores
+        uint32_t pk[2][2][8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) pk[j] = 0u;
+        for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int seg = (kb0 + kk) * 4 + 2 * half + j;
+            if (kk < nk && ri.valid) {
+              // h = tanh(F + G) in packed bf16 pairs (F, G already bf16; h is consumed as bf16)
+              const uint4 f0 = *(const uint4*)(frow + seg * 32), f1 = *(const uint4*)(frow + seg * 32 + 16);
+              const uint4 g0 = *(const uint4*)(grow + seg * 32), g1 = *(const uint4*)(grow + seg * 32 + 16);
+              pk[kk][j][0] = tanh_bf16x2(add_bf16x2(f0.x, g0.x));
+              pk[kk][j][1] = tanh_bf16x2(add_bf16x2(f0.y, g0.y));
+              pk[kk][j][2] = tanh_bf16x2(add_bf16x2(f0.z, g0.z));
+              pk[kk][j][3] = tanh_bf16x2(add_bf16x2(f0.w, g0.w));
+              pk[kk][j][4] = tanh_bf16x2(add_bf16x2(f1.x, g1.x));
+              pk[kk][j][5] = tanh_bf16x2(add_bf16x2(f1.y, g1.y));
+              pk[kk][j][6] = tanh_bf16x2(add_bf16x2(f1.z, g1.z));
+              pk[kk][j][7] = tanh_bf16x2(add_bf16x2(f1.w, g1.w));
+            } else {
+#pragma unroll
+              for (int w = 0; w < 8; ++w) pk[kk][j][w] = 0u;
+            }
+          }
         }
-        const int grp = kb / p.ks;
-        if ((si & 1) == 0 && kb % p.ks == 0 && !mbar_wait(&hempty[grp], hph ^ 1, abort_flag)) {
+        if (!mbar_wait(&hempty[g], hph ^ 1, abort_flag)) {
           ok = false;
           break;
         }
-        if (kb < kTmemKB) {
-          tmem_st8(tbase + lane_base + kHCol + kb * 32 + sub * 8, pk);
-        } else {
-          uint8_t* blk = hhi + (kb - kTmemKB) * 16384;
-          *(uint4*)(blk + sw128_offset(r, sub * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *(uint4*)(blk + sw128_offset(r, sub * 16 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-        if ((si & 1) == 1 && (kb % p.ks == p.ks - 1 || kb == p.KB - 1)) {
-          // last K block of the group (a group lies wholly in TMEM or wholly in shared memory)
-          if (kb < kTmemKB) {
-            tmem_wait_st();
-            tc_fence_before();
-          } else {
-            fence_proxy_async_smem();
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          if (kk >= nk) break;
+          const int kb = kb0 + kk;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int sub = 2 * half + j;
+            if (kb < kTmemKB) {
+              tmem_st8(tbase + lane_base + kHCol + kb * 32 + sub * 8, pk[kk][j]);
+            } else {
+              uint8_t* blk = hhi + (kb - kTmemKB) * 16384;
+              *(uint4*)(blk + sw128_offset(r, sub * 16)) = make_uint4(pk[kk][j][0], pk[kk][j][1], pk[kk][j][2], pk[kk][j][3]);
+              *(uint4*)(blk + sw128_offset(r, sub * 16 + 8)) =
+                  make_uint4(pk[kk][j][4], pk[kk][j][5], pk[kk][j][6], pk[kk][j][7]);
+            }
           }
-          __syncwarp();
-          if (lane == 0) arrive_leader(&hfull[grp]);
         }
+        // a group lies wholly in TMEM or wholly in shared memory
+        if (kb0 < kTmemKB) {
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) arrive_leader(&hfull[g]);
       }
       if (!ok) break;
       // this warp is done reading the tile's F/G rows
