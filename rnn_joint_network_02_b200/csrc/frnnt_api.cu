@@ -220,6 +220,34 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   return p;
 }
 
+// A second stream per device for work that runs beside the lattice DP (which
+// occupies one block per utterance and direction), forked from and joined
+// back to the caller's stream with events, so stream order, graph capture and
+// the caller's synchronisation are unaffected.  Shared by all calls on the
+// device: concurrent calls from several host threads stay correct and
+// serialise their side work.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ok = false;
+};
+
+SideStream* side_stream() {
+  static SideStream sides[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& x = sides[dev];
+  if (!x.ok && !x.s) {
+    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) == cudaSuccess &&
+        cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess)
+      x.ok = true;
+    else
+      cudaGetLastError();
+  }
+  return x.ok ? &x : nullptr;
+}
+
 int splits_for(int M, int N, int K) {
   const int BN = (N % 256 == 0 && N >= 256) ? 256 : 128;
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
@@ -272,6 +300,20 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     j.tile_end = (int)p.maxT;
     FRNNT_TRY(launch_joint_tc(j, st));
   }
+  // untiled: the h rows of the whole lattice do not depend on the DP; build
+  // them on the side stream while the DP runs
+  SideStream* side = untiled ? side_stream() : nullptr;
+  if (side) {
+    j.tile_begin = 0;
+    j.tile_end = (int)p.maxT;
+    cudaEventRecord(side->fork, st);
+    cudaStreamWaitEvent(side->s, side->fork, 0);
+    {
+      StageScope sc("bwd_hidden", side->s);
+      launch_hidden_rows(j, 0, side->s);
+    }
+    cudaEventRecord(side->join, side->s);
+  }
   {
     StageScope sc("lattice_dp", st);
     launch_dp(s, p.L, T_len, U_len, loss, st);
@@ -292,7 +334,9 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
         FRNNT_TRY(launch_joint_tc(j, st));
       }
     }
-    {
+    if (side) {
+      cudaStreamWaitEvent(st, side->join, 0);
+    } else {
       StageScope sc("bwd_hidden", st);
       launch_hidden_rows(j, untiled ? 0 : (int)c0, st);
     }

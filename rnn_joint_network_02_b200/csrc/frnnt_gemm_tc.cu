@@ -117,24 +117,43 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, int row, int
     for (int j = 0; j < 8; ++j)
       red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-  } else {                   // dtanh: out = acc * (1 - h^2), h read from and result written to out_bf16
-    uint4* hp = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 hv = hp[j];
-      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[q]);
-        float2 hf = __bfloat1622float2(h2);
-        float d0 = __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x);
-        float d1 = __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y);
-        o[q] = pack_bf16x2(d0, d1);
-      }
-      hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
   }
+}
+
+// dtanh epilogue: out = acc * (1 - h^2), with h (bf16) read from out_bf16 into
+// hv before the accumulator chunk is loaded from TMEM, and the result written
+// back in place.
+__device__ __forceinline__ void dtanh_load(const GemmParams& p, int row, int col0, uint4 (&hv)[4]) {
+  const uint4* hp = (const uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hv[j] = hp[j];
+}
+__device__ __forceinline__ void dtanh_store(const GemmParams& p, int row, int col0, const uint32_t (&r)[32],
+                                            const uint4 (&hv4)[4]) {
+  uint4* hp = (uint4*)(p.out_bf16 + (size_t)row * p.ldo + col0);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 hv = hv4[j];
+    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[q]);
+      float2 hf = __bfloat1622float2(h2);
+      float d0 = __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x);
+      float d1 = __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y);
+      o[q] = pack_bf16x2(d0, d1);
+    }
+    hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// dtanh epilogue: pull this thread's h row segment of a coming tile into L2
+// while the tile's MMAs run, so the epilogue's reads do not wait on HBM.
+__device__ __forceinline__ void dtanh_prefetch(const GemmParams& p, int row, int n0, int bn, int M) {
+  if (row >= M) return;
+  const __nv_bfloat16* base = (const __nv_bfloat16*)p.out_bf16 + (size_t)row * p.ldo;
+  for (int c = n0; c < n0 + bn && c < p.N; c += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + c));
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN>
@@ -272,23 +291,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
-      tc_fence_after();
       const int row = m0 + warp * 32 + lane;
       const bool row_ok = row < eff.M;
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0, BN, eff.M);
+      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
+        const int col0 = n0 + c * 32;
+        const bool st = row_ok && col0 < p.N;
+        uint4 hv[4];
+        if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
-        const int col0 = n0 + c * 32;
-        if (!row_ok || col0 >= p.N) continue;
-        epilogue_store(p, row, col0, r);
+        if (!st) continue;
+        if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
+        else epilogue_store(p, row, col0, r);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
       ++acc_i;
+      if (p.epi == GEMM_EPI_DTANH) {
+        int nm0, nnt, nkb0, nkb1;
+        if (unit + (int)gridDim.x < units && unit_coords(unit + gridDim.x, p, eff, nm0, nnt, nkb0, nkb1))
+          dtanh_prefetch(p, nm0 + warp * 32 + lane, nnt * BN, BN, eff.M);
+      }
     }
   }
 
@@ -473,23 +502,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
-      tc_fence_after();
       const int row = m0 + (int)rank * 128 + warp * 32 + lane;
       const bool row_ok = row < eff.M;
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0, BN, eff.M);
+      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
+        const int col0 = n0 + c * 32;
+        const bool st = row_ok && col0 < p.N;
+        uint4 hv[4];
+        if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
-        const int col0 = n0 + c * 32;
-        if (!row_ok || col0 >= p.N) continue;
-        epilogue_store(p, row, col0, r);
+        if (!st) continue;
+        if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
+        else epilogue_store(p, row, col0, r);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
       ++acc_i;
+      if (p.epi == GEMM_EPI_DTANH) {
+        int nm0, nnt, nkb0, nkb1;
+        if (unit + npairs < units && unit_coords2(unit + npairs, p, eff, nm0, nnt, nkb0, nkb1))
+          dtanh_prefetch(p, nm0 + (int)rank * 128 + warp * 32 + lane, nnt * BN, BN, eff.M);
+      }
     }
   }
 
