@@ -635,8 +635,8 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH) && (g.ldo % 8 || !g.out_bf16)) return FRNNT_ERR_DIMS;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
   const int BN = (g.N % 256 == 0 && g.N >= 256) ? 256 : 128;
-  // CTA pairs (M = 256 per MMA) unless the problem has too few rows to fill them
-  const bool pair = g.variant == 1 || (g.variant < 0 && g.M >= 512);
+  // CTA pairs (M = 256 per MMA) for 256-wide N tiles on problems with enough rows
+  const bool pair = g.variant == 1 || (g.variant < 0 && g.M >= 512 && BN == 256);
   CUtensorMap ta, tb;
   bool ok;
   if (!g.a_mn) ok = make_tmap_bf16_2d(&ta, g.A, g.K, g.M, (uint64_t)g.lda, 64, 128);
