@@ -183,7 +183,7 @@ struct TcPlan {
   int* ntiles;
   Lattice L;
   float *accWo, *db_part, *accWf, *accWg;
-  __nv_bfloat16 *zbuf, *hbuf, *Wo_pad;
+  __nv_bfloat16 *zbuf, *hbuf;
   size_t bytes;
 };
 
@@ -215,7 +215,6 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.V);
   p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * hidden_stride(s.H));
-  p.Wo_pad = dh_width(s.H) != s.H ? c.take<__nv_bfloat16>((size_t)s.V * dh_width(s.H)) : nullptr;
   p.bytes = c.off + 256;
   return p;
 }
@@ -276,7 +275,6 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     cudaMemsetAsync(p.dF, 0, s.BT * s.H * sizeof(float), st);
     cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accWo, 0, (size_t)s.V * hidden_stride(s.H) * sizeof(float), st);
-    if (p.Wo_pad) launch_pad_cols(W_o, s.V, s.H, p.Wo_pad, dh_width(s.H), st);
     cudaMemsetAsync(p.accWf, 0, (size_t)s.Dx * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accWg, 0, (size_t)s.Dy * s.H * sizeof(float), st);
   }
@@ -354,10 +352,9 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     {
       StageScope sc("bwd_dh", st);
       GemmTcArgs a{};
-      // N padded to a whole number of 256-wide tiles (W_o zero-padded) when H is not
-      const int NW = dh_width(s.H);
-      a.M = rows; a.N = NW; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = p.Wo_pad ? (const void*)p.Wo_pad : W_o;
-      a.b_mn = true; a.ldb = NW; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
+      // d_hidden = dz W_o, then (1 - h^2) in the epilogue, in place over h
+      a.M = rows; a.N = s.H; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = W_o;
+      a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
       a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
       FRNNT_TRY(gemm_tc(a, st));
     }

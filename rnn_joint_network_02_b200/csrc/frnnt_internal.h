@@ -131,10 +131,8 @@ struct JointLaunch {
 };
 bool joint_tc_supported(int H, int V, int U);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the
-// dW_o GEMM's N is a whole number of its N tiles; and the d_hidden GEMM's N (W_o zero-padded to it).
+// dW_o GEMM's N is a whole number of its N tiles.
 inline int hidden_stride(int H) { return H >= 512 ? ((H + 1 + 255) / 256) * 256 : ((H + 1 + 127) / 128) * 128; }
-inline int dh_width(int H) { return H; }
-void launch_pad_cols(const void* src, int rows, int cols, void* dst, int dcols, cudaStream_t st);
 void tile_shape(int U, int* TB, int* UB);
 long long max_tiles(const Shape& s, int TB, int UB);
 void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,

@@ -627,7 +627,9 @@ __global__ void tiles_kernel(int B, int T, int U, int TB, int UB, const int32_t*
 
 // ------------------------------------------------------------------ untiled backward: dz from stored z
 __global__ void dz_from_z_kernel(JointParams p) {
-  // one warp per row; rows of tiles [tile_begin, ntiles)
+  // one warp per row; rows of tiles [tile_begin, ntiles).  A row's z is read
+  // in batches of four 16-byte chunks per lane, all loads of a batch issued
+  // before any store (the row is rewritten in place).
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int V = p.V, Up1 = p.U + 1;
   const int lane = threadIdx.x & 31;
@@ -653,23 +655,33 @@ __global__ void dz_from_z_kernel(JointParams p) {
     const float lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) * w : 0.f;
     const float occ = bpost + lpost;
     const float lk = lse * kLog2e;
-    for (int k = lane * 8; k < V; k += 256) {
-      uint4 zv = *(const uint4*)(zr + k);
-      uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-      uint32_t o[4];
+    for (int k0 = 0; k0 < V; k0 += 4 * 256) {
+      uint4 zv[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[q]));
-        float d0 = occ * ex2(fmaf(zf.x, kLog2e, -lk));
-        float d1 = occ * ex2(fmaf(zf.y, kLog2e, -lk));
-        const int k0 = k + 2 * q;
-        if (k0 == p.blank) d0 -= bpost;
-        if (k0 + 1 == p.blank) d1 -= bpost;
-        if (k0 == ri.y) d0 -= lpost;
-        if (k0 + 1 == ri.y) d1 -= lpost;
-        o[q] = pack_bf16x2(d0, d1);
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i * 256 + lane * 8;
+        if (k < V) zv[i] = *(const uint4*)(zr + k);
       }
-      *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i * 256 + lane * 8;
+        if (k >= V) break;
+        const uint32_t zw[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[q]));
+          float d0 = occ * ex2(fmaf(zf.x, kLog2e, -lk));
+          float d1 = occ * ex2(fmaf(zf.y, kLog2e, -lk));
+          const int k2 = k + 2 * q;
+          if (k2 == p.blank) d0 -= bpost;
+          if (k2 + 1 == p.blank) d1 -= bpost;
+          if (k2 == ri.y) d0 -= lpost;
+          if (k2 + 1 == ri.y) d1 -= lpost;
+          o[q] = pack_bf16x2(d0, d1);
+        }
+        *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
@@ -1027,25 +1039,6 @@ void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, 
   if (blocks > 148 * 8) blocks = 148 * 8;
   wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), (__nv_bfloat16*)dW_o,
                                                        (__nv_bfloat16*)db_o);
-  note_launch();
-}
-
-// dst[r][0, cols) = src[r][0, cols), dst[r][cols, dcols) = 0 (bf16)
-__global__ void pad_cols_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
-                                __nv_bfloat16* __restrict__ dst, int dcols) {
-  const long long n = (long long)rows * dcols;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long r = i / dcols, c = i % dcols;
-    dst[i] = c < cols ? src[r * cols + c] : __float2bfloat16_rn(0.f);
-  }
-}
-
-void launch_pad_cols(const void* src, int rows, int cols, void* dst, int dcols, cudaStream_t st) {
-  long long n = (long long)rows * dcols;
-  long long blocks = (n + 255) / 256;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  pad_cols_kernel<<<(unsigned)blocks, 256, 0, st>>>((const __nv_bfloat16*)src, rows, cols, (__nv_bfloat16*)dst,
-                                                    dcols);
   note_launch();
 }
 
