@@ -703,16 +703,30 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
     __nv_bfloat16* hr = p.hbuf + ((size_t)(tile - row_tile0) * 128 + (row & 127)) * HS;
     const __nv_bfloat16* Fr = p.F + ((size_t)ri.b * p.T + (ri.valid ? ri.t : 0)) * H;
     const __nv_bfloat16* Gr = p.G + ((size_t)ri.b * Up1 + (ri.valid ? ri.u : 0)) * H;
-    for (int k = lane * 8; k < H; k += 256) {
-      uint4 o = make_uint4(0u, 0u, 0u, 0u);
-      if (ri.valid) {
-        const uint4 f = *(const uint4*)(Fr + k), g = *(const uint4*)(Gr + k);
-        o.x = tanh_bf16x2(add_bf16x2(f.x, g.x));
-        o.y = tanh_bf16x2(add_bf16x2(f.y, g.y));
-        o.z = tanh_bf16x2(add_bf16x2(f.z, g.z));
-        o.w = tanh_bf16x2(add_bf16x2(f.w, g.w));
+    // loads of up to four 16-byte chunks per lane issued before the stores
+    for (int k0 = 0; k0 < H; k0 += 4 * 256) {
+      uint4 f[4], g[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i * 256 + lane * 8;
+        if (k < H && ri.valid) {
+          f[i] = *(const uint4*)(Fr + k);
+          g[i] = *(const uint4*)(Gr + k);
+        }
       }
-      *(uint4*)(hr + k) = o;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i * 256 + lane * 8;
+        if (k >= H) break;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (ri.valid) {
+          o.x = tanh_bf16x2(add_bf16x2(f[i].x, g[i].x));
+          o.y = tanh_bf16x2(add_bf16x2(f[i].y, g[i].y));
+          o.z = tanh_bf16x2(add_bf16x2(f[i].z, g[i].z));
+          o.w = tanh_bf16x2(add_bf16x2(f[i].w, g[i].w));
+        }
+        *(uint4*)(hr + k) = o;
+      }
     }
     for (int k = H + lane * 8; k < HS; k += 256)
       *(uint4*)(hr + k) = make_uint4((k == H && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
@@ -733,44 +747,46 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
   const int HS = p.HS;
   const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * HS;
   // thread (c8, g): 8 consecutive columns, frame rows tl = g (mod 4) for dF and
-  // label rows ul = g (mod 4) for dG
+  // label rows ul = g (mod 4) for dG; rows are loaded four at a time before
+  // they are added, and rows outside the utterance are skipped
   const int g = threadIdx.y;
-  for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
-    for (int tl = g; tl < TB; tl += 4) {
-      const int t = td.y + tl;
-      if (t >= l.Tb) break;
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int ul = 0; ul < UB; ++ul) {
-        if (td.z + ul > l.Ub) break;
-        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * HS + c8 * 8);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  const int nt = min(TB, l.Tb - td.y), nu = min(UB, l.Ub + 1 - td.z);
+  auto add8 = [](float (&acc)[8], const uint4 v) {
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
-          acc[2 * q] += f.x;
-          acc[2 * q + 1] += f.y;
-        }
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
+      acc[2 * q] += f.x;
+      acc[2 * q + 1] += f.y;
+    }
+  };
+  for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
+    const __nv_bfloat16* col = base + c8 * 8;
+    for (int tl = g; tl < nt; tl += 4) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int u0 = 0; u0 < nu; u0 += 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          v[i] = u0 + i < nu ? *(const uint4*)(col + (size_t)(tl * UB + u0 + i) * HS) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) add8(acc, v[i]);
       }
-      float* dst = dF + ((size_t)td.x * p.T + t) * H + c8 * 8;
+      float* dst = dF + ((size_t)td.x * p.T + td.y + tl) * H + c8 * 8;
       red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
       red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
     }
-    for (int ul = g; ul < UB; ul += 4) {
-      const int u = td.z + ul;
-      if (u > l.Ub) break;
+    for (int ul = g; ul < nu; ul += 4) {
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int tl = 0; tl < TB; ++tl) {
-        if (td.y + tl >= l.Tb) break;
-        const uint4 v = *(const uint4*)(base + (size_t)(tl * UB + ul) * HS + c8 * 8);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      for (int t0 = 0; t0 < nt; t0 += 4) {
+        uint4 v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
-          acc[2 * q] += f.x;
-          acc[2 * q + 1] += f.y;
-        }
+        for (int i = 0; i < 4; ++i)
+          v[i] = t0 + i < nt ? *(const uint4*)(col + (size_t)((t0 + i) * UB + ul) * HS) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) add8(acc, v[i]);
       }
-      float* dst = dG + ((size_t)td.x * Up1 + u) * H + c8 * 8;
+      float* dst = dG + ((size_t)td.x * Up1 + td.z + ul) * H + c8 * 8;
       red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
       red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
     }
