@@ -1,10 +1,11 @@
 // Persistent, warp-specialised bf16 GEMM on the 5th-generation tensor cores:
 //   D[M,N] (fp32, TMEM) = A[M,K] * B[K,N]   with a fused epilogue.
 //
-// Roles (192 threads, one CTA per SM):
-//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld), then store / reduce
-//   warp 4     producer: TMA tile loads of A and B into a STAGES-deep ring
-//   warp 5     MMA issuer: one thread issues tcgen05.mma, commits to mbarriers
+// Roles (320 threads, one CTA per SM):
+//   warps 0-7  epilogue: TMEM -> registers (tcgen05.ld), then store / reduce;
+//              warp w reads TMEM lane quadrant w % 4, columns of half w / 4
+//   warp 8     producer: TMA tile loads of A and B into a STAGES-deep ring
+//   warp 9     MMA issuer: one elected lane issues tcgen05.mma, commits to mbarriers
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
 // of one output tile overlaps the main loop of the next.  Work units are
 // (m tile, n tile, k slice) triples handed out round-robin; split-K slices
@@ -27,7 +28,10 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+// warps 0-7 epilogue (two per TMEM lane quadrant, each half of the tile's
+// columns), warp 8 TMA producer, warp 9 MMA issuer
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8, kProdWarp = 8, kMmaWarp = 9;
 
 struct GemmParams {
   int M, N, K;
@@ -180,16 +184,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_base_p, 2 * BN);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProdWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ---------------------------------------------------------------- producer (warp polls, one lane issues)
     {
       int s = 0;
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer (warp polls, one lane issues)
     {
       constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 0-3)
+    // ---------------------------------------------------------------- epilogue (warps 0-7)
     int acc_i = 0;
     for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
       int m0, nt, kb0, kb1;
@@ -291,19 +295,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      const int row = m0 + warp * 32 + lane;
+      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column half
+      const int row = m0 + q * 32 + lane;
       const bool row_ok = row < eff.M;
-      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0, BN, eff.M);
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
       if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         const int col0 = n0 + c * 32;
         const bool st = row_ok && col0 < p.N;
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
-        tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
+        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (!st) continue;
         if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
@@ -316,13 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.epi == GEMM_EPI_DTANH) {
         int nm0, nnt, nkb0, nkb1;
         if (unit + (int)gridDim.x < units && unit_coords(unit + gridDim.x, p, eff, nm0, nnt, nkb0, nkb1))
-          dtanh_prefetch(p, nm0 + warp * 32 + lane, nnt * BN, BN, eff.M);
+          dtanh_prefetch(p, nm0 + q * 32 + lane, nnt * BN + half * (BN / 2), BN / 2, eff.M);
       }
     }
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tbase, 2 * BN);
   }
@@ -389,16 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);         // 4 epilogue warps in each CTA of the pair
+      mbar_init(&tempty[i], 2 * kEpiWarps);   // the epilogue warps of both CTAs of the pair
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc_pair(tmem_base_p, 2 * BN);
     tmem_relinquish_pair();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProdWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -406,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ---------------------------------------------------------------- producer (both CTAs; warp polls, one lane issues)
     {
       int s = 0;
@@ -449,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer (leader CTA only; warp polls, one lane issues)
     if (rank == 0) {
       constexpr uint32_t idesc = idesc_bf16(256, BN, A_MN, B_MN);
@@ -494,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 0-3, both CTAs)
+    // ---------------------------------------------------------------- epilogue (warps 0-7, both CTAs)
     int acc_i = 0;
     for (int unit = pair; unit < units; unit += npairs) {
       int m0, nt, kb0, kb1;
@@ -502,19 +507,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      const int row = m0 + (int)rank * 128 + warp * 32 + lane;
+      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column half
+      const int row = m0 + (int)rank * 128 + q * 32 + lane;
       const bool row_ok = row < eff.M;
-      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0, BN, eff.M);
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
       if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         const int col0 = n0 + c * 32;
         const bool st = row_ok && col0 < p.N;
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
-        tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + a * BN + c * 32, r);
+        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (!st) continue;
         if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
@@ -527,14 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.epi == GEMM_EPI_DTANH) {
         int nm0, nnt, nkb0, nkb1;
         if (unit + npairs < units && unit_coords2(unit + npairs, p, eff, nm0, nnt, nkb0, nkb1))
-          dtanh_prefetch(p, nm0 + (int)rank * 128 + warp * 32 + lane, nnt * BN, BN, eff.M);
+          dtanh_prefetch(p, nm0 + (int)rank * 128 + q * 32 + lane, nnt * BN + half * (BN / 2), BN / 2, eff.M);
       }
     }
   }
 
   __syncthreads();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tbase, 2 * BN);
   }
