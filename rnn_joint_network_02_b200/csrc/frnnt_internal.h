@@ -141,7 +141,8 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
 // Joint kernel variant for later calls: -1 automatic, 0 one CTA per cell tile, 1 CTA pairs; returns the previous one.
 int set_joint_variant(int variant);
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
-void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st);
+// blocks_per_sm: 256-thread blocks per SM of the grid (fewer leave room for work running beside it)
+void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
 void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);
 void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st);
 

@@ -1004,7 +1004,7 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   note_launch();
 }
 
-void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st) {
+void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm) {
   JointParams p{};
   p.T = j.s.T;
   p.U = j.s.U;
@@ -1023,7 +1023,7 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st) {
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
-  hidden_rows_kernel<<<sms() * 8, 256, 0, st>>>(p, row_tile0);
+  hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
   note_launch();
 }
 
