@@ -51,6 +51,17 @@ def parse():
     return p.parse_args()
 
 
+# DRAM bytes (read + write) per launch of a stage's kernel, from one ncu
+# capture of that kernel in the bench's own launch configuration (the file
+# under profiles/ gives the command).  An entry is removed whenever its kernel
+# changes, so the roofline's traffic is null rather than stale.
+MEASURED_TRAFFIC = {
+    ("medium", "untiled", "bwd_dh"): (1.010189e9 + 0.352219e9, "profiles/ncu_gemm_tc_medium_untiled.md"),
+    ("medium", "untiled", "joint_fwd"): (0.009213e9 + 0.570038e9, "profiles/ncu_joint_tc_medium_untiled.md"),
+    ("medium", "tiled", "joint_fwd"): (0.008490e9, "profiles/ncu_joint_tc_medium_tiled.md"),
+}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -310,16 +321,19 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         dom = max(stages, key=lambda k: stages[k]["ms"])
         kind, work = stage_work(batch, dom, mode)
         per_call_ms = stages[dom]["ms"] / args.steps
+        tr = MEASURED_TRAFFIC.get((args.workload, mode, dom))
         if kind == "tensor":
             achieved = work / (per_call_ms / 1e3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor_sustained"], "unit": "TFLOP/s",
-                        "frac": achieved / pk["tensor_sustained"], "traffic": None, "stage": dom,
+                        "frac": achieved / pk["tensor_sustained"], "traffic": tr[0] if tr else None,
+                        "traffic_source": tr[1] if tr else None, "stage": dom,
                         "launches_per_step": stages[dom]["launches"] / args.steps,
                         "peak_source": pk["source"] + " sustained dense bf16 (the stage runs inside a long step)"}
         elif kind == "hbm":
             achieved = work / (per_call_ms / 1e3) / 1e9
             roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                        "frac": achieved / pk["hbm"], "traffic": None, "stage": dom, "peak_source": pk["source"]}
+                        "frac": achieved / pk["hbm"], "traffic": tr[0] if tr else None,
+                        "traffic_source": tr[1] if tr else None, "stage": dom, "peak_source": pk["source"]}
     return {"ms": ms, "value": world * units / (ms / 1e3), "peak_bytes": peak_bytes,
             "valid_cells_per_s": world * batch.valid_cells() * batch.dims["V"] / (ms / 1e3),
             "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
