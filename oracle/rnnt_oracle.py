@@ -36,6 +36,19 @@ What it computes (the definitions, written out plainly, in float64):
   logits (dz = w_b (occ*softmax - bpost*e_blank - lpost*e_label)) and, by the
   chain rule through the joint, for b_o, W_o, the hidden pre-activation, f,
   g, W_f and W_g.
+* Maximum approximation (``loss="viterbi"``): the sum over alignments is
+  replaced by the single best alignment ("Daily Papers" page for the
+  CTC/RNN-T architecture search, the RNN-transducer abstract that compares
+  full marginalisation over alignments with the maximum approximation).
+  The pages give no recursion, so
+  the plainest reading is used: the same lattice with max in place of lae,
+      alpha(t,u) = max(alpha(t-1,u) + blank_lp(t-1,u),
+                       alpha(t,u-1) + label_lp(t,u-1)),
+      loss = -(alpha(T_len-1,U_len) + blank_lp(T_len-1,U_len)),
+  the best alignment recovered by backtracking from the last cell, and ties
+  broken towards the blank edge (arriving at (t,u) from (t-1,u)).  The loss
+  is -log p(best alignment), so its gradient is the marginal formula with
+  bpost / lpost the 0/1 indicators of the best alignment's edges.
 
 Every float op here is float64; inputs that the product path receives in
 bf16 are handed to the oracle already rounded to bf16 (by the shared seeded
@@ -139,6 +152,45 @@ def beta_lattice(blank_lp, label_lp, Tb: int, Ub: int):
     return Bt
 
 
+def viterbi_lattice(blank_lp, label_lp, Tb: int, Ub: int):
+    """Max-product forward variables and the best predecessor of every cell.
+
+    Returns (A, from_blank) with from_blank[t,u] True when the best way into
+    (t,u) is the blank edge from (t-1,u) (ties go to the blank edge)."""
+    A = np.full((Tb, Ub + 1), NEG_INF)
+    from_blank = np.zeros((Tb, Ub + 1), dtype=bool)
+    for t in range(Tb):
+        for u in range(Ub + 1):
+            if t == 0 and u == 0:
+                A[t, u] = 0.0
+                continue
+            by_blank = A[t - 1, u] + blank_lp[t - 1, u] if t > 0 else NEG_INF
+            by_label = A[t, u - 1] + label_lp[t, u - 1] if u > 0 else NEG_INF
+            if by_blank >= by_label:
+                A[t, u] = by_blank
+                from_blank[t, u] = True
+            else:
+                A[t, u] = by_label
+    return A, from_blank
+
+
+def best_alignment(from_blank, Tb: int, Ub: int):
+    """0/1 indicators of the edges leaving each cell on the best alignment:
+    (blank edge (t,u)->(t+1,u) incl. the final blank, label edge (t,u)->(t,u+1))."""
+    bpath = np.zeros((Tb, Ub + 1))
+    lpath = np.zeros((Tb, Ub + 1))
+    t, u = Tb - 1, Ub
+    bpath[t, u] = 1.0                      # the final blank that ends the last frame
+    while (t, u) != (0, 0):
+        if from_blank[t, u]:
+            t -= 1
+            bpath[t, u] = 1.0
+        else:
+            u -= 1
+            lpath[t, u] = 1.0
+    return bpath, lpath
+
+
 @dataclass
 class UtteranceLattice:
     """Per-cell quantities of one utterance, each of shape (Tb, Ub+1)."""
@@ -172,7 +224,8 @@ def _frame_block(Ub: int, V: int, H: int, budget_bytes: int = 1 << 28) -> int:
 
 
 def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
-            blank: int = 0, utterances=None, keep_lattice: bool = False) -> OracleResult:
+            blank: int = 0, utterances=None, keep_lattice: bool = False,
+            loss: str = "marginal") -> OracleResult:
     """Loss and gradients of sum_b w_b * loss_b, all in float64.
 
     f [B,T,D_enc], g [B,U+1,D_pred], W_f [D_enc,H], W_g [D_pred,H], W_o [V,H],
@@ -180,7 +233,10 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
     ``utterances`` restricts the work to a subset of b (the others get loss NaN
     and contribute nothing to the weight gradients; their df/dg rows are 0).
     Gradient rows for frames t >= T_len[b] and positions u > U_len[b] are 0.
+    ``loss`` is "marginal" (all alignments) or "viterbi" (the best one).
     """
+    if loss not in ("marginal", "viterbi"):
+        raise ValueError(f"unknown loss {loss!r}")
     f = np.asarray(f, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     W_f = np.asarray(W_f, dtype=np.float64)
@@ -222,23 +278,31 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
             for u in range(Ub):
                 label_lp[t0:t1, u] = z[:, u, y[u]] - blk_lse[:, u]
 
-        # transducer loss
-        A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
-        Bt = beta_lattice(blank_lp, label_lp, Tb, Ub)
-        log_p = A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub]
-        assert abs(Bt[0, 0] - log_p) <= 1e-9 * max(1.0, abs(log_p)), (Bt[0, 0], log_p)
-        res.loss[b] = -log_p
+        if loss == "viterbi":
+            # best alignment: its log-probability and its edges
+            A, from_blank = viterbi_lattice(blank_lp, label_lp, Tb, Ub)
+            log_p = A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub]
+            res.loss[b] = -log_p
+            bpost, lpost = best_alignment(from_blank, Tb, Ub)
+            Bt = np.full((Tb, Ub + 1), np.nan)              # no backward variables in this variant
+        else:
+            # transducer loss
+            A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
+            Bt = beta_lattice(blank_lp, label_lp, Tb, Ub)
+            log_p = A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub]
+            assert abs(Bt[0, 0] - log_p) <= 1e-9 * max(1.0, abs(log_p)), (Bt[0, 0], log_p)
+            res.loss[b] = -log_p
 
-        # alignment posteriors of each outgoing edge
-        beta_next_t = np.full((Tb, Ub + 1), NEG_INF)       # beta'(t+1, u)
-        beta_next_t[:-1] = Bt[1:]
-        beta_next_t[Tb - 1, Ub] = 0.0                       # terminal blank
-        beta_next_u = np.full((Tb, Ub + 1), NEG_INF)       # beta(t, u+1)
-        beta_next_u[:, :-1] = Bt[:, 1:]
-        bpost = np.exp(A + blank_lp + beta_next_t - log_p)
-        lpost = np.where(np.isfinite(label_lp), np.exp(A + label_lp + beta_next_u - log_p), 0.0)
-        occ = np.exp(A + Bt - log_p)
-        assert np.allclose(occ, bpost + lpost, rtol=1e-9, atol=1e-12)
+            # alignment posteriors of each outgoing edge
+            beta_next_t = np.full((Tb, Ub + 1), NEG_INF)       # beta'(t+1, u)
+            beta_next_t[:-1] = Bt[1:]
+            beta_next_t[Tb - 1, Ub] = 0.0                       # terminal blank
+            beta_next_u = np.full((Tb, Ub + 1), NEG_INF)       # beta(t, u+1)
+            beta_next_u[:, :-1] = Bt[:, 1:]
+            bpost = np.exp(A + blank_lp + beta_next_t - log_p)
+            lpost = np.where(np.isfinite(label_lp), np.exp(A + label_lp + beta_next_u - log_p), 0.0)
+            occ = np.exp(A + Bt - log_p)
+            assert np.allclose(occ, bpost + lpost, rtol=1e-9, atol=1e-12)
 
         # backward through the joint (logits recomputed per frame block)
         dF = np.zeros((Tb, H))
@@ -270,7 +334,7 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
     return res
 
 
-def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0):
+def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, loss: str = "marginal"):
     """Per-utterance losses (forward only), used by finite-difference checks."""
     f = np.asarray(f, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
@@ -289,6 +353,9 @@ def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0):
         label_lp = np.full((Tb, Ub + 1), NEG_INF)
         for u in range(Ub):
             label_lp[:, u] = z[:, u, int(labels[b, u])] - lse[:, u]
-        A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
+        if loss == "viterbi":
+            A, _ = viterbi_lattice(blank_lp, label_lp, Tb, Ub)
+        else:
+            A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
         out[b] = -(A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub])
     return out
