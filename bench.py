@@ -47,6 +47,8 @@ def parse():
                    help="both: untiled is the headline value, tiled is reported alongside")
     p.add_argument("--path", default="auto", choices=["auto", "simt"])
     p.add_argument("--chunk-cells", type=int, default=0)
+    p.add_argument("--loss", default="marginal", choices=["marginal", "viterbi"],
+                   help="training criterion: every alignment (default) or the best one")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -75,6 +77,7 @@ def config_of(batch, args, n_gpus):
     d = batch.dims
     return {"workload": args.workload, "B": d["B"], "T": d["T"], "U": d["U"], "D_enc": d["D_enc"],
             "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": args.mode, "path": args.path,
+            "loss": args.loss,
             "valid_cells": batch.valid_cells(), "padded_cells": batch.padded_cells(),
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{n_gpus}",
             "global_batch": d["B"] * n_gpus}
@@ -173,7 +176,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle (CPU) leg
 
-def oracle_sample(batch, utterance=0):
+def oracle_sample(batch, utterance=0, loss="marginal"):
     """Times the fp64 oracle on one utterance; returns (seconds, metric units)."""
     import numpy as np
 
@@ -183,7 +186,7 @@ def oracle_sample(batch, utterance=0):
     w[utterance] = 1.0
     t0 = time.perf_counter()
     oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
-                   grad_loss=w, utterances=[utterance])
+                   grad_loss=w, utterances=[utterance], loss=loss)
     dt = time.perf_counter() - t0
     d = batch.dims
     units = d["T"] * (d["U"] + 1) * d["V"]      # this utterance's share of B*T*(U+1)*V
@@ -203,11 +206,11 @@ def run_reference(args):
         return
     batch = synth.workload(args.workload)
     for _ in range(args.warmup):
-        oracle_sample(batch)
+        oracle_sample(batch, loss=args.loss)
     times = []
     units = 0
     for _ in range(args.steps):
-        dt, units = oracle_sample(batch)
+        dt, units = oracle_sample(batch, loss=args.loss)
         times.append(dt)
     sec = sum(times) / len(times)
     value = units / sec
@@ -229,13 +232,14 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     """Times one mode: warm-up, K timed steps (each after an L2 flush), the
     end-to-end variant with host buffers, per-stage device times."""
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
-    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank)
+    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank,
+                         args.loss)
     out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims)
     stream = torch.cuda.current_stream(dev)
 
     def call(check=False):
         res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
-                            d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells,
+                            d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells, loss=args.loss,
                             blank=batch.blank, out=out, check=check, stream=stream)
         if world > 1:
             # the data-parallel exchange: weight gradients summed over ranks
@@ -373,7 +377,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, u = oracle_sample(batch)
+        dt, u = oracle_sample(batch, loss=args.loss)
         Tb, Ub = int(batch.T_len[0]), int(batch.U_len[0])
         cpu = {"value": u / dt, "unit": UNIT, "cores": cores(), "kind": "oracle",
                "sample": f"utterance 0 of {args.workload} (T_len={Tb}, U_len={Ub}); units = T*(U+1)*V of one "

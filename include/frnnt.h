@@ -63,6 +63,15 @@ typedef enum { FRNNT_F32 = 0, FRNNT_BF16 = 1 } frnnt_dtype;
  * multiple of 128) and the CUDA-core kernels otherwise; SIMT forces the
  * CUDA-core kernels (fp32 arithmetic on bf16 or fp32 inputs). */
 typedef enum { FRNNT_PATH_AUTO = 0, FRNNT_PATH_SIMT = 1 } frnnt_path;
+/* Training criterion.  MARGINAL: -log of the probability summed over every
+ * alignment ("Sequence Transduction with Recurrent Neural Networks",
+ * abstract).  VITERBI: the maximum approximation, -log of the probability of
+ * the single best alignment ("Daily Papers" page, CTC/RNN-T architecture
+ * search, the RNN-transducer abstract comparing full marginalisation with the
+ * maximum approximation): the same lattice with max in place of log-add-exp,
+ * ties broken towards the blank edge, and the gradient taken along that one
+ * alignment (0/1 edge posteriors). */
+typedef enum { FRNNT_LOSS_MARGINAL = 0, FRNNT_LOSS_VITERBI = 1 } frnnt_loss;
 
 typedef struct {
   int B, T, U;            /* batch, max frames, max labels (g has U+1 rows) */
@@ -74,6 +83,7 @@ typedef struct {
   frnnt_path path;
   int chunk_cells;        /* FRNNT_TILED: lattice cells per backward chunk;
                              0 = default (65536).  Rounded up to whole tiles. */
+  frnnt_loss loss;        /* training criterion (MARGINAL unless set)         */
 } frnnt_dims;
 
 /* Host return codes. */

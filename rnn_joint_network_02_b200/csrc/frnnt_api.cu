@@ -40,6 +40,7 @@ bool enums_ok(const frnnt_dims* d) {
   if (d->dtype != FRNNT_F32 && d->dtype != FRNNT_BF16) return false;
   if (d->mode != FRNNT_UNTILED && d->mode != FRNNT_TILED) return false;
   if (d->path != FRNNT_PATH_AUTO && d->path != FRNNT_PATH_SIMT) return false;
+  if (d->loss != FRNNT_LOSS_MARGINAL && d->loss != FRNNT_LOSS_VITERBI) return false;
   return true;
 }
 
@@ -52,6 +53,7 @@ Shape shape_of(const frnnt_dims* d) {
   s.BU = (long long)d->B * (d->U + 1);
   s.Np = s.BT * s.Up1;
   s.bf16 = d->dtype == FRNNT_BF16;
+  s.viterbi = d->loss == FRNNT_LOSS_VITERBI;
   return s;
 }
 
@@ -83,6 +85,7 @@ SimtPlan plan_simt(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.label_lp = c.take<float>(s.Np);
   p.L.alpha = c.take<float>(s.Np);
   p.L.beta = c.take<float>(s.Np);
+  p.L.path = s.viterbi ? c.take<uint8_t>(s.Np) : nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   p.accWo = c.take<float>((size_t)s.V * s.H);
@@ -209,6 +212,7 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.label_lp = c.take<float>(s.Np);
   p.L.alpha = c.take<float>(s.Np);
   p.L.beta = c.take<float>(s.Np);
+  p.L.path = s.viterbi ? c.take<uint8_t>(s.Np) : nullptr;
   p.accWo = c.take<float>((size_t)s.V * hidden_stride(s.H));
   p.db_part = nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);

@@ -144,11 +144,130 @@ __global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, cons
   }
 }
 
+// Maximum approximation: the alpha wavefront with max in place of log-add-exp
+// (same schedule as dp_kernel's alpha block), recording for every cell
+// whether its best predecessor is the blank edge from (t-1, u) (ties go to
+// the blank edge); then one thread walks the best alignment back from
+// (T_len-1, U_len), marking the edge by which it leaves each cell on it.
+// The decisions go to a shared-memory bit array (one bit per padded cell of
+// the utterance) when `smem_bits`, so the walk reads no global memory;
+// otherwise to bit 2 of the path bytes.
+__global__ void dp_viterbi_kernel(int T, int U, const float* __restrict__ blank_lp,
+                                  const float* __restrict__ label_lp, float* __restrict__ alpha,
+                                  uint8_t* __restrict__ path, const int32_t* __restrict__ T_len,
+                                  const int32_t* __restrict__ U_len, float* __restrict__ loss, int smem_bits) {
+  __shared__ float xs[2][32];
+  extern __shared__ uint32_t dec_bits[];   // smem_bits: ceil(T (U+1) / 32) words
+  const int b = blockIdx.x;
+  const int u = threadIdx.x;
+  const int lane = u & 31, warp = u >> 5;
+  const Lengths l = lengths_of(T_len, U_len, b, T, U);
+  const int Tb = l.Tb, Ub = l.Ub;
+  const int Up1 = U + 1;
+  const size_t base = (size_t)b * T * Up1;
+  const int ndiag = Tb + Ub;
+  if (smem_bits) {
+    const int nwords = (T * Up1 + 31) / 32;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) dec_bits[i] = 0u;
+    __syncthreads();
+  }
+
+  float qb[kPrefetch], ql[kPrefetch];
+#pragma unroll
+  for (int i = 0; i < kPrefetch; ++i)
+    dp_operands(false, i, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
+
+  float cur = -INFINITY;
+  for (int step0 = 0; step0 < ndiag; step0 += kPrefetch) {
+#pragma unroll
+    for (int i = 0; i < kPrefetch; ++i) {
+      const int step = step0 + i;
+      if (step >= ndiag) break;     // uniform across the block
+      const float ob = qb[i], ol = ql[i];
+      dp_operands(false, step + kPrefetch, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
+      const int t = step - u;
+      const bool active = (u <= Ub) && (t >= 0) && (t < Tb);
+      float nb = __shfl_up_sync(0xffffffffu, cur, 1);
+      if (lane == 0) nb = warp > 0 ? xs[(step + 1) & 1][warp - 1] : -INFINITY;
+      float v = -INFINITY;
+      if (active) {
+        const size_t c = base + (size_t)t * Up1 + u;
+        bool from_blank = false;
+        if (t == 0 && u == 0) {
+          v = 0.f;
+        } else {
+          const float fb = t > 0 ? cur + ob : -INFINITY;   // from (t-1, u)
+          const float fl = u > 0 ? nb + ol : -INFINITY;    // from (t, u-1)
+          from_blank = fb >= fl;
+          v = from_blank ? fb : fl;
+        }
+        alpha[c] = v;
+        if (smem_bits) {
+          path[c] = 0;
+          if (from_blank) {
+            const int idx = t * Up1 + u;
+            atomicOr(&dec_bits[idx >> 5], 1u << (idx & 31));
+          }
+        } else {
+          path[c] = from_blank ? 4 : 0;
+        }
+      }
+      cur = v;
+      if (lane == 31) xs[step & 1][warp] = cur;
+      __syncthreads();
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const size_t cl = base + (size_t)(Tb - 1) * Up1 + Ub;
+    loss[b] = -(alpha[cl] + blank_lp[cl]);
+    path[cl] |= 1;                  // the final blank
+    int t = Tb - 1, uu = Ub;
+    while (t > 0 || uu > 0) {       // t + uu falls by one per step
+      const size_t c = base + (size_t)t * Up1 + uu;
+      const int idx = t * Up1 + uu;
+      const bool by_blank = smem_bits ? ((dec_bits[idx >> 5] >> (idx & 31)) & 1u) != 0 : (path[c] & 4) != 0;
+      // the predecessor's edge bit (a plain store when the decisions are in
+      // shared memory: the byte was zeroed by the wavefront)
+      size_t pc;
+      uint8_t bit;
+      if (by_blank && t > 0) {
+        --t;
+        pc = c - Up1;
+        bit = 1;
+      } else if (uu > 0) {
+        --uu;
+        pc = c - 1;
+        bit = 2;
+      } else {
+        --t;                        // not reached with finite log-probs
+        pc = c - Up1;
+        bit = 1;
+      }
+      if (smem_bits) path[pc] = bit;
+      else path[pc] |= bit;
+    }
+  }
+}
+
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
                cudaStream_t st) {
   int threads = ((s.Up1 + 31) / 32) * 32;
-  dim3 grid(s.B, 2);
-  dp_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
+  if (L.path) {
+    // decision bits in shared memory when they fit in 96 KB
+    const long long words = ((long long)s.T * s.Up1 + 31) / 32;
+    const int smem = words * 4 <= 96 * 1024 ? (int)(words * 4) : 0;
+    static bool attr = false;
+    if (!attr) {
+      cudaFuncSetAttribute(dp_viterbi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+      attr = true;
+    }
+    dp_viterbi_kernel<<<s.B, threads, smem, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.path, T_len,
+                                                  U_len, loss, smem > 0 ? 1 : 0);
+  } else {
+    dim3 grid(s.B, 2);
+    dp_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
+  }
   note_launch();
 }
 

@@ -37,6 +37,7 @@ struct Shape {
   long long BU;       // B * (U + 1)  (rows of g, G, dG, dg)
   long long Np;       // B * T * (U + 1) padded lattice cells
   bool bf16;
+  bool viterbi;       // maximum-approximation loss
 };
 
 // Lattice arrays, fp32, padded layout [b][t][u] with u fastest.
@@ -46,7 +47,35 @@ struct Lattice {
   float* label_lp;
   float* alpha;
   float* beta;
+  // Maximum approximation only (null otherwise): per cell, bit 0 = the best
+  // alignment leaves the cell by its blank edge, bit 1 = by its label edge,
+  // bit 2 = the best way into the cell is its blank edge (DP decision).
+  uint8_t* path;
 };
+
+#ifdef __CUDACC__
+// Posterior of the two edges leaving valid cell (t, u) at lattice index c
+// (padded layout, utterance base c0 = index of (0, 0)):
+//   marginal: bpost = exp(alpha + blank_lp + beta'(t+1,u) - logP) with
+//             beta'(T_len, U_len) = 0; lpost = exp(alpha + label_lp + beta(t,u+1) - logP);
+//   maximum approximation: the best alignment's 0/1 edge indicators.
+__device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size_t c0, int Up1, int t, int u, int Tb,
+                                                int Ub, float& bpost, float& lpost) {
+  if (L.path) {
+    const uint8_t e = L.path[c];
+    bpost = (e & 1) ? 1.f : 0.f;
+    lpost = (e & 2) ? 1.f : 0.f;
+    return;
+  }
+  const float logp = L.beta[c0];
+  const float al = L.alpha[c];
+  float beta_t1;
+  if (t + 1 < Tb) beta_t1 = L.beta[c + Up1];
+  else beta_t1 = (u == Ub) ? 0.f : -INFINITY;
+  bpost = __expf(al + L.blank_lp[c] + beta_t1 - logp);
+  lpost = u < Ub ? __expf(al + L.label_lp[c] + L.beta[c + 1] - logp) : 0.f;
+}
+#endif
 
 // ---------------------------------------------------------------- validation / DP
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,

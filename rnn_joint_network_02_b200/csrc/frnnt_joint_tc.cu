@@ -467,15 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       float lk = 0.f, bpost = 0.f, lpost = 0.f, occ = 0.f;
       if (MODE == MODE_BWD_DZ && ri.valid) {
         const size_t c = ri.cell;
-        const float logp = p.L.beta[(size_t)ri.b * p.T * Up1];
-        const float al = p.L.alpha[c];
-        float beta_t1;
-        if (ri.t + 1 < ri.Tb) beta_t1 = p.L.beta[c + Up1];
-        else beta_t1 = (ri.u == ri.Ub) ? 0.f : -INFINITY;
         lk = p.L.lse[c] * kLog2e;
         const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
-        bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp) * w;
-        lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) * w : 0.f;
+        edge_posteriors(p.L, c, (size_t)ri.b * p.T * Up1, Up1, ri.t, ri.u, ri.Tb, ri.Ub, bpost, lpost);
+        bpost *= w;
+        lpost *= w;
         occ = bpost + lpost;
       }
       bool ok = true;
@@ -644,15 +640,12 @@ __global__ void dz_from_z_kernel(JointParams p) {
       continue;
     }
     const size_t c = ri.cell;
-    const float logp = p.L.beta[(size_t)ri.b * p.T * Up1];
-    const float al = p.L.alpha[c];
-    float beta_t1;
-    if (ri.t + 1 < ri.Tb) beta_t1 = p.L.beta[c + Up1];
-    else beta_t1 = (ri.u == ri.Ub) ? 0.f : -INFINITY;
     const float lse = p.L.lse[c];
     const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
-    const float bpost = __expf(al + p.L.blank_lp[c] + beta_t1 - logp) * w;
-    const float lpost = ri.u < ri.Ub ? __expf(al + p.L.label_lp[c] + p.L.beta[c + 1] - logp) * w : 0.f;
+    float bpost, lpost;
+    edge_posteriors(p.L, c, (size_t)ri.b * p.T * Up1, Up1, ri.t, ri.u, ri.Tb, ri.Ub, bpost, lpost);
+    bpost *= w;
+    lpost *= w;
     const float occ = bpost + lpost;
     const float lk = lse * kLog2e;
     for (int k0 = 0; k0 < V; k0 += 4 * 256) {

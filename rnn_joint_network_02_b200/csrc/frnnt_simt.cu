@@ -218,14 +218,8 @@ __global__ void dz_simt_kernel(int T, int U, int V, int blank, float* __restrict
       for (int k = threadIdx.x; k < V; k += blockDim.x) zr[k] = 0.f;
       continue;
     }
-    const size_t ub = (size_t)b * T * Up1;
-    const float logp = L.beta[ub];
-    const float a = L.alpha[c];
-    float beta_t1;
-    if (t + 1 < l.Tb) beta_t1 = L.beta[c + Up1];
-    else beta_t1 = (u == l.Ub) ? 0.f : -INFINITY;
-    const float bpost = __expf(a + L.blank_lp[c] + beta_t1 - logp);
-    const float lpost = u < l.Ub ? __expf(a + L.label_lp[c] + L.beta[c + 1] - logp) : 0.f;
+    float bpost, lpost;
+    edge_posteriors(L, c, (size_t)b * T * Up1, Up1, t, u, l.Tb, l.Ub, bpost, lpost);
     const float occ = bpost + lpost;
     const float w = grad_loss ? grad_loss[b] : 1.f;
     const float lse = L.lse[c];

@@ -33,7 +33,7 @@ class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("U", ctypes.c_int), ("D_enc", ctypes.c_int),
                 ("D_pred", ctypes.c_int), ("H", ctypes.c_int), ("V", ctypes.c_int), ("blank", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("path", ctypes.c_int),
-                ("chunk_cells", ctypes.c_int)]
+                ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int)]
 
 
 class StageStat(ctypes.Structure):
@@ -121,11 +121,14 @@ def profile_read() -> dict:
     return out
 
 
+LOSSES = {"marginal": 0, "viterbi": 1}
+
+
 def make_dims(B, T, U, D_enc, D_pred, H, V, dtype="bf16", mode="tiled", path="auto", chunk_cells=0,
-              blank=0) -> Dims:
+              blank=0, loss="marginal") -> Dims:
     return Dims(B, T, U, D_enc, D_pred, H, V, blank, BF16 if dtype == "bf16" else F32,
                 TILED if mode == "tiled" else UNTILED, PATH_SIMT if path == "simt" else PATH_AUTO,
-                chunk_cells)
+                chunk_cells, LOSSES[loss])
 
 
 def workspace_size(dims: Dims) -> int:
@@ -140,11 +143,11 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank) -> Dims:
+def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal") -> Dims:
     B, T, D_enc = f.shape
     U = g.shape[1] - 1
     V, H = W_o.shape
-    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank)
+    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss)
 
 
 class Outputs:
@@ -168,16 +171,17 @@ class Outputs:
 
 
 def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
-            chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+            chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None, loss="marginal"):
     """One call of frnnt_fwd_bwd on CUDA tensors.
 
     Float tensors are all float32 or all bfloat16; labels/T_len/U_len int32.
+    ``loss`` is "marginal" (every alignment) or "viterbi" (the best one).
     Returns (loss [B] fp32, dict of gradients).  With ``check`` the device
     status word is read back (one 4-byte device-to-host copy, which
     synchronises the stream) and a non-zero status raises FrnntStatusError.
     """
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
-    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank)
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss)
     if out is None:
         out = Outputs(f, g, W_f, W_g, W_o, b_o, dims)
     if stream is None:
@@ -197,13 +201,14 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode
 
 
 def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
-                    chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+                    chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None,
+                    loss="marginal"):
     """frnnt_fwd_bwd_noalloc: like fwd_bwd, but the library's fixed scratch
     array replaces the workspace (``out.workspace`` is not used).  Raises
     FrnntError(FRNNT_ERR_WORKSPACE) when these dims need more than
     NOALLOC_MAX_BYTES of scratch."""
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
-    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank)
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss)
     if out is None:
         out = Outputs(f, g, W_f, W_g, W_o, b_o, dims, with_workspace=False)
     if stream is None:
