@@ -1,5 +1,5 @@
 """fp64 CPU oracle (test infrastructure only; see rnnt_oracle's header)."""
-from .rnnt_oracle import (STATUS_LABEL, STATUS_LENGTH, OracleResult, UtteranceLattice,  # noqa: F401
-                          alpha_lattice, beta_lattice, best_alignment, fwd_bwd, joint_logits, lae,
+from .rnnt_oracle import (STATUS_BOUNDS, STATUS_LABEL, STATUS_LENGTH, OracleResult, UtteranceLattice,  # noqa: F401
+                          alpha_lattice, band_mask, beta_lattice, best_alignment, fwd_bwd, joint_logits, lae,
                           log_sum_exp_last, loss_only, projections, validate,
-                          viterbi_lattice)
+                          validate_bounds, viterbi_lattice)

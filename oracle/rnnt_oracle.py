@@ -49,6 +49,16 @@ What it computes (the definitions, written out plainly, in float64):
   broken towards the blank edge (arriving at (t,u) from (t-1,u)).  The loss
   is -log p(best alignment), so its gradient is the marginal formula with
   bpost / lpost the 0/1 indicators of the best alignment's edges.
+* Pruning bounds (``bounds`` [B,T] int, ``S``): "Pruned RNN-T for fast,
+  memory-efficient ASR training" (abstract) evaluates the full non-linear
+  joiner only within pruning bounds; the bounds themselves (from a linear
+  joiner on the pages) are an input here.  Plainest reading: frame t of
+  utterance b keeps the S label positions s[b,t] <= u < s[b,t] + S, every
+  other cell is removed from the lattice (alpha = beta = -inf there, no
+  logits, no gradient), and the loss sums over the alignments that stay
+  inside the band.  Bounds are valid when s[b,0] = 0, s[b,t] <= U_len,
+  s[b,t] <= s[b,t+1] <= s[b,t] + S - 1 and s[b,T_len-1] + S - 1 >= U_len
+  (then a band alignment exists); otherwise STATUS_BOUNDS.
 
 Every float op here is float64; inputs that the product path receives in
 bf16 are handed to the oracle already rounded to bf16 (by the shared seeded
@@ -68,6 +78,7 @@ import numpy as np
 # a length outside its range, or a label outside the vocabulary / equal to blank.
 STATUS_LENGTH = 1
 STATUS_LABEL = 2
+STATUS_BOUNDS = 8
 
 NEG_INF = -math.inf
 
@@ -103,6 +114,31 @@ def validate(T: int, U: int, V: int, blank: int, labels, T_len, U_len) -> int:
     return status
 
 
+def validate_bounds(S: int, bounds, T_len, U_len) -> int:
+    """STATUS_BOUNDS unless every utterance's band is valid (see the header)."""
+    bounds = np.asarray(bounds)
+    for b in range(len(T_len)):
+        Tb, Ub = int(T_len[b]), int(U_len[b])
+        s = [int(bounds[b, t]) for t in range(Tb)]
+        if s[0] != 0 or s[Tb - 1] + S - 1 < Ub:
+            return STATUS_BOUNDS
+        for t in range(Tb):
+            if s[t] < 0 or s[t] > Ub:
+                return STATUS_BOUNDS
+            if t + 1 < Tb and not (s[t] <= s[t + 1] <= s[t] + S - 1):
+                return STATUS_BOUNDS
+    return 0
+
+
+def band_mask(bounds_b, S: int, Tb: int, Ub: int):
+    """True for the cells (t, u) of the (Tb, Ub+1) lattice inside the band."""
+    M = np.zeros((Tb, Ub + 1), dtype=bool)
+    for t in range(Tb):
+        s = int(bounds_b[t])
+        M[t, s:min(Ub + 1, s + S)] = True
+    return M
+
+
 def projections(f_b, g_b, W_f, W_g):
     """F = f W_f and G = g W_g for one utterance (float64 matmuls)."""
     return f_b @ W_f, g_b @ W_g
@@ -124,11 +160,14 @@ def log_sum_exp_last(z):
     return m + np.log(np.exp(z - m[..., None]).sum(axis=-1))
 
 
-def alpha_lattice(blank_lp, label_lp, Tb: int, Ub: int):
-    """Forward variables alpha(t,u) over the (Tb, Ub+1) lattice."""
+def alpha_lattice(blank_lp, label_lp, Tb: int, Ub: int, mask=None):
+    """Forward variables alpha(t,u) over the (Tb, Ub+1) lattice (cells outside
+    ``mask``, when given, are removed: -inf)."""
     A = np.full((Tb, Ub + 1), NEG_INF)
     for t in range(Tb):
         for u in range(Ub + 1):
+            if mask is not None and not mask[t, u]:
+                continue
             if t == 0 and u == 0:
                 A[t, u] = 0.0
                 continue
@@ -138,11 +177,13 @@ def alpha_lattice(blank_lp, label_lp, Tb: int, Ub: int):
     return A
 
 
-def beta_lattice(blank_lp, label_lp, Tb: int, Ub: int):
-    """Backward variables beta(t,u); beta(0,0) = log P."""
+def beta_lattice(blank_lp, label_lp, Tb: int, Ub: int, mask=None):
+    """Backward variables beta(t,u); beta(0,0) = log P (cells outside ``mask``: -inf)."""
     Bt = np.full((Tb, Ub + 1), NEG_INF)
     for t in range(Tb - 1, -1, -1):
         for u in range(Ub, -1, -1):
+            if mask is not None and not mask[t, u]:
+                continue
             if t == Tb - 1 and u == Ub:
                 Bt[t, u] = blank_lp[t, u]
                 continue
@@ -152,7 +193,7 @@ def beta_lattice(blank_lp, label_lp, Tb: int, Ub: int):
     return Bt
 
 
-def viterbi_lattice(blank_lp, label_lp, Tb: int, Ub: int):
+def viterbi_lattice(blank_lp, label_lp, Tb: int, Ub: int, mask=None):
     """Max-product forward variables and the best predecessor of every cell.
 
     Returns (A, from_blank) with from_blank[t,u] True when the best way into
@@ -161,6 +202,8 @@ def viterbi_lattice(blank_lp, label_lp, Tb: int, Ub: int):
     from_blank = np.zeros((Tb, Ub + 1), dtype=bool)
     for t in range(Tb):
         for u in range(Ub + 1):
+            if mask is not None and not mask[t, u]:
+                continue
             if t == 0 and u == 0:
                 A[t, u] = 0.0
                 continue
@@ -225,7 +268,7 @@ def _frame_block(Ub: int, V: int, H: int, budget_bytes: int = 1 << 28) -> int:
 
 def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
             blank: int = 0, utterances=None, keep_lattice: bool = False,
-            loss: str = "marginal") -> OracleResult:
+            loss: str = "marginal", bounds=None, S: int = 0) -> OracleResult:
     """Loss and gradients of sum_b w_b * loss_b, all in float64.
 
     f [B,T,D_enc], g [B,U+1,D_pred], W_f [D_enc,H], W_g [D_pred,H], W_o [V,H],
@@ -234,6 +277,7 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
     and contribute nothing to the weight gradients; their df/dg rows are 0).
     Gradient rows for frames t >= T_len[b] and positions u > U_len[b] are 0.
     ``loss`` is "marginal" (all alignments) or "viterbi" (the best one).
+    ``bounds`` [B,T] with band width ``S`` restricts the lattice (header).
     """
     if loss not in ("marginal", "viterbi"):
         raise ValueError(f"unknown loss {loss!r}")
@@ -250,6 +294,8 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
     U = g.shape[1] - 1
     V, H = W_o.shape
     status = validate(T, U, V, blank, labels, T_len, U_len)
+    if not status and bounds is not None:
+        status = validate_bounds(S, bounds, T_len, U_len)
     if status:
         return OracleResult(status=status)
     w = np.ones(B) if grad_loss is None else np.asarray(grad_loss, dtype=np.float64)
@@ -263,8 +309,9 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
         Tb, Ub = int(T_len[b]), int(U_len[b])
         y = [int(labels[b, u]) for u in range(Ub)]
         F, G = projections(f[b, :Tb], g[b, :Ub + 1], W_f, W_g)
+        mask = None if bounds is None else band_mask(bounds[b], S, Tb, Ub)
 
-        # forward: per-cell log-probabilities
+        # forward: per-cell log-probabilities (the band's cells only are used)
         lse = np.empty((Tb, Ub + 1))
         blank_lp = np.empty((Tb, Ub + 1))
         label_lp = np.full((Tb, Ub + 1), NEG_INF)
@@ -280,15 +327,15 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
 
         if loss == "viterbi":
             # best alignment: its log-probability and its edges
-            A, from_blank = viterbi_lattice(blank_lp, label_lp, Tb, Ub)
+            A, from_blank = viterbi_lattice(blank_lp, label_lp, Tb, Ub, mask)
             log_p = A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub]
             res.loss[b] = -log_p
             bpost, lpost = best_alignment(from_blank, Tb, Ub)
             Bt = np.full((Tb, Ub + 1), np.nan)              # no backward variables in this variant
         else:
             # transducer loss
-            A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
-            Bt = beta_lattice(blank_lp, label_lp, Tb, Ub)
+            A = alpha_lattice(blank_lp, label_lp, Tb, Ub, mask)
+            Bt = beta_lattice(blank_lp, label_lp, Tb, Ub, mask)
             log_p = A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub]
             assert abs(Bt[0, 0] - log_p) <= 1e-9 * max(1.0, abs(log_p)), (Bt[0, 0], log_p)
             res.loss[b] = -log_p
@@ -334,7 +381,8 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
     return res
 
 
-def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, loss: str = "marginal"):
+def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, loss: str = "marginal",
+              bounds=None, S: int = 0):
     """Per-utterance losses (forward only), used by finite-difference checks."""
     f = np.asarray(f, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
@@ -353,9 +401,10 @@ def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, lo
         label_lp = np.full((Tb, Ub + 1), NEG_INF)
         for u in range(Ub):
             label_lp[:, u] = z[:, u, int(labels[b, u])] - lse[:, u]
+        mask = None if bounds is None else band_mask(bounds[b], S, Tb, Ub)
         if loss == "viterbi":
-            A, _ = viterbi_lattice(blank_lp, label_lp, Tb, Ub)
+            A, _ = viterbi_lattice(blank_lp, label_lp, Tb, Ub, mask)
         else:
-            A = alpha_lattice(blank_lp, label_lp, Tb, Ub)
+            A = alpha_lattice(blank_lp, label_lp, Tb, Ub, mask)
         out[b] = -(A[Tb - 1, Ub] + blank_lp[Tb - 1, Ub])
     return out

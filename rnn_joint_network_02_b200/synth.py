@@ -153,3 +153,18 @@ def redraw_padding(batch: Batch, seed: int) -> Batch:
     return Batch(f=f, g=g, W_f=batch.W_f, W_g=batch.W_g, W_o=batch.W_o, b_o=batch.b_o,
                  labels=lab, T_len=batch.T_len, U_len=batch.U_len, dtype=batch.dtype,
                  blank=batch.blank)
+
+
+def diagonal_bounds(T_len, U_len, T: int, S: int) -> torch.Tensor:
+    """Pruning-bound inputs: a band of S label positions per frame that follows
+    the lattice's diagonal, s[b,t] = min(U_len, max(0, floor(t (U_len+1) / T_len) - S // 2)),
+    int32 [B, T]; padding frames repeat the last frame's start.  (The pages
+    obtain bounds from a linear joiner; here they are synthetic inputs.)"""
+    B = len(T_len)
+    s = torch.zeros(B, T, dtype=torch.int32)
+    for b in range(B):
+        Tb, Ub = int(T_len[b]), int(U_len[b])
+        for t in range(T):
+            tt = min(t, Tb - 1)
+            s[b, t] = min(Ub, max(0, (tt * (Ub + 1)) // Tb - S // 2))
+    return s
