@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--chunk-cells", type=int, default=0)
     p.add_argument("--loss", default="marginal", choices=["marginal", "viterbi"],
                    help="training criterion: every alignment (default) or the best one")
+    p.add_argument("--prune", type=int, default=0,
+                   help="pruned lattice: S label positions per frame on a band along the diagonal (0: whole lattice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -77,7 +79,7 @@ def config_of(batch, args, n_gpus):
     d = batch.dims
     return {"workload": args.workload, "B": d["B"], "T": d["T"], "U": d["U"], "D_enc": d["D_enc"],
             "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": args.mode, "path": args.path,
-            "loss": args.loss,
+            "loss": args.loss, "prune_S": args.prune,
             "valid_cells": batch.valid_cells(), "padded_cells": batch.padded_cells(),
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{n_gpus}",
             "global_batch": d["B"] * n_gpus}
@@ -85,12 +87,13 @@ def config_of(batch, args, n_gpus):
 
 # ------------------------------------------------------------------ algorithmic work per stage
 
-def stage_work(batch, stage, mode):
+def stage_work(batch, stage, mode, cells=None):
     """(kind, amount per call): tensor flops or HBM bytes that the stage must
-    do by definition (recomputation excluded)."""
+    do by definition (recomputation excluded); ``cells`` = the valid cells of
+    the lattice computed (default: the whole lattice's)."""
     d = batch.dims
     H, V = d["H"], d["V"]
-    cells = batch.valid_cells()
+    cells = batch.valid_cells() if cells is None else cells
     if stage in ("joint_fwd", "bwd_dWo", "bwd_dh"):
         return "tensor", 2.0 * H * V * cells
     if stage == "joint_bwd_dz":
@@ -233,14 +236,27 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     end-to-end variant with host buffers, per-stage device times."""
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
     dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank,
-                         args.loss)
+                         args.loss, args.prune)
+    bounds = None
+    valid = batch.valid_cells()
+    if args.prune:
+        hb = synth.diagonal_bounds(batch.T_len, batch.U_len, batch.f.shape[1], args.prune)
+        valid = sum(min(args.prune, int(batch.U_len[b]) - int(hb[b, t]) + 1)
+                    for b in range(batch.dims["B"]) for t in range(int(batch.T_len[b])))
+        bounds = hb.to(dev)
     out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims)
     stream = torch.cuda.current_stream(dev)
 
     def call(check=False):
-        res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
-                            d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells, loss=args.loss,
-                            blank=batch.blank, out=out, check=check, stream=stream)
+        if bounds is not None:
+            res = frnnt.fwd_bwd_pruned(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"],
+                                       d["T_len"], d["U_len"], bounds, args.prune, mode=mode, path=args.path,
+                                       chunk_cells=args.chunk_cells, loss=args.loss, blank=batch.blank, out=out,
+                                       check=check, stream=stream)
+        else:
+            res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                                d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells, loss=args.loss,
+                                blank=batch.blank, out=out, check=check, stream=stream)
         if world > 1:
             # the data-parallel exchange: weight gradients summed over ranks
             rdist.allreduce_weight_grads(res[1])
@@ -317,13 +333,14 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e = float(t.item())
 
-    units = batch.padded_cells() * batch.dims["V"]
+    # cells of the lattice that is computed: B*T*(U+1), or B*T*S when pruned
+    units = (batch.dims["B"] * batch.dims["T"] * args.prune if args.prune else batch.padded_cells()) * batch.dims["V"]
     launches = sum(v["launches"] for v in stages.values())
     roofline = None
     pk = peaks()
     if stages:
         dom = max(stages, key=lambda k: stages[k]["ms"])
-        kind, work = stage_work(batch, dom, mode)
+        kind, work = stage_work(batch, dom, mode, valid)
         per_call_ms = stages[dom]["ms"] / args.steps
         tr = MEASURED_TRAFFIC.get((args.workload, mode, dom))
         if kind == "tensor":
@@ -339,7 +356,7 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
                         "frac": achieved / pk["hbm"], "traffic": tr[0] if tr else None,
                         "traffic_source": tr[1] if tr else None, "stage": dom, "peak_source": pk["source"]}
     return {"ms": ms, "value": world * units / (ms / 1e3), "peak_bytes": peak_bytes,
-            "valid_cells_per_s": world * batch.valid_cells() * batch.dims["V"] / (ms / 1e3),
+            "valid_cells_per_s": world * valid * batch.dims["V"] / (ms / 1e3),
             "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
             "launches": launches, "roofline": roofline, "clocks": clocks,

@@ -84,6 +84,15 @@ typedef struct {
   int chunk_cells;        /* FRNNT_TILED: lattice cells per backward chunk;
                              0 = default (65536).  Rounded up to whole tiles. */
   frnnt_loss loss;        /* training criterion (MARGINAL unless set)         */
+  int prune_S;            /* 0: the whole lattice.  S > 0 (S <= 32): pruned
+                             lattice, frame t of utterance b keeps only the S
+                             label positions bounds[b,t] <= u < bounds[b,t]+S
+                             ("Pruned RNN-T for fast, memory-efficient ASR
+                             training", abstract: the non-linear joiner is
+                             evaluated only within pruning bounds, which are
+                             an input here).  Call frnnt_fwd_bwd_pruned.
+                             Needs FRNNT_BF16 on the tensor-core kernels
+                             (FRNNT_ERR_UNSUPPORTED otherwise).               */
 } frnnt_dims;
 
 /* Host return codes. */
@@ -101,7 +110,10 @@ enum {
 enum {
   FRNNT_STATUS_LENGTH = 1,     /* T_len[b] outside [1,T] or U_len[b] outside [0,U] */
   FRNNT_STATUS_LABEL = 2,      /* labels[b,u] (u < U_len[b]) outside [0,V) or == blank */
-  FRNNT_STATUS_TIMEOUT = 4     /* a bounded device-side wait gave up           */
+  FRNNT_STATUS_TIMEOUT = 4,    /* a bounded device-side wait gave up           */
+  FRNNT_STATUS_BOUNDS = 8      /* pruned: bounds[b,0] != 0, a start outside [0,U_len[b]],
+                                  bounds[b,t+1] outside [bounds[b,t], bounds[b,t]+S-1],
+                                  or bounds[b,T_len[b]-1]+S-1 < U_len[b] (t < T_len[b]) */
 };
 
 /* Bytes of device workspace frnnt_fwd_bwd needs for these dims.  Host-only:
@@ -130,6 +142,24 @@ FRNNT_API int frnnt_fwd_bwd(const frnnt_dims* d,
                   const void* f, const void* g, const void* W_f, const void* W_g,
                   const void* W_o, const void* b_o,
                   const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                  const float* grad_loss, float* loss,
+                  void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream);
+
+/* frnnt_fwd_bwd on the pruned lattice of d->prune_S > 0 (frnnt_fwd_bwd itself
+ * returns FRNNT_ERR_DIMS for such dims, and this call for d->prune_S == 0).
+ *   bounds      [B, T] int32 device array: first label position of frame t's
+ *               band; rows past T_len[b] are padding and not read.
+ * The loss sums over the alignments that stay inside the band (maximum over
+ * them with FRNNT_LOSS_VITERBI); cells outside it have no logits and no
+ * gradient.  Invalid bounds set FRNNT_STATUS_BOUNDS.  Everything else as
+ * frnnt_fwd_bwd (same workspace size query: frnnt_workspace_size(d)). */
+FRNNT_API int frnnt_fwd_bwd_pruned(const frnnt_dims* d,
+                  const void* f, const void* g, const void* W_f, const void* W_g,
+                  const void* W_o, const void* b_o,
+                  const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                  const int32_t* bounds,
                   const float* grad_loss, float* loss,
                   void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
                   void* workspace, size_t workspace_bytes,

@@ -33,6 +33,7 @@ bool dims_ok(const frnnt_dims* d) {
   if (d->blank < 0 || d->blank >= d->V) return false;
   if (d->U + 1 > 1024) return false;
   if (d->chunk_cells < 0) return false;
+  if (d->prune_S < 0 || d->prune_S > 32) return false;
   return true;
 }
 
@@ -54,6 +55,8 @@ Shape shape_of(const frnnt_dims* d) {
   s.Np = s.BT * s.Up1;
   s.bf16 = d->dtype == FRNNT_BF16;
   s.viterbi = d->loss == FRNNT_LOSS_VITERBI;
+  s.S = d->prune_S;
+  s.Nlat = s.S > 0 ? s.BT * s.S : s.Np;
   return s;
 }
 
@@ -108,7 +111,7 @@ int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, 
   const bool untiled = d->mode == FRNNT_UNTILED;
   {
     StageScope sc("validate", st);
-    launch_validate(s, labels, T_len, U_len, status, st);
+    launch_validate(s, labels, T_len, U_len, nullptr, status, st);
     cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accWo, 0, (size_t)s.V * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accbo, 0, (size_t)s.V * sizeof(float), st);
@@ -132,7 +135,7 @@ int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, 
 
   {  // transducer forward-backward
     StageScope sc("lattice_dp", st);
-    launch_dp(s, p.L, T_len, U_len, loss, st);
+    launch_dp(s, p.L, T_len, U_len, nullptr, loss, st);
   }
 
   // backward through the joint
@@ -173,7 +176,7 @@ bool use_tc(const frnnt_dims* d) {
   if (d->dtype != FRNNT_BF16 || d->path != FRNNT_PATH_AUTO) return false;
   if (d->B > 1024) return false;
   if (d->H % 64 || d->D_enc % 32 || d->D_pred % 32) return false;
-  return joint_tc_supported(d->H, d->V, d->U);
+  return joint_tc_supported(d->H, d->V, d->U, d->prune_S);
 }
 
 struct TcPlan {
@@ -193,7 +196,7 @@ struct TcPlan {
 TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   TcPlan p;
   Carver c(ws);
-  tile_shape(s.U, &p.TB, &p.UB);
+  tile_shape_of(s, &p.TB, &p.UB);
   p.maxT = max_tiles(s, p.TB, p.UB);
   const long long cells = d->chunk_cells > 0 ? d->chunk_cells : kDefaultChunkCells;
   p.chunkT = (cells + 127) / 128;
@@ -207,12 +210,12 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.dGb = c.take<__nv_bfloat16>(s.BU * s.H);
   p.tiles = c.take<int4>(p.maxT);
   p.ntiles = c.take<int>(4);
-  p.L.lse = c.take<float>(s.Np);
-  p.L.blank_lp = c.take<float>(s.Np);
-  p.L.label_lp = c.take<float>(s.Np);
-  p.L.alpha = c.take<float>(s.Np);
-  p.L.beta = c.take<float>(s.Np);
-  p.L.path = s.viterbi ? c.take<uint8_t>(s.Np) : nullptr;
+  p.L.lse = c.take<float>(s.Nlat);
+  p.L.blank_lp = c.take<float>(s.Nlat);
+  p.L.label_lp = c.take<float>(s.Nlat);
+  p.L.alpha = c.take<float>(s.Nlat);
+  p.L.beta = c.take<float>(s.Nlat);
+  p.L.path = s.viterbi ? c.take<uint8_t>(s.Nlat) : nullptr;
   p.accWo = c.take<float>((size_t)s.V * hidden_stride(s.H));
   p.db_part = nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
@@ -262,7 +265,7 @@ int splits_for(int M, int N, int K) {
 
 int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, const void* W_f, const void* W_g,
            const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
-           const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+           const int32_t* bounds, const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
            void* ws, int32_t* status, cudaStream_t st) {
   TcPlan p = plan_tc(d, s, ws);
   const bool untiled = d->mode == FRNNT_UNTILED;
@@ -274,7 +277,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   } while (0)
   {
     StageScope sc("validate", st);
-    launch_validate(s, labels, T_len, U_len, status, st);
+    launch_validate(s, labels, T_len, U_len, bounds, status, st);
     launch_tiles(s, p.TB, p.UB, T_len, U_len, p.tiles, p.ntiles, st);
     cudaMemsetAsync(p.dF, 0, s.BT * s.H * sizeof(float), st);
     cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
@@ -294,7 +297,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   JointLaunch j{};
   j.s = s; j.TB = p.TB; j.UB = p.UB; j.F = p.F; j.G = p.G; j.W_o = W_o; j.b_o = b_o; j.labels = labels;
   j.T_len = T_len; j.U_len = U_len; j.grad_loss = grad_loss; j.tiles = p.tiles; j.ntiles = p.ntiles; j.L = p.L;
-  j.zbuf = p.zbuf; j.hbuf = p.hbuf; j.db_part = p.db_part; j.status = status;
+  j.zbuf = p.zbuf; j.hbuf = p.hbuf; j.db_part = p.db_part; j.status = status; j.bounds = bounds;
   {
     StageScope sc("joint_fwd", st);
     j.mode = untiled ? 1 : 0;
@@ -318,7 +321,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   }
   {
     StageScope sc("lattice_dp", st);
-    launch_dp(s, p.L, T_len, U_len, loss, st);
+    launch_dp(s, p.L, T_len, U_len, bounds, loss, st);
   }
   for (long long c0 = 0; c0 < p.maxT; c0 += p.chunkT) {
     const long long c1 = (c0 + p.chunkT < p.maxT) ? c0 + p.chunkT : p.maxT;
@@ -406,25 +409,30 @@ extern "C" int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes) {
   if (!d || !bytes) return FRNNT_ERR_NULL;
   if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
   if (!dims_ok(d)) return FRNNT_ERR_DIMS;
+  if (d->prune_S > 0 && !use_tc(d)) return FRNNT_ERR_UNSUPPORTED;
   Shape s = shape_of(d);
   *bytes = use_tc(d) ? plan_tc(d, s, nullptr).bytes : plan_simt(d, s, nullptr).bytes;
   return FRNNT_OK;
 }
 
-extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g,
-                             const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len,
-                             const int32_t* U_len, const float* grad_loss, float* loss, void* df, void* dg,
-                             void* dW_f, void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes,
-                             int32_t* status, void* stream) {
+namespace {
+
+int fwd_bwd_impl(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g, const void* W_o,
+                 const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                 const int32_t* bounds, const float* grad_loss, float* loss, void* df, void* dg, void* dW_f,
+                 void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes, int32_t* status,
+                 void* stream) {
   if (!d) return FRNNT_ERR_NULL;
   if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
   if (!dims_ok(d)) return FRNNT_ERR_DIMS;
+  if (d->prune_S > 0 && !use_tc(d)) return FRNNT_ERR_UNSUPPORTED;
   const void* req[] = {f, g, W_f, W_g, W_o, b_o, T_len, U_len, loss, df, dg, dW_f, dW_g, dW_o, db_o, workspace, status};
   for (const void* p : req)
     if (!p) return FRNNT_ERR_NULL;
   if (!labels && d->U > 0) return FRNNT_ERR_NULL;
-  const void* al[] = {f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
-                      db_o, workspace, status};
+  if (d->prune_S > 0 && !bounds) return FRNNT_ERR_NULL;
+  const void* al[] = {f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
+                      dW_o, db_o, workspace, status};
   for (const void* p : al)
     if (p && !aligned16(p)) return FRNNT_ERR_ALIGN;
   size_t need = 0;
@@ -435,10 +443,33 @@ extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, 
   cudaGetLastError();   // clear a stale error so it is not reported as ours
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return FRNNT_ERR_CUDA;
   if (use_tc(d))
-    return run_tc(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o, db_o,
-                  workspace, status, st);
+    return run_tc(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
+                  dW_o, db_o, workspace, status, st);
   return run_simt(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
                   db_o, workspace, status, st);
+}
+
+}  // namespace
+
+extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g,
+                             const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len,
+                             const int32_t* U_len, const float* grad_loss, float* loss, void* df, void* dg,
+                             void* dW_f, void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes,
+                             int32_t* status, void* stream) {
+  if (d && d->prune_S != 0) return FRNNT_ERR_DIMS;   // pruned dims go through frnnt_fwd_bwd_pruned
+  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, nullptr, grad_loss, loss, df, dg, dW_f, dW_g,
+                      dW_o, db_o, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int frnnt_fwd_bwd_pruned(const frnnt_dims* d, const void* f, const void* g, const void* W_f,
+                                    const void* W_g, const void* W_o, const void* b_o, const int32_t* labels,
+                                    const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
+                                    const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g,
+                                    void* dW_o, void* db_o, void* workspace, size_t workspace_bytes, int32_t* status,
+                                    void* stream) {
+  if (d && d->prune_S <= 0) return FRNNT_ERR_DIMS;
+  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
+                      dW_o, db_o, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" const char* frnnt_error_string(int code) {

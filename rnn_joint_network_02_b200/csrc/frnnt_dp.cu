@@ -40,10 +40,43 @@ __global__ void validate_kernel(int B, int T, int U, int V, int blank, const int
   if ((threadIdx.x & 31) == 0 && bits) atomicOr(status, bits);
 }
 
+// Pruned lattice: the bands of every utterance with valid lengths must start
+// at 0, stay within [0, U_len], advance by 0 .. S-1 per frame and reach U_len
+// in the last frame (then an alignment inside the band exists).
+__global__ void validate_bounds_kernel(int B, int T, int U, int S, const int32_t* __restrict__ bounds,
+                                       const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
+                                       int32_t* __restrict__ status) {
+  int bad = 0;
+  const long long n = (long long)B * T;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int b = (int)(i / T), t = (int)(i % T);
+    const int tl = T_len[b], ul = U_len[b];
+    if (tl < 1 || tl > T || ul < 0 || ul > U) continue;   // length already flagged
+    if (t >= tl) continue;                                // padding frame
+    const int s = bounds[i];
+    if (s < 0 || s > ul) bad = 1;
+    if (t == 0 && s != 0) bad = 1;
+    if (t + 1 < tl) {
+      const int sn = bounds[i + 1];
+      if (sn < s || sn > s + S - 1) bad = 1;
+    } else if (s + S - 1 < ul) {
+      bad = 1;
+    }
+  }
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if ((threadIdx.x & 31) == 0 && bad) atomicOr(status, FRNNT_STATUS_BOUNDS);
+}
+
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
-                     int32_t* status, cudaStream_t st) {
+                     const int32_t* bounds, int32_t* status, cudaStream_t st) {
   validate_kernel<<<1, 256, 0, st>>>(s.B, s.T, s.U, s.V, s.blank, labels, T_len, U_len, status);
   note_launch();
+  if (s.S > 0) {
+    const long long n = (long long)s.B * s.T;
+    const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+    validate_bounds_kernel<<<blocks, 256, 0, st>>>(s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
+    note_launch();
+  }
 }
 
 // Operands of step `step` for thread u: alpha needs blank_lp(t-1,u) and
@@ -250,10 +283,295 @@ __global__ void dp_viterbi_kernel(int T, int U, const float* __restrict__ blank_
   }
 }
 
-void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
-               cudaStream_t st) {
+// Pruned lattice (layout [b][t][j], label position u = s[b,t] + j, j < S).
+// One thread per (utterance, direction) walks the band row by row; the
+// previous row (alpha) or next row (beta) is kept in shared memory.  A cell
+// (t, u) is in the lattice when t < T_len, j < S and u <= U_len; its blank
+// predecessor (t-1, u) sits at j' = u - s[b,t-1] of the previous row when
+// 0 <= j' < S.  With `viterbi`, alpha takes the max (ties to the blank edge),
+// the decision goes to bit 2 of the path byte, and the alpha thread then walks
+// the best alignment back, marking the edge that leaves each cell on it.
+__global__ void dp_band_kernel(int T, int U, int S, const int32_t* __restrict__ bounds,
+                               const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
+                               float* __restrict__ alpha, float* __restrict__ beta, uint8_t* __restrict__ path,
+                               const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
+                               float* __restrict__ loss) {
+  __shared__ float row[2][32];      // [direction][j] of the neighbouring row
+  const int b = blockIdx.x;
+  const int dir = threadIdx.x;      // 0 alpha, 1 beta
+  const bool viterbi = path != nullptr;
+  if (dir > 1 || (viterbi && dir == 1)) return;
+  const Lengths l = lengths_of(T_len, U_len, b, T, U);
+  const int Tb = l.Tb, Ub = l.Ub;
+  const size_t base = (size_t)b * T * S;
+  const int32_t* sb = bounds + (size_t)b * T;
+  float* prev = row[dir];
+  if (dir == 0) {
+    int sp = 0;
+    for (int t = 0; t < Tb; ++t) {
+      const int s = clampi(sb[t], 0, U);
+      float left = -INFINITY;       // alpha(t, u-1) within this row
+      float cur_row[32];
+#pragma unroll 1
+      for (int j = 0; j < S; ++j) {
+        const int u = s + j;
+        const size_t c = base + (size_t)t * S + j;
+        float v = -INFINITY;
+        bool from_blank = false;
+        if (u <= Ub) {
+          if (t == 0 && u == 0) {
+            v = 0.f;
+          } else {
+            float fb = -INFINITY;
+            const int jp = u - sp;
+            if (t > 0 && jp >= 0 && jp < S) fb = prev[jp] + __ldg(blank_lp + base + (size_t)(t - 1) * S + jp);
+            const float fl = j > 0 ? left + __ldg(label_lp + c - 1) : -INFINITY;
+            if (viterbi) {
+              from_blank = fb >= fl;
+              v = from_blank ? fb : fl;
+            } else {
+              v = log_add_exp(fb, fl);
+            }
+          }
+        }
+        alpha[c] = v;
+        if (viterbi) path[c] = from_blank ? 4 : 0;
+        cur_row[j] = v;
+        left = v;
+      }
+#pragma unroll 1
+      for (int j = 0; j < S; ++j) prev[j] = cur_row[j];
+      sp = s;
+    }
+    const int jl = Ub - clampi(sb[Tb - 1], 0, U);
+    if (viterbi && jl >= 0 && jl < S) {   // (invalid bounds are flagged; nothing to walk then)
+      size_t c = base + (size_t)(Tb - 1) * S + jl;
+      loss[b] = -(alpha[c] + __ldg(blank_lp + c));
+      path[c] |= 1;                 // the final blank
+      int t = Tb - 1, u = Ub;
+      while (t > 0 || u > 0) {      // t + u falls by one per step
+        const int s = clampi(sb[t], 0, U);
+        if ((path[c] & 4) && t > 0) {
+          const int jp = u - clampi(sb[t - 1], 0, U);
+          if (jp < 0 || jp >= S) break;   // not reached with valid bounds
+          --t;
+          c = base + (size_t)t * S + jp;
+          path[c] |= 1;
+        } else if (u > s) {
+          --u;
+          c -= 1;
+          path[c] |= 2;
+        } else {
+          break;                    // not reached with valid bounds
+        }
+      }
+    }
+  } else {
+    int sn = 0;
+    for (int t = Tb - 1; t >= 0; --t) {
+      const int s = clampi(sb[t], 0, U);
+      float right = -INFINITY;      // beta(t, u+1) within this row
+      float cur_row[32];
+#pragma unroll 1
+      for (int j = S - 1; j >= 0; --j) {
+        const int u = s + j;
+        const size_t c = base + (size_t)t * S + j;
+        float v = -INFINITY;
+        if (u <= Ub) {
+          if (t == Tb - 1 && u == Ub) {
+            v = __ldg(blank_lp + c);
+          } else {
+            float bb = -INFINITY;
+            const int jn = u - sn;
+            if (t + 1 < Tb && jn >= 0 && jn < S) bb = prev[jn] + __ldg(blank_lp + c);
+            const float bl = (j + 1 < S && u + 1 <= Ub) ? right + __ldg(label_lp + c) : -INFINITY;
+            v = log_add_exp(bb, bl);
+          }
+        }
+        beta[c] = v;
+        cur_row[j] = v;
+        right = v;
+      }
+#pragma unroll 1
+      for (int j = 0; j < S; ++j) prev[j] = cur_row[j];
+      sn = s;
+    }
+    loss[b] = -beta[base];
+  }
+}
+
+// The same pruned recursion with one warp per (utterance, direction) and lane
+// j = band position (S <= 32): a frame's blank-edge terms come from the
+// neighbouring frame by one shuffle (the band moves by bounds[t] - bounds[t-1],
+// the same for every lane); the label-edge recurrence along the frame,
+// x_j = lae(a_j, x_{j-1} + l_{j-1}), is an inclusive scan over lanes with the
+// associative composition of the maps x -> lae(a, x + l):
+//   (a1, l1) then (a2, l2)  =  (lae(a2, a1 + l2), l1 + l2)
+// (max for the maximum approximation).  Beta runs the mirrored scan from the
+// right.  The next frame's operands are fetched one frame ahead.  With
+// `viterbi` the decision bits of each frame (a ballot) go to shared memory and
+// lane 0 walks the best alignment back.
+__device__ __forceinline__ float comb(bool viterbi, float a, float b) { return viterbi ? fmaxf(a, b) : log_add_exp(a, b); }
+
+__global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, const int32_t* __restrict__ bounds,
+                                                          const float* __restrict__ blank_lp,
+                                                          const float* __restrict__ label_lp, float* __restrict__ alpha,
+                                                          float* __restrict__ beta, uint8_t* __restrict__ path,
+                                                          const int32_t* __restrict__ T_len,
+                                                          const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  extern __shared__ uint32_t dec[];   // viterbi: one ballot of decisions per frame
+  const int b = blockIdx.x;
+  const bool is_beta = blockIdx.y == 1;
+  const bool viterbi = path != nullptr;
+  const int lane = threadIdx.x;
+  const Lengths l = lengths_of(T_len, U_len, b, T, U);
+  const int Tb = l.Tb, Ub = l.Ub;
+  const size_t base = (size_t)b * T * S;
+  const int32_t* sb = bounds + (size_t)b * T;
+  auto start = [&](int t) { return clampi(sb[t], 0, U); };
+  if (!is_beta) {
+    // operands of frame t: blank_lp(t-1, u) at the previous frame's position and label_lp(t, u-1)
+    auto fetch = [&](int t, float& ob, float& ol) {
+      ob = -INFINITY;
+      ol = -INFINITY;
+      if (t >= Tb) return;
+      const int s = start(t), u = s + lane;
+      if (lane >= S || u > Ub) return;
+      if (t > 0) {
+        const int jp = u - start(t - 1);
+        if (jp >= 0 && jp < S) ob = __ldg(blank_lp + base + (size_t)(t - 1) * S + jp);
+      }
+      if (lane > 0) ol = __ldg(label_lp + base + (size_t)t * S + lane - 1);
+    };
+    float ob, ol, nob, nol;
+    fetch(0, ob, ol);
+    float prev = -INFINITY;
+    int sp = 0;
+    for (int t = 0; t < Tb; ++t) {
+      fetch(t + 1, nob, nol);
+      const int s = start(t), u = s + lane;
+      const bool valid = lane < S && u <= Ub;
+      const int delta = s - sp;
+      const int src = lane + delta < 32 ? lane + delta : 31;
+      const float pv = __shfl_sync(0xffffffffu, prev, src);
+      const float fb = (t > 0 && valid && lane + delta < S) ? pv + ob : -INFINITY;
+      float a = (t == 0 && u == 0) ? 0.f : fb;
+      float c = ol;
+      float x = a;
+      // inclusive scan over lanes (the band's S lanes need log2 S steps)
+      for (int off = 1; off < S; off <<= 1) {
+        const float xa = __shfl_up_sync(0xffffffffu, x, off);
+        const float xc = __shfl_up_sync(0xffffffffu, c, off);
+        if (lane >= off) {
+          x = comb(viterbi, x, xa + c);
+          c = xc + c;
+        }
+      }
+      if (!valid) x = -INFINITY;
+      if (lane < S) {
+        alpha[base + (size_t)t * S + lane] = x;
+        if (viterbi) path[base + (size_t)t * S + lane] = 0;
+      }
+      if (viterbi) {
+        const float left = __shfl_up_sync(0xffffffffu, x, 1);
+        const bool from_blank = valid && (lane == 0 || fb >= left + ol);
+        const uint32_t bits = __ballot_sync(0xffffffffu, from_blank);
+        if (lane == 0) dec[t] = bits;
+      }
+      prev = x;
+      sp = s;
+      ob = nob;
+      ol = nol;
+    }
+    if (viterbi) {
+      __syncwarp();
+      if (lane == 0) {
+        int t = Tb - 1;
+        int j = Ub - start(t);
+        if (j >= 0 && j < S) {
+          size_t c = base + (size_t)t * S + j;
+          loss[b] = -(alpha[c] + __ldg(blank_lp + c));
+          path[c] = 1;              // the final blank
+          while (t > 0 || start(t) + j > 0) {
+            if (((dec[t] >> j) & 1u) && t > 0) {
+              const int u = start(t) + j;
+              const int jp = u - start(t - 1);
+              if (jp < 0 || jp >= S) break;   // not reached with valid bounds
+              --t;
+              j = jp;
+              c = base + (size_t)t * S + j;
+              path[c] = 1;
+            } else if (j > 0) {
+              --j;
+              c -= 1;
+              path[c] = 2;
+            } else {
+              break;                // not reached with valid bounds
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // operands of frame t: blank_lp(t, u) and label_lp(t, u)
+    auto fetch = [&](int t, float& ob, float& ol) {
+      ob = -INFINITY;
+      ol = -INFINITY;
+      if (t < 0) return;
+      const int u = start(t) + lane;
+      if (lane >= S || u > Ub) return;
+      ob = __ldg(blank_lp + base + (size_t)t * S + lane);
+      if (lane + 1 < S && u < Ub) ol = __ldg(label_lp + base + (size_t)t * S + lane);
+    };
+    float ob, ol, nob, nol;
+    fetch(Tb - 1, ob, ol);
+    float next = -INFINITY;
+    int sn = 0;
+    for (int t = Tb - 1; t >= 0; --t) {
+      fetch(t - 1, nob, nol);
+      const int s = start(t), u = s + lane;
+      const bool valid = lane < S && u <= Ub;
+      const int d2 = (t + 1 < Tb) ? sn - s : 0;
+      const int src = lane - d2 >= 0 ? lane - d2 : 0;
+      const float nv = __shfl_sync(0xffffffffu, next, src);
+      float bb = (t + 1 < Tb && valid && lane - d2 >= 0) ? nv + ob : -INFINITY;
+      if (t == Tb - 1 && u == Ub) bb = ob;   // the final blank
+      float y = valid ? bb : -INFINITY;
+      float c = ol;
+      // inclusive scan from the right
+      for (int off = 1; off < S; off <<= 1) {
+        const float ya = __shfl_down_sync(0xffffffffu, y, off);
+        const float yc = __shfl_down_sync(0xffffffffu, c, off);
+        if (lane + off < 32) {
+          y = comb(false, y, c + ya);
+          c = c + yc;
+        }
+      }
+      if (!valid) y = -INFINITY;
+      if (lane < S) beta[base + (size_t)t * S + lane] = y;
+      next = y;
+      sn = s;
+      ob = nob;
+      ol = nol;
+    }
+    if (lane == 0) loss[b] = -beta[base];
+  }
+}
+
+void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
+               float* loss, cudaStream_t st) {
   int threads = ((s.Up1 + 31) / 32) * 32;
-  if (L.path) {
+  if (s.S > 0) {
+    const int smem = L.path ? s.T * 4 : 0;
+    if (smem <= 48 * 1024) {
+      dim3 grid(s.B, L.path ? 1 : 2);
+      dp_band_warp_kernel<<<grid, 32, smem, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
+                                                  L.path, T_len, U_len, loss);
+    } else {
+      dp_band_kernel<<<s.B, 32, 0, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta, L.path,
+                                         T_len, U_len, loss);
+    }
+  } else if (L.path) {
     // decision bits in shared memory when they fit in 96 KB
     const long long words = ((long long)s.T * s.Up1 + 31) / 32;
     const int smem = words * 4 <= 96 * 1024 ? (int)(words * 4) : 0;

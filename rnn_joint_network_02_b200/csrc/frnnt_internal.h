@@ -38,6 +38,8 @@ struct Shape {
   long long Np;       // B * T * (U + 1) padded lattice cells
   bool bf16;
   bool viterbi;       // maximum-approximation loss
+  int S;              // pruned lattice: label positions kept per frame (0 = the whole lattice)
+  long long Nlat;     // entries of one lattice array: B*T*(U+1), or B*T*S when pruned
 };
 
 // Lattice arrays, fp32, padded layout [b][t][u] with u fastest.
@@ -55,12 +57,14 @@ struct Lattice {
 
 #ifdef __CUDACC__
 // Posterior of the two edges leaving valid cell (t, u) at lattice index c
-// (padded layout, utterance base c0 = index of (0, 0)):
+// (c0 = index of the utterance's cell (0, 0); c_t1 / c_u1 = index of (t+1, u)
+// / (t, u+1), or -1 where that cell is not in the lattice; `last` marks
+// (T_len-1, U_len), whose blank edge ends the alignment):
 //   marginal: bpost = exp(alpha + blank_lp + beta'(t+1,u) - logP) with
-//             beta'(T_len, U_len) = 0; lpost = exp(alpha + label_lp + beta(t,u+1) - logP);
+//             beta' = 0 after the last cell; lpost = exp(alpha + label_lp + beta(t,u+1) - logP);
 //   maximum approximation: the best alignment's 0/1 edge indicators.
-__device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size_t c0, int Up1, int t, int u, int Tb,
-                                                int Ub, float& bpost, float& lpost) {
+__device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size_t c0, long long c_t1,
+                                                long long c_u1, bool last, float& bpost, float& lpost) {
   if (L.path) {
     const uint8_t e = L.path[c];
     bpost = (e & 1) ? 1.f : 0.f;
@@ -69,19 +73,18 @@ __device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size
   }
   const float logp = L.beta[c0];
   const float al = L.alpha[c];
-  float beta_t1;
-  if (t + 1 < Tb) beta_t1 = L.beta[c + Up1];
-  else beta_t1 = (u == Ub) ? 0.f : -INFINITY;
+  const float beta_t1 = c_t1 >= 0 ? L.beta[c_t1] : (last ? 0.f : -INFINITY);
   bpost = __expf(al + L.blank_lp[c] + beta_t1 - logp);
-  lpost = u < Ub ? __expf(al + L.label_lp[c] + L.beta[c + 1] - logp) : 0.f;
+  lpost = c_u1 >= 0 ? __expf(al + L.label_lp[c] + L.beta[c_u1] - logp) : 0.f;
 }
 #endif
 
 // ---------------------------------------------------------------- validation / DP
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
-                     int32_t* status, cudaStream_t st);
-void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
-               cudaStream_t st);
+                     const int32_t* bounds, int32_t* status, cudaStream_t st);
+// bounds: the pruned lattice's per-frame starts (s.S > 0), else null
+void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
+               float* loss, cudaStream_t st);
 
 // ---------------------------------------------------------------- CUDA-core kernels
 // C[M,N] (fp32, row stride ldc) = op(A)[M,K] * op(B)[K,N]  (+ C when accumulate)
@@ -157,12 +160,16 @@ struct JointLaunch {
   void* hbuf;                   // h rows, same indexing, bf16 [.][hidden_stride(H)]; column H is 1 (cell count column)
   float* db_part;               // unused
   int32_t* status;
+  const int32_t* bounds;        // pruned lattice (s.S > 0): [B][T] first label position of each frame's band
 };
-bool joint_tc_supported(int H, int V, int U);
+bool joint_tc_supported(int H, int V, int U, int S);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the
 // dW_o GEMM's N is a whole number of its N tiles.
 inline int hidden_stride(int H) { return H >= 512 ? ((H + 1 + 255) / 256) * 256 : ((H + 1 + 127) / 128) * 128; }
 void tile_shape(int U, int* TB, int* UB);
+// Cell tile of the shape: TB frames x UB label positions, or for a pruned
+// lattice TB frames x (S rounded up to a power of two) band positions.
+void tile_shape_of(const Shape& s, int* TB, int* UB);
 long long max_tiles(const Shape& s, int TB, int UB);
 void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
                   cudaStream_t st);

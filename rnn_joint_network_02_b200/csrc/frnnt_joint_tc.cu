@@ -82,26 +82,60 @@ struct JointParams {
   int srows;              // rows per epilogue store-staging pass (8 or 32)
   float* db_part;         // unused
   int32_t* status;
+  const int32_t* bounds;  // pruned lattice: [B][T] band starts; S = band width (0: whole lattice)
+  int S;
 };
 
 struct RowInfo {
   bool valid;
-  int b, t, u, Tb, Ub, y;
-  size_t cell;            // padded lattice index
+  int b, t, u, j, Tb, Ub, y;
+  size_t cell;            // lattice index: [b][t][u] (padded), or [b][t][j] on a pruned lattice
 };
 
+// Cell of tile row r: frame t0 + r / UB and label position u0 + r % UB, or on
+// a pruned lattice band position j = r % UB of frame t, u = bounds[b,t] + j.
 __device__ __forceinline__ RowInfo row_info(const JointParams& p, int4 tile, int r) {
   RowInfo ri;
   ri.b = tile.x;
   ri.t = tile.y + r / p.UB;
-  ri.u = tile.z + r % p.UB;
   const Lengths l = lengths_of(p.T_len, p.U_len, ri.b, p.T, p.U);
   ri.Tb = l.Tb;
   ri.Ub = l.Ub;
-  ri.valid = ri.t < l.Tb && ri.u <= l.Ub;
+  if (p.S) {
+    ri.j = r % p.UB;
+    const int tc = min(ri.t, l.Tb - 1);
+    ri.u = clampi(p.bounds[(size_t)ri.b * p.T + tc], 0, p.U) + ri.j;
+    ri.valid = ri.t < l.Tb && ri.j < p.S && ri.u <= l.Ub;
+    ri.cell = ((size_t)ri.b * p.T + (ri.valid ? ri.t : 0)) * p.S + (ri.valid ? ri.j : 0);
+  } else {
+    ri.u = tile.z + r % p.UB;
+    ri.j = ri.u;
+    ri.valid = ri.t < l.Tb && ri.u <= l.Ub;
+    ri.cell = ((size_t)ri.b * p.T + (ri.valid ? ri.t : 0)) * (p.U + 1) + (ri.valid ? ri.u : 0);
+  }
   ri.y = (ri.valid && ri.u < l.Ub) ? label_of(p.labels, ri.b, ri.u, p.U, p.V) : -1;
-  ri.cell = ((size_t)ri.b * p.T + (ri.valid ? ri.t : 0)) * (p.U + 1) + (ri.valid ? ri.u : 0);
   return ri;
+}
+
+// Lattice indices around a valid cell: the utterance's (0, 0), (t+1, u) and
+// (t, u+1) (-1 when not in the lattice), and whether it is (T_len-1, U_len).
+__device__ __forceinline__ void lattice_neighbors(const JointParams& p, const RowInfo& ri, size_t& c0, long long& c_t1,
+                                                  long long& c_u1, bool& last) {
+  last = ri.t == ri.Tb - 1 && ri.u == ri.Ub;
+  if (p.S) {
+    c0 = (size_t)ri.b * p.T * p.S;
+    c_t1 = -1;
+    if (ri.t + 1 < ri.Tb) {
+      const int jn = ri.u - clampi(p.bounds[(size_t)ri.b * p.T + ri.t + 1], 0, p.U);
+      if (jn >= 0 && jn < p.S) c_t1 = (long long)(c0 + (size_t)(ri.t + 1) * p.S + jn);
+    }
+    c_u1 = (ri.j + 1 < p.S && ri.u < ri.Ub) ? (long long)ri.cell + 1 : -1;
+  } else {
+    const int Up1 = p.U + 1;
+    c0 = (size_t)ri.b * p.T * Up1;
+    c_t1 = ri.t + 1 < ri.Tb ? (long long)(ri.cell + Up1) : -1;
+    c_u1 = ri.u < ri.Ub ? (long long)ri.cell + 1 : -1;
+  }
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -362,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     auto issue_fg = [&](int tile, uint32_t empty_parity) {
       const bool dummy = tile >= ntiles;
       const int4 td = dummy ? make_int4(0, p.T, 0, 0) : p.tiles[tile];
-      const int nF = dummy ? 0 : min(p.TB, p.T - td.y), nG = dummy ? 0 : min(p.UB, Up1 - td.z);
+      // (a pruned lattice's G rows differ per frame: the generators read them from global memory)
+      const int nF = dummy ? 0 : min(p.TB, p.T - td.y), nG = (dummy || p.S) ? 0 : min(p.UB, Up1 - td.z);
       if (!mbar_wait(fg_empty, empty_parity, abort_flag)) return false;
       if (lane == 0) mbar_arrive_expect_tx(fg_full, (uint32_t)(nF + nG) * H * 2);
       __syncwarp();
@@ -381,7 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       const int4 td = tile < ntiles ? p.tiles[tile] : make_int4(0, p.T, 0, 0);
       const RowInfo ri = row_info(p, td, r);
       const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
-      const uint8_t* grow = fgs + (p.TB + r % p.UB) * fg_stride;
+      const uint8_t* grow = p.S ? (const uint8_t*)(p.G + ((size_t)ri.b * Up1 + min(ri.u, p.U)) * H)
+                                : fgs + (p.TB + r % p.UB) * fg_stride;
       if (!mbar_wait(fg_full, fph, abort_flag)) break;
       for (int g = 0; g < ngrp; ++g) {
         const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
@@ -454,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     const int q = warp & 3;                   // TMEM lane quadrant
     const int half = warp >> 2;               // columns [64 half, 64 half + 64) of each V tile
     const int r = q * 32 + lane;
-    const int V = p.V, Up1 = p.U + 1;
+    const int V = p.V;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     int acc_i = 0;
     for (int it = slot; it < niter; it += nslots) {
@@ -469,7 +505,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
         const size_t c = ri.cell;
         lk = p.L.lse[c] * kLog2e;
         const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
-        edge_posteriors(p.L, c, (size_t)ri.b * p.T * Up1, Up1, ri.t, ri.u, ri.Tb, ri.Ub, bpost, lpost);
+        size_t c0;
+        long long c_t1, c_u1;
+        bool last;
+        lattice_neighbors(p, ri, c0, c_t1, c_u1, last);
+        edge_posteriors(p.L, c, c0, c_t1, c_u1, last, bpost, lpost);
         bpost *= w;
         lpost *= w;
         occ = bpost + lpost;
@@ -592,13 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ tile list
 // Tiles of utterance b: ceil(T_len/TB) x ceil((U_len+1)/UB) blocks, u-blocks fastest.
-__global__ void tiles_kernel(int B, int T, int U, int TB, int UB, const int32_t* __restrict__ T_len,
+// (pruned: one tile per TB frames, its UB rows per frame being band positions)
+__global__ void tiles_kernel(int B, int T, int U, int TB, int UB, int pruned, const int32_t* __restrict__ T_len,
                              const int32_t* __restrict__ U_len, int4* __restrict__ tiles, int* __restrict__ ntiles) {
   __shared__ int offs[1025];
   __shared__ int counts[1024];
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const Lengths l = lengths_of(T_len, U_len, b, T, U);
-    counts[b] = ((l.Tb + TB - 1) / TB) * ((l.Ub + 1 + UB - 1) / UB);
+    counts[b] = ((l.Tb + TB - 1) / TB) * (pruned ? 1 : (l.Ub + 1 + UB - 1) / UB);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -613,7 +654,7 @@ __global__ void tiles_kernel(int B, int T, int U, int TB, int UB, const int32_t*
   __syncthreads();
   for (int b = 0; b < B; ++b) {
     const Lengths l = lengths_of(T_len, U_len, b, T, U);
-    const int nu = (l.Ub + 1 + UB - 1) / UB;
+    const int nu = pruned ? 1 : (l.Ub + 1 + UB - 1) / UB;
     for (int i = threadIdx.x; i < counts[b]; i += blockDim.x) {
       const int it = i / nu, iu = i % nu;
       tiles[offs[b] + i] = make_int4(b, it * TB, iu * UB, 0);
@@ -627,7 +668,7 @@ __global__ void dz_from_z_kernel(JointParams p) {
   // in batches of four 16-byte chunks per lane, all loads of a batch issued
   // before any store (the row is rewritten in place).
   const int ntiles = min(p.tile_end, *p.ntiles);
-  const int V = p.V, Up1 = p.U + 1;
+  const int V = p.V;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
   for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows;
@@ -643,7 +684,11 @@ __global__ void dz_from_z_kernel(JointParams p) {
     const float lse = p.L.lse[c];
     const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
     float bpost, lpost;
-    edge_posteriors(p.L, c, (size_t)ri.b * p.T * Up1, Up1, ri.t, ri.u, ri.Tb, ri.Ub, bpost, lpost);
+    size_t c0;
+    long long c_t1, c_u1;
+    bool last;
+    lattice_neighbors(p, ri, c0, c_t1, c_u1, last);
+    edge_posteriors(p.L, c, c0, c_t1, c_u1, last, bpost, lpost);
     bpost *= w;
     lpost *= w;
     const float occ = bpost + lpost;
@@ -786,6 +831,52 @@ __global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict
   }
 }
 
+// Pruned lattice: tile row r is band position j = r % UB of frame t = t0 + r / UB,
+// label position u = bounds[b,t] + j.  dF[b,t] += sum over the frame's valid
+// positions; dG[b,u] += every valid row (u differs per frame, so per row).
+__global__ void seg_reduce_band_kernel(JointParams p, const __nv_bfloat16* __restrict__ dpre, int row_tile0,
+                                       float* dF, float* dG) {
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int tile = p.tile_begin + blockIdx.x;
+  if (tile >= ntiles) return;
+  const int4 td = p.tiles[tile];
+  const int H = p.H, UB = p.UB, TB = p.TB, Up1 = p.U + 1, HS = p.HS;
+  const Lengths l = lengths_of(p.T_len, p.U_len, td.x, p.T, p.U);
+  const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * HS;
+  const int nt = min(TB, l.Tb - td.y);
+  const int g = threadIdx.y;
+  for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
+    const __nv_bfloat16* col = base + c8 * 8;
+    for (int tl = g; tl < nt; tl += 4) {
+      const int t = td.y + tl;
+      const int st = clampi(p.bounds[(size_t)td.x * p.T + t], 0, p.U);
+      const int nj = min(p.S, l.Ub - st + 1);      // band positions of this frame inside the utterance
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < nj; ++j) {
+        const uint4 v = *(const uint4*)(col + (size_t)(tl * UB + j) * HS);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        float row[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
+          row[2 * q] = f.x;
+          row[2 * q + 1] = f.y;
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+        float* dg = dG + ((size_t)td.x * Up1 + st + j) * H + c8 * 8;
+        red_add_v4(dg, row[0], row[1], row[2], row[3]);
+        red_add_v4(dg + 4, row[4], row[5], row[6], row[7]);
+      }
+      if (nj > 0) {
+        float* dst = dF + ((size_t)td.x * p.T + t) * H + c8 * 8;
+        red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
+        red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
+      }
+    }
+  }
+}
+
 // dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
 // whose column H is the sum of dz over cells.
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, __nv_bfloat16* __restrict__ dW_o,
@@ -892,10 +983,13 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
 }  // namespace
 
 // ------------------------------------------------------------------ host entry points
-bool joint_tc_supported(int H, int V, int U) {
+bool joint_tc_supported(int H, int V, int U, int S) {
   if (H % 64 || H > 1024 || V % 128) return false;
+  Shape s{};
+  s.U = U;
+  s.S = S;
   int TB, UB;
-  tile_shape(U, &TB, &UB);
+  tile_shape_of(s, &TB, &UB);
   return stages_for(H / 64, V, TB, UB) >= 2;
 }
 
@@ -910,13 +1004,24 @@ void tile_shape(int U, int* TB, int* UB) {
   *TB = 128 / ub;
 }
 
+void tile_shape_of(const Shape& s, int* TB, int* UB) {
+  if (s.S > 0) {
+    int sp = 4;                     // at most 32 frames per tile (their F rows are staged)
+    while (sp < s.S) sp *= 2;
+    *UB = sp;
+    *TB = 128 / sp;
+  } else {
+    tile_shape(s.U, TB, UB);
+  }
+}
+
 long long max_tiles(const Shape& s, int TB, int UB) {
-  return (long long)s.B * ((s.T + TB - 1) / TB) * ((s.Up1 + UB - 1) / UB);
+  return (long long)s.B * ((s.T + TB - 1) / TB) * (s.S > 0 ? 1 : (s.Up1 + UB - 1) / UB);
 }
 
 void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
                   cudaStream_t st) {
-  tiles_kernel<<<1, 1024, 0, st>>>(s.B, s.T, s.U, TB, UB, T_len, U_len, tiles, ntiles);
+  tiles_kernel<<<1, 1024, 0, st>>>(s.B, s.T, s.U, TB, UB, s.S > 0 ? 1 : 0, T_len, U_len, tiles, ntiles);
   note_launch();
 }
 
@@ -941,6 +1046,8 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
@@ -991,6 +1098,8 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   dz_from_z_kernel<<<sms() * 4, 256, 0, st>>>(p);
@@ -1015,6 +1124,8 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
   hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
   note_launch();
@@ -1033,12 +1144,17 @@ void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, fl
   p.ntiles = j.ntiles;
   p.tile_begin = j.tile_begin;
   p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
   p.HS = hidden_stride(j.s.H);
   const int n = j.tile_end - j.tile_begin;
   if (n <= 0) return;
   int threads = (p.H / 8 + 31) / 32 * 32;
   if (threads > 128) threads = 128;
-  seg_reduce_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
+  if (p.S)
+    seg_reduce_band_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
+  else
+    seg_reduce_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
   note_launch();
 }
 

@@ -219,7 +219,8 @@ __global__ void dz_simt_kernel(int T, int U, int V, int blank, float* __restrict
       continue;
     }
     float bpost, lpost;
-    edge_posteriors(L, c, (size_t)b * T * Up1, Up1, t, u, l.Tb, l.Ub, bpost, lpost);
+    edge_posteriors(L, c, (size_t)b * T * Up1, t + 1 < l.Tb ? (long long)(c + Up1) : -1LL,
+                    u < l.Ub ? (long long)(c + 1) : -1LL, t == l.Tb - 1 && u == l.Ub, bpost, lpost);
     const float occ = bpost + lpost;
     const float w = grad_loss ? grad_loss[b] : 1.f;
     const float lse = L.lse[c];

@@ -21,10 +21,10 @@ F32, BF16 = 0, 1
 PATH_AUTO, PATH_SIMT = 0, 1
 
 OK = 0
-STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT = 1, 2, 4
+STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT, STATUS_BOUNDS = 1, 2, 4, 8
 
 EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
-            "frnnt_profile_read", "frnnt_fwd_bwd_noalloc")
+            "frnnt_profile_read", "frnnt_fwd_bwd_noalloc", "frnnt_fwd_bwd_pruned")
 NOALLOC_MAX_BYTES = 64 * 1024 * 1024
 TEST_HOOKS = ("frnnt_test_gemm_bf16", "frnnt_test_joint_variant")
 
@@ -33,7 +33,7 @@ class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("U", ctypes.c_int), ("D_enc", ctypes.c_int),
                 ("D_pred", ctypes.c_int), ("H", ctypes.c_int), ("V", ctypes.c_int), ("blank", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("path", ctypes.c_int),
-                ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int)]
+                ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int), ("prune_S", ctypes.c_int)]
 
 
 class StageStat(ctypes.Structure):
@@ -49,7 +49,8 @@ class FrnntError(RuntimeError):
 
 class FrnntStatusError(RuntimeError):
     def __init__(self, bits: int):
-        names = [n for n, v in (("length", STATUS_LENGTH), ("label", STATUS_LABEL), ("timeout", STATUS_TIMEOUT))
+        names = [n for n, v in (("length", STATUS_LENGTH), ("label", STATUS_LABEL), ("timeout", STATUS_TIMEOUT),
+                                ("bounds", STATUS_BOUNDS))
                  if bits & v]
         super().__init__(f"frnnt device status {bits}: invalid {', '.join(names)}")
         self.bits = bits
@@ -71,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.frnnt_fwd_bwd.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] + [vp] * 6 +
                                     [vp, ctypes.c_size_t, i32p, vp])
         L.frnnt_fwd_bwd.restype = ctypes.c_int
+        L.frnnt_fwd_bwd_pruned.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 4 + [f32p, f32p] + [vp] * 6 +
+                                           [vp, ctypes.c_size_t, i32p, vp])
+        L.frnnt_fwd_bwd_pruned.restype = ctypes.c_int
         L.frnnt_fwd_bwd_noalloc.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] +
                                             [vp] * 6 + [i32p, vp])
         L.frnnt_fwd_bwd_noalloc.restype = ctypes.c_int
@@ -125,10 +129,10 @@ LOSSES = {"marginal": 0, "viterbi": 1}
 
 
 def make_dims(B, T, U, D_enc, D_pred, H, V, dtype="bf16", mode="tiled", path="auto", chunk_cells=0,
-              blank=0, loss="marginal") -> Dims:
+              blank=0, loss="marginal", prune_S=0) -> Dims:
     return Dims(B, T, U, D_enc, D_pred, H, V, blank, BF16 if dtype == "bf16" else F32,
                 TILED if mode == "tiled" else UNTILED, PATH_SIMT if path == "simt" else PATH_AUTO,
-                chunk_cells, LOSSES[loss])
+                chunk_cells, LOSSES[loss], prune_S)
 
 
 def workspace_size(dims: Dims) -> int:
@@ -143,11 +147,11 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal") -> Dims:
+def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", prune_S=0) -> Dims:
     B, T, D_enc = f.shape
     U = g.shape[1] - 1
     V, H = W_o.shape
-    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss)
+    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss, prune_S)
 
 
 class Outputs:
@@ -250,3 +254,29 @@ def set_joint_variant(variant: int) -> int:
     """Test hook: fused joint kernel variant for later calls (-1 automatic,
     0 one CTA per cell tile, 1 CTA pairs); returns the previous setting."""
     return int(lib().frnnt_test_joint_variant(int(variant)))
+
+
+def fwd_bwd_pruned(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, S: int, grad_loss=None, mode="tiled",
+                   path="auto", chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None,
+                   loss="marginal"):
+    """frnnt_fwd_bwd_pruned: the loss and gradients on the pruned lattice that
+    keeps, for frame t of utterance b, the S label positions
+    bounds[b,t] <= u < bounds[b,t] + S (bounds: int32 [B, T] on the device)."""
+    dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss, S)
+    if out is None:
+        out = Outputs(f, g, W_f, W_g, W_o, b_o, dims)
+    if stream is None:
+        stream = torch.cuda.current_stream(f.device)
+    rc = lib().frnnt_fwd_bwd_pruned(ctypes.byref(dims), _ptr(f), _ptr(g), _ptr(W_f), _ptr(W_g), _ptr(W_o),
+                                    _ptr(b_o), _ptr(labels), _ptr(T_len), _ptr(U_len), _ptr(bounds),
+                                    _ptr(grad_loss), _ptr(out.loss), _ptr(out.df), _ptr(out.dg), _ptr(out.dW_f),
+                                    _ptr(out.dW_g), _ptr(out.dW_o), _ptr(out.db_o), _ptr(out.workspace),
+                                    out.workspace.numel(), _ptr(out.status), ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    if check:
+        bits = int(out.status[0].item())
+        if bits:
+            raise FrnntStatusError(bits)
+    return out.loss, out.grads()

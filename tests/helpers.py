@@ -20,12 +20,13 @@ def to_device(batch, device="cuda"):
     return d
 
 
-def run_oracle(batch, grad_loss=None, utterances=None, keep_lattice=False, loss="marginal"):
+def run_oracle(batch, grad_loss=None, utterances=None, keep_lattice=False, loss="marginal", bounds=None, S=0):
     f, g, W_f, W_g, W_o, b_o = (t.numpy() for t in batch.float64())
     w = None if grad_loss is None else np.asarray(grad_loss, dtype=np.float64)
     return oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(),
                           batch.U_len.numpy(), grad_loss=w, blank=batch.blank, utterances=utterances,
-                          keep_lattice=keep_lattice, loss=loss)
+                          keep_lattice=keep_lattice, loss=loss,
+                          bounds=None if bounds is None else np.asarray(bounds), S=S)
 
 
 def rel_l2(a, b) -> float:

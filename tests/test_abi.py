@@ -88,3 +88,30 @@ def test_small_workspace_rejected_before_any_launch():
     args = ([ctypes.byref(d)] + fake[:6] + fake[6:9] + [None, fake[9]] + fake[10:16] +
             [fake[16], 16, fake[17], None])
     assert lib.frnnt_fwd_bwd(*args) == 3
+
+
+def test_pruned_dims_rules():
+    """prune_S: 0..32; pruned needs the bf16 tensor-core kernels; the plain
+    entry refuses pruned dims and the pruned entry refuses unpruned ones."""
+    lib = frnnt.lib()
+    n = ctypes.c_size_t(0)
+    d = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16", prune_S=33)
+    assert lib.frnnt_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 2
+    d = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="f32", prune_S=4)
+    assert lib.frnnt_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 4
+    d = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16", prune_S=4)
+    assert lib.frnnt_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0
+    full = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16", mode="untiled")
+    pruned = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16", mode="untiled", prune_S=4)
+    assert frnnt.workspace_size(pruned) < frnnt.workspace_size(full)
+    fake = [ctypes.c_void_p(4096 * (i + 1)) for i in range(20)]
+    args = ([ctypes.byref(d)] + fake[:6] + fake[6:9] + [None, fake[9]] + fake[10:16] +
+            [fake[16], 1 << 40, fake[17], None])
+    assert lib.frnnt_fwd_bwd(*args) == 2            # pruned dims on the plain entry
+    u = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16")
+    pargs = ([ctypes.byref(u)] + fake[:6] + fake[6:9] + [fake[19]] + [None, fake[9]] + fake[10:16] +
+             [fake[16], 1 << 40, fake[17], None])
+    assert lib.frnnt_fwd_bwd_pruned(*pargs) == 2    # unpruned dims on the pruned entry
+    pargs[0] = ctypes.byref(d)
+    pargs[10] = None                                # missing bounds
+    assert lib.frnnt_fwd_bwd_pruned(*pargs) == 1
