@@ -419,7 +419,11 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
                                                           float* __restrict__ beta, uint8_t* __restrict__ path,
                                                           const int32_t* __restrict__ T_len,
                                                           const int32_t* __restrict__ U_len, float* __restrict__ loss) {
-  extern __shared__ uint32_t dec[];   // viterbi: one ballot of decisions per frame
+  // shared memory: the utterance's band starts (T ints), then (viterbi) one
+  // ballot of decisions per frame (T words)
+  extern __shared__ int32_t dsm[];
+  int32_t* starts = dsm;
+  uint32_t* dec = (uint32_t*)(dsm + T);
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
   const bool viterbi = path != nullptr;
@@ -427,8 +431,9 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
   const Lengths l = lengths_of(T_len, U_len, b, T, U);
   const int Tb = l.Tb, Ub = l.Ub;
   const size_t base = (size_t)b * T * S;
-  const int32_t* sb = bounds + (size_t)b * T;
-  auto start = [&](int t) { return clampi(sb[t], 0, U); };
+  for (int t = lane; t < Tb; t += 32) starts[t] = clampi(bounds[(size_t)b * T + t], 0, U);
+  __syncwarp();
+  auto start = [&](int t) { return starts[t]; };
   if (!is_beta) {
     // operands of frame t: blank_lp(t-1, u) at the previous frame's position and label_lp(t, u-1)
     auto fetch = [&](int t, float& ob, float& ol) {
@@ -443,12 +448,14 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       }
       if (lane > 0) ol = __ldg(label_lp + base + (size_t)t * S + lane - 1);
     };
-    float ob, ol, nob, nol;
+    // operands fetched two frames ahead
+    float ob, ol, ob1, ol1, ob2, ol2;
     fetch(0, ob, ol);
+    fetch(1, ob1, ol1);
     float prev = -INFINITY;
     int sp = 0;
     for (int t = 0; t < Tb; ++t) {
-      fetch(t + 1, nob, nol);
+      fetch(t + 2, ob2, ol2);
       const int s = start(t), u = s + lane;
       const bool valid = lane < S && u <= Ub;
       const int delta = s - sp;
@@ -480,8 +487,10 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       }
       prev = x;
       sp = s;
-      ob = nob;
-      ol = nol;
+      ob = ob1;
+      ol = ol1;
+      ob1 = ob2;
+      ol1 = ol2;
     }
     if (viterbi) {
       __syncwarp();
@@ -523,12 +532,13 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       ob = __ldg(blank_lp + base + (size_t)t * S + lane);
       if (lane + 1 < S && u < Ub) ol = __ldg(label_lp + base + (size_t)t * S + lane);
     };
-    float ob, ol, nob, nol;
+    float ob, ol, ob1, ol1, ob2, ol2;
     fetch(Tb - 1, ob, ol);
+    fetch(Tb - 2, ob1, ol1);
     float next = -INFINITY;
     int sn = 0;
     for (int t = Tb - 1; t >= 0; --t) {
-      fetch(t - 1, nob, nol);
+      fetch(t - 2, ob2, ol2);
       const int s = start(t), u = s + lane;
       const bool valid = lane < S && u <= Ub;
       const int d2 = (t + 1 < Tb) ? sn - s : 0;
@@ -551,8 +561,10 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       if (lane < S) beta[base + (size_t)t * S + lane] = y;
       next = y;
       sn = s;
-      ob = nob;
-      ol = nol;
+      ob = ob1;
+      ol = ol1;
+      ob1 = ob2;
+      ol1 = ol2;
     }
     if (lane == 0) loss[b] = -beta[base];
   }
@@ -562,7 +574,7 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
                float* loss, cudaStream_t st) {
   int threads = ((s.Up1 + 31) / 32) * 32;
   if (s.S > 0) {
-    const int smem = L.path ? s.T * 4 : 0;
+    const int smem = s.T * 4 * (L.path ? 2 : 1);
     if (smem <= 48 * 1024) {
       dim3 grid(s.B, L.path ? 1 : 2);
       dp_band_warp_kernel<<<grid, 32, smem, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
