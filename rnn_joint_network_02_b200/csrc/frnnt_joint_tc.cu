@@ -476,7 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) arrive_leader(&hfull[g]);
+        // TMEM groups are complete once tcgen05.wait::st returns (a relaxed
+        // signal suffices); shared-memory groups are published with release
+        if (lane == 0) {
+          if (PAIR && kb0 < kTmemKB) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&hfull[g]), 0));
+          else arrive_leader(&hfull[g]);
+        }
       }
       if (!ok) break;
       // this warp is done reading the tile's F/G rows
@@ -593,7 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(&tempty[a]);
+        // the accumulator is free (only TMEM was read: a relaxed signal suffices)
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[a]), 0));
+          else mbar_arrive(&tempty[a]);
+        }
       }
       if (!ok || *abort_flag) break;
       if (MODE != MODE_BWD_DZ) {
