@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[a]), 0));   // only TMEM was read
       ++acc_i;
       if (p.epi == GEMM_EPI_DTANH) {
         int nm0, nnt, nkb0, nkb1;
