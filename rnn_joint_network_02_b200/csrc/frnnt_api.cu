@@ -361,7 +361,11 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       GemmTcArgs a{};
       // d_hidden = dz W_o, then (1 - h^2) in the epilogue, in place over h
       a.M = rows; a.N = s.H; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = W_o;
-      a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
+      a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH_FG; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
+      // (1 - h^2) with h recomputed from the L2-resident F and G rows of each cell, not read back
+      a.cells.tiles = p.tiles; a.cells.tile0 = (int)c0; a.cells.T = s.T; a.cells.U = s.U; a.cells.H = s.H;
+      a.cells.UB = p.UB; a.cells.S = s.S; a.cells.bounds = bounds; a.cells.T_len = T_len; a.cells.U_len = U_len;
+      a.cells.F = p.F; a.cells.G = p.G;
       a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
       FRNNT_TRY(gemm_tc(a, st));
     }

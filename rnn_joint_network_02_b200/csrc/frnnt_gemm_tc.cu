@@ -43,6 +43,7 @@ struct GemmParams {
   int32_t* status;
   const int* dyn_count;
   int dyn_base, dyn_scale, dyn_dim;
+  CellMap cells;
 };
 
 // Effective problem after the optional device-side limit on M or K.
@@ -149,6 +150,71 @@ __device__ __forceinline__ void dtanh_store(const GemmParams& p, int row, int co
       o[q] = pack_bf16x2(d0, d1);
     }
     hp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Recompute-h dtanh epilogue: the F and G rows behind GEMM row `row` (null
+// when the row is no lattice cell: its accumulator is zero, so is its result).
+struct FgRows {
+  const __nv_bfloat16* f;
+  const __nv_bfloat16* g;
+};
+__device__ __forceinline__ FgRows fg_rows(const CellMap& m, int row) {
+  const int4 td = m.tiles[m.tile0 + (row >> 7)];
+  const int r = row & 127;
+  const int b = td.x, t = td.y + r / m.UB;
+  const int Tb = clampi(m.T_len[b], 1, m.T), Ub = clampi(m.U_len[b], 0, m.U);
+  int u;
+  bool valid;
+  if (m.S) {
+    const int j = r % m.UB;
+    u = clampi(m.bounds[(size_t)b * m.T + min(t, Tb - 1)], 0, m.U) + j;
+    valid = t < Tb && j < m.S && u <= Ub;
+  } else {
+    u = td.z + r % m.UB;
+    valid = t < Tb && u <= Ub;
+  }
+  FgRows fr{nullptr, nullptr};
+  if (valid) {
+    fr.f = (const __nv_bfloat16*)m.F + ((size_t)b * m.T + t) * m.H;
+    fr.g = (const __nv_bfloat16*)m.G + ((size_t)b * (m.U + 1) + u) * m.H;
+  }
+  return fr;
+}
+__device__ __forceinline__ uint32_t tanh_bf16x2_g(uint32_t x) {
+  uint32_t y;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// h (bf16, as the joint kernel and the h rows compute it) of 32 columns from
+// col0, into hv (same layout as dtanh_load's: 4 x 8 bf16)
+__device__ __forceinline__ void h_from_fg(const FgRows& fr, int col0, uint4 (&hv)[4]) {
+  if (!fr.f) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) hv[j] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* fp = (const uint4*)(fr.f + col0);
+  const uint4* gp = (const uint4*)(fr.g + col0);
+  uint4 fv[4], gv[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    fv[j] = __ldg(fp + j);
+    gv[j] = __ldg(gp + j);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 a, c;
+    uint32_t o[4];
+    const uint32_t fw[4] = {fv[j].x, fv[j].y, fv[j].z, fv[j].w}, gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      a = *reinterpret_cast<const __nv_bfloat162*>(&fw[q]);
+      c = *reinterpret_cast<const __nv_bfloat162*>(&gw[q]);
+      __nv_bfloat162 sum = __hadd2(a, c);
+      o[q] = tanh_bf16x2_g(*reinterpret_cast<uint32_t*>(&sum));
+    }
+    hv[j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -299,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = m0 + q * 32 + lane;
       const bool row_ok = row < eff.M;
       if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
+      const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
       if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -308,10 +375,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool st = row_ok && col0 < p.N;
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (!st) continue;
-        if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
+        if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
         else epilogue_store(p, row, col0, r);
       }
       tc_fence_before();
@@ -511,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = m0 + (int)rank * 128 + q * 32 + lane;
       const bool row_ok = row < eff.M;
       if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
+      const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
       if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -520,10 +589,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool st = row_ok && col0 < p.N;
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (!st) continue;
-        if (p.epi == GEMM_EPI_DTANH) dtanh_store(p, row, col0, r, hv);
+        if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
         else epilogue_store(p, row, col0, r);
       }
       tc_fence_before();
@@ -638,7 +708,9 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return FRNNT_OK;
   if ((g.lda % 8) || (g.ldb % 8) || (g.N % 32)) return FRNNT_ERR_DIMS;
   if ((g.epi == GEMM_EPI_STORE_F32 || g.epi == GEMM_EPI_RED_F32) && (g.ldo % 4 || !g.out_f32)) return FRNNT_ERR_DIMS;
-  if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH) && (g.ldo % 8 || !g.out_bf16)) return FRNNT_ERR_DIMS;
+  if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH || g.epi == GEMM_EPI_DTANH_FG) &&
+      (g.ldo % 8 || !g.out_bf16))
+    return FRNNT_ERR_DIMS;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
   const int BN = (g.N % 256 == 0 && g.N >= 256) ? 256 : 128;
   // CTA pairs (M = 256 per MMA) for 256-wide N tiles on problems with enough rows
@@ -675,6 +747,7 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   p.dyn_base = g.dyn_base;
   p.dyn_scale = g.dyn_scale;
   p.dyn_dim = g.dyn_dim;
+  p.cells = g.cells;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
   bool launched;
   if (pair) {

@@ -113,7 +113,22 @@ void launch_dtanh_reduce_simt(const Shape& s, const float* dh, const float* h, l
 // ---------------------------------------------------------------- tensor-core GEMM
 // D[M,N] = A[M,K] * B[K,N] in bf16 with fp32 accumulation (tcgen05, TMA).
 // A: K-major [M][lda] or MN-major [K][lda]; B: K-major [N][ldb] or MN-major [K][ldb].
-enum GemmEpilogue { GEMM_EPI_STORE_F32 = 0, GEMM_EPI_STORE_BF16 = 1, GEMM_EPI_RED_F32 = 2, GEMM_EPI_DTANH = 3 };
+enum GemmEpilogue { GEMM_EPI_STORE_F32 = 0, GEMM_EPI_STORE_BF16 = 1, GEMM_EPI_RED_F32 = 2, GEMM_EPI_DTANH = 3,
+                    GEMM_EPI_DTANH_FG = 4 };
+
+// Lattice cells behind the rows of a GEMM whose 128-row M tiles are cell tiles
+// (row m of the GEMM = row m % 128 of cell tile tile0 + m / 128), for the
+// d_hidden epilogue that recomputes h = tanh(F[t] + G[u]) instead of reading it.
+struct CellMap {
+  const int4* tiles = nullptr;    // (b, t0, u0, -)
+  int tile0 = 0;
+  int T = 0, U = 0, H = 0, UB = 0, S = 0;
+  const int32_t* bounds = nullptr;
+  const int32_t* T_len = nullptr;
+  const int32_t* U_len = nullptr;
+  const void* F = nullptr;        // [B*T][H] bf16
+  const void* G = nullptr;        // [B*(U+1)][H] bf16
+};
 struct GemmTcArgs {
   int M, N, K;
   const void* A;
@@ -133,6 +148,7 @@ struct GemmTcArgs {
   const int* dyn_count = nullptr;
   int dyn_base = 0, dyn_scale = 0, dyn_dim = 0;
   int variant = -1;    // -1 auto, 0 one CTA per tile (M = 128), 1 CTA pairs (M = 256, cta_group::2)
+  CellMap cells;       // GEMM_EPI_DTANH_FG: out = acc * (1 - h^2), h recomputed from F and G
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
 
