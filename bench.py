@@ -60,9 +60,9 @@ def parse():
 # under profiles/ gives the command).  An entry is removed whenever its kernel
 # changes, so the roofline's traffic is null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dh"): (1.010189e9 + 0.352219e9, "profiles/ncu_gemm_tc_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd"): (0.009213e9 + 0.570038e9, "profiles/ncu_joint_tc_medium_untiled.md"),
-    ("medium", "tiled", "joint_fwd"): (0.008490e9, "profiles/ncu_joint_tc_medium_tiled.md"),
+    ("medium", "untiled", "bwd_dh"): (0.629034e9 + 0.354387e9, "profiles/ncu_gemm_tc_medium_untiled.md"),
+    ("medium", "untiled", "bwd_dWo"): (1.175207e9 + 0.010739e9, "profiles/ncu_gemm2_tc_medium_untiled.md"),
+    ("medium", "untiled", "joint_fwd"): (0.009159e9 + 0.570264e9, "profiles/ncu_joint_tc_medium_untiled.md"),
 }
 
 
