@@ -13,7 +13,9 @@
 // u-1 (alpha) or u+1 (beta) is the neighbour's result on the previous
 // diagonal, passed by a warp shuffle, and across a warp boundary by a
 // parity-double-buffered shared-memory slot.  One block per (utterance,
-// direction): alpha and beta run concurrently.
+// direction): alpha and beta run concurrently.  The marginal kernel
+// (dp2_kernel) advances two diagonals per dependent step; the maximum
+// approximation and the pruned band keep one.
 #include "frnnt_common.cuh"
 #include "frnnt_internal.h"
 
@@ -104,10 +106,68 @@ __device__ __forceinline__ void dp_operands(bool is_beta, int step, int ndiag, i
   }
 }
 
-__global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
-                          float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
-                          const int32_t* __restrict__ U_len, float* __restrict__ loss) {
-  __shared__ float xs[2][32];
+// Two diagonals per step.  A cell on diagonal d+2 is reached from diagonal d
+// by three two-edge paths whose weights use only the log-probabilities:
+//   alpha(t,u) = lae(alpha(t-2,u)   + b(t-2,u) + b(t-1,u),
+//                    alpha(t-1,u-1) + lae(b(t-1,u-1) + l(t,u-1), l(t-1,u-1) + b(t-1,u)),
+//                    alpha(t,u-2)   + l(t,u-2) + l(t,u-1))
+// (b = blank_lp, l = label_lp, -inf outside the lattice), and the middle
+// diagonal d+1 takes the usual one-edge step from d as well.  Both depend on
+// diagonal d only, so the dependent chain is one diagonal pair long instead
+// of two diagonals.  Beta mirrors it:
+//   beta(t,u)  = lae(beta(t+2,u)   + b(t,u) + b(t+1,u),
+//                    beta(t+1,u+1) + lae(b(t,u) + l(t+1,u), l(t,u) + b(t,u+1)),
+//                    beta(t,u+2)   + l(t,u) + l(t,u+1)).
+// A thread owns label position u; the values of u-1, u-2 (alpha) or u+1, u+2
+// (beta) on the previous diagonal pair come by shuffles, across a warp
+// boundary through shared memory.  The six log-probabilities of a step are
+// fetched kPrefetch2 steps ahead.
+constexpr int kPrefetch2 = 4;
+
+struct DpOps {
+  float bA, bB, bC, lA, lB, lC;
+};
+
+// alpha, cell (t,u) on diagonal d+2 (t = d + 2 - u):
+//   bA = b(t-2,u), bB = b(t-1,u), bC = b(t-1,u-1), lA = l(t,u-1), lB = l(t-1,u-1), lC = l(t,u-2)
+// beta, cell (t,u) on diagonal d-2:
+//   bA = b(t,u), bB = b(t+1,u), bC = b(t,u+1), lA = l(t+1,u), lB = l(t,u), lC = l(t,u+1)
+__device__ __forceinline__ float lp_at(const float* __restrict__ a, size_t base, int Up1, int t, int u, int Tb,
+                                       int umax) {
+  return (t >= 0 && t < Tb && u >= 0 && u <= umax) ? __ldg(a + base + (size_t)t * Up1 + u) : -INFINITY;
+}
+
+__device__ __forceinline__ DpOps dp2_operands(bool is_beta, int step, int nsteps, int u, int Tb, int Ub, int Up1,
+                                              int last, size_t base, const float* __restrict__ blank_lp,
+                                              const float* __restrict__ label_lp) {
+  DpOps o{-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  if (step >= nsteps || u > Ub) return o;
+  if (!is_beta) {
+    const int t = 2 * step + 2 - u;           // cell on the far diagonal of this step
+    o.bA = lp_at(blank_lp, base, Up1, t - 2, u, Tb, Ub);
+    o.bB = lp_at(blank_lp, base, Up1, t - 1, u, Tb, Ub);
+    o.bC = lp_at(blank_lp, base, Up1, t - 1, u - 1, Tb, Ub);
+    o.lA = lp_at(label_lp, base, Up1, t, u - 1, Tb, Ub - 1);
+    o.lB = lp_at(label_lp, base, Up1, t - 1, u - 1, Tb, Ub - 1);
+    o.lC = lp_at(label_lp, base, Up1, t, u - 2, Tb, Ub - 1);
+  } else {
+    const int t = last - 2 * step - 2 - u;    // cell on the far diagonal of this step
+    o.bA = lp_at(blank_lp, base, Up1, t, u, Tb, Ub);
+    o.bB = lp_at(blank_lp, base, Up1, t + 1, u, Tb, Ub);
+    o.bC = lp_at(blank_lp, base, Up1, t, u + 1, Tb, Ub);
+    o.lA = lp_at(label_lp, base, Up1, t + 1, u, Tb, Ub - 1);
+    o.lB = lp_at(label_lp, base, Up1, t, u, Tb, Ub - 1);
+    o.lC = lp_at(label_lp, base, Up1, t, u + 1, Tb, Ub - 1);
+  }
+  return o;
+}
+
+__device__ __forceinline__ float lae3(float a, float b, float c) { return log_add_exp(log_add_exp(a, b), c); }
+
+__global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
+                           float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
+                           const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  __shared__ float xs[2][32][2];    // [parity][warp][edge lane]: values handed across warp boundaries
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
   const int u = threadIdx.x;
@@ -116,61 +176,103 @@ __global__ void dp_kernel(int T, int U, const float* __restrict__ blank_lp, cons
   const int Tb = l.Tb, Ub = l.Ub;
   const int Up1 = U + 1;
   const size_t base = (size_t)b * T * Up1;
-  const int ndiag = Tb + Ub;        // diagonals d = 0 .. Tb-1+Ub
+  const int last = Tb - 1 + Ub;             // the last diagonal
+  const int nsteps = (last + 1) / 2;        // steps of two diagonals after diagonal 0 (alpha) / `last` (beta)
+  const bool in_u = u <= Ub;
 
-  float qb[kPrefetch], ql[kPrefetch];
-#pragma unroll
-  for (int i = 0; i < kPrefetch; ++i)
-    dp_operands(is_beta, i, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
+  // the first diagonal: (0,0) for alpha, (Tb-1, Ub) for beta
+  float cur = -INFINITY;
+  if (!is_beta) {
+    if (u == 0) {
+      cur = 0.f;
+      alpha[base] = 0.f;
+    }
+  } else if (u == Ub) {
+    const size_t c = base + (size_t)(Tb - 1) * Up1 + Ub;
+    cur = __ldg(blank_lp + c);
+    beta[c] = cur;
+    if (last == 0) loss[b] = -cur;
+  }
 
-  float cur = -INFINITY;            // this thread's value on the previous diagonal
-  for (int step0 = 0; step0 < ndiag; step0 += kPrefetch) {
+  DpOps q[kPrefetch2];
 #pragma unroll
-    for (int i = 0; i < kPrefetch; ++i) {
+  for (int i = 0; i < kPrefetch2; ++i)
+    q[i] = dp2_operands(is_beta, i, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+
+  // parity 1 holds the first diagonal's edge values
+  if (!is_beta) {
+    if (lane >= 30) xs[1][warp][lane - 30] = cur;
+  } else {
+    if (lane < 2) xs[1][warp][lane] = cur;
+  }
+  __syncthreads();
+
+  for (int step0 = 0; step0 < nsteps; step0 += kPrefetch2) {
+#pragma unroll
+    for (int i = 0; i < kPrefetch2; ++i) {
       const int step = step0 + i;
-      if (step >= ndiag) break;     // uniform across the block
-      const float ob = qb[i], ol = ql[i];
-      dp_operands(is_beta, step + kPrefetch, ndiag, u, Tb, Ub, Up1, base, blank_lp, label_lp, qb[i], ql[i]);
-      const int d = is_beta ? (ndiag - 1 - step) : step;
-      const int t = d - u;
-      const bool active = (u <= Ub) && (t >= 0) && (t < Tb);
-      float nb;                     // neighbour's value on the previous diagonal
+      if (step >= nsteps) break;    // uniform across the block
+      const DpOps o = q[i];
+      q[i] = dp2_operands(is_beta, step + kPrefetch2, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+      const int par = (step + 1) & 1;       // parity holding the previous pair's edge values
+      float n1, n2;                          // neighbours at distance 1 and 2 on the previous far diagonal
       if (!is_beta) {
-        nb = __shfl_up_sync(0xffffffffu, cur, 1);
-        if (lane == 0) nb = warp > 0 ? xs[(step + 1) & 1][warp - 1] : -INFINITY;
+        n1 = __shfl_up_sync(0xffffffffu, cur, 1);
+        n2 = __shfl_up_sync(0xffffffffu, cur, 2);
+        if (lane == 0) {
+          n1 = warp > 0 ? xs[par][warp - 1][1] : -INFINITY;
+          n2 = warp > 0 ? xs[par][warp - 1][0] : -INFINITY;
+        } else if (lane == 1) {
+          n2 = warp > 0 ? xs[par][warp - 1][1] : -INFINITY;
+        }
       } else {
-        nb = __shfl_down_sync(0xffffffffu, cur, 1);
-        if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1] : -INFINITY;
-      }
-      float v = -INFINITY;
-      if (active) {
-        const size_t c = base + (size_t)t * Up1 + u;
-        if (!is_beta) {
-          if (t == 0 && u == 0) {
-            v = 0.f;
-          } else {
-            const float fb = t > 0 ? cur + ob : -INFINITY;   // from (t-1, u)
-            const float fl = u > 0 ? nb + ol : -INFINITY;    // from (t, u-1)
-            v = log_add_exp(fb, fl);
-          }
-          alpha[c] = v;
-        } else {
-          if (t == Tb - 1 && u == Ub) {
-            v = ob;
-          } else {
-            const float bb = t + 1 < Tb ? cur + ob : -INFINITY;    // to (t+1, u)
-            const float bl = u < Ub ? nb + ol : -INFINITY;         // to (t, u+1)
-            v = log_add_exp(bb, bl);
-          }
-          beta[c] = v;
-          if (t == 0 && u == 0) loss[b] = -v;
+        n1 = __shfl_down_sync(0xffffffffu, cur, 1);
+        n2 = __shfl_down_sync(0xffffffffu, cur, 2);
+        if (lane == 31) {
+          n1 = warp + 1 < nwarps ? xs[par][warp + 1][0] : -INFINITY;
+          n2 = warp + 1 < nwarps ? xs[par][warp + 1][1] : -INFINITY;
+        } else if (lane == 30) {
+          n2 = warp + 1 < nwarps ? xs[par][warp + 1][0] : -INFINITY;
         }
       }
-      cur = v;
+      float v1 = -INFINITY, v2 = -INFINITY;
+      if (in_u) {
+        if (!is_beta) {
+          const int d1 = 2 * step + 1, d2 = d1 + 1;
+          const int t1 = d1 - u, t2 = d2 - u;
+          if (t1 >= 0 && t1 < Tb) {
+            // one edge from diagonal d1 - 1: (t1-1,u) by blank (operand b(t1-1,u) = bA), (t1,u-1) by label (lB)
+            v1 = log_add_exp(cur + o.bA, n1 + o.lB);
+            alpha[base + (size_t)t1 * Up1 + u] = v1;
+          }
+          if (d2 <= last && t2 >= 0 && t2 < Tb) {
+            v2 = lae3(cur + o.bA + o.bB, n1 + log_add_exp(o.bC + o.lA, o.lB + o.bB), n2 + o.lC + o.lA);
+            alpha[base + (size_t)t2 * Up1 + u] = v2;
+          }
+        } else {
+          const int d1 = last - 2 * step - 1, d2 = d1 - 1;
+          const int t1 = d1 - u, t2 = d2 - u;
+          if (t1 >= 0 && t1 < Tb) {
+            // cell (t1,u) = (t2+1,u): one edge to (t1+1,u) by blank (bB), (t1,u+1) by label (lA)
+            v1 = log_add_exp(cur + o.bB, n1 + o.lA);
+            beta[base + (size_t)t1 * Up1 + u] = v1;
+          }
+          if (d2 >= 0 && t2 >= 0 && t2 < Tb) {
+            v2 = lae3(cur + o.bA + o.bB, n1 + log_add_exp(o.bA + o.lA, o.lB + o.bC), n2 + o.lB + o.lC);
+            beta[base + (size_t)t2 * Up1 + u] = v2;
+            if (t2 == 0 && u == 0) loss[b] = -v2;
+          }
+          if (d2 < 0 && t1 == 0 && u == 0) loss[b] = -v1;
+        }
+      }
+      // the far diagonal of this step becomes the previous one (the middle one
+      // when the far one is past the lattice's end)
+      const bool far_exists = is_beta ? (last - 2 * step - 2 >= 0) : (2 * step + 2 <= last);
+      cur = far_exists ? v2 : v1;
       if (!is_beta) {
-        if (lane == 31) xs[step & 1][warp] = cur;
+        if (lane >= 30) xs[step & 1][warp][lane - 30] = cur;
       } else {
-        if (lane == 0) xs[step & 1][warp] = cur;
+        if (lane < 2) xs[step & 1][warp][lane] = cur;
       }
       __syncthreads();
     }
@@ -596,7 +698,7 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
                                                   U_len, loss, smem > 0 ? 1 : 0);
   } else {
     dim3 grid(s.B, 2);
-    dp_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
+    dp2_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
   }
   note_launch();
 }
