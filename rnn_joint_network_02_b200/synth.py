@@ -168,3 +168,19 @@ def diagonal_bounds(T_len, U_len, T: int, S: int) -> torch.Tensor:
             tt = min(t, Tb - 1)
             s[b, t] = min(Ub, max(0, (tt * (Ub + 1)) // Tb - S // 2))
     return s
+
+
+# Duration set of the token-and-duration transducer workloads: 0 .. 4 frames.
+TDT_DURATIONS = (0, 1, 2, 3, 4)
+
+
+def duration_head(batch: Batch, n_dur: int, seed: int, bias_std: float = 0.5):
+    """Weights of a duration output head for ``batch``: W_d ~ N(0, 1/H) of shape
+    [n_dur, H] and b_d ~ N(0, bias_std^2) of shape [n_dur], from their own
+    generator (seeded ``seed``), rounded to the batch's float type."""
+    gen = torch.Generator().manual_seed(seed)
+    H = batch.W_o.shape[1]
+    W_d = torch.randn(n_dur, H, generator=gen, dtype=torch.float32) / H ** 0.5
+    b_d = torch.randn(n_dur, generator=gen, dtype=torch.float32) * bias_std
+    tt = torch.bfloat16 if batch.dtype == "bf16" else torch.float32
+    return W_d.to(tt), b_d.to(tt)
