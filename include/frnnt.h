@@ -73,6 +73,10 @@ typedef enum { FRNNT_PATH_AUTO = 0, FRNNT_PATH_SIMT = 1 } frnnt_path;
  * alignment (0/1 edge posteriors). */
 typedef enum { FRNNT_LOSS_MARGINAL = 0, FRNNT_LOSS_VITERBI = 1 } frnnt_loss;
 
+/* Token-and-duration transducer limits: at most 8 durations, none above 8 frames. */
+#define FRNNT_MAX_DURATIONS 8
+#define FRNNT_MAX_DURATION 8
+
 typedef struct {
   int B, T, U;            /* batch, max frames, max labels (g has U+1 rows) */
   int D_enc, D_pred;      /* encoder / prediction feature sizes              */
@@ -93,6 +97,13 @@ typedef struct {
                              an input here).  Call frnnt_fwd_bwd_pruned.
                              Needs FRNNT_BF16 on the tensor-core kernels
                              (FRNNT_ERR_UNSUPPORTED otherwise).               */
+  int n_dur;              /* 0: the transducer.  n_dur > 0: the token-and-
+                             duration transducer with the n_dur durations
+                             below (call frnnt_fwd_bwd_tdt).                  */
+  int durations[FRNNT_MAX_DURATIONS];
+                          /* strictly increasing frame counts, durations[0] = 0,
+                             durations[1] = 1, durations[n_dur-1] <=
+                             FRNNT_MAX_DURATION; entries past n_dur unused    */
 } frnnt_dims;
 
 /* Host return codes. */
@@ -162,6 +173,36 @@ FRNNT_API int frnnt_fwd_bwd_pruned(const frnnt_dims* d,
                   const int32_t* bounds,
                   const float* grad_loss, float* loss,
                   void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* status, void* stream);
+
+/* The token-and-duration transducer (TDT) of "Efficient Sequence Transduction
+ * by Jointly Predicting Tokens and Durations" (abstract: the joint network has
+ * two outputs, normalised independently, one over the labels and one over
+ * durations, a duration being the number of input frames the emitted symbol
+ * covers).  With the hidden h of every cell as above:
+ *   z  = W_o h + b_o   (V label logits, blank included)
+ *   zd = W_d h + b_d   (n_dur duration logits)
+ * A label y_u emitted at (t,u) with duration durations[i] moves to
+ * (t + durations[i], u+1); a blank with a duration >= 1 moves to
+ * (t + durations[i], u) (a zero-frame blank would be a self-loop); each edge
+ * weighs P(symbol) * P(duration).  An alignment starts at (0,0) and ends with
+ * a blank from (t, U_len) that lands exactly on frame T_len; loss[b] = -log of
+ * the summed weight of all alignments.  The gradients of sum_b w_b loss[b]
+ * come back for f, g, W_f, W_g, W_o, b_o and the duration head:
+ *   W_d [n_dur, H], b_d [n_dur]  inputs;  dW_d, db_d  outputs, same shapes.
+ * Needs d->n_dur in [2, FRNNT_MAX_DURATIONS] with valid durations (else
+ * FRNNT_ERR_DIMS; frnnt_fwd_bwd returns FRNNT_ERR_DIMS for n_dur != 0),
+ * FRNNT_BF16 on the tensor-core kernels, the marginal loss and the whole
+ * lattice (FRNNT_ERR_UNSUPPORTED otherwise).  Workspace:
+ * frnnt_workspace_size(d).  Everything else as frnnt_fwd_bwd. */
+FRNNT_API int frnnt_fwd_bwd_tdt(const frnnt_dims* d,
+                  const void* f, const void* g, const void* W_f, const void* W_g,
+                  const void* W_o, const void* b_o, const void* W_d, const void* b_d,
+                  const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                  const float* grad_loss, float* loss,
+                  void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
+                  void* dW_d, void* db_d,
                   void* workspace, size_t workspace_bytes,
                   int32_t* status, void* stream);
 

@@ -34,6 +34,14 @@ bool dims_ok(const frnnt_dims* d) {
   if (d->U + 1 > 1024) return false;
   if (d->chunk_cells < 0) return false;
   if (d->prune_S < 0 || d->prune_S > 32) return false;
+  if (d->n_dur != 0) {
+    // token-and-duration transducer: 0 and 1 frames first, strictly increasing, at most 8 frames
+    if (d->n_dur < 2 || d->n_dur > FRNNT_MAX_DURATIONS) return false;
+    if (d->durations[0] != 0 || d->durations[1] != 1) return false;
+    for (int i = 2; i < d->n_dur; ++i)
+      if (d->durations[i] <= d->durations[i - 1]) return false;
+    if (d->durations[d->n_dur - 1] > FRNNT_MAX_DURATION) return false;
+  }
   return true;
 }
 
@@ -57,6 +65,14 @@ Shape shape_of(const frnnt_dims* d) {
   s.viterbi = d->loss == FRNNT_LOSS_VITERBI;
   s.S = d->prune_S;
   s.Nlat = s.S > 0 ? s.BT * s.S : s.Np;
+  s.n_dur = d->n_dur;
+  s.dmask = 0;
+  s.dmax = 0;
+  for (int i = 0; i < d->n_dur; ++i) {
+    s.dmask |= 1u << d->durations[i];
+    s.dmax = d->durations[i] > s.dmax ? d->durations[i] : s.dmax;
+  }
+  s.Vx = d->n_dur > 0 ? d->V + 128 : d->V;
   return s;
 }
 
@@ -176,7 +192,13 @@ bool use_tc(const frnnt_dims* d) {
   if (d->dtype != FRNNT_BF16 || d->path != FRNNT_PATH_AUTO) return false;
   if (d->B > 1024) return false;
   if (d->H % 64 || d->D_enc % 32 || d->D_pred % 32) return false;
-  return joint_tc_supported(d->H, d->V, d->U, d->prune_S);
+  return joint_tc_supported(d->H, d->n_dur > 0 ? d->V + 128 : d->V, d->U, d->prune_S);
+}
+
+// The token-and-duration transducer runs on the tensor-core kernels, with the
+// marginal loss, over the whole lattice.
+bool tdt_supported(const frnnt_dims* d) {
+  return use_tc(d) && d->loss == FRNNT_LOSS_MARGINAL && d->prune_S == 0;
 }
 
 struct TcPlan {
@@ -190,6 +212,10 @@ struct TcPlan {
   Lattice L;
   float *accWo, *db_part, *accWf, *accWg;
   __nv_bfloat16 *zbuf, *hbuf;
+  // token-and-duration transducer: [W_o; W_d; 0], [b_o; b_d; 0] and the
+  // duration head's weight-gradient accumulator (64 rows, n_dur used)
+  __nv_bfloat16 *Wx = nullptr, *bx = nullptr;
+  float* accWd = nullptr;
   size_t bytes;
 };
 
@@ -216,11 +242,20 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.alpha = c.take<float>(s.Nlat);
   p.L.beta = c.take<float>(s.Nlat);
   p.L.path = s.viterbi ? c.take<uint8_t>(s.Nlat) : nullptr;
+  if (s.n_dur > 0) {
+    p.L.beta_l = c.take<float>(s.Nlat);
+    p.L.dur_lp = c.take<float>((size_t)s.n_dur * s.Nlat);
+    p.L.tdt_q = c.take<float>((size_t)s.n_dur * s.Nlat);
+    p.L.plane = s.Nlat;
+    p.Wx = c.take<__nv_bfloat16>((size_t)s.Vx * s.H);
+    p.bx = c.take<__nv_bfloat16>(s.Vx);
+    p.accWd = c.take<float>((size_t)64 * hidden_stride(s.H));
+  }
   p.accWo = c.take<float>((size_t)s.V * hidden_stride(s.H));
   p.db_part = nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
-  p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.V);
+  p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.Vx);
   p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * hidden_stride(s.H));
   p.bytes = c.off + 256;
   return p;
@@ -264,11 +299,13 @@ int splits_for(int M, int N, int K) {
 }
 
 int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, const void* W_f, const void* W_g,
-           const void* W_o, const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
-           const int32_t* bounds, const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o,
-           void* ws, int32_t* status, cudaStream_t st) {
+           const void* W_o, const void* b_o, const void* W_d, const void* b_d, const int32_t* labels,
+           const int32_t* T_len, const int32_t* U_len, const int32_t* bounds, const float* grad_loss, float* loss,
+           void* df, void* dg, void* dW_f, void* dW_g, void* dW_o, void* db_o, void* dW_d, void* db_d, void* ws,
+           int32_t* status, cudaStream_t st) {
   TcPlan p = plan_tc(d, s, ws);
   const bool untiled = d->mode == FRNNT_UNTILED;
+  const bool tdt = s.n_dur > 0;
   int rc = FRNNT_OK;
 #define FRNNT_TRY(x)            \
   do {                          \
@@ -284,6 +321,10 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     cudaMemsetAsync(p.accWo, 0, (size_t)s.V * hidden_stride(s.H) * sizeof(float), st);
     cudaMemsetAsync(p.accWf, 0, (size_t)s.Dx * s.H * sizeof(float), st);
     cudaMemsetAsync(p.accWg, 0, (size_t)s.Dy * s.H * sizeof(float), st);
+    if (tdt) {
+      cudaMemsetAsync(p.accWd, 0, (size_t)64 * hidden_stride(s.H) * sizeof(float), st);
+      launch_tdt_weights(s, W_o, b_o, W_d, b_d, p.Wx, p.bx, st);
+    }
   }
   {
     StageScope sc("projection", st);
@@ -295,7 +336,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     FRNNT_TRY(gemm_tc(a, st));
   }
   JointLaunch j{};
-  j.s = s; j.TB = p.TB; j.UB = p.UB; j.F = p.F; j.G = p.G; j.W_o = W_o; j.b_o = b_o; j.labels = labels;
+  j.s = s; j.TB = p.TB; j.UB = p.UB; j.F = p.F; j.G = p.G; j.W_o = tdt ? (const void*)p.Wx : W_o;
+  j.b_o = tdt ? (const void*)p.bx : b_o; j.labels = labels;
   j.T_len = T_len; j.U_len = U_len; j.grad_loss = grad_loss; j.tiles = p.tiles; j.ntiles = p.ntiles; j.L = p.L;
   j.zbuf = p.zbuf; j.hbuf = p.hbuf; j.db_part = p.db_part; j.status = status; j.bounds = bounds;
   {
@@ -327,7 +369,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     const long long c1 = (c0 + p.chunkT < p.maxT) ? c0 + p.chunkT : p.maxT;
     j.tile_begin = (int)c0;
     j.tile_end = (int)c1;
-    __nv_bfloat16* zrows = untiled ? p.zbuf + (size_t)c0 * 128 * s.V : p.zbuf;
+    __nv_bfloat16* zrows = untiled ? p.zbuf + (size_t)c0 * 128 * s.Vx : p.zbuf;
     const int HS = hidden_stride(s.H);
     __nv_bfloat16* hrows = untiled ? p.hbuf + (size_t)c0 * 128 * HS : p.hbuf;
     {
@@ -337,6 +379,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       } else {
         j.mode = 2;
         FRNNT_TRY(launch_joint_tc(j, st));
+        if (tdt) launch_tdt_dzd(j, st);
       }
     }
     if (side) {
@@ -350,18 +393,24 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       StageScope sc("bwd_dWo", st);
       GemmTcArgs a{};
       // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias gradient
-      a.M = s.V; a.N = HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.V; a.B = hrows; a.b_mn = true;
+      a.M = s.V; a.N = HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.Vx; a.B = hrows; a.b_mn = true;
       a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, HS, rows); a.out_f32 = p.accWo;
       a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;
       FRNNT_TRY(gemm_tc(a, st));
+      if (tdt) {
+        // dW_d | db_d from the duration columns (64 of them, zero past n_dur)
+        a.M = 64; a.A = zrows + s.V; a.k_splits = splits_for(64, HS, rows); a.out_f32 = p.accWd;
+        FRNNT_TRY(gemm_tc(a, st));
+      }
     }
     {
       StageScope sc("bwd_dh", st);
       GemmTcArgs a{};
       // d_hidden = dz W_o, then (1 - h^2) in the epilogue, in place over h
-      a.M = rows; a.N = s.H; a.K = s.V; a.A = zrows; a.a_mn = false; a.lda = s.V; a.B = W_o;
-      a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH_FG; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
+      // (token-and-duration transducer: dz | dzd against [W_o; W_d], K = V + 64)
+      a.M = rows; a.N = s.H; a.K = tdt ? s.V + 64 : s.V; a.A = zrows; a.a_mn = false; a.lda = s.Vx;
+      a.B = tdt ? (const void*)p.Wx : W_o; a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH_FG; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
       // (1 - h^2) with h recomputed from the L2-resident F and G rows of each cell, not read back
       a.cells.tiles = p.tiles; a.cells.tile0 = (int)c0; a.cells.T = s.T; a.cells.U = s.U; a.cells.H = s.H;
       a.cells.UB = p.UB; a.cells.S = s.S; a.cells.bounds = bounds; a.cells.T_len = T_len; a.cells.U_len = U_len;
@@ -377,6 +426,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   {
     StageScope sc("projection_bwd", st);
     launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st);
+    if (tdt) launch_wo_finalize(p.accWd, s.n_dur, s.H, dW_d, db_d, st);
     launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
     launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, st);
     GemmTcArgs a{};
@@ -414,6 +464,7 @@ extern "C" int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes) {
   if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
   if (!dims_ok(d)) return FRNNT_ERR_DIMS;
   if (d->prune_S > 0 && !use_tc(d)) return FRNNT_ERR_UNSUPPORTED;
+  if (d->n_dur > 0 && !tdt_supported(d)) return FRNNT_ERR_UNSUPPORTED;
   Shape s = shape_of(d);
   *bytes = use_tc(d) ? plan_tc(d, s, nullptr).bytes : plan_simt(d, s, nullptr).bytes;
   return FRNNT_OK;
@@ -422,21 +473,23 @@ extern "C" int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes) {
 namespace {
 
 int fwd_bwd_impl(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g, const void* W_o,
-                 const void* b_o, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
-                 const int32_t* bounds, const float* grad_loss, float* loss, void* df, void* dg, void* dW_f,
-                 void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes, int32_t* status,
-                 void* stream) {
+                 const void* b_o, const void* W_d, const void* b_d, const int32_t* labels, const int32_t* T_len,
+                 const int32_t* U_len, const int32_t* bounds, const float* grad_loss, float* loss, void* df, void* dg,
+                 void* dW_f, void* dW_g, void* dW_o, void* db_o, void* dW_d, void* db_d, void* workspace,
+                 size_t workspace_bytes, int32_t* status, void* stream) {
   if (!d) return FRNNT_ERR_NULL;
   if (!enums_ok(d)) return FRNNT_ERR_UNSUPPORTED;
   if (!dims_ok(d)) return FRNNT_ERR_DIMS;
   if (d->prune_S > 0 && !use_tc(d)) return FRNNT_ERR_UNSUPPORTED;
+  if (d->n_dur > 0 && !tdt_supported(d)) return FRNNT_ERR_UNSUPPORTED;
   const void* req[] = {f, g, W_f, W_g, W_o, b_o, T_len, U_len, loss, df, dg, dW_f, dW_g, dW_o, db_o, workspace, status};
   for (const void* p : req)
     if (!p) return FRNNT_ERR_NULL;
   if (!labels && d->U > 0) return FRNNT_ERR_NULL;
   if (d->prune_S > 0 && !bounds) return FRNNT_ERR_NULL;
-  const void* al[] = {f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
-                      dW_o, db_o, workspace, status};
+  if (d->n_dur > 0 && (!W_d || !b_d || !dW_d || !db_d)) return FRNNT_ERR_NULL;
+  const void* al[] = {f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, bounds, grad_loss, loss, df, dg,
+                      dW_f, dW_g, dW_o, db_o, dW_d, db_d, workspace, status};
   for (const void* p : al)
     if (p && !aligned16(p)) return FRNNT_ERR_ALIGN;
   size_t need = 0;
@@ -447,8 +500,8 @@ int fwd_bwd_impl(const frnnt_dims* d, const void* f, const void* g, const void* 
   cudaGetLastError();   // clear a stale error so it is not reported as ours
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return FRNNT_ERR_CUDA;
   if (use_tc(d))
-    return run_tc(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
-                  dW_o, db_o, workspace, status, st);
+    return run_tc(d, s, f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, bounds, grad_loss, loss, df, dg,
+                  dW_f, dW_g, dW_o, db_o, dW_d, db_d, workspace, status, st);
   return run_simt(d, s, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, loss, df, dg, dW_f, dW_g, dW_o,
                   db_o, workspace, status, st);
 }
@@ -460,9 +513,10 @@ extern "C" int frnnt_fwd_bwd(const frnnt_dims* d, const void* f, const void* g, 
                              const int32_t* U_len, const float* grad_loss, float* loss, void* df, void* dg,
                              void* dW_f, void* dW_g, void* dW_o, void* db_o, void* workspace, size_t workspace_bytes,
                              int32_t* status, void* stream) {
-  if (d && d->prune_S != 0) return FRNNT_ERR_DIMS;   // pruned dims go through frnnt_fwd_bwd_pruned
-  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, nullptr, grad_loss, loss, df, dg, dW_f, dW_g,
-                      dW_o, db_o, workspace, workspace_bytes, status, stream);
+  // pruned dims go through frnnt_fwd_bwd_pruned, duration sets through frnnt_fwd_bwd_tdt
+  if (d && (d->prune_S != 0 || d->n_dur != 0)) return FRNNT_ERR_DIMS;
+  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, nullptr, nullptr, labels, T_len, U_len, nullptr, grad_loss, loss,
+                      df, dg, dW_f, dW_g, dW_o, db_o, nullptr, nullptr, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" int frnnt_fwd_bwd_pruned(const frnnt_dims* d, const void* f, const void* g, const void* W_f,
@@ -471,9 +525,20 @@ extern "C" int frnnt_fwd_bwd_pruned(const frnnt_dims* d, const void* f, const vo
                                     const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g,
                                     void* dW_o, void* db_o, void* workspace, size_t workspace_bytes, int32_t* status,
                                     void* stream) {
-  if (d && d->prune_S <= 0) return FRNNT_ERR_DIMS;
-  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, grad_loss, loss, df, dg, dW_f, dW_g,
-                      dW_o, db_o, workspace, workspace_bytes, status, stream);
+  if (d && (d->prune_S <= 0 || d->n_dur != 0)) return FRNNT_ERR_DIMS;
+  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, nullptr, nullptr, labels, T_len, U_len, bounds, grad_loss, loss,
+                      df, dg, dW_f, dW_g, dW_o, db_o, nullptr, nullptr, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int frnnt_fwd_bwd_tdt(const frnnt_dims* d, const void* f, const void* g, const void* W_f, const void* W_g,
+                                 const void* W_o, const void* b_o, const void* W_d, const void* b_d,
+                                 const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
+                                 const float* grad_loss, float* loss, void* df, void* dg, void* dW_f, void* dW_g,
+                                 void* dW_o, void* db_o, void* dW_d, void* db_d, void* workspace,
+                                 size_t workspace_bytes, int32_t* status, void* stream) {
+  if (d && d->n_dur == 0) return FRNNT_ERR_DIMS;
+  return fwd_bwd_impl(d, f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, nullptr, grad_loss, loss, df, dg,
+                      dW_f, dW_g, dW_o, db_o, dW_d, db_d, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" const char* frnnt_error_string(int code) {

@@ -672,10 +672,219 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
   }
 }
 
+// ------------------------------------------------------------------ token-and-duration lattice
+// "Efficient Sequence Transduction by Jointly Predicting Tokens and Durations"
+// (abstract): every emission also draws a duration, the number of frames it
+// covers.  From cell (t,u) a label with duration k goes to (t+k, u+1), a blank
+// with duration k >= 1 to (t+k, u), each edge weighing
+// token_lp + dur_lp(k); alignments end with a blank from (t, U_len) that lands
+// exactly on frame T_len.
+//
+// Cells still form anti-diagonal wavefronts (an edge of duration k advances
+// the diagonal by k or k+1), so one thread again owns one label position u:
+//  * alpha pushes.  Once alpha(t,u) is known the thread adds its blank edges
+//    into a shift register of its own future diagonals (fut[k] = diagonal
+//    s+k) and hands its label edges, one per duration, to thread u+1 (warp
+//    shuffle, shared memory across a warp boundary), which adds them to its
+//    own register one diagonal later.  Only the cell's own log-probs are read.
+//  * beta pulls.  The thread keeps its own beta of the last DM+1 diagonals in
+//    a shift register (hist[k] = diagonal s+k) and reads thread u+1's
+//    register for the label edges; (T_len, U_len) after the final blank is a
+//    virtual cell with beta 0 on diagonal T_len + U_len.  It stores PB / PL
+//    (the blank / label parts of beta) and, per duration, the log posterior
+//    numerator without alpha and log P.
+// DM = the largest duration (1..8): register arrays are indexed by compile-time k.
+template <int DM>
+struct TdtOps {
+  float bl, ll;
+  float dl[DM + 1];    // -inf for durations outside the set
+};
+
+template <int DM>
+__device__ __forceinline__ void tdt_operands(TdtOps<DM>& o, bool live, int t, int u, int Tb, int Ub, int Up1,
+                                             size_t base, long long plane, uint32_t dmask,
+                                             const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
+                                             const float* __restrict__ dur_lp) {
+  o.bl = -INFINITY;
+  o.ll = -INFINITY;
+#pragma unroll
+  for (int k = 0; k <= DM; ++k) o.dl[k] = -INFINITY;
+  if (!live || u > Ub || t < 0 || t >= Tb) return;
+  const size_t c = base + (size_t)t * Up1 + u;
+  o.bl = __ldg(blank_lp + c);
+  if (u < Ub) o.ll = __ldg(label_lp + c);
+  int i = 0;
+#pragma unroll
+  for (int k = 0; k <= DM; ++k)
+    if ((dmask >> k) & 1u) {
+      o.dl[k] = __ldg(dur_lp + (size_t)i * plane + c);
+      ++i;
+    }
+}
+
+constexpr int tdt_prefetch(int DM) { return DM <= 4 ? 4 : 2; }
+
+// MAXT: the block size bound (256 lets the registers hold every array without spilling).
+template <int DM, int MAXT>
+__global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dmask, long long plane,
+                                                      const float* __restrict__ blank_lp,
+                                                      const float* __restrict__ label_lp,
+                                                      const float* __restrict__ dur_lp, float* __restrict__ alpha,
+                                                      float* __restrict__ beta_b, float* __restrict__ beta_l,
+                                                      float* __restrict__ q, const int32_t* __restrict__ T_len,
+                                                      const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  constexpr int P = tdt_prefetch(DM);
+  __shared__ float xs[2][32][DM + 2];     // [parity][warp][k]: values handed across warp boundaries
+  const int b = blockIdx.x;
+  const bool is_beta = blockIdx.y == 1;
+  const int u = threadIdx.x;
+  const int lane = u & 31, warp = u >> 5, nwarps = blockDim.x >> 5;
+  const Lengths l = lengths_of(T_len, U_len, b, T, U);
+  const int Tb = l.Tb, Ub = l.Ub;
+  const int Up1 = U + 1;
+  const size_t base = (size_t)b * T * Up1;
+  const int last = Tb - 1 + Ub;           // the last diagonal
+  const int nsteps = last + 1;
+  // diagonal of step i: i (alpha) or last - i (beta); the thread's cell on it has t = diagonal - u
+  auto cell_t = [&](int i) { return (is_beta ? last - i : i) - u; };
+
+  TdtOps<DM> ops[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    tdt_operands<DM>(ops[i], i < nsteps, cell_t(i), u, Tb, Ub, Up1, base, plane, dmask, blank_lp, label_lp, dur_lp);
+
+  if (!is_beta) {
+    float fut[DM + 1];    // incoming weight of this thread's cell on diagonal s + k
+    float outl[DM + 1];   // this thread's label edges of the previous step, by duration
+#pragma unroll
+    for (int k = 0; k <= DM; ++k) {
+      fut[k] = -INFINITY;
+      outl[k] = -INFINITY;
+    }
+    for (int k = threadIdx.x; k < 2 * 32 * (DM + 2); k += blockDim.x) (&xs[0][0][0])[k] = -INFINITY;
+    __syncthreads();
+    for (int s0 = 0; s0 < nsteps; s0 += P) {
+#pragma unroll
+      for (int i = 0; i < P; ++i) {
+        const int s = s0 + i;
+        if (s >= nsteps) break;           // uniform across the block
+        const TdtOps<DM> o = ops[i];
+        tdt_operands<DM>(ops[i], s + P < nsteps, cell_t(s + P), u, Tb, Ub, Up1, base, plane, dmask, blank_lp,
+                         label_lp, dur_lp);
+        // label edges of thread u-1 from diagonal s-1 with duration k land on diagonal s + k
+#pragma unroll
+        for (int k = 0; k <= DM; ++k) {
+          if (!((dmask >> k) & 1u)) continue;
+          float nl = __shfl_up_sync(0xffffffffu, outl[k], 1);
+          if (lane == 0) nl = warp > 0 ? xs[(s + 1) & 1][warp - 1][k] : -INFINITY;
+          fut[k] = log_add_exp(fut[k], nl);
+        }
+        const int t = s - u;
+        const bool valid = u <= Ub && t >= 0 && t < Tb;
+        const float v = valid ? ((t == 0 && u == 0) ? 0.f : fut[0]) : -INFINITY;
+        if (valid) alpha[base + (size_t)t * Up1 + u] = v;
+        // own blank edges (duration >= 1) to diagonal s + k
+#pragma unroll
+        for (int k = 1; k <= DM; ++k)
+          if ((dmask >> k) & 1u) fut[k] = log_add_exp(fut[k], v + o.bl + o.dl[k]);
+#pragma unroll
+        for (int k = 0; k <= DM; ++k) outl[k] = v + o.ll + o.dl[k];
+        if (lane == 31) {
+#pragma unroll
+          for (int k = 0; k <= DM; ++k) xs[s & 1][warp][k] = outl[k];
+        }
+#pragma unroll
+        for (int k = 0; k < DM; ++k) fut[k] = fut[k + 1];
+        fut[DM] = -INFINITY;
+        __syncthreads();
+      }
+    }
+  } else {
+    float hist[DM + 2];   // this thread's beta on diagonal s + k (k >= 1)
+#pragma unroll
+    for (int k = 0; k < DM + 2; ++k) hist[k] = -INFINITY;
+    if (u == Ub) hist[1] = 0.f;           // the virtual cell after the final blank
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < DM + 2; ++k) xs[1][warp][k] = hist[k];
+    }
+    __syncthreads();
+    for (int i0 = 0; i0 < nsteps; i0 += P) {
+#pragma unroll
+      for (int i = 0; i < P; ++i) {
+        const int step = i0 + i;
+        if (step >= nsteps) break;        // uniform across the block
+        const TdtOps<DM> o = ops[i];
+        tdt_operands<DM>(ops[i], step + P < nsteps, cell_t(step + P), u, Tb, Ub, Up1, base, plane, dmask, blank_lp,
+                         label_lp, dur_lp);
+        const int t = cell_t(step);
+        const bool valid = u <= Ub && t >= 0 && t < Tb;
+        float pb = -INFINITY, pl = -INFINITY, qk[DM + 1];
+#pragma unroll
+        for (int k = 0; k <= DM; ++k) {
+          // thread u+1's beta on diagonal s + k + 1, i.e. at (t + k, u + 1)
+          float nb = __shfl_down_sync(0xffffffffu, hist[k + 1], 1);
+          if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1][k + 1] : -INFINITY;
+          const float eb = k >= 1 ? o.bl + o.dl[k] + hist[k] : -INFINITY;
+          const float el = (u < Ub && t + k < Tb) ? o.ll + o.dl[k] + nb : -INFINITY;
+          pb = log_add_exp(pb, eb);
+          pl = log_add_exp(pl, el);
+          qk[k] = log_add_exp(eb, el);
+        }
+        const float bt = log_add_exp(pb, pl);
+        if (valid) {
+          const size_t c = base + (size_t)t * Up1 + u;
+          beta_b[c] = pb;
+          beta_l[c] = pl;
+          int j = 0;
+#pragma unroll
+          for (int k = 0; k <= DM; ++k)
+            if ((dmask >> k) & 1u) {
+              q[(size_t)j * plane + c] = qk[k];
+              ++j;
+            }
+          if (t == 0 && u == 0) loss[b] = -bt;
+        }
+#pragma unroll
+        for (int k = DM + 1; k >= 2; --k) hist[k] = hist[k - 1];
+        hist[1] = valid ? bt : -INFINITY;
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < DM + 2; ++k) xs[step & 1][warp][k] = hist[k];
+        }
+        __syncthreads();
+      }
+    }
+  }
+}
+
+template <int DM>
+void launch_tdt_dp_t(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
+                     int threads, cudaStream_t st) {
+  dim3 grid(s.B, 2);
+  if (threads <= 256)
+    tdt_dp_kernel<DM, 256><<<grid, threads, 0, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+                                                     L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
+  else
+    tdt_dp_kernel<DM, 1024><<<grid, threads, 0, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+                                                      L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
+}
+
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
                float* loss, cudaStream_t st) {
   int threads = ((s.Up1 + 31) / 32) * 32;
-  if (s.S > 0) {
+  if (s.n_dur > 0) {
+    switch (s.dmax) {
+      case 1: launch_tdt_dp_t<1>(s, L, T_len, U_len, loss, threads, st); break;
+      case 2: launch_tdt_dp_t<2>(s, L, T_len, U_len, loss, threads, st); break;
+      case 3: launch_tdt_dp_t<3>(s, L, T_len, U_len, loss, threads, st); break;
+      case 4: launch_tdt_dp_t<4>(s, L, T_len, U_len, loss, threads, st); break;
+      case 5: launch_tdt_dp_t<5>(s, L, T_len, U_len, loss, threads, st); break;
+      case 6: launch_tdt_dp_t<6>(s, L, T_len, U_len, loss, threads, st); break;
+      case 7: launch_tdt_dp_t<7>(s, L, T_len, U_len, loss, threads, st); break;
+      default: launch_tdt_dp_t<8>(s, L, T_len, U_len, loss, threads, st); break;
+    }
+  } else if (s.S > 0) {
     const int smem = s.T * 4 * (L.path ? 2 : 1);
     if (smem <= 48 * 1024) {
       dim3 grid(s.B, L.path ? 1 : 2);

@@ -40,6 +40,14 @@ struct Shape {
   bool viterbi;       // maximum-approximation loss
   int S;              // pruned lattice: label positions kept per frame (0 = the whole lattice)
   long long Nlat;     // entries of one lattice array: B*T*(U+1), or B*T*S when pruned
+  // token-and-duration transducer (n_dur > 0): the duration set as a bit mask
+  // (bit k = duration k frames), its largest entry, and Vx = V + 128: the
+  // columns of [W_o; W_d; 0] and the row stride of the logit buffers, whose
+  // columns V .. V+n_dur-1 carry the duration head
+  int n_dur = 0;
+  uint32_t dmask = 0;
+  int dmax = 0;
+  int Vx = 0;
 };
 
 // Lattice arrays, fp32, padded layout [b][t][u] with u fastest.
@@ -53,6 +61,15 @@ struct Lattice {
   // alignment leaves the cell by its blank edge, bit 1 = by its label edge,
   // bit 2 = the best way into the cell is its blank edge (DP decision).
   uint8_t* path;
+  // Token-and-duration transducer only (null otherwise).  beta then holds
+  // PB(c) = log of the weight of finishing from c through one of its blank
+  // edges, beta_l the same through its label edges (beta(c) = lae(PB, PL));
+  // dur_lp [n_dur][plane] the duration log-probs and tdt_q [n_dur][plane]
+  // the log posterior numerator of each duration at c without alpha and log P.
+  float* beta_l = nullptr;
+  float* dur_lp = nullptr;
+  float* tdt_q = nullptr;
+  long long plane = 0;
 };
 
 #ifdef __CUDACC__
@@ -65,6 +82,17 @@ struct Lattice {
 //   maximum approximation: the best alignment's 0/1 edge indicators.
 __device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size_t c0, long long c_t1,
                                                 long long c_u1, bool last, float& bpost, float& lpost) {
+  if (L.beta_l) {
+    // token-and-duration transducer: the summed posteriors of the blank and
+    // of the label edges of every duration, with log P = lae(PB, PL) at (0,0)
+    const float x = L.beta[c0], y = L.beta_l[c0];
+    const float m = fmaxf(x, y);
+    const float logp = m + __logf(__expf(x - m) + __expf(y - m));
+    const float al = L.alpha[c] - logp;
+    bpost = __expf(al + L.beta[c]);
+    lpost = __expf(al + L.beta_l[c]);
+    return;
+  }
   if (L.path) {
     const uint8_t e = L.path[c];
     bpost = (e & 1) ? 1.f : 0.f;
@@ -193,6 +221,13 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
 // Joint kernel variant for later calls: -1 automatic, 0 one CTA per cell tile, 1 CTA pairs; returns the previous one.
 int set_joint_variant(int variant);
 void launch_dz_from_z(const JointLaunch& j, cudaStream_t st);
+// Token-and-duration transducer: the duration-head logit gradient of the
+// launch's rows into columns [V, V + 128) of their dz rows (zeros past n_dur
+// and for cells outside the lattice); rows (tile - tile_begin) * 128 + r.
+void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st);
+// W_x = [W_o; W_d; 0] [Vx][H] and b_x = [b_o; b_d; 0] [Vx] (bf16).
+void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const void* W_d, const void* b_d, void* W_x,
+                        void* b_x, cudaStream_t st);
 // blocks_per_sm: 256-thread blocks per SM of the grid (fewer leave room for work running beside it)
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
 void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);

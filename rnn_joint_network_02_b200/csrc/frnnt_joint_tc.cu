@@ -84,6 +84,11 @@ struct JointParams {
   int32_t* status;
   const int32_t* bounds;  // pruned lattice: [B][T] band starts; S = band width (0: whole lattice)
   int S;
+  // columns of the joint's output weights and row stride of zbuf: V, or for the
+  // token-and-duration transducer (n_dur > 0) V + 128, the last 128-column tile
+  // holding the duration head (columns V .. V + n_dur - 1)
+  int Vx;
+  int n_dur;
 };
 
 struct RowInfo {
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   const int ngrp = (p.KB + p.ks - 1) / p.ks;                      // K-block groups (one ring stage each)
   uint8_t* fgs = ring + p.stages * STAGE;                         // TB F rows then UB G rows of this tile
   __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + fg_bytes(p.TB, p.UB, p.H));   // b_o (bf16)
-  uint8_t* stage_s = (uint8_t*)(bias_s + ((p.V + 511) & ~511));   // per epilogue warp: srows x 80 B
+  uint8_t* stage_s = (uint8_t*)(bias_s + ((p.Vx + 511) & ~511));  // per epilogue warp: srows x 80 B
   uint64_t* full = (uint64_t*)(stage_s + kEpiWarps * p.srows * 80);
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int k = threadIdx.x; k < p.V; k += blockDim.x) bias_s[k] = p.b_o[k];
+  for (int k = threadIdx.x; k < p.Vx; k += blockDim.x) bias_s[k] = p.b_o[k];
   if (warp == kMmaWarp) {
     if (PAIR) {
       tmem_alloc_pair(tmem_base_p, 512);
@@ -495,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     const int q = warp & 3;                   // TMEM lane quadrant
     const int half = warp >> 2;               // columns [64 half, 64 half + 64) of each V tile
     const int r = q * 32 + lane;
-    const int V = p.V;
+    const int V = p.Vx;                       // row stride of zbuf
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     int acc_i = 0;
     for (int it = slot; it < niter; it += nslots) {
@@ -547,7 +552,24 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               v[8 * j + 2 * q + 1] = __uint_as_float(buf[8 * j + 2 * q + 1]) + bf.y;
             }
           }
-          if (MODE != MODE_BWD_DZ) {
+          if (MODE != MODE_BWD_DZ && p.n_dur > 0 && n == p.nV - 1) {
+            // the duration head: its own log-softmax over columns 0 .. n_dur-1
+            // of the last tile, not part of the label log-sum-exp, not stored
+            if (c == 0 && half == 0 && real && ri.valid) {
+              float md = v[0];
+#pragma unroll
+              for (int i = 1; i < FRNNT_MAX_DURATIONS; ++i)
+                if (i < p.n_dur) md = fmaxf(md, v[i]);
+              float sd = 0.f;
+#pragma unroll
+              for (int i = 0; i < FRNNT_MAX_DURATIONS; ++i)
+                if (i < p.n_dur) sd += ex2((v[i] - md) * kLog2e);
+              const float ld = md + __logf(sd);
+#pragma unroll
+              for (int i = 0; i < FRNNT_MAX_DURATIONS; ++i)
+                if (i < p.n_dur) p.L.dur_lp[(size_t)i * p.L.plane + ri.cell] = v[i] - ld;
+            }
+          } else if (MODE != MODE_BWD_DZ) {
             float t0 = fmaxf(v[0], v[1]), t1 = fmaxf(v[2], v[3]);
 #pragma unroll
             for (int j = 4; j < 32; j += 4) {
@@ -672,19 +694,51 @@ __global__ void tiles_kernel(int B, int T, int U, int TB, int UB, int pruned, co
 }
 
 // ------------------------------------------------------------------ untiled backward: dz from stored z
+// Token-and-duration transducer: the duration-head logit gradient of the cell
+// behind row ri into the 128 bf16 columns at `out` (lane l writes columns
+// 4l .. 4l+3):  dzd_i = w (occ P_dur(i) - exp(alpha - log P + q_i)) for
+// i < n_dur, 0 past n_dur and for cells outside the lattice.
+__device__ __forceinline__ void tdt_dzd_row(const JointParams& p, const RowInfo& ri, __nv_bfloat16* out, int lane) {
+  float vals[4] = {0.f, 0.f, 0.f, 0.f};
+  if (ri.valid && 4 * lane < p.n_dur) {
+    size_t c0;
+    long long c_t1, c_u1;
+    bool last;
+    lattice_neighbors(p, ri, c0, c_t1, c_u1, last);
+    const size_t c = ri.cell;
+    const float x = p.L.beta[c0], y = p.L.beta_l[c0];
+    const float m = fmaxf(x, y);
+    const float logp = m + __logf(__expf(x - m) + __expf(y - m));
+    const float a = p.L.alpha[c] - logp;
+    const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
+    const float occ = __expf(a + p.L.beta[c]) + __expf(a + p.L.beta_l[c]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = 4 * lane + j;
+      if (i < p.n_dur) {
+        const size_t o = (size_t)i * p.L.plane + c;
+        vals[j] = w * (occ * __expf(p.L.dur_lp[o]) - __expf(a + p.L.tdt_q[o]));
+      }
+    }
+  }
+  *(uint2*)(out + 4 * lane) = make_uint2(pack_bf16x2(vals[0], vals[1]), pack_bf16x2(vals[2], vals[3]));
+}
+
 __global__ void dz_from_z_kernel(JointParams p) {
   // one warp per row; rows of tiles [tile_begin, ntiles).  A row's z is read
   // in batches of four 16-byte chunks per lane, all loads of a batch issued
   // before any store (the row is rewritten in place).
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int V = p.V;
+  const int ldz = p.Vx;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
   for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows;
        row += (long long)gridDim.x * (blockDim.x >> 5)) {
     const int tile = p.tile_begin + (int)(row >> 7);
     const RowInfo ri = row_info(p, p.tiles[tile], (int)(row & 127));
-    __nv_bfloat16* zr = p.zbuf + (size_t)tile * 128 * V + (size_t)(row & 127) * V;
+    __nv_bfloat16* zr = p.zbuf + (size_t)tile * 128 * ldz + (size_t)(row & 127) * ldz;
+    if (p.n_dur > 0) tdt_dzd_row(p, ri, zr + V, lane);
     if (!ri.valid) {
       for (int k = lane * 8; k < V; k += 256) *(uint4*)(zr + k) = make_uint4(0, 0, 0, 0);
       continue;
@@ -730,6 +784,40 @@ __global__ void dz_from_z_kernel(JointParams p) {
         *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
+  }
+}
+
+// Tiled backward of the token-and-duration transducer: the duration columns of
+// the chunk's dz rows (the label columns come from the joint kernel's dz pass).
+__global__ void tdt_dzd_kernel(JointParams p) {
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows;
+       row += (long long)gridDim.x * (blockDim.x >> 5)) {
+    const int tile = p.tile_begin + (int)(row >> 7);
+    const RowInfo ri = row_info(p, p.tiles[tile], (int)(row & 127));
+    tdt_dzd_row(p, ri, p.zbuf + (size_t)row * p.Vx + p.V, lane);
+  }
+}
+
+// W_x = [W_o; W_d; 0] (Vx rows of H) and b_x = [b_o; b_d; 0], bf16.
+__global__ void tdt_weights_kernel(int V, int H, int n_dur, int Vx, const __nv_bfloat16* __restrict__ W_o,
+                                   const __nv_bfloat16* __restrict__ b_o, const __nv_bfloat16* __restrict__ W_d,
+                                   const __nv_bfloat16* __restrict__ b_d, __nv_bfloat16* __restrict__ W_x,
+                                   __nv_bfloat16* __restrict__ b_x) {
+  const int cpr = H / 8;                          // 16-byte chunks per row
+  const long long n = (long long)Vx * cpr;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / cpr), k = (int)(i % cpr) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < V) v = *(const uint4*)(W_o + (size_t)r * H + k);
+    else if (r < V + n_dur) v = *(const uint4*)(W_d + (size_t)(r - V) * H + k);
+    *(uint4*)(W_x + (size_t)r * H + k) = v;
+  }
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < Vx; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)i;
+    b_x[r] = r < V ? b_o[r] : (r < V + n_dur ? b_d[r - V] : __float2bfloat16_rn(0.f));
   }
 }
 
@@ -934,14 +1022,14 @@ int g_joint_variant = -1;   // -1 automatic, 0 one CTA per tile, 1 CTA pairs
 template <int MODE, bool PAIR>
 int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStream_t st) {
   constexpr int kb_bytes = PAIR ? kStageBytes / 2 : kStageBytes;
-  p.srows = staging_rows(p.KB, p.V, p.TB, p.UB);
+  p.srows = staging_rows(p.KB, p.Vx, p.TB, p.UB);
   // two K blocks per ring stage (half as many barrier polls in the MMA issuer)
   // while that still leaves at least three stages
-  p.ks = stages_for(p.KB, p.V, p.TB, p.UB, 2 * kb_bytes) >= 3 ? 2 : 1;
+  p.ks = stages_for(p.KB, p.Vx, p.TB, p.UB, 2 * kb_bytes) >= 3 ? 2 : 1;
   const int stage_bytes = p.ks * kb_bytes;
-  p.stages = stages_for(p.KB, p.V, p.TB, p.UB, stage_bytes);
+  p.stages = stages_for(p.KB, p.Vx, p.TB, p.UB, stage_bytes);
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
-  const int smem = smem_fixed(p.KB, p.V, p.TB, p.UB, p.srows) + p.stages * stage_bytes;
+  const int smem = smem_fixed(p.KB, p.Vx, p.TB, p.UB, p.srows) + p.stages * stage_bytes;
   auto kern = joint_tc_kernel<MODE, PAIR>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1063,17 +1151,21 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.HS = hidden_stride(j.s.H);
   p.db_part = j.db_part;
   p.status = j.status;
-  p.nV = p.V / BN;
+  p.Vx = j.s.Vx;
+  p.n_dur = j.s.n_dur;
+  // the backward dz pass covers the label tiles only (the duration head's
+  // gradient comes from the stored duration log-probs)
+  p.nV = (j.mode == MODE_BWD_DZ ? p.V : p.Vx) / BN;
   // upper bound of this launch's tile count (the exact count is on the device)
   const long long span = (long long)std::min<long long>(j.tile_end, max_tiles(j.s, j.TB, j.UB)) - j.tile_begin;
   const int ntiles_max = (int)std::max<long long>(0, span);
   // CTA pairs pay off when W_o is large (each CTA then streams half of it);
   // for small W_o the coupling of the two CTAs' h generation costs more
   const bool pair = g_joint_variant == 1 ||
-                    (g_joint_variant < 0 && ntiles_max >= sms() && (long long)p.V * p.H >= (1LL << 21));
+                    (g_joint_variant < 0 && ntiles_max >= sms() && (long long)p.Vx * p.H >= (1LL << 21));
   CUtensorMap tm;
   // a pair CTA stages 64 of the BN rows of every W_o tile
-  if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.V, p.H, 64, pair ? BN / 2 : BN)) return FRNNT_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.Vx, p.H, 64, pair ? BN / 2 : BN)) return FRNNT_ERR_CUDA;
   if (pair) {
     if (j.mode == MODE_FWD) return launch_joint_t<MODE_FWD, true>(tm, p, ntiles_max, st);
     if (j.mode == MODE_FWD_STORE) return launch_joint_t<MODE_FWD_STORE, true>(tm, p, ntiles_max, st);
@@ -1111,7 +1203,42 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.S = j.s.S;
   p.L = j.L;
   p.zbuf = (__nv_bfloat16*)j.zbuf;
+  p.Vx = j.s.Vx;
+  p.n_dur = j.s.n_dur;
   dz_from_z_kernel<<<sms() * 4, 256, 0, st>>>(p);
+  note_launch();
+}
+
+void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st) {
+  JointParams p{};
+  p.T = j.s.T;
+  p.U = j.s.U;
+  p.V = j.s.V;
+  p.TB = j.TB;
+  p.UB = j.UB;
+  p.labels = j.labels;
+  p.T_len = j.T_len;
+  p.U_len = j.U_len;
+  p.grad_loss = j.grad_loss;
+  p.tiles = j.tiles;
+  p.ntiles = j.ntiles;
+  p.tile_begin = j.tile_begin;
+  p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
+  p.L = j.L;
+  p.zbuf = (__nv_bfloat16*)j.zbuf;
+  p.Vx = j.s.Vx;
+  p.n_dur = j.s.n_dur;
+  tdt_dzd_kernel<<<sms() * 4, 256, 0, st>>>(p);
+  note_launch();
+}
+
+void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const void* W_d, const void* b_d, void* W_x,
+                        void* b_x, cudaStream_t st) {
+  tdt_weights_kernel<<<sms() * 2, 256, 0, st>>>(s.V, s.H, s.n_dur, s.Vx, (const __nv_bfloat16*)W_o,
+                                                (const __nv_bfloat16*)b_o, (const __nv_bfloat16*)W_d,
+                                                (const __nv_bfloat16*)b_d, (__nv_bfloat16*)W_x, (__nv_bfloat16*)b_x);
   note_launch();
 }
 

@@ -24,7 +24,8 @@ OK = 0
 STATUS_LENGTH, STATUS_LABEL, STATUS_TIMEOUT, STATUS_BOUNDS = 1, 2, 4, 8
 
 EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnnt_version", "frnnt_profile",
-            "frnnt_profile_read", "frnnt_fwd_bwd_noalloc", "frnnt_fwd_bwd_pruned")
+            "frnnt_profile_read", "frnnt_fwd_bwd_noalloc", "frnnt_fwd_bwd_pruned", "frnnt_fwd_bwd_tdt")
+MAX_DURATIONS = 8
 NOALLOC_MAX_BYTES = 64 * 1024 * 1024
 TEST_HOOKS = ("frnnt_test_gemm_bf16", "frnnt_test_joint_variant")
 
@@ -33,7 +34,8 @@ class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("U", ctypes.c_int), ("D_enc", ctypes.c_int),
                 ("D_pred", ctypes.c_int), ("H", ctypes.c_int), ("V", ctypes.c_int), ("blank", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("path", ctypes.c_int),
-                ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int), ("prune_S", ctypes.c_int)]
+                ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int), ("prune_S", ctypes.c_int),
+                ("n_dur", ctypes.c_int), ("durations", ctypes.c_int * 8)]
 
 
 class StageStat(ctypes.Structure):
@@ -75,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.frnnt_fwd_bwd_pruned.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 4 + [f32p, f32p] + [vp] * 6 +
                                            [vp, ctypes.c_size_t, i32p, vp])
         L.frnnt_fwd_bwd_pruned.restype = ctypes.c_int
+        L.frnnt_fwd_bwd_tdt.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 8 + [i32p] * 3 + [f32p, f32p] + [vp] * 8 +
+                                        [vp, ctypes.c_size_t, i32p, vp])
+        L.frnnt_fwd_bwd_tdt.restype = ctypes.c_int
         L.frnnt_fwd_bwd_noalloc.argtypes = ([ctypes.POINTER(Dims)] + [vp] * 6 + [i32p] * 3 + [f32p, f32p] +
                                             [vp] * 6 + [i32p, vp])
         L.frnnt_fwd_bwd_noalloc.restype = ctypes.c_int
@@ -129,10 +134,14 @@ LOSSES = {"marginal": 0, "viterbi": 1}
 
 
 def make_dims(B, T, U, D_enc, D_pred, H, V, dtype="bf16", mode="tiled", path="auto", chunk_cells=0,
-              blank=0, loss="marginal", prune_S=0) -> Dims:
+              blank=0, loss="marginal", prune_S=0, durations=()) -> Dims:
+    """``durations`` (token-and-duration transducer): the duration set, or () for the transducer."""
+    if len(durations) > MAX_DURATIONS:
+        raise ValueError(f"at most {MAX_DURATIONS} durations")
+    dur = (ctypes.c_int * 8)(*[int(x) for x in durations])
     return Dims(B, T, U, D_enc, D_pred, H, V, blank, BF16 if dtype == "bf16" else F32,
                 TILED if mode == "tiled" else UNTILED, PATH_SIMT if path == "simt" else PATH_AUTO,
-                chunk_cells, LOSSES[loss], prune_S)
+                chunk_cells, LOSSES[loss], prune_S, len(durations), dur)
 
 
 def workspace_size(dims: Dims) -> int:
@@ -147,18 +156,21 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", prune_S=0) -> Dims:
+def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", prune_S=0, durations=()) -> Dims:
     B, T, D_enc = f.shape
     U = g.shape[1] - 1
     V, H = W_o.shape
-    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss, prune_S)
+    return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss, prune_S,
+                     durations)
 
 
 class Outputs:
     """Preallocated outputs and workspace of one call shape."""
 
-    def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims, with_workspace: bool = True):
+    def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims, with_workspace: bool = True, W_d=None, b_d=None):
         dev = f.device
+        self.dW_d = None if W_d is None else torch.empty_like(W_d)
+        self.db_d = None if b_d is None else torch.empty_like(b_d)
         self.loss = torch.empty(f.shape[0], dtype=torch.float32, device=dev)
         self.df = torch.empty_like(f)
         self.dg = torch.empty_like(g)
@@ -171,7 +183,10 @@ class Outputs:
         self.workspace = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def grads(self):
-        return dict(df=self.df, dg=self.dg, dW_f=self.dW_f, dW_g=self.dW_g, dW_o=self.dW_o, db_o=self.db_o)
+        d = dict(df=self.df, dg=self.dg, dW_f=self.dW_f, dW_g=self.dW_g, dW_o=self.dW_o, db_o=self.db_o)
+        if self.dW_d is not None:
+            d.update(dW_d=self.dW_d, db_d=self.db_d)
+        return d
 
 
 def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
@@ -273,6 +288,35 @@ def fwd_bwd_pruned(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, S: in
                                     _ptr(grad_loss), _ptr(out.loss), _ptr(out.df), _ptr(out.dg), _ptr(out.dW_f),
                                     _ptr(out.dW_g), _ptr(out.dW_o), _ptr(out.db_o), _ptr(out.workspace),
                                     out.workspace.numel(), _ptr(out.status), ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        raise FrnntError(rc, error_string(rc))
+    if check:
+        bits = int(out.status[0].item())
+        if bits:
+            raise FrnntStatusError(bits)
+    return out.loss, out.grads()
+
+
+def fwd_bwd_tdt(f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, durations, grad_loss=None,
+                mode="tiled", chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+    """frnnt_fwd_bwd_tdt: the token-and-duration transducer loss and gradients.
+
+    W_d [n_dur, H] and b_d [n_dur] are the duration head (bf16, like the other
+    weights); ``durations`` is the duration set (frame counts, increasing,
+    starting 0, 1).  Returns (loss [B] fp32, dict of gradients including dW_d
+    and db_d)."""
+    dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
+    dims = dims_of(f, g, W_o, dtype, mode, "auto", chunk_cells, blank, "marginal", 0, tuple(durations))
+    if out is None:
+        out = Outputs(f, g, W_f, W_g, W_o, b_o, dims, W_d=W_d, b_d=b_d)
+    if stream is None:
+        stream = torch.cuda.current_stream(f.device)
+    rc = lib().frnnt_fwd_bwd_tdt(ctypes.byref(dims), _ptr(f), _ptr(g), _ptr(W_f), _ptr(W_g), _ptr(W_o), _ptr(b_o),
+                                 _ptr(W_d), _ptr(b_d), _ptr(labels), _ptr(T_len), _ptr(U_len), _ptr(grad_loss),
+                                 _ptr(out.loss), _ptr(out.df), _ptr(out.dg), _ptr(out.dW_f), _ptr(out.dW_g),
+                                 _ptr(out.dW_o), _ptr(out.db_o), _ptr(out.dW_d), _ptr(out.db_d),
+                                 _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
+                                 ctypes.c_void_p(stream.cuda_stream))
     if rc != OK:
         raise FrnntError(rc, error_string(rc))
     if check:

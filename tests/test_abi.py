@@ -115,3 +115,42 @@ def test_pruned_dims_rules():
     pargs[0] = ctypes.byref(d)
     pargs[10] = None                                # missing bounds
     assert lib.frnnt_fwd_bwd_pruned(*pargs) == 1
+
+
+def test_tdt_dims_rules():
+    """Duration sets: 2..8 strictly increasing frame counts starting 0, 1 and at
+    most 8; the token-and-duration entry needs the bf16 tensor-core kernels, the
+    marginal loss and the whole lattice; the plain entry refuses duration sets,
+    the duration entry refuses dims without one, and a missing head is NULL."""
+    lib = frnnt.lib()
+    n = ctypes.c_size_t(0)
+
+    def ws(**kw):
+        args = dict(dtype="bf16", mode="untiled")
+        args.update(kw)
+        d = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, **args)
+        return lib.frnnt_workspace_size(ctypes.byref(d), ctypes.byref(n))
+
+    for bad in [(0,), (1, 2), (0, 2), (0, 1, 1), (0, 1, 3, 2), (0, 1, 9), tuple(range(8)) + (8,)][:6]:
+        assert ws(durations=bad) == 2, bad
+    assert ws(durations=(0, 1, 2, 3, 4)) == 0
+    assert ws(durations=(0, 1, 2, 4, 8)) == 0
+    assert ws(durations=tuple(range(8))) == 0
+    assert ws(durations=(0, 1, 2), dtype="f32") == 4
+    assert ws(durations=(0, 1, 2), loss="viterbi") == 4
+    assert ws(durations=(0, 1, 2), prune_S=4) == 4
+    with pytest.raises(ValueError):
+        frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, durations=tuple(range(9)))
+    plain = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16")
+    tdt = frnnt.make_dims(8, 100, 20, 256, 256, 256, 128, dtype="bf16", durations=(0, 1, 2))
+    assert frnnt.workspace_size(tdt) > frnnt.workspace_size(plain)
+    fake = [ctypes.c_void_p(4096 * (i + 1)) for i in range(24)]
+    args = ([ctypes.byref(tdt)] + fake[:6] + fake[6:9] + [None, fake[9]] + fake[10:16] +
+            [fake[16], 1 << 40, fake[17], None])
+    assert lib.frnnt_fwd_bwd(*args) == 2                # duration set on the plain entry
+    targs = ([ctypes.byref(plain)] + fake[:8] + fake[8:11] + [None, fake[11]] + fake[12:20] +
+             [fake[20], 1 << 40, fake[21], None])
+    assert lib.frnnt_fwd_bwd_tdt(*targs) == 2           # no duration set on the duration entry
+    targs[0] = ctypes.byref(tdt)
+    targs[7] = None                                     # missing W_d
+    assert lib.frnnt_fwd_bwd_tdt(*targs) == 1
