@@ -47,8 +47,9 @@ def parse():
                    help="both: untiled is the headline value, tiled is reported alongside")
     p.add_argument("--path", default="auto", choices=["auto", "simt"])
     p.add_argument("--chunk-cells", type=int, default=0)
-    p.add_argument("--loss", default="marginal", choices=["marginal", "viterbi"],
-                   help="training criterion: every alignment (default) or the best one")
+    p.add_argument("--loss", default="marginal", choices=["marginal", "viterbi", "tdt"],
+                   help="training criterion: every alignment (default), the best one, or the token-and-duration "
+                        "transducer (durations 0..4 frames, a duration head beside the label head)")
     p.add_argument("--prune", type=int, default=0,
                    help="pruned lattice: S label positions per frame on a band along the diagonal (0: whole lattice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -80,6 +81,7 @@ def config_of(batch, args, n_gpus):
     return {"workload": args.workload, "B": d["B"], "T": d["T"], "U": d["U"], "D_enc": d["D_enc"],
             "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": args.mode, "path": args.path,
             "loss": args.loss, "prune_S": args.prune,
+            "durations": list(synth.TDT_DURATIONS) if args.loss == "tdt" else None,
             "valid_cells": batch.valid_cells(), "padded_cells": batch.padded_cells(),
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{n_gpus}",
             "global_batch": d["B"] * n_gpus}
@@ -87,12 +89,13 @@ def config_of(batch, args, n_gpus):
 
 # ------------------------------------------------------------------ algorithmic work per stage
 
-def stage_work(batch, stage, mode, cells=None):
+def stage_work(batch, stage, mode, cells=None, n_dur=0):
     """(kind, amount per call): tensor flops or HBM bytes that the stage must
-    do by definition (recomputation excluded); ``cells`` = the valid cells of
-    the lattice computed (default: the whole lattice's)."""
+    do by definition (recomputation and tile padding excluded); ``cells`` = the
+    valid cells of the lattice computed (default: the whole lattice's);
+    ``n_dur`` = outputs of a duration head beside the V label logits."""
     d = batch.dims
-    H, V = d["H"], d["V"]
+    H, V = d["H"], d["V"] + n_dur
     cells = batch.valid_cells() if cells is None else cells
     if stage in ("joint_fwd", "bwd_dWo", "bwd_dh"):
         return "tensor", 2.0 * H * V * cells
@@ -179,6 +182,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle (CPU) leg
 
+def duration_head(batch):
+    """The token-and-duration workloads' duration head (seeded, like the other inputs)."""
+    return synth.duration_head(batch, len(synth.TDT_DURATIONS), seed=5)
+
+
 def oracle_sample(batch, utterance=0, loss="marginal"):
     """Times the fp64 oracle on one utterance; returns (seconds, metric units)."""
     import numpy as np
@@ -188,8 +196,13 @@ def oracle_sample(batch, utterance=0, loss="marginal"):
     w = np.zeros(batch.f.shape[0])
     w[utterance] = 1.0
     t0 = time.perf_counter()
-    oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
-                   grad_loss=w, utterances=[utterance], loss=loss)
+    if loss == "tdt":
+        W_d, b_d = (t.double().numpy() for t in duration_head(batch))
+        oracle.tdt_fwd_bwd(f, g, W_f, W_g, W_o, b_o, W_d, b_d, batch.labels.numpy(), batch.T_len.numpy(),
+                           batch.U_len.numpy(), synth.TDT_DURATIONS, grad_loss=w, utterances=[utterance])
+    else:
+        oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                       grad_loss=w, utterances=[utterance], loss=loss)
     dt = time.perf_counter() - t0
     d = batch.dims
     units = d["T"] * (d["U"] + 1) * d["V"]      # this utterance's share of B*T*(U+1)*V
@@ -235,8 +248,10 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     """Times one mode: warm-up, K timed steps (each after an L2 flush), the
     end-to-end variant with host buffers, per-stage device times."""
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
+    tdt = args.loss == "tdt"
+    durations = tuple(synth.TDT_DURATIONS) if tdt else ()
     dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank,
-                         args.loss, args.prune)
+                         "marginal" if tdt else args.loss, args.prune, durations)
     bounds = None
     valid = batch.valid_cells()
     if args.prune:
@@ -244,11 +259,17 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         valid = sum(min(args.prune, int(batch.U_len[b]) - int(hb[b, t]) + 1)
                     for b in range(batch.dims["B"]) for t in range(int(batch.T_len[b])))
         bounds = hb.to(dev)
-    out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims)
+    out = frnnt.Outputs(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], dims, W_d=d.get("W_d"),
+                        b_d=d.get("b_d"))
     stream = torch.cuda.current_stream(dev)
 
     def call(check=False):
-        if bounds is not None:
+        if tdt:
+            res = frnnt.fwd_bwd_tdt(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["W_d"], d["b_d"],
+                                    d["labels"], d["T_len"], d["U_len"], durations, mode=mode,
+                                    chunk_cells=args.chunk_cells, blank=batch.blank, out=out, check=check,
+                                    stream=stream)
+        elif bounds is not None:
             res = frnnt.fwd_bwd_pruned(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"],
                                        d["T_len"], d["U_len"], bounds, args.prune, mode=mode, path=args.path,
                                        chunk_cells=args.chunk_cells, loss=args.loss, blank=batch.blank, out=out,
@@ -340,7 +361,7 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     pk = peaks()
     if stages:
         dom = max(stages, key=lambda k: stages[k]["ms"])
-        kind, work = stage_work(batch, dom, mode, valid)
+        kind, work = stage_work(batch, dom, mode, valid, len(durations))
         per_call_ms = stages[dom]["ms"] / args.steps
         tr = MEASURED_TRAFFIC.get((args.workload, mode, dom))
         if kind == "tensor":
@@ -380,6 +401,9 @@ def run_ours(args):
     batch = synth.workload(args.workload, seed=1000 + idx + 7919 * rank)
     d = {k: getattr(batch, k).to(dev).contiguous()
          for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+    if args.loss == "tdt":
+        W_d, b_d = duration_head(batch)
+        d["W_d"], d["b_d"] = W_d.to(dev).contiguous(), b_d.to(dev).contiguous()
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
     elt = 2 if dtype == "bf16" else 4
     footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +

@@ -30,10 +30,12 @@ __device__ inline int label_of(const int32_t* labels, int b, int u, int U, int V
 // log(exp(a) + exp(b)) in fp32, exact for -inf operands: max + ln(1 + e^-|a-b|),
 // with the 1 + e^-d in [1, 2] taken by the hardware exp2 / log2 (absolute error
 // of the correction term ~1e-7, far below fp32 rounding of the running sums).
+// Both -inf: the correction is NaN and the select returns -inf.  A select, not
+// a branch, so that independent calls interleave (a branch per call serialises them).
 __device__ __forceinline__ float log_add_exp(float a, float b) {
-  float m = fmaxf(a, b);
-  if (m == -INFINITY) return -INFINITY;
-  return m + __logf(1.f + __expf(-fabsf(a - b)));
+  const float m = fmaxf(a, b);
+  const float r = m + __logf(1.f + __expf(-fabsf(a - b)));
+  return m == -INFINITY ? m : r;
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

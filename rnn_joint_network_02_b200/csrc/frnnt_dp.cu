@@ -684,16 +684,19 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
 // the diagonal by k or k+1), so one thread again owns one label position u:
 //  * alpha pushes.  Once alpha(t,u) is known the thread adds its blank edges
 //    into a shift register of its own future diagonals (fut[k] = diagonal
-//    s+k) and hands its label edges, one per duration, to thread u+1 (warp
-//    shuffle, shared memory across a warp boundary), which adds them to its
-//    own register one diagonal later.  Only the cell's own log-probs are read.
+//    s+k) and hands its label edges, one per duration, to thread u+1 through
+//    shared memory, which adds them to its own register one diagonal later.
+//    Only the cell's own log-probs are read.
 //  * beta pulls.  The thread keeps its own beta of the last DM+1 diagonals in
 //    a shift register (hist[k] = diagonal s+k) and reads thread u+1's
-//    register for the label edges; (T_len, U_len) after the final blank is a
+//    register (through shared memory) for the label edges; (T_len, U_len) after the final blank is a
 //    virtual cell with beta 0 on diagonal T_len + U_len.  It stores PB / PL
 //    (the blank / label parts of beta) and, per duration, the log posterior
 //    numerator without alpha and log P.
 // DM = the largest duration (1..8): register arrays are indexed by compile-time k.
+// Every thread exchanges through a parity-double-buffered shared array
+// xa[parity][k][thread] (one barrier per step, no shuffles): dynamic shared
+// memory of 2 (DM+2) blockDim floats.
 template <int DM>
 struct TdtOps {
   float bl, ll;
@@ -724,7 +727,7 @@ __device__ __forceinline__ void tdt_operands(TdtOps<DM>& o, bool live, int t, in
 
 constexpr int tdt_prefetch(int DM) { return DM <= 4 ? 4 : 2; }
 
-// MAXT: the block size bound (256 lets the registers hold every array without spilling).
+// MAXT: the block size bound (256 and 512 let the registers hold every array without spilling).
 template <int DM, int MAXT>
 __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dmask, long long plane,
                                                       const float* __restrict__ blank_lp,
@@ -734,11 +737,12 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
                                                       float* __restrict__ q, const int32_t* __restrict__ T_len,
                                                       const int32_t* __restrict__ U_len, float* __restrict__ loss) {
   constexpr int P = tdt_prefetch(DM);
-  __shared__ float xs[2][32][DM + 2];     // [parity][warp][k]: values handed across warp boundaries
+  extern __shared__ float xa[];           // [2][DM+2][blockDim]
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
   const int u = threadIdx.x;
-  const int lane = u & 31, warp = u >> 5, nwarps = blockDim.x >> 5;
+  const int nth = blockDim.x;
+  auto X = [&](int par, int k, int i) -> float& { return xa[(par * (DM + 2) + k) * nth + i]; };
   const Lengths l = lengths_of(T_len, U_len, b, T, U);
   const int Tb = l.Tb, Ub = l.Ub;
   const int Up1 = U + 1;
@@ -755,13 +759,10 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
 
   if (!is_beta) {
     float fut[DM + 1];    // incoming weight of this thread's cell on diagonal s + k
-    float outl[DM + 1];   // this thread's label edges of the previous step, by duration
 #pragma unroll
-    for (int k = 0; k <= DM; ++k) {
-      fut[k] = -INFINITY;
-      outl[k] = -INFINITY;
-    }
-    for (int k = threadIdx.x; k < 2 * 32 * (DM + 2); k += blockDim.x) (&xs[0][0][0])[k] = -INFINITY;
+    for (int k = 0; k <= DM; ++k) fut[k] = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < DM + 2; ++k) X(1, k, u) = -INFINITY;
     __syncthreads();
     for (int s0 = 0; s0 < nsteps; s0 += P) {
 #pragma unroll
@@ -775,8 +776,7 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
 #pragma unroll
         for (int k = 0; k <= DM; ++k) {
           if (!((dmask >> k) & 1u)) continue;
-          float nl = __shfl_up_sync(0xffffffffu, outl[k], 1);
-          if (lane == 0) nl = warp > 0 ? xs[(s + 1) & 1][warp - 1][k] : -INFINITY;
+          const float nl = u > 0 ? X((s + 1) & 1, k, u - 1) : -INFINITY;
           fut[k] = log_add_exp(fut[k], nl);
         }
         const int t = s - u;
@@ -788,11 +788,7 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
         for (int k = 1; k <= DM; ++k)
           if ((dmask >> k) & 1u) fut[k] = log_add_exp(fut[k], v + o.bl + o.dl[k]);
 #pragma unroll
-        for (int k = 0; k <= DM; ++k) outl[k] = v + o.ll + o.dl[k];
-        if (lane == 31) {
-#pragma unroll
-          for (int k = 0; k <= DM; ++k) xs[s & 1][warp][k] = outl[k];
-        }
+        for (int k = 0; k <= DM; ++k) X(s & 1, k, u) = v + o.ll + o.dl[k];
 #pragma unroll
         for (int k = 0; k < DM; ++k) fut[k] = fut[k + 1];
         fut[DM] = -INFINITY;
@@ -804,10 +800,8 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
 #pragma unroll
     for (int k = 0; k < DM + 2; ++k) hist[k] = -INFINITY;
     if (u == Ub) hist[1] = 0.f;           // the virtual cell after the final blank
-    if (lane == 0) {
 #pragma unroll
-      for (int k = 0; k < DM + 2; ++k) xs[1][warp][k] = hist[k];
-    }
+    for (int k = 0; k < DM + 2; ++k) X(1, k, u) = hist[k];
     __syncthreads();
     for (int i0 = 0; i0 < nsteps; i0 += P) {
 #pragma unroll
@@ -823,8 +817,7 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
 #pragma unroll
         for (int k = 0; k <= DM; ++k) {
           // thread u+1's beta on diagonal s + k + 1, i.e. at (t + k, u + 1)
-          float nb = __shfl_down_sync(0xffffffffu, hist[k + 1], 1);
-          if (lane == 31) nb = warp + 1 < nwarps ? xs[(step + 1) & 1][warp + 1][k + 1] : -INFINITY;
+          const float nb = u + 1 < nth ? X((step + 1) & 1, k + 1, u + 1) : -INFINITY;
           const float eb = k >= 1 ? o.bl + o.dl[k] + hist[k] : -INFINITY;
           const float el = (u < Ub && t + k < Tb) ? o.ll + o.dl[k] + nb : -INFINITY;
           pb = log_add_exp(pb, eb);
@@ -848,10 +841,8 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
 #pragma unroll
         for (int k = DM + 1; k >= 2; --k) hist[k] = hist[k - 1];
         hist[1] = valid ? bt : -INFINITY;
-        if (lane == 0) {
 #pragma unroll
-          for (int k = 0; k < DM + 2; ++k) xs[step & 1][warp][k] = hist[k];
-        }
+        for (int k = 0; k < DM + 2; ++k) X(step & 1, k, u) = hist[k];
         __syncthreads();
       }
     }
@@ -862,12 +853,24 @@ template <int DM>
 void launch_tdt_dp_t(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, float* loss,
                      int threads, cudaStream_t st) {
   dim3 grid(s.B, 2);
+  const int smem = 2 * (DM + 2) * threads * (int)sizeof(float);   // <= 80 KB (DM 8, 1024 threads)
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(tdt_dp_kernel<DM, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 256 * 4);
+    cudaFuncSetAttribute(tdt_dp_kernel<DM, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 512 * 4);
+    cudaFuncSetAttribute(tdt_dp_kernel<DM, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 1024 * 4);
+    attr = true;
+  }
   if (threads <= 256)
-    tdt_dp_kernel<DM, 256><<<grid, threads, 0, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
-                                                     L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
+    tdt_dp_kernel<DM, 256><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+                                                        L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
+  else if (threads <= 512)
+    tdt_dp_kernel<DM, 512><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+                                                        L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
   else
-    tdt_dp_kernel<DM, 1024><<<grid, threads, 0, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
-                                                      L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
+    tdt_dp_kernel<DM, 1024><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp,
+                                                         L.dur_lp, L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len,
+                                                         loss);
 }
 
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,

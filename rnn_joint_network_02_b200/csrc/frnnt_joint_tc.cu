@@ -724,7 +724,10 @@ __device__ __forceinline__ void tdt_dzd_row(const JointParams& p, const RowInfo&
   *(uint2*)(out + 4 * lane) = make_uint2(pack_bf16x2(vals[0], vals[1]), pack_bf16x2(vals[2], vals[3]));
 }
 
-__global__ void dz_from_z_kernel(JointParams p) {
+// TDT: also write the duration columns (a separate instantiation, so the
+// transducer's kernel keeps its register count and occupancy).
+template <bool TDT>
+__global__ void __launch_bounds__(256, 4) dz_from_z_kernel(JointParams p) {
   // one warp per row; rows of tiles [tile_begin, ntiles).  A row's z is read
   // in batches of four 16-byte chunks per lane, all loads of a batch issued
   // before any store (the row is rewritten in place).
@@ -738,7 +741,7 @@ __global__ void dz_from_z_kernel(JointParams p) {
     const int tile = p.tile_begin + (int)(row >> 7);
     const RowInfo ri = row_info(p, p.tiles[tile], (int)(row & 127));
     __nv_bfloat16* zr = p.zbuf + (size_t)tile * 128 * ldz + (size_t)(row & 127) * ldz;
-    if (p.n_dur > 0) tdt_dzd_row(p, ri, zr + V, lane);
+    if (TDT) tdt_dzd_row(p, ri, zr + V, lane);
     if (!ri.valid) {
       for (int k = lane * 8; k < V; k += 256) *(uint4*)(zr + k) = make_uint4(0, 0, 0, 0);
       continue;
@@ -1205,7 +1208,8 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.Vx = j.s.Vx;
   p.n_dur = j.s.n_dur;
-  dz_from_z_kernel<<<sms() * 4, 256, 0, st>>>(p);
+  if (p.n_dur > 0) dz_from_z_kernel<true><<<sms() * 4, 256, 0, st>>>(p);
+  else dz_from_z_kernel<false><<<sms() * 4, 256, 0, st>>>(p);
   note_launch();
 }
 

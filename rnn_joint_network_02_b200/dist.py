@@ -65,11 +65,11 @@ def take_shard(tensors: dict, idx: list[int], trim: bool = True) -> dict:
 
 
 def allreduce_weight_grads(grads: dict, group=None) -> dict:
-    """Sums dW_f, dW_g, dW_o, db_o over the ranks of `group` in at least fp32
-    (16-bit gradients are widened for the sum, then rounded back).  df / dg
-    are left as they are."""
+    """Sums dW_f, dW_g, dW_o, db_o (and the duration head's dW_d, db_d when
+    present) over the ranks of `group` in at least fp32 (16-bit gradients are
+    widened for the sum, then rounded back).  df / dg are left as they are."""
     out = dict(grads)
-    for k in WEIGHT_GRADS:
+    for k in WEIGHT_GRADS + tuple(k for k in ("dW_d", "db_d") if k in grads):
         g = grads[k]
         acc = g.float() if g.element_size() < 4 else g.clone()
         dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
@@ -98,11 +98,16 @@ def fwd_bwd_sharded(tensors: dict, compute, rank: int, world: int, group=None, g
     return idx, loss, grads
 
 
-def gpu_compute(mode: str = "tiled", **kw):
-    """The CUDA library as the per-rank compute of fwd_bwd_sharded."""
+def gpu_compute(mode: str = "tiled", durations=None, **kw):
+    """The CUDA library as the per-rank compute of fwd_bwd_sharded (with
+    ``durations``: the token-and-duration transducer, whose duration head
+    W_d / b_d travels in the tensors dict like the other weights)."""
     from . import frnnt
 
     def run(t, w):
+        if durations is not None:
+            return frnnt.fwd_bwd_tdt(t["f"], t["g"], t["W_f"], t["W_g"], t["W_o"], t["b_o"], t["W_d"], t["b_d"],
+                                     t["labels"], t["T_len"], t["U_len"], durations, grad_loss=w, mode=mode, **kw)
         return frnnt.fwd_bwd(t["f"], t["g"], t["W_f"], t["W_g"], t["W_o"], t["b_o"], t["labels"], t["T_len"],
                              t["U_len"], grad_loss=w, mode=mode, **kw)
     return run

@@ -102,3 +102,61 @@ def test_two_gloo_ranks_match_single_process(tmp_path):
             np.testing.assert_allclose(d["grads"]["dg"][j, :Ub + 1].numpy(), ref.dg[b, :Ub + 1], rtol=1e-10,
                                        atol=1e-12)
     assert sorted(seen) == list(range(5))
+
+
+TDT_D = (0, 1, 2)
+
+
+def _tdt_batch():
+    batch = synth.make(B=5, T=7, U=4, D_enc=4, D_pred=3, H=6, V=7, dtype="f32", seed=78, T_range=(2, 7),
+                       U_range=(0, 4), bias_std=0.3)
+    W_d, b_d = synth.duration_head(batch, len(TDT_D), seed=4)
+    return batch, W_d, b_d
+
+
+def _oracle_tdt_compute(shard, w):
+    import oracle
+    f, g, W_f, W_g, W_o, b_o, W_d, b_d = (shard[k].double().numpy()
+                                          for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "W_d", "b_d"))
+    res = oracle.tdt_fwd_bwd(f, g, W_f, W_g, W_o, b_o, W_d, b_d, shard["labels"].numpy(), shard["T_len"].numpy(),
+                             shard["U_len"].numpy(), TDT_D, grad_loss=None if w is None else w.double().numpy())
+    grads = {k: torch.from_numpy(getattr(res, k))
+             for k in ("df", "dg", "dW_f", "dW_g", "dW_o", "db_o", "dW_d", "db_d")}
+    return torch.from_numpy(res.loss), grads
+
+
+def _tdt_worker(rank, world, port, out_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        batch, W_d, b_d = _tdt_batch()
+        t = {k: getattr(batch, k) for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+        t["W_d"], t["b_d"] = W_d, b_d
+        idx, loss, grads = rdist.fwd_bwd_sharded(t, _oracle_tdt_compute, rank, world,
+                                                 grad_loss=torch.linspace(0.5, 1.5, 5))
+        torch.save({"idx": idx, "loss": loss, "grads": grads}, f"{out_path}.{rank}")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_tdt_duration_head_grads_summed(tmp_path):
+    """The token-and-duration transducer's duration-head gradients take part
+    in the weight-gradient exchange like the label head's."""
+    world = 2
+    out = str(tmp_path / "tdt")
+    mp.start_processes(_tdt_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
+    import oracle
+    batch, W_d, b_d = _tdt_batch()
+    f, g, W_f, W_g, W_o, b_o = (x.numpy() for x in batch.float64())
+    ref = oracle.tdt_fwd_bwd(f, g, W_f, W_g, W_o, b_o, W_d.double().numpy(), b_d.double().numpy(),
+                             batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(), TDT_D,
+                             grad_loss=np.linspace(0.5, 1.5, 5))
+    seen = []
+    for r in range(world):
+        d = torch.load(f"{out}.{r}")
+        seen += d["idx"]
+        np.testing.assert_allclose(d["loss"].numpy(), ref.loss[d["idx"]], rtol=1e-12)
+        for k in ("dW_f", "dW_g", "dW_o", "db_o", "dW_d", "db_d"):
+            np.testing.assert_allclose(d["grads"][k].numpy(), getattr(ref, k), rtol=1e-10, atol=1e-12)
+    assert sorted(seen) == list(range(5))
