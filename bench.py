@@ -58,12 +58,13 @@ def parse():
 
 # DRAM bytes (read + write) per launch of a stage's kernel, from one ncu
 # capture of that kernel in the bench's own launch configuration (the file
-# under profiles/ gives the command).  An entry is removed whenever its kernel
-# changes, so the roofline's traffic is null rather than stale.
+# under profiles/ gives the command), keyed by (workload, mode, stage, loss).
+# An entry is removed whenever its kernel changes, so the roofline's traffic is
+# null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dh"): (0.629034e9 + 0.354387e9, "profiles/ncu_gemm_tc_medium_untiled.md"),
-    ("medium", "untiled", "bwd_dWo"): (1.175207e9 + 0.010739e9, "profiles/ncu_gemm2_tc_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd"): (0.009159e9 + 0.570264e9, "profiles/ncu_joint_tc_medium_untiled.md"),
+    ("medium", "untiled", "bwd_dWo", "marginal"): (1.175207e9 + 0.010739e9, "profiles/ncu_gemm2_tc_medium_untiled.md"),
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009159e9 + 0.570264e9,
+                                                     "profiles/ncu_joint_tc_medium_untiled.md"),
 }
 
 
@@ -363,7 +364,7 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         dom = max(stages, key=lambda k: stages[k]["ms"])
         kind, work = stage_work(batch, dom, mode, valid, len(durations))
         per_call_ms = stages[dom]["ms"] / args.steps
-        tr = MEASURED_TRAFFIC.get((args.workload, mode, dom))
+        tr = None if args.prune else MEASURED_TRAFFIC.get((args.workload, mode, dom, args.loss))
         if kind == "tensor":
             achieved = work / (per_call_ms / 1e3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor_sustained"], "unit": "TFLOP/s",

@@ -21,8 +21,9 @@ extern "C" {
  * into out (k_splits >= 1 K slices); 3 = out (bf16, holding h on entry)
  * becomes D * (1 - h*h).  Requires lda, ldb multiples of 8, N a multiple of
  * 32, 16-byte aligned pointers.  variant: -1 automatic, 0 one CTA per 128-row
- * tile, 1 CTA pairs sharing 256-row tiles (cta_group::2).  Returns FRNNT_OK or
- * an FRNNT_ERR_* code. */
+ * tile, 1 CTA pairs sharing 256-row tiles (cta_group::2); 2 / 3 as 0 / 1 with
+ * 256-wide N tiles whatever N (a ragged last tile).  Returns FRNNT_OK or an
+ * FRNNT_ERR_* code. */
 FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn, long long lda,
                                    const void* B, int b_mn, long long ldb, int epi, int k_splits,
                                    void* out, long long ldo, int variant, int32_t* status, void* stream);

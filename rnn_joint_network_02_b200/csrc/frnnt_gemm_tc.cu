@@ -712,9 +712,16 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
       (g.ldo % 8 || !g.out_bf16))
     return FRNNT_ERR_DIMS;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
-  const int BN = (g.N % 256 == 0 && g.N >= 256) ? 256 : 128;
+  // variants 2 / 3: 256-wide N tiles even when N is not a multiple of 256 (the
+  // last tile's missing B rows are zero-filled by TMA; its extra columns are
+  // computed and not stored), one CTA / CTA pairs
+  // (automatic: also for tall GEMMs with N > 512 and N % 256 >= 128, e.g. the
+  // d_hidden GEMM at H = 640, where the wider tiles' halved L2 traffic outweighs
+  // the last tile's extra columns; short ones such as the projections keep 128)
+  const bool wide = (g.N % 256 == 0 && g.N >= 256) || (g.M >= 65536 && g.N > 512 && g.N % 256 >= 128);
+  const int BN = (wide || g.variant >= 2) ? 256 : 128;
   // CTA pairs (M = 256 per MMA) for 256-wide N tiles on problems with enough rows
-  const bool pair = g.variant == 1 || (g.variant < 0 && g.M >= 512 && BN == 256);
+  const bool pair = g.variant == 1 || g.variant == 3 || (g.variant < 0 && g.M >= 512 && BN == 256);
   CUtensorMap ta, tb;
   bool ok;
   if (!g.a_mn) ok = make_tmap_bf16_2d(&ta, g.A, g.K, g.M, (uint64_t)g.lda, 64, 128);

@@ -175,7 +175,8 @@ struct GemmTcArgs {
   // is min(static, (*dyn_count - dyn_base) * dyn_scale), read by the kernel.
   const int* dyn_count = nullptr;
   int dyn_base = 0, dyn_scale = 0, dyn_dim = 0;
-  int variant = -1;    // -1 auto, 0 one CTA per tile (M = 128), 1 CTA pairs (M = 256, cta_group::2)
+  int variant = -1;    // -1 auto, 0 one CTA per tile (M = 128), 1 CTA pairs (M = 256, cta_group::2);
+                       // 2 / 3: as 0 / 1 with 256-wide N tiles also for N not a multiple of 256
   CellMap cells;       // GEMM_EPI_DTANH_FG: out = acc * (1 - h^2), h recomputed from F and G
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);

@@ -24,7 +24,7 @@ extern "C" FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A
   g.out_bf16 = (epi == 1 || epi == 3) ? out : nullptr;
   g.ldo = ldo;
   g.status = status;
-  g.variant = variant < -1 || variant > 1 ? -1 : variant;
+  g.variant = variant < -1 || variant > 3 ? -1 : variant;
   cudaGetLastError();
   return frnnt::gemm_tc(g, (cudaStream_t)stream);
 }

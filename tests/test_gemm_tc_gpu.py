@@ -24,12 +24,13 @@ def _check(out, ref, tol=2e-3):
     assert err.item() <= tol, err.item()
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
 @pytest.mark.parametrize("a_mn", [False, True])
 @pytest.mark.parametrize("b_mn", [False, True])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 256, 128), (296, 640, 520), (1000, 512, 256)])
 def test_store_f32(cuda_ok, a_mn, b_mn, M, N, K, variant):
-    """variant 0: one CTA per 128-row tile; 1: CTA pairs on 256-row tiles (cta_group::2)."""
+    """variant 0: one CTA per 128-row tile; 1: CTA pairs on 256-row tiles (cta_group::2);
+    2 / 3: the same with 256-wide N tiles whatever N (a ragged last tile)."""
     A, B, ref = _operands(M, N, K, a_mn, b_mn)
     out = frnnt.test_gemm_bf16(A, B, a_mn, b_mn, M, N, K, epi=0, variant=variant)
     torch.cuda.synchronize()
@@ -46,7 +47,7 @@ def test_store_bf16(cuda_ok, a_mn, b_mn, variant):
     _check(out, ref, 8e-3)
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
 @pytest.mark.parametrize("splits", [1, 3, 7])
 def test_split_k_reduce(cuda_ok, splits, variant):
     M, N, K = 1024, 640, 4096 + 64
@@ -57,7 +58,7 @@ def test_split_k_reduce(cuda_ok, splits, variant):
     _check(out - 0.5, ref, 1e-5)
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
 def test_dtanh_epilogue(cuda_ok, variant):
     M, N, K = 512, 640, 1024
     A, B, ref = _operands(M, N, K, False, True, seed=3)
@@ -69,7 +70,7 @@ def test_dtanh_epilogue(cuda_ok, variant):
     _check(out, expect, 8e-3)
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
 def test_many_tiles_persistent(cuda_ok, variant):
     """More output tiles than SMs: every CTA walks several tiles and both TMEM buffers."""
     M, N, K = 6400, 640, 512
