@@ -407,20 +407,19 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     {
       StageScope sc("bwd_dh", st);
       GemmTcArgs a{};
-      // d_hidden = dz W_o, then (1 - h^2) in the epilogue, in place over h
+      // d_hidden = dz W_o; the epilogue forms dpre = d_hidden (1 - h^2), with h
+      // recomputed from the L2-resident F and G rows of each cell (not read
+      // back), and sums it into dF (per frame) and dG (per label position):
+      // dpre is never stored
       // (token-and-duration transducer: dz | dzd against [W_o; W_d], K = V + 64)
       a.M = rows; a.N = s.H; a.K = tdt ? s.V + 64 : s.V; a.A = zrows; a.a_mn = false; a.lda = s.Vx;
-      a.B = tdt ? (const void*)p.Wx : W_o; a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH_FG; a.k_splits = 1; a.out_bf16 = hrows; a.ldo = HS; a.status = status;
-      // (1 - h^2) with h recomputed from the L2-resident F and G rows of each cell, not read back
+      a.B = tdt ? (const void*)p.Wx : W_o; a.b_mn = true; a.ldb = s.H; a.epi = GEMM_EPI_DTANH_SEG; a.k_splits = 1;
+      a.status = status;
       a.cells.tiles = p.tiles; a.cells.tile0 = (int)c0; a.cells.T = s.T; a.cells.U = s.U; a.cells.H = s.H;
       a.cells.UB = p.UB; a.cells.S = s.S; a.cells.bounds = bounds; a.cells.T_len = T_len; a.cells.U_len = U_len;
-      a.cells.F = p.F; a.cells.G = p.G;
+      a.cells.F = p.F; a.cells.G = p.G; a.cells.dF = p.dF; a.cells.dG = p.dG;
       a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
       FRNNT_TRY(gemm_tc(a, st));
-    }
-    {
-      StageScope sc("bwd_seg_reduce", st);
-      launch_seg_reduce(j, hrows, (int)c0, p.dF, p.dG, st);
     }
   }
   {

@@ -181,6 +181,129 @@ __device__ __forceinline__ FgRows fg_rows(const CellMap& m, int row) {
   }
   return fr;
 }
+// Fused segment reduction (GEMM_EPI_DTANH_SEG).  The rows of a 128-row M tile
+// are one cell tile: row r = frame t0 + r / UB and label (or band) position
+// r % UB, so the UB consecutive lanes of a warp share a frame and, on the whole
+// lattice, lanes UB apart share a label position.  A 32-column chunk of dpre is
+// summed over a frame's lanes by recursive halving (each lane ends with 32/UB
+// columns of the frame's sum) and over a label position's lanes likewise (UB
+// columns each), then added to dF / dG with vector reductions.  On a pruned
+// lattice the label positions differ per frame: every cell adds its own dG row.
+struct SegRow {
+  const __nv_bfloat16* f;   // F and G rows of the cell (null: no lattice cell, dpre = 0)
+  const __nv_bfloat16* g;
+  float* df;                // dF row of the lane's frame (null: the frame is outside the utterance)
+  float* dg;                // dG row of the lane's label position (null: outside, or no cell when pruned)
+};
+__device__ __forceinline__ SegRow seg_row(const CellMap& m, int row, bool row_ok) {
+  SegRow s{nullptr, nullptr, nullptr, nullptr};
+  if (!row_ok) return s;
+  const int4 td = m.tiles[m.tile0 + (row >> 7)];
+  const int r = row & 127;
+  const int b = td.x, t = td.y + r / m.UB;
+  const int Tb = clampi(m.T_len[b], 1, m.T), Ub = clampi(m.U_len[b], 0, m.U);
+  int u;
+  bool uok;
+  if (m.S) {
+    const int j = r % m.UB;
+    u = clampi(m.bounds[(size_t)b * m.T + min(t, Tb - 1)], 0, m.U) + j;
+    uok = j < m.S && u <= Ub;
+  } else {
+    u = td.z + r % m.UB;
+    uok = u <= Ub;
+  }
+  const bool tok = t < Tb;
+  if (tok) s.df = m.dF + ((size_t)b * m.T + t) * m.H;
+  if (uok && (m.S == 0 || tok)) s.dg = m.dG + ((size_t)b * (m.U + 1) + u) * m.H;
+  if (tok && uok) {
+    s.f = (const __nv_bfloat16*)m.F + ((size_t)b * m.T + t) * m.H;
+    s.g = (const __nv_bfloat16*)m.G + ((size_t)b * (m.U + 1) + u) * m.H;
+  }
+  return s;
+}
+
+// One recursive-halving level over lanes s apart: of the first N values a
+// lane keeps the upper half when (lane & s), the lower one otherwise, plus
+// its partner's copy of that half.
+template <int N>
+__device__ __forceinline__ void rs_level(float (&v)[32], int s, bool upper) {
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float give = upper ? v[i] : v[i + N / 2];
+    const float keep = upper ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, give, s);
+  }
+}
+// Sum over each group of G consecutive lanes: v[0 .. 32/G) becomes the sum of
+// columns (32/G) (lane % G) + i.
+template <int G, int N = 32>
+__device__ __forceinline__ void rs_within(float (&v)[32], int lane) {
+  if constexpr (G > 1) {
+    rs_level<N>(v, G / 2, (lane & (G / 2)) != 0);
+    rs_within<G / 2, N / 2>(v, lane);
+  }
+}
+// Sum over the lanes congruent modulo G: v[0 .. G) becomes the sum of columns G (lane / G) + i.
+template <int G, int S = 16, int N = 32>
+__device__ __forceinline__ void rs_across(float (&v)[32], int lane) {
+  if constexpr (S >= G) {
+    rs_level<N>(v, S, (lane & S) != 0);
+    rs_across<G, S / 2, N / 2>(v, lane);
+  }
+}
+template <int NV>
+__device__ __forceinline__ void red_add_n(float* dst, const float (&v)[32]) {
+  if constexpr (NV == 1) {
+    red_add_f32(dst, v[0]);
+  } else if constexpr (NV == 2) {
+    red_add_v2(dst, v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NV; i += 4) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+  }
+}
+template <int G>
+__device__ __forceinline__ void seg_chunk_g(const CellMap& m, const SegRow& sr, int col0, const float (&d)[32],
+                                            int lane) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = d[i];
+  rs_within<G>(v, lane);
+  if (sr.df) red_add_n<32 / G>(sr.df + col0 + (32 / G) * (lane & (G - 1)), v);
+  if constexpr (G < 32) {
+    if (m.S == 0) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = d[i];
+      rs_across<G>(v, lane);
+      if (sr.dg) red_add_n<G>(sr.dg + col0 + G * (lane / G), v);
+      return;
+    }
+  }
+  if (sr.dg) red_add_n<32>(sr.dg + col0, d);
+}
+// dpre = acc (1 - h^2) of the lane's row (0 when it is no cell), then the sums.
+// Every lane of the warp calls this for the same chunk (the shuffles need all).
+__device__ __forceinline__ void seg_chunk(const CellMap& m, const SegRow& sr, int col0, const uint32_t (&r)[32],
+                                          const uint4 (&hv4)[4], int lane) {
+  float d[32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t hw[4] = {hv4[j].x, hv4[j].y, hv4[j].z, hv4[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[q]));
+      d[8 * j + 2 * q] = sr.f ? __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x) : 0.f;
+      d[8 * j + 2 * q + 1] = sr.f ? __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y) : 0.f;
+    }
+  }
+  switch (m.UB) {
+    case 4: seg_chunk_g<4>(m, sr, col0, d, lane); break;
+    case 8: seg_chunk_g<8>(m, sr, col0, d, lane); break;
+    case 16: seg_chunk_g<16>(m, sr, col0, d, lane); break;
+    default: seg_chunk_g<32>(m, sr, col0, d, lane); break;
+  }
+}
+
 __device__ __forceinline__ uint32_t tanh_bf16x2_g(uint32_t x) {
   uint32_t y;
   asm("tanh.approx.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
@@ -366,7 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < eff.M;
       if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
       const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
-      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
+      if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
 #pragma unroll 1
       for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
@@ -376,8 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) h_from_fg(FgRows{sr.f, sr.g}, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
+        if (p.epi == GEMM_EPI_DTANH_SEG) {
+          if (col0 < p.N) seg_chunk(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
+          continue;
+        }
         if (!st) continue;
         if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
         else epilogue_store(p, row, col0, r);
@@ -580,7 +709,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < eff.M;
       if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
       const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
-      if (!mbar_wait(&tfull[a], aph, abort_flag)) break;
+      const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
+      if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
 #pragma unroll 1
       for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
@@ -590,8 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) h_from_fg(FgRows{sr.f, sr.g}, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
+        if (p.epi == GEMM_EPI_DTANH_SEG) {
+          if (col0 < p.N) seg_chunk(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
+          continue;
+        }
         if (!st) continue;
         if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
         else epilogue_store(p, row, col0, r);
@@ -710,6 +845,8 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   if ((g.epi == GEMM_EPI_STORE_F32 || g.epi == GEMM_EPI_RED_F32) && (g.ldo % 4 || !g.out_f32)) return FRNNT_ERR_DIMS;
   if ((g.epi == GEMM_EPI_STORE_BF16 || g.epi == GEMM_EPI_DTANH || g.epi == GEMM_EPI_DTANH_FG) &&
       (g.ldo % 8 || !g.out_bf16))
+    return FRNNT_ERR_DIMS;
+  if (g.epi == GEMM_EPI_DTANH_SEG && (!g.cells.tiles || !g.cells.F || !g.cells.G || !g.cells.dF || !g.cells.dG))
     return FRNNT_ERR_DIMS;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.out_f32 | (uintptr_t)g.out_bf16) & 15u) return FRNNT_ERR_ALIGN;
   // variants 2 / 3: 256-wide N tiles even when N is not a multiple of 256 (the

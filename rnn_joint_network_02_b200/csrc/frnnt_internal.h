@@ -142,7 +142,7 @@ void launch_dtanh_reduce_simt(const Shape& s, const float* dh, const float* h, l
 // D[M,N] = A[M,K] * B[K,N] in bf16 with fp32 accumulation (tcgen05, TMA).
 // A: K-major [M][lda] or MN-major [K][lda]; B: K-major [N][ldb] or MN-major [K][ldb].
 enum GemmEpilogue { GEMM_EPI_STORE_F32 = 0, GEMM_EPI_STORE_BF16 = 1, GEMM_EPI_RED_F32 = 2, GEMM_EPI_DTANH = 3,
-                    GEMM_EPI_DTANH_FG = 4 };
+                    GEMM_EPI_DTANH_FG = 4, GEMM_EPI_DTANH_SEG = 5 };
 
 // Lattice cells behind the rows of a GEMM whose 128-row M tiles are cell tiles
 // (row m of the GEMM = row m % 128 of cell tile tile0 + m / 128), for the
@@ -156,6 +156,8 @@ struct CellMap {
   const int32_t* U_len = nullptr;
   const void* F = nullptr;        // [B*T][H] bf16
   const void* G = nullptr;        // [B*(U+1)][H] bf16
+  float* dF = nullptr;            // GEMM_EPI_DTANH_SEG: [B*T][H] fp32, += sum over each frame's cells
+  float* dG = nullptr;            //                     [B*(U+1)][H] fp32, += sum over each label position's cells
 };
 struct GemmTcArgs {
   int M, N, K;
@@ -177,7 +179,8 @@ struct GemmTcArgs {
   int dyn_base = 0, dyn_scale = 0, dyn_dim = 0;
   int variant = -1;    // -1 auto, 0 one CTA per tile (M = 128), 1 CTA pairs (M = 256, cta_group::2);
                        // 2 / 3: as 0 / 1 with 256-wide N tiles also for N not a multiple of 256
-  CellMap cells;       // GEMM_EPI_DTANH_FG: out = acc * (1 - h^2), h recomputed from F and G
+  CellMap cells;       // GEMM_EPI_DTANH_FG: out = acc * (1 - h^2), h recomputed from F and G;
+                       // GEMM_EPI_DTANH_SEG: the same dpre summed into cells.dF / cells.dG, nothing stored
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
 
@@ -231,7 +234,6 @@ void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const 
                         void* b_x, cudaStream_t st);
 // blocks_per_sm: 256-thread blocks per SM of the grid (fewer leave room for work running beside it)
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
-void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st);
 void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st);
 
 // out[i] = (dtype) in[i]

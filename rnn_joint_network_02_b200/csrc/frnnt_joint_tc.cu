@@ -871,112 +871,6 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
   }
 }
 
-// ------------------------------------------------------------------ dtanh'd hidden gradient -> dF, dG
-// dpre rows of the tiles in [tile_begin, ntiles) (bf16, rows (tile - row_tile0) * 128 + r):
-// dF[b, t] += sum over the tile's u of dpre, dG[b, u] += sum over the tile's t.
-__global__ void seg_reduce_kernel(JointParams p, const __nv_bfloat16* __restrict__ dpre, int row_tile0, float* dF,
-                                  float* dG) {
-  const int ntiles = min(p.tile_end, *p.ntiles);
-  const int tile = p.tile_begin + blockIdx.x;
-  if (tile >= ntiles) return;
-  const int4 td = p.tiles[tile];
-  const int H = p.H, TB = p.TB, UB = p.UB, Up1 = p.U + 1;
-  const Lengths l = lengths_of(p.T_len, p.U_len, td.x, p.T, p.U);
-  const int HS = p.HS;
-  const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * HS;
-  // thread (c8, g): 8 consecutive columns, frame rows tl = g (mod 4) for dF and
-  // label rows ul = g (mod 4) for dG; rows are loaded four at a time before
-  // they are added, and rows outside the utterance are skipped
-  const int g = threadIdx.y;
-  const int nt = min(TB, l.Tb - td.y), nu = min(UB, l.Ub + 1 - td.z);
-  auto add8 = [](float (&acc)[8], const uint4 v) {
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
-      acc[2 * q] += f.x;
-      acc[2 * q + 1] += f.y;
-    }
-  };
-  for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
-    const __nv_bfloat16* col = base + c8 * 8;
-    for (int tl = g; tl < nt; tl += 4) {
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int u0 = 0; u0 < nu; u0 += 4) {
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          v[i] = u0 + i < nu ? *(const uint4*)(col + (size_t)(tl * UB + u0 + i) * HS) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) add8(acc, v[i]);
-      }
-      float* dst = dF + ((size_t)td.x * p.T + td.y + tl) * H + c8 * 8;
-      red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
-      red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
-    }
-    for (int ul = g; ul < nu; ul += 4) {
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int t0 = 0; t0 < nt; t0 += 4) {
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          v[i] = t0 + i < nt ? *(const uint4*)(col + (size_t)((t0 + i) * UB + ul) * HS) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) add8(acc, v[i]);
-      }
-      float* dst = dG + ((size_t)td.x * Up1 + td.z + ul) * H + c8 * 8;
-      red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
-      red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
-    }
-  }
-}
-
-// Pruned lattice: tile row r is band position j = r % UB of frame t = t0 + r / UB,
-// label position u = bounds[b,t] + j.  dF[b,t] += sum over the frame's valid
-// positions; dG[b,u] += every valid row (u differs per frame, so per row).
-__global__ void seg_reduce_band_kernel(JointParams p, const __nv_bfloat16* __restrict__ dpre, int row_tile0,
-                                       float* dF, float* dG) {
-  const int ntiles = min(p.tile_end, *p.ntiles);
-  const int tile = p.tile_begin + blockIdx.x;
-  if (tile >= ntiles) return;
-  const int4 td = p.tiles[tile];
-  const int H = p.H, UB = p.UB, TB = p.TB, Up1 = p.U + 1, HS = p.HS;
-  const Lengths l = lengths_of(p.T_len, p.U_len, td.x, p.T, p.U);
-  const __nv_bfloat16* base = dpre + (size_t)(tile - row_tile0) * 128 * HS;
-  const int nt = min(TB, l.Tb - td.y);
-  const int g = threadIdx.y;
-  for (int c8 = threadIdx.x; c8 * 8 < H; c8 += blockDim.x) {
-    const __nv_bfloat16* col = base + c8 * 8;
-    for (int tl = g; tl < nt; tl += 4) {
-      const int t = td.y + tl;
-      const int st = clampi(p.bounds[(size_t)td.x * p.T + t], 0, p.U);
-      const int nj = min(p.S, l.Ub - st + 1);      // band positions of this frame inside the utterance
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int j = 0; j < nj; ++j) {
-        const uint4 v = *(const uint4*)(col + (size_t)(tl * UB + j) * HS);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        float row[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
-          row[2 * q] = f.x;
-          row[2 * q + 1] = f.y;
-          acc[2 * q] += f.x;
-          acc[2 * q + 1] += f.y;
-        }
-        float* dg = dG + ((size_t)td.x * Up1 + st + j) * H + c8 * 8;
-        red_add_v4(dg, row[0], row[1], row[2], row[3]);
-        red_add_v4(dg + 4, row[4], row[5], row[6], row[7]);
-      }
-      if (nj > 0) {
-        float* dst = dF + ((size_t)td.x * p.T + t) * H + c8 * 8;
-        red_add_v4(dst, acc[0], acc[1], acc[2], acc[3]);
-        red_add_v4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
-      }
-    }
-  }
-}
-
 // dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
 // whose column H is the sum of dz over cells.
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, __nv_bfloat16* __restrict__ dW_o,
@@ -1268,33 +1162,6 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   p.S = j.s.S;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
   hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
-  note_launch();
-}
-
-void launch_seg_reduce(const JointLaunch& j, const void* dpre, int row_tile0, float* dF, float* dG, cudaStream_t st) {
-  JointParams p{};
-  p.T = j.s.T;
-  p.U = j.s.U;
-  p.H = j.s.H;
-  p.TB = j.TB;
-  p.UB = j.UB;
-  p.T_len = j.T_len;
-  p.U_len = j.U_len;
-  p.tiles = j.tiles;
-  p.ntiles = j.ntiles;
-  p.tile_begin = j.tile_begin;
-  p.tile_end = j.tile_end;
-  p.bounds = j.bounds;
-  p.S = j.s.S;
-  p.HS = hidden_stride(j.s.H);
-  const int n = j.tile_end - j.tile_begin;
-  if (n <= 0) return;
-  int threads = (p.H / 8 + 31) / 32 * 32;
-  if (threads > 128) threads = 128;
-  if (p.S)
-    seg_reduce_band_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
-  else
-    seg_reduce_kernel<<<n, dim3(threads, 4), 0, st>>>(p, (const __nv_bfloat16*)dpre, row_tile0, dF, dG);
   note_launch();
 }
 

@@ -315,6 +315,12 @@ __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gaddr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
+__device__ __forceinline__ void red_add_v2(float* gaddr, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(gaddr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float* gaddr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(gaddr), "f"(a) : "memory");
+}
 
 }  // namespace sm100
 }  // namespace frnnt
