@@ -269,7 +269,8 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
 // serialise their side work.
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;     // hidden rows beside the lattice DP
+  cudaEvent_t fork2 = nullptr, join2 = nullptr;   // the G-side projection backward beside the F side
   bool ok = false;
 };
 
@@ -281,7 +282,9 @@ SideStream* side_stream() {
   if (!x.ok && !x.s) {
     if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) == cudaSuccess &&
         cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
-        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess)
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&x.fork2, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&x.join2, cudaEventDisableTiming) == cudaSuccess)
       x.ok = true;
     else
       cudaGetLastError();
@@ -314,17 +317,22 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   } while (0)
   {
     StageScope sc("validate", st);
-    launch_validate(s, labels, T_len, U_len, bounds, status, st);
-    launch_tiles(s, p.TB, p.UB, T_len, U_len, p.tiles, p.ntiles, st);
-    cudaMemsetAsync(p.dF, 0, s.BT * s.H * sizeof(float), st);
-    cudaMemsetAsync(p.dG, 0, s.BU * s.H * sizeof(float), st);
-    cudaMemsetAsync(p.accWo, 0, (size_t)s.V * hidden_stride(s.H) * sizeof(float), st);
-    cudaMemsetAsync(p.accWf, 0, (size_t)s.Dx * s.H * sizeof(float), st);
-    cudaMemsetAsync(p.accWg, 0, (size_t)s.Dy * s.H * sizeof(float), st);
-    if (tdt) {
-      cudaMemsetAsync(p.accWd, 0, (size_t)64 * hidden_stride(s.H) * sizeof(float), st);
-      launch_tdt_weights(s, W_o, b_o, W_d, b_d, p.Wx, p.bx, st);
-    }
+    // validation, tile list and cleared accumulators in one launch
+    ZeroList z{};
+    auto add = [&](float* ptr, long long n) {
+      z.ptr[z.count] = ptr;
+      z.n[z.count] = n;
+      ++z.count;
+    };
+    add(p.dF, s.BT * s.H);
+    add(p.dG, s.BU * s.H);
+    add(p.accWo, (long long)s.V * hidden_stride(s.H));
+    add(p.accWf, (long long)s.Dx * s.H);
+    add(p.accWg, (long long)s.Dy * s.H);
+    if (tdt) add(p.accWd, 64LL * hidden_stride(s.H));
+    launch_prologue(s, p.TB, p.UB, labels, T_len, U_len, status, p.tiles, p.ntiles, z, st);
+    if (s.S > 0) launch_validate_bounds(s, bounds, T_len, U_len, status, st);
+    if (tdt) launch_tdt_weights(s, W_o, b_o, W_d, b_d, p.Wx, p.bx, st);
   }
   {
     StageScope sc("projection", st);
@@ -424,28 +432,42 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   }
   {
     StageScope sc("projection_bwd", st);
+    // the G side (dg, dW_g) runs on the side stream beside the F side (df,
+    // dW_f); forked from and joined back to the caller's stream by events
+    SideStream* ps = side_stream();
+    cudaStream_t gs = ps ? ps->s : st;
+    if (ps) {
+      cudaEventRecord(ps->fork2, st);
+      cudaStreamWaitEvent(gs, ps->fork2, 0);
+    }
     launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st);
     if (tdt) launch_wo_finalize(p.accWd, s.n_dur, s.H, dW_d, db_d, st);
     launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
-    launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, st);
+    launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, gs);
     GemmTcArgs a{};
     // df = dF W_f^T : B = W_f read as K-major [D_enc][H]
     a.M = (int)s.BT; a.N = s.Dx; a.K = s.H; a.A = p.dFb; a.a_mn = false; a.lda = s.H; a.B = W_f; a.b_mn = false;
     a.ldb = s.H; a.epi = GEMM_EPI_STORE_BF16; a.k_splits = 1; a.out_bf16 = df; a.ldo = s.Dx; a.status = status;
-    FRNNT_TRY(gemm_tc(a, st));
+    int rc_f = gemm_tc(a, st);
     a.M = (int)s.BU; a.N = s.Dy; a.A = p.dGb; a.B = W_g; a.out_bf16 = dg; a.ldo = s.Dy;
-    FRNNT_TRY(gemm_tc(a, st));
+    int rc_g = gemm_tc(a, gs);
     // dW_f = f^T dF : A = f read as MN-major [BT][D_enc], B = dF MN-major [BT][H]
     GemmTcArgs w{};
     w.M = s.Dx; w.N = s.H; w.K = (int)s.BT; w.A = f; w.a_mn = true; w.lda = s.Dx; w.B = p.dFb; w.b_mn = true;
     w.ldb = s.H; w.epi = GEMM_EPI_RED_F32; w.k_splits = splits_for(s.Dx, s.H, (int)s.BT); w.out_f32 = p.accWf;
     w.ldo = s.H; w.status = status;
-    FRNNT_TRY(gemm_tc(w, st));
+    if (rc_f == FRNNT_OK) rc_f = gemm_tc(w, st);
     w.M = s.Dy; w.K = (int)s.BU; w.A = g; w.lda = s.Dy; w.B = p.dGb; w.k_splits = splits_for(s.Dy, s.H, (int)s.BU);
     w.out_f32 = p.accWg;
-    FRNNT_TRY(gemm_tc(w, st));
+    if (rc_g == FRNNT_OK) rc_g = gemm_tc(w, gs);
     launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, true, st);
-    launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, true, st);
+    launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, true, gs);
+    if (ps) {   // joined on every path, so the caller's stream never runs ahead of the side work
+      cudaEventRecord(ps->join2, gs);
+      cudaStreamWaitEvent(st, ps->join2, 0);
+    }
+    FRNNT_TRY(rc_f);
+    FRNNT_TRY(rc_g);
   }
 #undef FRNNT_TRY
   return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;

@@ -23,6 +23,28 @@ __device__ inline Lengths lengths_of(const int32_t* T_len, const int32_t* U_len,
   l.Ub = clampi(U_len[b], 0, U);
   return l;
 }
+// Status bits found by one thread of a block that checks the lengths and
+// labels (strided by nthreads): FRNNT_STATUS_LENGTH for T_len outside [1,T] or
+// U_len outside [0,U], FRNNT_STATUS_LABEL for a label (u < U_len) outside
+// [0,V) or equal to blank.
+__device__ inline int validate_bits(int B, int T, int U, int V, int blank, const int32_t* labels,
+                                    const int32_t* T_len, const int32_t* U_len, int tid, int nthreads) {
+  int bits = 0;
+  for (int b = tid; b < B; b += nthreads) {
+    const int tl = T_len[b], ul = U_len[b];
+    if (tl < 1 || tl > T || ul < 0 || ul > U) bits |= FRNNT_STATUS_LENGTH;
+  }
+  const long long n = (long long)B * U;
+  for (long long i = tid; i < n; i += nthreads) {
+    const int b = (int)(i / U), u = (int)(i % U);
+    const int tl = T_len[b], ul = U_len[b];
+    if (tl < 1 || tl > T || ul < 0 || ul > U) continue;   // length already flagged
+    if (u >= ul) continue;                                // padding label
+    const int y = labels[i];
+    if (y < 0 || y >= V || y == blank) bits |= FRNNT_STATUS_LABEL;
+  }
+  return bits;
+}
 __device__ inline int label_of(const int32_t* labels, int b, int u, int U, int V) {
   return clampi(labels[(size_t)b * U + u], 0, V - 1);
 }

@@ -24,20 +24,7 @@ namespace frnnt {
 __global__ void validate_kernel(int B, int T, int U, int V, int blank, const int32_t* __restrict__ labels,
                                 const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
                                 int32_t* __restrict__ status) {
-  int bits = 0;
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    int tl = T_len[b], ul = U_len[b];
-    if (tl < 1 || tl > T || ul < 0 || ul > U) bits |= FRNNT_STATUS_LENGTH;
-  }
-  long long n = (long long)B * U;
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-    int b = (int)(i / U), u = (int)(i % U);
-    int tl = T_len[b], ul = U_len[b];
-    if (tl < 1 || tl > T || ul < 0 || ul > U) continue;   // length already flagged
-    if (u >= ul) continue;                                // padding label
-    int y = labels[i];
-    if (y < 0 || y >= V || y == blank) bits |= FRNNT_STATUS_LABEL;
-  }
+  int bits = validate_bits(B, T, U, V, blank, labels, T_len, U_len, threadIdx.x, blockDim.x);
   bits = __reduce_or_sync(0xffffffffu, bits);
   if ((threadIdx.x & 31) == 0 && bits) atomicOr(status, bits);
 }
@@ -67,6 +54,14 @@ __global__ void validate_bounds_kernel(int B, int T, int U, int S, const int32_t
   }
   bad = __reduce_or_sync(0xffffffffu, bad);
   if ((threadIdx.x & 31) == 0 && bad) atomicOr(status, FRNNT_STATUS_BOUNDS);
+}
+
+void launch_validate_bounds(const Shape& s, const int32_t* bounds, const int32_t* T_len, const int32_t* U_len,
+                            int32_t* status, cudaStream_t st) {
+  const long long n = (long long)s.B * s.T;
+  const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+  validate_bounds_kernel<<<blocks, 256, 0, st>>>(s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
+  note_launch();
 }
 
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
@@ -119,9 +114,9 @@ __device__ __forceinline__ void dp_operands(bool is_beta, int step, int ndiag, i
 //                    beta(t+1,u+1) + lae(b(t,u) + l(t+1,u), l(t,u) + b(t,u+1)),
 //                    beta(t,u+2)   + l(t,u) + l(t,u+1)).
 // A thread owns label position u; the values of u-1, u-2 (alpha) or u+1, u+2
-// (beta) on the previous diagonal pair come by shuffles, across a warp
-// boundary through shared memory.  The six log-probabilities of a step are
-// fetched kPrefetch2 steps ahead.
+// (beta) on the previous diagonal pair come through a parity-double-buffered
+// shared array with one entry per thread (one barrier per step, no shuffles).
+// The six log-probabilities of a step are fetched kPrefetch2 steps ahead.
 constexpr int kPrefetch2 = 4;
 
 struct DpOps {
@@ -167,11 +162,11 @@ __device__ __forceinline__ float lae3(float a, float b, float c) { return log_ad
 __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
                            float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
                            const int32_t* __restrict__ U_len, float* __restrict__ loss) {
-  __shared__ float xs[2][32][2];    // [parity][warp][edge lane]: values handed across warp boundaries
+  __shared__ float xa[2][1024];     // [parity][thread]: each thread's value on the last far diagonal
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
   const int u = threadIdx.x;
-  const int lane = u & 31, warp = u >> 5, nwarps = blockDim.x >> 5;
+  const int nth = blockDim.x;
   const Lengths l = lengths_of(T_len, U_len, b, T, U);
   const int Tb = l.Tb, Ub = l.Ub;
   const int Up1 = U + 1;
@@ -199,12 +194,8 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
   for (int i = 0; i < kPrefetch2; ++i)
     q[i] = dp2_operands(is_beta, i, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
 
-  // parity 1 holds the first diagonal's edge values
-  if (!is_beta) {
-    if (lane >= 30) xs[1][warp][lane - 30] = cur;
-  } else {
-    if (lane < 2) xs[1][warp][lane] = cur;
-  }
+  // parity 1 holds the first diagonal
+  xa[1][u] = cur;
   __syncthreads();
 
   for (int step0 = 0; step0 < nsteps; step0 += kPrefetch2) {
@@ -217,23 +208,11 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
       const int par = (step + 1) & 1;       // parity holding the previous pair's edge values
       float n1, n2;                          // neighbours at distance 1 and 2 on the previous far diagonal
       if (!is_beta) {
-        n1 = __shfl_up_sync(0xffffffffu, cur, 1);
-        n2 = __shfl_up_sync(0xffffffffu, cur, 2);
-        if (lane == 0) {
-          n1 = warp > 0 ? xs[par][warp - 1][1] : -INFINITY;
-          n2 = warp > 0 ? xs[par][warp - 1][0] : -INFINITY;
-        } else if (lane == 1) {
-          n2 = warp > 0 ? xs[par][warp - 1][1] : -INFINITY;
-        }
+        n1 = u >= 1 ? xa[par][u - 1] : -INFINITY;
+        n2 = u >= 2 ? xa[par][u - 2] : -INFINITY;
       } else {
-        n1 = __shfl_down_sync(0xffffffffu, cur, 1);
-        n2 = __shfl_down_sync(0xffffffffu, cur, 2);
-        if (lane == 31) {
-          n1 = warp + 1 < nwarps ? xs[par][warp + 1][0] : -INFINITY;
-          n2 = warp + 1 < nwarps ? xs[par][warp + 1][1] : -INFINITY;
-        } else if (lane == 30) {
-          n2 = warp + 1 < nwarps ? xs[par][warp + 1][0] : -INFINITY;
-        }
+        n1 = u + 1 < nth ? xa[par][u + 1] : -INFINITY;
+        n2 = u + 2 < nth ? xa[par][u + 2] : -INFINITY;
       }
       float v1 = -INFINITY, v2 = -INFINITY;
       if (in_u) {
@@ -269,11 +248,7 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
       // when the far one is past the lattice's end)
       const bool far_exists = is_beta ? (last - 2 * step - 2 >= 0) : (2 * step + 2 <= last);
       cur = far_exists ? v2 : v1;
-      if (!is_beta) {
-        if (lane >= 30) xs[step & 1][warp][lane - 30] = cur;
-      } else {
-        if (lane < 2) xs[step & 1][warp][lane] = cur;
-      }
+      xa[step & 1][u] = cur;
       __syncthreads();
     }
   }

@@ -110,6 +110,8 @@ __device__ __forceinline__ void edge_posteriors(const Lattice& L, size_t c, size
 // ---------------------------------------------------------------- validation / DP
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
                      const int32_t* bounds, int32_t* status, cudaStream_t st);
+void launch_validate_bounds(const Shape& s, const int32_t* bounds, const int32_t* T_len, const int32_t* U_len,
+                            int32_t* status, cudaStream_t st);
 // bounds: the pruned lattice's per-frame starts (s.S > 0), else null
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
                float* loss, cudaStream_t st);
@@ -219,8 +221,17 @@ void tile_shape(int U, int* TB, int* UB);
 // lattice TB frames x (S rounded up to a power of two) band positions.
 void tile_shape_of(const Shape& s, int* TB, int* UB);
 long long max_tiles(const Shape& s, int TB, int UB);
-void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
-                  cudaStream_t st);
+// Regions of fp32 accumulators to clear (16-byte aligned, a multiple of 4 floats each).
+struct ZeroList {
+  float* ptr[8];
+  long long n[8];
+  int count;
+};
+// One launch: the length / label validation (status bits), the tile list and
+// the clearing of the accumulators in `z`.
+void launch_prologue(const Shape& s, int TB, int UB, const int32_t* labels, const int32_t* T_len,
+                     const int32_t* U_len, int32_t* status, int4* tiles, int* ntiles, const ZeroList& z,
+                     cudaStream_t st);
 int launch_joint_tc(const JointLaunch& j, cudaStream_t st);
 // Joint kernel variant for later calls: -1 automatic, 0 one CTA per cell tile, 1 CTA pairs; returns the previous one.
 int set_joint_variant(int variant);

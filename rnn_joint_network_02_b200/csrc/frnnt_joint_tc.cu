@@ -662,36 +662,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
 }
 
 // ------------------------------------------------------------------ tile list
-// Tiles of utterance b: ceil(T_len/TB) x ceil((U_len+1)/UB) blocks, u-blocks fastest.
-// (pruned: one tile per TB frames, its UB rows per frame being band positions)
-__global__ void tiles_kernel(int B, int T, int U, int TB, int UB, int pruned, const int32_t* __restrict__ T_len,
-                             const int32_t* __restrict__ U_len, int4* __restrict__ tiles, int* __restrict__ ntiles) {
-  __shared__ int offs[1025];
-  __shared__ int counts[1024];
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const Lengths l = lengths_of(T_len, U_len, b, T, U);
-    counts[b] = ((l.Tb + TB - 1) / TB) * (pruned ? 1 : (l.Ub + 1 + UB - 1) / UB);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int b = 0; b < B; ++b) {
-      offs[b] = acc;
-      acc += counts[b];
-    }
-    offs[B] = acc;
-    *ntiles = acc;
-  }
-  __syncthreads();
-  for (int b = 0; b < B; ++b) {
-    const Lengths l = lengths_of(T_len, U_len, b, T, U);
-    const int nu = pruned ? 1 : (l.Ub + 1 + UB - 1) / UB;
-    for (int i = threadIdx.x; i < counts[b]; i += blockDim.x) {
-      const int it = i / nu, iu = i % nu;
-      tiles[offs[b] + i] = make_int4(b, it * TB, iu * UB, 0);
-    }
-  }
-}
+// Tiles of utterance b: ceil(T_len/TB) x ceil((U_len+1)/UB) blocks, u-blocks fastest
+// (pruned: one tile per TB frames, its UB rows per frame being band positions);
+// built by prologue_kernel below.
 
 // ------------------------------------------------------------------ untiled backward: dz from stored z
 // Token-and-duration transducer: the duration-head logit gradient of the cell
@@ -1013,9 +986,64 @@ long long max_tiles(const Shape& s, int TB, int UB) {
   return (long long)s.B * ((s.T + TB - 1) / TB) * (s.S > 0 ? 1 : (s.Up1 + UB - 1) / UB);
 }
 
-void launch_tiles(const Shape& s, int TB, int UB, const int32_t* T_len, const int32_t* U_len, int4* tiles, int* ntiles,
-                  cudaStream_t st) {
-  tiles_kernel<<<1, 1024, 0, st>>>(s.B, s.T, s.U, TB, UB, s.S > 0 ? 1 : 0, T_len, U_len, tiles, ntiles);
+// Block 0: the length / label validation and the tile list (a prefix sum of
+// the per-utterance tile counts); the other blocks clear the accumulators.
+__global__ void __launch_bounds__(1024) prologue_kernel(int B, int T, int U, int V, int blank, int TB, int UB,
+                                                        int pruned, const int32_t* __restrict__ labels,
+                                                        const int32_t* __restrict__ T_len,
+                                                        const int32_t* __restrict__ U_len, int32_t* status,
+                                                        int4* __restrict__ tiles, int* __restrict__ ntiles,
+                                                        ZeroList z) {
+  if (blockIdx.x > 0) {
+    const long long stride = (long long)(gridDim.x - 1) * blockDim.x;
+    const long long tid = (long long)(blockIdx.x - 1) * blockDim.x + threadIdx.x;
+    for (int k = 0; k < z.count; ++k) {
+      float4* p = (float4*)z.ptr[k];
+      const long long n4 = z.n[k] / 4;
+      for (long long i = tid; i < n4; i += stride) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+  int bits = validate_bits(B, T, U, V, blank, labels, T_len, U_len, threadIdx.x, blockDim.x);
+  bits = __reduce_or_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0 && bits) atomicOr(status, bits);
+  __shared__ int offs[1025];
+  __shared__ int counts[1024];
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const Lengths l = lengths_of(T_len, U_len, b, T, U);
+    counts[b] = ((l.Tb + TB - 1) / TB) * (pruned ? 1 : (l.Ub + 1 + UB - 1) / UB);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = 0; b < B; ++b) {
+      offs[b] = acc;
+      acc += counts[b];
+    }
+    offs[B] = acc;
+    *ntiles = acc;
+  }
+  __syncthreads();
+  for (int b = 0; b < B; ++b) {
+    const Lengths l = lengths_of(T_len, U_len, b, T, U);
+    const int nu = pruned ? 1 : (l.Ub + 1 + UB - 1) / UB;
+    for (int i = threadIdx.x; i < counts[b]; i += blockDim.x) {
+      const int it = i / nu, iu = i % nu;
+      tiles[offs[b] + i] = make_int4(b, it * TB, iu * UB, 0);
+    }
+  }
+}
+
+void launch_prologue(const Shape& s, int TB, int UB, const int32_t* labels, const int32_t* T_len,
+                     const int32_t* U_len, int32_t* status, int4* tiles, int* ntiles, const ZeroList& z,
+                     cudaStream_t st) {
+  long long total = 0;
+  for (int k = 0; k < z.count; ++k) total += z.n[k];
+  int zb = (int)((total / 4 + 1023) / 1024);
+  if (zb > 2 * sms()) zb = 2 * sms();
+  if (zb < 1) zb = 1;
+  prologue_kernel<<<1 + zb, 1024, 0, st>>>(s.B, s.T, s.U, s.V, s.blank, TB, UB, s.S > 0 ? 1 : 0, labels, T_len,
+                                           U_len, status, tiles, ntiles, z);
   note_launch();
 }
 
