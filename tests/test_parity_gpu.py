@@ -182,3 +182,18 @@ def test_joint_variants_short(cuda_ok, joint_variant, variant):
     for mode in ("tiled", "untiled"):
         loss, grads = _call(batch, mode=mode)
         compare(loss, grads, run_oracle(batch), "bf16", extra_note=f"short/{mode}/v{variant}")
+
+
+@pytest.mark.parametrize("loss", ["marginal", "viterbi"])
+def test_wide_label_lattice(cuda_ok, loss):
+    """More than 512 label positions: the DP blocks of up to 1024 threads
+    (U + 1 = 701 here), both modes."""
+    batch = synth.make(B=2, T=12, U=700, D_enc=64, D_pred=64, H=128, V=128, dtype="bf16", seed=77,
+                       T_range=(6, 12), U_range=(660, 700), bias_std=0.3)
+    ref = run_oracle(batch, loss=loss)
+    for mode in ("untiled", "tiled"):
+        d = to_device(batch)
+        l, g = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                             d["U_len"], mode=mode, chunk_cells=4096, blank=batch.blank, loss=loss)
+        torch.cuda.synchronize()
+        compare(l, g, ref, "bf16", extra_note=f"wide lattice {loss}/{mode}")

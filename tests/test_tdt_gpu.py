@@ -100,3 +100,16 @@ def test_modes_agree_and_padding_ignored(cuda_ok):
         assert rel_l2(gt[k].float().cpu().numpy(), gu[k].float().cpu().numpy()) <= 1e-2, k
     for k in ("df", "dg"):
         assert rel_l2(gt[k].float().cpu().numpy(), gu[k].float().cpu().numpy()) <= 1e-2, k
+
+
+@pytest.mark.parametrize("U,D", [(300, (0, 1, 2, 3, 4)), (700, (0, 1, 2, 3, 4)), (700, (0, 1, 2, 4, 8))])
+def test_wide_label_lattice(cuda_ok, U, D):
+    """Label positions past 256 and 512 (the DP's 512- and 1024-thread
+    instantiations, the latter with the largest duration set), both modes."""
+    batch = synth.make(B=2, T=12, U=U, D_enc=64, D_pred=64, H=128, V=128, dtype="bf16", seed=900 + U,
+                       T_range=(6, 12), U_range=(U - 40, U), bias_std=0.3)
+    W_d, b_d = synth.duration_head(batch, len(D), seed=U)
+    ref = _oracle(batch, W_d, b_d, D)
+    for mode in ("untiled", "tiled"):
+        l, g = _call(batch, W_d, b_d, D, mode=mode, chunk_cells=4096)
+        _compare(l, g, ref, f"tdt U{U} {D}/{mode}")
