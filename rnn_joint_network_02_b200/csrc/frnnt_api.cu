@@ -348,6 +348,11 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   j.b_o = tdt ? (const void*)p.bx : b_o; j.labels = labels;
   j.T_len = T_len; j.U_len = U_len; j.grad_loss = grad_loss; j.tiles = p.tiles; j.ntiles = p.ntiles; j.L = p.L;
   j.zbuf = p.zbuf; j.hbuf = p.hbuf; j.db_part = p.db_part; j.status = status; j.bounds = bounds;
+  // tiled: the backward joint pass (mode 2) also stores the h rows of each
+  // chunk (its generators have the time; a separate pass would re-read F and
+  // G); untiled: the forward pass already stores z, and a second stream of
+  // stores there costs more than the hidden-row kernel beside the DP
+  j.store_h = 0;
   {
     StageScope sc("joint_fwd", st);
     j.mode = untiled ? 1 : 0;
@@ -386,15 +391,16 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
         launch_dz_from_z(j, st);
       } else {
         j.mode = 2;
+        j.store_h = 1;
         FRNNT_TRY(launch_joint_tc(j, st));
         if (tdt) launch_tdt_dzd(j, st);
       }
     }
     if (side) {
       cudaStreamWaitEvent(st, side->join, 0);
-    } else {
+    } else if (untiled) {   // no side stream could be created: build the h rows here
       StageScope sc("bwd_hidden", st);
-      launch_hidden_rows(j, untiled ? 0 : (int)c0, st);
+      launch_hidden_rows(j, 0, st);
     }
     const int rows = (int)((c1 - c0) * 128);
     {

@@ -211,6 +211,7 @@ struct JointLaunch {
   float* db_part;               // unused
   int32_t* status;
   const int32_t* bounds;        // pruned lattice (s.S > 0): [B][T] first label position of each frame's band
+  int store_h = 0;              // modes 1 and 2: the generators also write the h rows of hbuf
 };
 bool joint_tc_supported(int H, int V, int U, int S);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the

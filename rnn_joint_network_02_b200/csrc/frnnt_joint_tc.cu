@@ -89,6 +89,10 @@ struct JointParams {
   // holding the duration head (columns V .. V + n_dur - 1)
   int Vx;
   int n_dur;
+  // FWD_STORE / BWD_DZ: the generators also store the h rows they build into
+  // hbuf (rows as zbuf's), with the column block [1, 0, ...] (0 outside the
+  // lattice) after column H, for the backward GEMMs
+  int store_h;
 };
 
 struct RowInfo {
@@ -424,6 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       const uint8_t* grow = p.S ? (const uint8_t*)(p.G + ((size_t)ri.b * Up1 + min(ri.u, p.U)) * H)
                                 : fgs + (p.TB + r % p.UB) * fg_stride;
       if (!mbar_wait(fg_full, fph, abort_flag)) break;
+      // h rows for the backward GEMMs (real tiles only; a pair's dummy tile has no rows)
+      __nv_bfloat16* hrow = nullptr;
+      if (MODE != MODE_FWD && p.store_h && tile < ntiles) {
+        const size_t row0 = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
+        hrow = p.hbuf + (row0 + r) * p.HS;
+        if (half == 0) {
+          const uint4 one = make_uint4(ri.valid ? 0x3F80u : 0u, 0u, 0u, 0u);   // bf16 1.0 in column H
+          for (int c = H; c < p.HS; c += 8) *(uint4*)(hrow + c) = c == H ? one : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       for (int g = 0; g < ngrp; ++g) {
         const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
         // the whole group's values first (loads and MUFU work overlap the
@@ -449,6 +463,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
             } else {
 #pragma unroll
               for (int w = 0; w < 8; ++w) pk[kk][j][w] = 0u;
+            }
+            if (hrow && kk < nk) {
+              uint4* dst = (uint4*)(hrow + seg * 16);
+              dst[0] = make_uint4(pk[kk][j][0], pk[kk][j][1], pk[kk][j][2], pk[kk][j][3]);
+              dst[1] = make_uint4(pk[kk][j][4], pk[kk][j][5], pk[kk][j][6], pk[kk][j][7]);
             }
           }
         }
@@ -1078,6 +1097,7 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.status = j.status;
   p.Vx = j.s.Vx;
   p.n_dur = j.s.n_dur;
+  p.store_h = j.store_h;
   // the backward dz pass covers the label tiles only (the duration head's
   // gradient comes from the stored duration log-probs)
   p.nV = (j.mode == MODE_BWD_DZ ? p.V : p.Vx) / BN;
