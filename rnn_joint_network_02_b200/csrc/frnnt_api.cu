@@ -105,6 +105,7 @@ SimtPlan plan_simt(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.alpha = c.take<float>(s.Np);
   p.L.beta = c.take<float>(s.Np);
   p.L.path = s.viterbi ? c.take<uint8_t>(s.Np) : nullptr;
+  p.L.dpw = s.viterbi ? nullptr : c.take<float>(dp2_weight_floats(s.B, s.T, s.U));
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   p.accWo = c.take<float>((size_t)s.V * s.H);
@@ -151,6 +152,7 @@ int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, 
 
   {  // transducer forward-backward
     StageScope sc("lattice_dp", st);
+    launch_dp_weights(s, p.L, T_len, U_len, st);
     launch_dp(s, p.L, T_len, U_len, nullptr, loss, st);
   }
 
@@ -242,6 +244,8 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.alpha = c.take<float>(s.Nlat);
   p.L.beta = c.take<float>(s.Nlat);
   p.L.path = s.viterbi ? c.take<uint8_t>(s.Nlat) : nullptr;
+  // the two-diagonal DP's step weights (marginal loss, whole lattice, no durations)
+  p.L.dpw = (!s.viterbi && s.S == 0 && s.n_dur == 0) ? c.take<float>(dp2_weight_floats(s.B, s.T, s.U)) : nullptr;
   if (s.n_dur > 0) {
     p.L.beta_l = c.take<float>(s.Nlat);
     p.L.dur_lp = c.take<float>((size_t)s.n_dur * s.Nlat);
@@ -359,6 +363,12 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     j.tile_begin = 0;
     j.tile_end = (int)p.maxT;
     FRNNT_TRY(launch_joint_tc(j, st));
+  }
+  {
+    // the DP's step weights first: a short full-GPU pass, done before the
+    // hidden rows below take the SMs
+    StageScope sc("lattice_dp", st);
+    launch_dp_weights(s, p.L, T_len, U_len, st);
   }
   // untiled: the h rows of the whole lattice do not depend on the DP; build
   // them on the side stream while the DP runs

@@ -117,7 +117,7 @@ __device__ __forceinline__ void dp_operands(bool is_beta, int step, int ndiag, i
 // (beta) on the previous diagonal pair come through a parity-double-buffered
 // shared array with one entry per thread (one barrier per step, no shuffles).
 // The six log-probabilities of a step are fetched kPrefetch2 steps ahead.
-constexpr int kPrefetch2 = 4;
+constexpr int kPrefetch2 = kDp2Prefetch;
 
 struct DpOps {
   float bA, bB, bC, lA, lB, lC;
@@ -157,16 +157,76 @@ __device__ __forceinline__ DpOps dp2_operands(bool is_beta, int step, int nsteps
   return o;
 }
 
-__device__ __forceinline__ float lae3(float a, float b, float c) { return log_add_exp(log_add_exp(a, b), c); }
+// The step's weights, precomputed for every (utterance, direction, step, label
+// position) by a parallel kernel, so that the serial wavefront loads five
+// numbers per step with no index arithmetic or bounds checks on them:
+//   alpha, far cell (t,u), t = 2 step + 2 - u, middle cell (t-1,u):
+//     M1 = b(t-2,u), M2 = l(t-1,u-1);  W1 = b(t-2,u) + b(t-1,u),
+//     W2 = lae(b(t-1,u-1) + l(t,u-1), l(t-1,u-1) + b(t-1,u)),  W3 = l(t,u-2) + l(t,u-1)
+//   beta, far cell (t,u), t = last - 2 step - 2 - u, middle cell (t+1,u):
+//     M1 = b(t+1,u), M2 = l(t+1,u);  W1 = b(t,u) + b(t+1,u),
+//     W2 = lae(b(t,u) + l(t+1,u), l(t,u) + b(t,u+1)),  W3 = l(t,u) + l(t,u+1)
+// so that middle = lae(cur + M1, n1 + M2) and far = lae(lae(cur + W1, n1 + W2), n2 + W3)
+// (cur, n1, n2: the previous far diagonal at u and at u -/+ 1, 2), with all
+// weights -inf for a cell outside the lattice, whose value then is -inf too.
+// Layout [b][direction][step][5][UP] (UP = the DP's block size), with
+// kPrefetch2 extra steps so that the prefetch never needs a bound.
+__global__ void dp2_weights_kernel(int B, int T, int U, int NS, int UP, const float* __restrict__ blank_lp,
+                                   const float* __restrict__ label_lp, const int32_t* __restrict__ T_len,
+                                   const int32_t* __restrict__ U_len, float* __restrict__ w) {
+  const long long n = (long long)B * 2 * NS * UP;
+  const int Up1 = U + 1;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(i % UP);
+    long long r = i / UP;
+    const int step = (int)(r % NS);
+    r /= NS;
+    const bool is_beta = (r & 1) != 0;
+    const int b = (int)(r >> 1);
+    const Lengths l = lengths_of(T_len, U_len, b, T, U);
+    const int Tb = l.Tb, Ub = l.Ub;
+    const int last = Tb - 1 + Ub;
+    const int nsteps = (last + 1) / 2;
+    const size_t base = (size_t)b * T * Up1;
+    const DpOps o = dp2_operands(is_beta, step, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+    const bool live = step < nsteps && u <= Ub;
+    float m1, m2, w1, w2, w3;
+    if (!is_beta) {
+      const int t = 2 * step + 2 - u;
+      const bool mid = live && t - 1 >= 0 && t - 1 < Tb;
+      const bool far = live && 2 * step + 2 <= last && t >= 0 && t < Tb;
+      m1 = mid ? o.bA : -INFINITY;
+      m2 = mid ? o.lB : -INFINITY;
+      w1 = far ? o.bA + o.bB : -INFINITY;
+      w2 = far ? log_add_exp(o.bC + o.lA, o.lB + o.bB) : -INFINITY;
+      w3 = far ? o.lC + o.lA : -INFINITY;
+    } else {
+      const int t = last - 2 * step - 2 - u;
+      const bool mid = live && t + 1 >= 0 && t + 1 < Tb;
+      const bool far = live && last - 2 * step - 2 >= 0 && t >= 0 && t < Tb;
+      m1 = mid ? o.bB : -INFINITY;
+      m2 = mid ? o.lA : -INFINITY;
+      w1 = far ? o.bA + o.bB : -INFINITY;
+      w2 = far ? log_add_exp(o.bA + o.lA, o.lB + o.bC) : -INFINITY;
+      w3 = far ? o.lB + o.lC : -INFINITY;
+    }
+    float* dst = w + ((size_t)(((long long)b * 2 + (is_beta ? 1 : 0)) * NS + step) * 5) * UP + u;
+    dst[0] = m1;
+    dst[UP] = m2;
+    dst[2 * UP] = w1;
+    dst[3 * UP] = w2;
+    dst[4 * UP] = w3;
+  }
+}
 
-__global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, const float* __restrict__ label_lp,
+__global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank_lp, const float* __restrict__ wts,
                            float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
                            const int32_t* __restrict__ U_len, float* __restrict__ loss) {
   __shared__ float xa[2][1024];     // [parity][thread]: each thread's value on the last far diagonal
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
   const int u = threadIdx.x;
-  const int nth = blockDim.x;
+  const int nth = blockDim.x;       // = the weights' UP
   const Lengths l = lengths_of(T_len, U_len, b, T, U);
   const int Tb = l.Tb, Ub = l.Ub;
   const int Up1 = U + 1;
@@ -174,6 +234,7 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
   const int last = Tb - 1 + Ub;             // the last diagonal
   const int nsteps = (last + 1) / 2;        // steps of two diagonals after diagonal 0 (alpha) / `last` (beta)
   const bool in_u = u <= Ub;
+  const float* wp = wts + (size_t)((long long)b * 2 + (is_beta ? 1 : 0)) * NS * 5 * nth + u;
 
   // the first diagonal: (0,0) for alpha, (Tb-1, Ub) for beta
   float cur = -INFINITY;
@@ -189,10 +250,11 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
     if (last == 0) loss[b] = -cur;
   }
 
-  DpOps q[kPrefetch2];
+  float q[kPrefetch2][5];
 #pragma unroll
   for (int i = 0; i < kPrefetch2; ++i)
-    q[i] = dp2_operands(is_beta, i, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)(i * 5 + k) * nth);
 
   // parity 1 holds the first diagonal
   xa[1][u] = cur;
@@ -203,9 +265,11 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
     for (int i = 0; i < kPrefetch2; ++i) {
       const int step = step0 + i;
       if (step >= nsteps) break;    // uniform across the block
-      const DpOps o = q[i];
-      q[i] = dp2_operands(is_beta, step + kPrefetch2, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
-      const int par = (step + 1) & 1;       // parity holding the previous pair's edge values
+      const float m1 = q[i][0], m2 = q[i][1], w1 = q[i][2], w2 = q[i][3], w3 = q[i][4];
+      // (NS covers nsteps + kPrefetch2 steps: no bound on the prefetch)
+#pragma unroll
+      for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)((step + kPrefetch2) * 5 + k) * nth);
+      const int par = (step + 1) & 1;       // parity holding the previous pair's far values
       float n1, n2;                          // neighbours at distance 1 and 2 on the previous far diagonal
       if (!is_beta) {
         n1 = u >= 1 ? xa[par][u - 1] : -INFINITY;
@@ -214,30 +278,18 @@ __global__ void dp2_kernel(int T, int U, const float* __restrict__ blank_lp, con
         n1 = u + 1 < nth ? xa[par][u + 1] : -INFINITY;
         n2 = u + 2 < nth ? xa[par][u + 2] : -INFINITY;
       }
-      float v1 = -INFINITY, v2 = -INFINITY;
+      const float v1 = log_add_exp(cur + m1, n1 + m2);
+      const float v2 = log_add_exp(log_add_exp(cur + w1, n1 + w2), n2 + w3);
       if (in_u) {
         if (!is_beta) {
-          const int d1 = 2 * step + 1, d2 = d1 + 1;
-          const int t1 = d1 - u, t2 = d2 - u;
-          if (t1 >= 0 && t1 < Tb) {
-            // one edge from diagonal d1 - 1: (t1-1,u) by blank (operand b(t1-1,u) = bA), (t1,u-1) by label (lB)
-            v1 = log_add_exp(cur + o.bA, n1 + o.lB);
-            alpha[base + (size_t)t1 * Up1 + u] = v1;
-          }
-          if (d2 <= last && t2 >= 0 && t2 < Tb) {
-            v2 = lae3(cur + o.bA + o.bB, n1 + log_add_exp(o.bC + o.lA, o.lB + o.bB), n2 + o.lC + o.lA);
-            alpha[base + (size_t)t2 * Up1 + u] = v2;
-          }
+          const int t1 = 2 * step + 1 - u, t2 = t1 + 1;
+          if (t1 >= 0 && t1 < Tb) alpha[base + (size_t)t1 * Up1 + u] = v1;
+          if (2 * step + 2 <= last && t2 >= 0 && t2 < Tb) alpha[base + (size_t)t2 * Up1 + u] = v2;
         } else {
-          const int d1 = last - 2 * step - 1, d2 = d1 - 1;
-          const int t1 = d1 - u, t2 = d2 - u;
-          if (t1 >= 0 && t1 < Tb) {
-            // cell (t1,u) = (t2+1,u): one edge to (t1+1,u) by blank (bB), (t1,u+1) by label (lA)
-            v1 = log_add_exp(cur + o.bB, n1 + o.lA);
-            beta[base + (size_t)t1 * Up1 + u] = v1;
-          }
+          const int d2 = last - 2 * step - 2;
+          const int t2 = d2 - u, t1 = t2 + 1;
+          if (t1 >= 0 && t1 < Tb) beta[base + (size_t)t1 * Up1 + u] = v1;
           if (d2 >= 0 && t2 >= 0 && t2 < Tb) {
-            v2 = lae3(cur + o.bA + o.bB, n1 + log_add_exp(o.bA + o.lA, o.lB + o.bC), n2 + o.lB + o.lC);
             beta[base + (size_t)t2 * Up1 + u] = v2;
             if (t2 == 0 && u == 0) loss[b] = -v2;
           }
@@ -848,6 +900,17 @@ void launch_tdt_dp_t(const Shape& s, const Lattice& L, const int32_t* T_len, con
                                                          loss);
 }
 
+void launch_dp_weights(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len,
+                       cudaStream_t st) {
+  if (!L.dpw) return;
+  const int threads = ((s.Up1 + 31) / 32) * 32;
+  const int NS = dp2_weight_steps(s.T, s.U);
+  const long long n = (long long)s.B * 2 * NS * threads;
+  const int wb = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+  dp2_weights_kernel<<<wb, 256, 0, st>>>(s.B, s.T, s.U, NS, threads, L.blank_lp, L.label_lp, T_len, U_len, L.dpw);
+  note_launch();
+}
+
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
                float* loss, cudaStream_t st) {
   int threads = ((s.Up1 + 31) / 32) * 32;
@@ -885,7 +948,8 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
                                                   U_len, loss, smem > 0 ? 1 : 0);
   } else {
     dim3 grid(s.B, 2);
-    dp2_kernel<<<grid, threads, 0, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.beta, T_len, U_len, loss);
+    dp2_kernel<<<grid, threads, 0, st>>>(s.T, s.U, dp2_weight_steps(s.T, s.U), L.blank_lp, L.dpw, L.alpha, L.beta,
+                                         T_len, U_len, loss);
   }
   note_launch();
 }

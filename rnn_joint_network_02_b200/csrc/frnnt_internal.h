@@ -70,7 +70,17 @@ struct Lattice {
   float* dur_lp = nullptr;
   float* tdt_q = nullptr;
   long long plane = 0;
+  // the two-diagonal DP's precomputed step weights (marginal loss on the
+  // whole lattice): dp2_weight_floats(s) floats, else null
+  float* dpw = nullptr;
 };
+
+// Steps (with the prefetch margin) and floats of the two-diagonal DP's weights.
+constexpr int kDp2Prefetch = 4;   // steps the two-diagonal DP loads ahead
+inline int dp2_weight_steps(int T, int U) { return (T + U) / 2 + 1 + kDp2Prefetch; }
+inline long long dp2_weight_floats(int B, int T, int U) {
+  return (long long)B * 2 * dp2_weight_steps(T, U) * 5 * (((U + 1 + 31) / 32) * 32);
+}
 
 #ifdef __CUDACC__
 // Posterior of the two edges leaving valid cell (t, u) at lattice index c
@@ -112,6 +122,9 @@ void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len
                      const int32_t* bounds, int32_t* status, cudaStream_t st);
 void launch_validate_bounds(const Shape& s, const int32_t* bounds, const int32_t* T_len, const int32_t* U_len,
                             int32_t* status, cudaStream_t st);
+// The two-diagonal DP's step weights (when L.dpw is set); must precede launch_dp.
+void launch_dp_weights(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len,
+                       cudaStream_t st);
 // bounds: the pruned lattice's per-frame starts (s.S > 0), else null
 void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int32_t* U_len, const int32_t* bounds,
                float* loss, cudaStream_t st);
