@@ -217,6 +217,7 @@ struct TcPlan {
   // token-and-duration transducer: [W_o; W_d; 0], [b_o; b_d; 0] and the
   // duration head's weight-gradient accumulator (64 rows, n_dur used)
   __nv_bfloat16 *Wx = nullptr, *bx = nullptr;
+  float4* row_params = nullptr;   // the dz pass with bias sums: per-row scalars
   float* accWd = nullptr;
   size_t bytes;
 };
@@ -256,7 +257,10 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
     p.accWd = c.take<float>((size_t)64 * hidden_stride(s.H));
   }
   p.accWo = c.take<float>((size_t)s.V * hidden_stride(s.H));
-  p.db_part = nullptr;
+  // untiled with H a multiple of 256: db_o is summed by the dz pass, so the
+  // dW_o GEMM runs on N = H (whole 256-wide tiles) without the ones column
+  p.db_part = (d->mode == FRNNT_UNTILED && dz_db_supported(s.V, s.H)) ? c.take<float>(s.V) : nullptr;
+  p.row_params = p.db_part ? c.take<float4>((size_t)p.maxT * 128) : nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.Vx);
@@ -334,6 +338,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     add(p.accWf, (long long)s.Dx * s.H);
     add(p.accWg, (long long)s.Dy * s.H);
     if (tdt) add(p.accWd, 64LL * hidden_stride(s.H));
+    if (p.db_part) add(p.db_part, (s.V + 3) / 4 * 4);
     launch_prologue(s, p.TB, p.UB, labels, T_len, U_len, status, p.tiles, p.ntiles, z, st);
     if (s.S > 0) launch_validate_bounds(s, bounds, T_len, U_len, status, st);
     if (tdt) launch_tdt_weights(s, W_o, b_o, W_d, b_d, p.Wx, p.bx, st);
@@ -398,7 +403,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     {
       StageScope sc("joint_bwd_dz", st);
       if (untiled) {
-        launch_dz_from_z(j, st);
+        if (p.db_part) launch_dz_db(j, p.db_part, p.row_params, st);
+        else launch_dz_from_z(j, st);
       } else {
         j.mode = 2;
         j.store_h = 1;
@@ -416,15 +422,17 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     {
       StageScope sc("bwd_dWo", st);
       GemmTcArgs a{};
-      // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias gradient
-      a.M = s.V; a.N = HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.Vx; a.B = hrows; a.b_mn = true;
-      a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, HS, rows); a.out_f32 = p.accWo;
+      // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias
+      // gradient, unless the dz pass summed it (then N = H)
+      a.M = s.V; a.N = p.db_part ? s.H : HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.Vx; a.B = hrows;
+      a.b_mn = true; a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, a.N, rows);
+      a.out_f32 = p.accWo;
       a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;
       FRNNT_TRY(gemm_tc(a, st));
       if (tdt) {
         // dW_d | db_d from the duration columns (64 of them, zero past n_dur)
-        a.M = 64; a.A = zrows + s.V; a.k_splits = splits_for(64, HS, rows); a.out_f32 = p.accWd;
+        a.M = 64; a.N = HS; a.A = zrows + s.V; a.k_splits = splits_for(64, HS, rows); a.out_f32 = p.accWd;
         FRNNT_TRY(gemm_tc(a, st));
       }
     }
@@ -456,7 +464,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       cudaEventRecord(ps->fork2, st);
       cudaStreamWaitEvent(gs, ps->fork2, 0);
     }
-    launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st);
+    launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st, p.db_part);
     if (tdt) launch_wo_finalize(p.accWd, s.n_dur, s.H, dW_d, db_d, st);
     launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
     launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, gs);

@@ -259,7 +259,14 @@ void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const 
                         void* b_x, cudaStream_t st);
 // blocks_per_sm: 256-thread blocks per SM of the grid (fewer leave room for work running beside it)
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
-void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st);
+// dW_o = acc[:, :H]; db_o = db (when non-null) or acc[:, H]; acc rows of hidden_stride(H)
+void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st,
+                        const float* db = nullptr);
+// Untiled dz pass that also sums db_o into db_acc [V] (cleared beforehand), for
+// dz_db_supported(V, H): the dW_o GEMM then runs on N = H.
+bool dz_db_supported(int V, int H);
+// row_params: scratch of one float4 per row of the launch's tiles.
+void launch_dz_db(const JointLaunch& j, float* db_acc, float4* row_params, cudaStream_t st);
 
 // out[i] = (dtype) in[i]
 void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaStream_t st);

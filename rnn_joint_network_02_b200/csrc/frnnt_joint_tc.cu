@@ -80,7 +80,7 @@ struct JointParams {
   __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
   int HS;                 // row stride of hbuf (hidden_stride(H))
   int srows;              // rows per epilogue store-staging pass (8 or 32)
-  float* db_part;         // unused
+  float* db_part;         // dz_db_kernel: db_o accumulator [V] (column sums of dz), else unused
   int32_t* status;
   const int32_t* bounds;  // pruned lattice: [B][T] band starts; S = band width (0: whole lattice)
   int S;
@@ -782,6 +782,117 @@ __global__ void __launch_bounds__(256, 4) dz_from_z_kernel(JointParams p) {
   }
 }
 
+// dz_from_z with the bias gradient: warps are split over the 1024-column ranges
+// of the vocabulary, each warp owning one range (32 columns per lane) for all
+// the rows it visits, so its column sums stay in registers; at the end every
+// warp adds them to p.db_part.  Lets the dW_o GEMM run on N = H instead of a
+// padded h with a ones column.  Rows: absolute tile rows (untiled).  TDT: the
+// warps of range 0 also write the rows' duration columns.  The grid's warp
+// count is a multiple of the number of ranges.
+// Per-row scalars of the dz pass, computed once per row (the dz warps of
+// several column ranges share them): {lse log2(e), w bpost, w lpost, label}
+// with the label -2 for a row that is no lattice cell (-1: a cell without a
+// label edge).
+__global__ void row_params_kernel(JointParams p, float4* __restrict__ rp) {
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
+  for (long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x; row < nrows;
+       row += (long long)gridDim.x * blockDim.x) {
+    const int tile = p.tile_begin + (int)(row >> 7);
+    const RowInfo ri = row_info(p, p.tiles[tile], (int)(row & 127));
+    float4 v = make_float4(0.f, 0.f, 0.f, __int_as_float(-2));
+    if (ri.valid) {
+      const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
+      float bpost, lpost;
+      size_t c0;
+      long long c_t1, c_u1;
+      bool last;
+      lattice_neighbors(p, ri, c0, c_t1, c_u1, last);
+      edge_posteriors(p.L, ri.cell, c0, c_t1, c_u1, last, bpost, lpost);
+      v = make_float4(p.L.lse[ri.cell] * kLog2e, w * bpost, w * lpost, __int_as_float(ri.y));
+    }
+    rp[row] = v;
+  }
+}
+
+template <bool TDT>
+__global__ void __launch_bounds__(256, 3) dz_db_kernel(JointParams p, const float4* __restrict__ rp) {
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int V = p.V, ldz = p.Vx;
+  const int lane = threadIdx.x & 31;
+  const int ncr = (V + 1023) / 1024;
+  const long long gw = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int cr = (int)(gw % ncr);
+  const long long nw = (long long)gridDim.x * (blockDim.x >> 5) / ncr;
+  const int k0 = cr * 1024;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
+  // each row's scalars are fetched one iteration ahead, so the z loads of a
+  // valid row (only those: rows that are no cell are just cleared) issue at once
+  long long row = gw / ncr;
+  float4 rv_next = row < nrows ? rp[row] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (; row < nrows; row += nw) {
+    const float4 rv = rv_next;
+    if (row + nw < nrows) rv_next = rp[row + nw];
+    const int tile = p.tile_begin + (int)(row >> 7);
+    __nv_bfloat16* zr = p.zbuf + (size_t)tile * 128 * ldz + (size_t)(row & 127) * ldz;
+    if (TDT && cr == 0) tdt_dzd_row(p, row_info(p, p.tiles[tile], (int)(row & 127)), zr + V, lane);
+    const int y = __float_as_int(rv.w);
+    if (y == -2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i * 256 + lane * 8;
+        if (k < V) *(uint4*)(zr + k) = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
+    uint4 zv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int k = k0 + i * 256 + lane * 8;
+      if (k < V) zv[i] = *(const uint4*)(zr + k);
+    }
+    const float lk = rv.x, bpost = rv.y, lpost = rv.z;
+    const float occ = bpost + lpost;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int k = k0 + i * 256 + lane * 8;
+      if (k >= V) break;
+      const uint32_t zw[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[q]));
+        float d0 = occ * ex2(fmaf(zf.x, kLog2e, -lk));
+        float d1 = occ * ex2(fmaf(zf.y, kLog2e, -lk));
+        const int k2 = k + 2 * q;
+        if (k2 == p.blank) d0 -= bpost;
+        if (k2 + 1 == p.blank) d1 -= bpost;
+        if (k2 == y) d0 -= lpost;
+        if (k2 + 1 == y) d1 -= lpost;
+        o[q] = pack_bf16x2(d0, d1);
+        // the bias gradient sums what the GEMMs read: the bf16-rounded dz
+        const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o[q]));
+        acc[i][2 * q] += r.x;
+        acc[i][2 * q + 1] += r.y;
+      }
+      *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = k0 + i * 256 + lane * 8;
+    if (k < V) {
+      red_add_v4(p.db_part + k, acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      red_add_v4(p.db_part + k + 4, acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+  }
+}
+
 // Tiled backward of the token-and-duration transducer: the duration columns of
 // the chunk's dz rows (the label columns come from the joint kernel's dz pass).
 __global__ void tdt_dzd_kernel(JointParams p) {
@@ -865,13 +976,13 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
 
 // dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
 // whose column H is the sum of dz over cells.
-__global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, __nv_bfloat16* __restrict__ dW_o,
-                                   __nv_bfloat16* __restrict__ db_o) {
+__global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, const float* __restrict__ db,
+                                   __nv_bfloat16* __restrict__ dW_o, __nv_bfloat16* __restrict__ db_o) {
   const long long n = (long long)V * H;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const long long k = i / H, j = i % H;
     dW_o[i] = __float2bfloat16_rn(acc[k * HS + j]);
-    if (j == 0) db_o[k] = __float2bfloat16_rn(acc[k * HS + H]);
+    if (j == 0) db_o[k] = __float2bfloat16_rn(db ? db[k] : acc[k * HS + H]);
   }
 }
 
@@ -1155,6 +1266,43 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   note_launch();
 }
 
+void launch_dz_db(const JointLaunch& j, float* db_acc, float4* row_params, cudaStream_t st) {
+  JointParams p{};
+  p.T = j.s.T;
+  p.U = j.s.U;
+  p.H = j.s.H;
+  p.V = j.s.V;
+  p.blank = j.s.blank;
+  p.TB = j.TB;
+  p.UB = j.UB;
+  p.labels = j.labels;
+  p.T_len = j.T_len;
+  p.U_len = j.U_len;
+  p.grad_loss = j.grad_loss;
+  p.tiles = j.tiles;
+  p.ntiles = j.ntiles;
+  p.tile_begin = j.tile_begin;
+  p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
+  p.L = j.L;
+  p.zbuf = (__nv_bfloat16*)j.zbuf;
+  p.Vx = j.s.Vx;
+  p.n_dur = j.s.n_dur;
+  p.db_part = db_acc;
+  // 8 warps per block: the warp count sms * 3 * 8 is a multiple of the range count (1..4)
+  const int ncr = (j.s.V + 1023) / 1024;
+  int blocks = sms() * 3;
+  blocks -= blocks % (ncr == 3 ? 3 : 1);
+  row_params_kernel<<<sms() * 8, 256, 0, st>>>(p, row_params);
+  note_launch();
+  if (p.n_dur > 0) dz_db_kernel<true><<<blocks, 256, 0, st>>>(p, row_params);
+  else dz_db_kernel<false><<<blocks, 256, 0, st>>>(p, row_params);
+  note_launch();
+}
+
+bool dz_db_supported(int V, int H) { return V % 256 == 0 && V <= 4096 && H % 256 == 0; }
+
 void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st) {
   JointParams p{};
   p.T = j.s.T;
@@ -1213,11 +1361,11 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   note_launch();
 }
 
-void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st) {
+void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st, const float* db) {
   long long n = (long long)V * H;
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), (__nv_bfloat16*)dW_o,
+  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, (__nv_bfloat16*)dW_o,
                                                        (__nv_bfloat16*)db_o);
   note_launch();
 }
