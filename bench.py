@@ -62,9 +62,11 @@ def parse():
 # An entry is removed whenever its kernel changes, so the roofline's traffic is
 # null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dWo", "marginal"): (1.175207e9 + 0.010739e9, "profiles/ncu_gemm2_tc_medium_untiled.md"),
-    ("medium", "untiled", "bwd_dh", "marginal"): (0.629206e9 + 0.356382e9, "profiles/ncu_gemm2_dh_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd", "marginal"): (0.009145e9 + 0.572019e9,
+    ("medium", "untiled", "bwd_dWo", "marginal"): (1.181477e9 + 0.011693e9,
+                                                   "profiles/ncu_gemm2_backward_medium_untiled.md"),
+    ("medium", "untiled", "bwd_dh", "marginal"): (0.642829e9 + 0.016059e9,
+                                                  "profiles/ncu_gemm2_backward_medium_untiled.md"),
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009251e9 + 0.570488e9,
                                                      "profiles/ncu_joint_tc_medium_untiled.md"),
 }
 
