@@ -93,6 +93,10 @@ struct JointParams {
   // hbuf (rows as zbuf's), with the column block [1, 0, ...] (0 outside the
   // lattice) after column H, for the backward GEMMs
   int store_h;
+  // 1: the tile's F and G rows are bulk-copied into shared memory one tile
+  // ahead; 0 (when shared memory is better spent on the W_o ring): the
+  // generators read them from global memory (L2-resident)
+  int stage_fg;
 };
 
 struct RowInfo {
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   const int STAGE = p.ks * KBB;
   const int ngrp = (p.KB + p.ks - 1) / p.ks;                      // K-block groups (one ring stage each)
   uint8_t* fgs = ring + p.stages * STAGE;                         // TB F rows then UB G rows of this tile
-  __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + fg_bytes(p.TB, p.UB, p.H));   // b_o (bf16)
+  __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + (p.stage_fg ? fg_bytes(p.TB, p.UB, p.H) : 0));   // b_o (bf16)
   uint8_t* stage_s = (uint8_t*)(bias_s + ((p.Vx + 511) & ~511));  // per epilogue warp: srows x 80 B
   uint64_t* full = (uint64_t*)(stage_s + kEpiWarps * p.srows * 80);
   uint64_t* empty = full + kMaxStages;
@@ -389,10 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   } else if (warp >= kGen0) {
     // ------------------------------------------------------------ h generators (warps 10-17)
     // The tile's TB rows of F and UB rows of G are bulk-copied into shared
-    // memory (by warp kGen0, one tile ahead), then every thread builds its row
-    // h[r, :] = tanh(F[t] + G[u]) 16 columns at a time (half of each 64-wide
-    // K block per warp), into TMEM (first 512 columns of h) or the swizzled
-    // shared-memory operand (the rest).
+    // memory (by warp kGen0, one tile ahead; without p.stage_fg every thread
+    // reads its rows from global memory instead), then every thread builds its
+    // row h[r, :] = tanh(F[t] + G[u]) 16 columns at a time (half of each
+    // 64-wide K block per warp), into TMEM (first 512 columns of h) or the
+    // swizzled shared-memory operand (the rest).
     const int q = warp & 3;                  // TMEM lane quadrant this warp may access
     const int half = (warp - kGen0) >> 2;    // which two of the four 16-column segments of each K block
     const int r = q * 32 + lane;             // tile row generated by this thread
@@ -418,16 +423,18 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       return true;
     };
     bool ok = true;
-    if (warp == kGen0 && slot < niter) ok = issue_fg(tile_of(slot), 1u);
+    if (p.stage_fg && warp == kGen0 && slot < niter) ok = issue_fg(tile_of(slot), 1u);
     for (int it = slot; it < niter && ok; it += nslots, hph ^= 1, fph ^= 1) {
       const int tile = tile_of(it);
       // a dummy tile (the odd one out of a pair) has no valid row: its h is zero
       const int4 td = tile < ntiles ? p.tiles[tile] : make_int4(0, p.T, 0, 0);
       const RowInfo ri = row_info(p, td, r);
-      const uint8_t* frow = fgs + (r / p.UB) * fg_stride;
-      const uint8_t* grow = p.S ? (const uint8_t*)(p.G + ((size_t)ri.b * Up1 + min(ri.u, p.U)) * H)
-                                : fgs + (p.TB + r % p.UB) * fg_stride;
-      if (!mbar_wait(fg_full, fph, abort_flag)) break;
+      // (global rows are read only for valid cells; the clamps keep the pointers in range regardless)
+      const uint8_t* frow = p.stage_fg ? fgs + (r / p.UB) * fg_stride
+                                       : (const uint8_t*)(p.F + ((size_t)ri.b * p.T + min(ri.t, p.T - 1)) * H);
+      const uint8_t* grow = (p.S || !p.stage_fg) ? (const uint8_t*)(p.G + ((size_t)ri.b * Up1 + min(ri.u, p.U)) * H)
+                                                 : fgs + (p.TB + r % p.UB) * fg_stride;
+      if (p.stage_fg && !mbar_wait(fg_full, fph, abort_flag)) break;
       // h rows for the backward GEMMs (real tiles only; a pair's dummy tile has no rows)
       __nv_bfloat16* hrow = nullptr;
       if (MODE != MODE_FWD && p.store_h && tile < ntiles) {
@@ -508,10 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
         }
       }
       if (!ok) break;
-      // this warp is done reading the tile's F/G rows
-      __syncwarp();
-      if (lane == 0) mbar_arrive(fg_empty);
-      if (warp == kGen0 && it + nslots < niter) ok = issue_fg(tile_of(it + nslots), fph);
+      if (p.stage_fg) {
+        // this warp is done reading the tile's F/G rows
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fg_empty);
+        if (warp == kGen0 && it + nslots < niter) ok = issue_fg(tile_of(it + nslots), fph);
+      }
       if (*abort_flag) break;
     }
   } else {
@@ -1000,20 +1009,20 @@ int sms() {
 constexpr int kSmemLimit = 232448;   // max dynamic shared memory per block on sm_100
 constexpr int kBarBytes = 3072;   // mbarriers + TMEM address + abort flag + 2 KB epilogue combine area
 
-int smem_fixed(int KB, int V, int TB, int UB, int srows) {
+int smem_fixed(int KB, int V, int TB, int UB, int srows, bool stage_fg = true) {
   const int KB_hi = KB > kTmemKB ? KB - kTmemKB : 0;
-  return 1024 + KB_hi * 16384 + fg_bytes(TB, UB, KB * 64) + ((V + 511) & ~511) * 2 + kEpiWarps * srows * 80 +
-         kBarBytes;
+  return 1024 + KB_hi * 16384 + (stage_fg ? fg_bytes(TB, UB, KB * 64) : 0) + ((V + 511) & ~511) * 2 +
+         kEpiWarps * srows * 80 + kBarBytes;
 }
 
 // Staging rows: 32 when that still leaves at least 6 full W_o tiles of ring, else 8.
-int staging_rows(int KB, int V, int TB, int UB) {
-  return (kSmemLimit - smem_fixed(KB, V, TB, UB, 32)) / kStageBytes >= 6 ? 32 : 8;
+int staging_rows(int KB, int V, int TB, int UB, bool stage_fg = true) {
+  return (kSmemLimit - smem_fixed(KB, V, TB, UB, 32, stage_fg)) / kStageBytes >= 6 ? 32 : 8;
 }
 
 // Ring stages of stage_bytes each (a full W_o tile, or half of one per CTA of a pair).
-int stages_for(int KB, int V, int TB, int UB, int stage_bytes = kStageBytes) {
-  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB, staging_rows(KB, V, TB, UB))) / stage_bytes;
+int stages_for(int KB, int V, int TB, int UB, int stage_bytes = kStageBytes, bool stage_fg = true) {
+  int st = (kSmemLimit - smem_fixed(KB, V, TB, UB, staging_rows(KB, V, TB, UB, stage_fg), stage_fg)) / stage_bytes;
   return st > kMaxStages ? kMaxStages : st;
 }
 
@@ -1022,14 +1031,23 @@ int g_joint_variant = -1;   // -1 automatic, 0 one CTA per tile, 1 CTA pairs
 template <int MODE, bool PAIR>
 int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStream_t st) {
   constexpr int kb_bytes = PAIR ? kStageBytes / 2 : kStageBytes;
-  p.srows = staging_rows(p.KB, p.Vx, p.TB, p.UB);
-  // two K blocks per ring stage (half as many barrier polls in the MMA issuer)
-  // while that still leaves at least three stages
-  p.ks = stages_for(p.KB, p.Vx, p.TB, p.UB, 2 * kb_bytes) >= 3 ? 2 : 1;
-  const int stage_bytes = p.ks * kb_bytes;
-  p.stages = stages_for(p.KB, p.Vx, p.TB, p.UB, stage_bytes);
+  int stage_bytes = 0;
+  auto plan = [&](bool fg) {
+    p.stage_fg = fg ? 1 : 0;
+    p.srows = staging_rows(p.KB, p.Vx, p.TB, p.UB, fg);
+    // two K blocks per ring stage (half as many barrier polls in the MMA issuer)
+    // while that still leaves at least three stages
+    p.ks = stages_for(p.KB, p.Vx, p.TB, p.UB, 2 * kb_bytes, fg) >= 3 ? 2 : 1;
+    stage_bytes = p.ks * kb_bytes;
+    p.stages = stages_for(p.KB, p.Vx, p.TB, p.UB, stage_bytes, fg);
+  };
+  // stage the F / G rows in shared memory unless that leaves the W_o ring
+  // under 96 KB (large H: then the ring's depth matters more than the
+  // generators' load latency, measured on H = 1024 vs 640)
+  plan(true);
+  if (p.stages * stage_bytes < 96 * 1024) plan(false);
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
-  const int smem = smem_fixed(p.KB, p.Vx, p.TB, p.UB, p.srows) + p.stages * stage_bytes;
+  const int smem = smem_fixed(p.KB, p.Vx, p.TB, p.UB, p.srows, p.stage_fg != 0) + p.stages * stage_bytes;
   auto kern = joint_tc_kernel<MODE, PAIR>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1087,7 +1105,7 @@ bool joint_tc_supported(int H, int V, int U, int S) {
   s.S = S;
   int TB, UB;
   tile_shape_of(s, &TB, &UB);
-  return stages_for(H / 64, V, TB, UB) >= 2;
+  return stages_for(H / 64, V, TB, UB, kStageBytes, false) >= 2;
 }
 
 void tile_shape(int U, int* TB, int* UB) {
