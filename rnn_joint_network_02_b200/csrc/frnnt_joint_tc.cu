@@ -64,7 +64,8 @@ struct JointParams {
   int KB;                 // H / 64
   int nV;                 // V / BN
   int stages;
-  int ks;                 // 64-wide K blocks per ring stage and per h signal (1 or 2)
+  int ks;                 // 64-wide K blocks per h group (one generator signal; 1 or 2)
+  int kr;                 // 64-wide K blocks per W_o ring stage (>= ks; one TMA / MMA hand-off)
   const __nv_bfloat16* F;   // [B*T][H] bf16
   const __nv_bfloat16* G;   // [B*(U+1)][H] bf16
   const __nv_bfloat16* b_o;
@@ -208,8 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   uint8_t* ring = hhi + KB_hi * 16384;                            // stages x ks K blocks of W_o
   const int fg_stride = 2 * p.H + 16;                             // padded bf16 row (bank spread)
   constexpr int KBB = PAIR ? kStageBytes / 2 : kStageBytes;      // this CTA's rows of one K block of a W_o tile
-  const int STAGE = p.ks * KBB;
-  const int ngrp = (p.KB + p.ks - 1) / p.ks;                      // K-block groups (one ring stage each)
+  const int STAGE = p.kr * KBB;
+  const int ngrp = (p.KB + p.ks - 1) / p.ks;                      // h groups of ks K blocks
+  const int nst = (p.KB + p.kr - 1) / p.kr;                       // ring stages per V tile
   uint8_t* fgs = ring + p.stages * STAGE;                         // TB F rows then UB G rows of this tile
   __nv_bfloat16* bias_s = (__nv_bfloat16*)(fgs + (p.stage_fg ? fg_bytes(p.TB, p.UB, p.H) : 0));   // b_o (bf16)
   uint8_t* stage_s = (uint8_t*)(bias_s + ((p.Vx + 511) & ~511));  // per epilogue warp: srows x 80 B
@@ -288,12 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       bool ok = true;
       for (int it = slot; it < niter && ok; it += nslots) {
         for (int n = 0; n < p.nV && ok; ++n) {
-          for (int g = 0; g < ngrp; ++g) {
+          for (int si = 0; si < nst; ++si) {
             if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) {
               ok = false;
               break;
             }
-            const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
+            const int kb0 = si * p.kr, nk = min(p.kr, p.KB - kb0);
             if (!elect_one()) {
               // other lanes: nothing to issue
             } else if (PAIR) {
@@ -337,13 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
           }
           tc_fence_after();
           const uint32_t dt = tbase + a * BN;
-          for (int g = 0; g < ngrp; ++g) {
+          int g_ready = 0;                  // h groups waited for in this tile (first V tile only)
+          for (int si = 0; si < nst; ++si) {
+            const int kb0 = si * p.kr, nk = min(p.kr, p.KB - kb0);
             if (n == 0) {
-              // h blocks of group g written by the generators (TMEM stores / shared stores)
-              if (!(PAIR ? warp_wait_cluster(&hfull[g], hph, abort_flag) : warp_wait(&hfull[g], hph, abort_flag))) {
-                ok = false;
-                break;
+              // h groups the stage's K blocks belong to, written by the generators
+              const int g_last = (kb0 + nk - 1) / p.ks;
+              for (; g_ready <= g_last && ok; ++g_ready) {
+                if (!(PAIR ? warp_wait_cluster(&hfull[g_ready], hph, abort_flag)
+                           : warp_wait(&hfull[g_ready], hph, abort_flag)))
+                  ok = false;
               }
+              if (!ok) break;
               tc_fence_after();
             }
             // W_o stage landed (TMA completion is ordered by the mbarrier itself)
@@ -351,7 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               ok = false;
               break;
             }
-            const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
             if (elect_one()) {
               for (int kk = 0; kk < nk; ++kk) {
                 const int kb = kb0 + kk;
@@ -376,7 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
                 }
               }
               commit_all(&empty[s]);
-              if (n == p.nV - 1) commit_all(&hempty[g]);   // h group g is free once these MMAs finish
+              if (n == p.nV - 1) {
+                // an h group is free once the MMAs of its last K block finish
+                for (int g = kb0 / p.ks; g < ngrp; ++g) {
+                  const int g_end = min((g + 1) * p.ks, p.KB) - 1;
+                  if (g_end >= kb0 + nk) break;
+                  commit_all(&hempty[g]);
+                }
+              }
             }
             __syncwarp();
             if (++s == p.stages) {
@@ -1038,7 +1051,16 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
     // two K blocks per ring stage (half as many barrier polls in the MMA issuer)
     // while that still leaves at least three stages
     p.ks = stages_for(p.KB, p.Vx, p.TB, p.UB, 2 * kb_bytes, fg) >= 3 ? 2 : 1;
-    stage_bytes = p.ks * kb_bytes;
+    // ring stages of up to 4 K blocks while two stages still fit: fewer
+    // stage hand-offs per MMA (measured: 4 blocks beat 2 on medium and large,
+    // most in the forward pass without z stores)
+    p.kr = p.ks;
+    for (int kr = 4; kr > p.ks; --kr)
+      if (stages_for(p.KB, p.Vx, p.TB, p.UB, kr * kb_bytes, fg) >= 2) {
+        p.kr = kr;
+        break;
+      }
+    stage_bytes = p.kr * kb_bytes;
     p.stages = stages_for(p.KB, p.Vx, p.TB, p.UB, stage_bytes, fg);
   };
   // stage the F / G rows in shared memory unless that leaves the W_o ring
