@@ -724,6 +724,20 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
 // Every thread exchanges through a parity-double-buffered shared array
 // xa[parity][k][thread] (one barrier per step, no shuffles): dynamic shared
 // memory of 2 (DM+2) blockDim floats.
+// exp2 / log2 by the hardware approximations (ex2(-inf) = 0, lg2(0) = -inf)
+constexpr float kLog2eDp = 1.4426950408889634f;
+constexpr float kLn2Dp = 0.6931471805599453f;
+__device__ __forceinline__ float ex2_dp(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_dp(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int DM>
 struct TdtOps {
   float bl, ll;
@@ -840,18 +854,35 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
                          label_lp, dur_lp);
         const int t = cell_t(step);
         const bool valid = u <= Ub && t >= 0 && t < Tb;
-        float pb = -INFINITY, pl = -INFINITY, qk[DM + 1];
+        // the cell's edge terms (blank eb[k], label el[k]) against one shared
+        // maximum: one exp2 per term and one log per sum needed (PB, PL, each
+        // duration's q, beta) instead of a log-add-exp per term and sum; a
+        // term that underflows against the maximum would vanish from every
+        // posterior anyway
+        float eb[DM + 1], el[DM + 1];
+        float mx = -INFINITY;
 #pragma unroll
         for (int k = 0; k <= DM; ++k) {
           // thread u+1's beta on diagonal s + k + 1, i.e. at (t + k, u + 1)
           const float nb = u + 1 < nth ? X((step + 1) & 1, k + 1, u + 1) : -INFINITY;
-          const float eb = k >= 1 ? o.bl + o.dl[k] + hist[k] : -INFINITY;
-          const float el = (u < Ub && t + k < Tb) ? o.ll + o.dl[k] + nb : -INFINITY;
-          pb = log_add_exp(pb, eb);
-          pl = log_add_exp(pl, el);
-          qk[k] = log_add_exp(eb, el);
+          eb[k] = k >= 1 ? o.bl + o.dl[k] + hist[k] : -INFINITY;
+          el[k] = (u < Ub && t + k < Tb) ? o.ll + o.dl[k] + nb : -INFINITY;
+          mx = fmaxf(mx, fmaxf(eb[k], el[k]));
         }
-        const float bt = log_add_exp(pb, pl);
+        const bool none = mx == -INFINITY;        // no edge leaves the cell: everything -inf
+        const float mk = none ? 0.f : mx * kLog2eDp;
+        float sb = 0.f, sl = 0.f, qk[DM + 1];
+#pragma unroll
+        for (int k = 0; k <= DM; ++k) {
+          const float xb = ex2_dp(fmaf(eb[k], kLog2eDp, -mk));   // 0 for -inf terms
+          const float xl = ex2_dp(fmaf(el[k], kLog2eDp, -mk));
+          sb += xb;
+          sl += xl;
+          qk[k] = none ? -INFINITY : mx + lg2_dp(xb + xl) * kLn2Dp;
+        }
+        const float pb = none ? -INFINITY : mx + lg2_dp(sb) * kLn2Dp;
+        const float pl = none ? -INFINITY : mx + lg2_dp(sl) * kLn2Dp;
+        const float bt = none ? -INFINITY : mx + lg2_dp(sb + sl) * kLn2Dp;
         if (valid) {
           const size_t c = base + (size_t)t * Up1 + u;
           beta_b[c] = pb;
