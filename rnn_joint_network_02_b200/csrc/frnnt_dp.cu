@@ -542,6 +542,10 @@ __global__ void dp_band_kernel(int T, int U, int S, const int32_t* __restrict__ 
 // lane 0 walks the best alignment back.
 __device__ __forceinline__ float comb(bool viterbi, float a, float b) { return viterbi ? fmaxf(a, b) : log_add_exp(a, b); }
 
+// SP: the band width rounded up to a power of two (4 .. 32): the scan's levels
+// are unrolled (levels past S leave the band's lanes unchanged), and a lane
+// that takes no part in a level keeps its value by a select, not a branch.
+template <int SP>
 __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, const int32_t* __restrict__ bounds,
                                                           const float* __restrict__ blank_lp,
                                                           const float* __restrict__ label_lp, float* __restrict__ alpha,
@@ -595,13 +599,14 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       float c = ol;
       float x = a;
       // inclusive scan over lanes (the band's S lanes need log2 S steps)
-      for (int off = 1; off < S; off <<= 1) {
+#pragma unroll
+      for (int off = 1; off < SP; off <<= 1) {
         const float xa = __shfl_up_sync(0xffffffffu, x, off);
         const float xc = __shfl_up_sync(0xffffffffu, c, off);
-        if (lane >= off) {
-          x = comb(viterbi, x, xa + c);
-          c = xc + c;
-        }
+        const bool in = lane >= off;
+        const float xn = comb(viterbi, x, xa + c);
+        c = in ? xc + c : c;
+        x = in ? xn : x;
       }
       if (!valid) x = -INFINITY;
       if (lane < S) {
@@ -678,13 +683,14 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
       float y = valid ? bb : -INFINITY;
       float c = ol;
       // inclusive scan from the right
-      for (int off = 1; off < S; off <<= 1) {
+#pragma unroll
+      for (int off = 1; off < SP; off <<= 1) {
         const float ya = __shfl_down_sync(0xffffffffu, y, off);
         const float yc = __shfl_down_sync(0xffffffffu, c, off);
-        if (lane + off < 32) {
-          y = comb(false, y, c + ya);
-          c = c + yc;
-        }
+        const bool in = lane + off < 32;
+        const float yn = comb(false, y, c + ya);
+        c = in ? c + yc : c;
+        y = in ? yn : y;
       }
       if (!valid) y = -INFINITY;
       if (lane < S) beta[base + (size_t)t * S + lane] = y;
@@ -960,7 +966,10 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
     const int smem = s.T * 4 * (L.path ? 2 : 1);
     if (smem <= 48 * 1024) {
       dim3 grid(s.B, L.path ? 1 : 2);
-      dp_band_warp_kernel<<<grid, 32, smem, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
+      const int sp = s.S <= 4 ? 4 : s.S <= 8 ? 8 : s.S <= 16 ? 16 : 32;
+      auto kern = sp == 4 ? dp_band_warp_kernel<4> : sp == 8 ? dp_band_warp_kernel<8>
+                : sp == 16 ? dp_band_warp_kernel<16> : dp_band_warp_kernel<32>;
+      kern<<<grid, 32, smem, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
                                                   L.path, T_len, U_len, loss);
     } else {
       dp_band_kernel<<<s.B, 32, 0, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta, L.path,
