@@ -996,6 +996,48 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
   }
 }
 
+// The same h rows, one block per cell tile (whole lattice): the tile's TB F rows
+// and UB G rows are read once into shared memory (instead of once per row:
+// each F row serves UB rows, each G row TB rows), then 8 warps write the
+// tile's 128 rows, 16-byte stores.  Dynamic shared memory (TB + UB) H bf16.
+__global__ void __launch_bounds__(256) hidden_tiles_kernel(JointParams p, int row_tile0) {
+  extern __shared__ __align__(16) __nv_bfloat16 fg_s[];   // [TB][H] F rows, then [UB][H] G rows
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int H = p.H, HS = p.HS, Up1 = p.U + 1, TB = p.TB, UB = p.UB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cpr = H / 8;                                    // 16-byte chunks per row
+  for (int tile = p.tile_begin + blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int4 td = p.tiles[tile];
+    __syncthreads();                                        // the previous tile's rows are written
+    for (int i = threadIdx.x; i < (TB + UB) * cpr; i += blockDim.x) {
+      const int rr = i / cpr, k = (i % cpr) * 8;
+      const __nv_bfloat16* src = rr < TB ? p.F + ((size_t)td.x * p.T + min(td.y + rr, p.T - 1)) * H
+                                         : p.G + ((size_t)td.x * Up1 + min(td.z + rr - TB, p.U)) * H;
+      *(uint4*)(fg_s + (size_t)rr * H + k) = __ldg((const uint4*)(src + k));
+    }
+    __syncthreads();
+    for (int r = warp; r < 128; r += blockDim.x >> 5) {
+      const RowInfo ri = row_info(p, td, r);
+      __nv_bfloat16* hr = p.hbuf + ((size_t)(tile - row_tile0) * 128 + r) * HS;
+      const __nv_bfloat16* Fr = fg_s + (size_t)(r / UB) * H;
+      const __nv_bfloat16* Gr = fg_s + (size_t)(TB + r % UB) * H;
+      for (int k = lane * 8; k < H; k += 256) {
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (ri.valid) {
+          const uint4 f = *(const uint4*)(Fr + k), g = *(const uint4*)(Gr + k);
+          o.x = tanh_bf16x2(add_bf16x2(f.x, g.x));
+          o.y = tanh_bf16x2(add_bf16x2(f.y, g.y));
+          o.z = tanh_bf16x2(add_bf16x2(f.z, g.z));
+          o.w = tanh_bf16x2(add_bf16x2(f.w, g.w));
+        }
+        *(uint4*)(hr + k) = o;
+      }
+      for (int k = H + lane * 8; k < HS; k += 256)
+        *(uint4*)(hr + k) = make_uint4((k == H && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 // dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
 // whose column H is the sum of dz over cells.
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, const float* __restrict__ db,
@@ -1397,7 +1439,18 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   p.bounds = j.bounds;
   p.S = j.s.S;
   p.hbuf = (__nv_bfloat16*)j.hbuf;
-  hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
+  if (j.s.S == 0) {
+    // whole lattice: one block per cell tile, F and G rows read once per tile
+    const int smem = (j.TB + j.UB) * j.s.H * 2;
+    static int smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+      cudaFuncSetAttribute(hidden_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      smem_set = smem;
+    }
+    hidden_tiles_kernel<<<sms() * (blocks_per_sm >= 4 ? 4 : blocks_per_sm), 256, smem, st>>>(p, row_tile0);
+  } else {
+    hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
+  }
   note_launch();
 }
 
