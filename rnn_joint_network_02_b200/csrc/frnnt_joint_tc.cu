@@ -1030,10 +1030,12 @@ __global__ void __launch_bounds__(256) hidden_tiles_kernel(JointParams p, int ro
           o.z = tanh_bf16x2(add_bf16x2(f.z, g.z));
           o.w = tanh_bf16x2(add_bf16x2(f.w, g.w));
         }
-        *(uint4*)(hr + k) = o;
+        // streaming stores (evict first): the rows are read back only by the
+        // later GEMMs, and should not push the concurrent DP's data out of L2
+        __stcs((uint4*)(hr + k), o);
       }
       for (int k = H + lane * 8; k < HS; k += 256)
-        *(uint4*)(hr + k) = make_uint4((k == H && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u);
+        __stcs((uint4*)(hr + k), make_uint4((k == H && ri.valid) ? 0x3F80u : 0u, 0u, 0u, 0u));
     }
   }
 }
