@@ -257,7 +257,8 @@ void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st);
 // W_x = [W_o; W_d; 0] [Vx][H] and b_x = [b_o; b_d; 0] [Vx] (bf16).
 void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const void* W_d, const void* b_d, void* W_x,
                         void* b_x, cudaStream_t st);
-// blocks_per_sm: 256-thread blocks per SM of the grid (fewer leave room for work running beside it)
+// blocks_per_sm: 256-thread blocks per SM of the row-by-row kernel (pruned lattice); the whole
+// lattice's tile-by-tile kernel sizes its own grid (up to 6 blocks per SM, as its shared memory allows)
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
 // dW_o = acc[:, :H]; db_o = db (when non-null) or acc[:, H]; acc rows of hidden_stride(H)
 void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st,

@@ -1449,7 +1449,11 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
       cudaFuncSetAttribute(hidden_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       smem_set = smem;
     }
-    hidden_tiles_kernel<<<sms() * (blocks_per_sm >= 4 ? 4 : blocks_per_sm), 256, smem, st>>>(p, row_tile0);
+    // up to 6 resident blocks per SM (measured best beside the DP on medium),
+    // fewer when their shared memory does not fit: one full wave
+    int hb = (220 * 1024) / smem;
+    hb = hb < 1 ? 1 : (hb > 6 ? 6 : hb);
+    hidden_tiles_kernel<<<sms() * hb, 256, smem, st>>>(p, row_tile0);
   } else {
     hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
   }
