@@ -27,7 +27,8 @@ def _check(out, ref, tol=2e-3):
 @pytest.mark.parametrize("variant", [0, 1, 2, 3])
 @pytest.mark.parametrize("a_mn", [False, True])
 @pytest.mark.parametrize("b_mn", [False, True])
-@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 256, 128), (296, 640, 520), (1000, 512, 256)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 256, 128), (296, 640, 520), (1000, 512, 256), (200, 608, 192),
+                                   (312, 448, 128)])
 def test_store_f32(cuda_ok, a_mn, b_mn, M, N, K, variant):
     """variant 0: one CTA per 128-row tile; 1: CTA pairs on 256-row tiles (cta_group::2);
     2 / 3: the same with 256-wide N tiles whatever N (a ragged last tile)."""
