@@ -110,7 +110,8 @@ typedef struct {
 enum {
   FRNNT_OK = 0,
   FRNNT_ERR_NULL = 1,          /* a required pointer is NULL                  */
-  FRNNT_ERR_DIMS = 2,          /* a size <= 0, blank outside [0,V), U+1 > 1024 */
+  FRNNT_ERR_DIMS = 2,          /* a size <= 0, blank outside [0,V), U+1 > 1024, or dims that break
+                                  the pruned / duration rules or go to the wrong entry point */
   FRNNT_ERR_WORKSPACE = 3,     /* workspace_bytes smaller than required       */
   FRNNT_ERR_UNSUPPORTED = 4,   /* unknown dtype / mode / path value            */
   FRNNT_ERR_CUDA = 5,          /* a CUDA launch or query failed                */

@@ -590,7 +590,9 @@ extern "C" const char* frnnt_error_string(int code) {
   switch (code) {
     case FRNNT_OK: return "ok";
     case FRNNT_ERR_NULL: return "a required pointer is NULL";
-    case FRNNT_ERR_DIMS: return "invalid dimensions (size <= 0, blank outside [0,V), or U+1 > 1024)";
+    case FRNNT_ERR_DIMS:
+      return "invalid dimensions (a size <= 0, blank outside [0,V), U+1 > 1024, a pruned / duration rule "
+             "broken, or dims for another entry point)";
     case FRNNT_ERR_WORKSPACE: return "workspace smaller than frnnt_workspace_size";
     case FRNNT_ERR_UNSUPPORTED: return "unsupported dtype, mode or path";
     case FRNNT_ERR_CUDA: return "a CUDA launch failed";
