@@ -194,7 +194,7 @@ bool use_tc(const frnnt_dims* d) {
   if (d->dtype != FRNNT_BF16 || d->path != FRNNT_PATH_AUTO) return false;
   if (d->B > 1024) return false;
   if (d->H % 64 || d->D_enc % 32 || d->D_pred % 32) return false;
-  return joint_tc_supported(d->H, d->n_dur > 0 ? d->V + 128 : d->V, d->U, d->prune_S);
+  return joint_tc_supported(d->H, d->n_dur > 0 ? d->V + 128 : d->V, d->T, d->U, d->prune_S);
 }
 
 // The token-and-duration transducer runs on the tensor-core kernels, with the

@@ -226,11 +226,11 @@ struct JointLaunch {
   const int32_t* bounds;        // pruned lattice (s.S > 0): [B][T] first label position of each frame's band
   int store_h = 0;              // modes 1 and 2: the generators also write the h rows of hbuf
 };
-bool joint_tc_supported(int H, int V, int U, int S);
+bool joint_tc_supported(int H, int V, int T, int U, int S);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the
 // dW_o GEMM's N is a whole number of its N tiles.
 inline int hidden_stride(int H) { return H >= 512 ? ((H + 1 + 255) / 256) * 256 : ((H + 1 + 127) / 128) * 128; }
-void tile_shape(int U, int* TB, int* UB);
+void tile_shape(int T, int U, int* TB, int* UB);
 // Cell tile of the shape: TB frames x UB label positions, or for a pruned
 // lattice TB frames x (S rounded up to a power of two) band positions.
 void tile_shape_of(const Shape& s, int* TB, int* UB);

@@ -37,7 +37,7 @@ namespace frnnt {
 
 using namespace sm100;
 
-void tile_shape(int U, int* TB, int* UB);
+void tile_shape(int T, int U, int* TB, int* UB);
 
 namespace {
 
@@ -1164,9 +1164,10 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
 }  // namespace
 
 // ------------------------------------------------------------------ host entry points
-bool joint_tc_supported(int H, int V, int U, int S) {
+bool joint_tc_supported(int H, int V, int T, int U, int S) {
   if (H % 64 || H > 1024 || V % 128) return false;
   Shape s{};
+  s.T = T;
   s.U = U;
   s.S = S;
   int TB, UB;
@@ -1174,13 +1175,17 @@ bool joint_tc_supported(int H, int V, int U, int S) {
   return stages_for(H / 64, V, TB, UB, kStageBytes, false) >= 2;
 }
 
-void tile_shape(int U, int* TB, int* UB) {
-  // label positions per tile: a power of two near U+1 so ragged u-blocks waste little
+void tile_shape(int T, int U, int* TB, int* UB) {
+  // label positions per tile.  Up to 16 positions fit one u-block (8 when
+  // that is enough, with 16 frames); above that, the padding of the ragged
+  // tiles at an utterance's edges grows as TB * (U_len+1) + UB * T_len, so
+  // for lengths in proportion to T and U+1 eight positions by 16 frames pad
+  // less than 16 by 8 whenever U+1 < T (both keep 24 F and G rows per tile)
   const int Up1 = U + 1;
-  int ub = 16;
+  int ub;
   if (Up1 <= 8) ub = 8;
   else if (Up1 <= 16) ub = 16;
-  else if (Up1 <= 24) ub = 8;
+  else ub = Up1 < T ? 8 : 16;
   *UB = ub;
   *TB = 128 / ub;
 }
@@ -1192,7 +1197,7 @@ void tile_shape_of(const Shape& s, int* TB, int* UB) {
     *UB = sp;
     *TB = 128 / sp;
   } else {
-    tile_shape(s.U, TB, UB);
+    tile_shape(s.T, s.U, TB, UB);
   }
 }
 
