@@ -62,11 +62,11 @@ def parse():
 # An entry is removed whenever its kernel changes, so the roofline's traffic is
 # null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dWo", "marginal"): (1.176242e9 + 0.009391e9,
+    ("medium", "untiled", "bwd_dWo", "marginal"): (1.204969e9 + 0.008939e9,
                                                    "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "bwd_dh", "marginal"): (0.642734e9 + 0.019768e9,
+    ("medium", "untiled", "bwd_dh", "marginal"): (0.628156e9 + 0.015830e9,
                                                   "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd", "marginal"): (0.009256e9 + 0.572416e9,
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009181e9 + 0.556763e9,
                                                      "profiles/ncu_joint_tc_medium_untiled.md"),
 }
 
