@@ -37,6 +37,17 @@ FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A, int a_mn,
  * additions. */
 FRNNT_API int frnnt_test_joint_variant(int variant);
 
+/* Failure-detection test setting: each of the next n tensor-core GEMM launches
+ * (frnnt_test_gemm_bf16, or the GEMMs inside frnnt_fwd_bwd*) has every CTA
+ * skip the load of its first K block, and the arrival that would announce it,
+ * so the MMA issuer's bounded wait on that stage runs out (about 2 s).  The
+ * kernel then stops every role, frees its tensor memory and ORs
+ * FRNNT_STATUS_TIMEOUT into the call's status word (when one is given); the
+ * context stays usable and later launches run normally.  That GEMM's output is
+ * left incomplete.  n <= 0 clears the setting.  Process-wide, not thread-safe
+ * (set it between calls).  Returns the previous count. */
+FRNNT_API int frnnt_test_lose_gemm_loads(int n);
+
 #ifdef __cplusplus
 }
 #endif

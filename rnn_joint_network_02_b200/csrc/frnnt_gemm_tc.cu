@@ -44,6 +44,7 @@ struct GemmParams {
   const int* dyn_count;
   int dyn_base, dyn_scale, dyn_dim;
   CellMap cells;
+  int lose_first_load;   // test setting: no CTA loads (or announces) its first K block
 };
 
 // Effective problem after the optional device-side limit on M or K.
@@ -396,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      bool lose = p.lose_first_load != 0;
       for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
         int m0, nt, kb0, kb1;
         if (!unit_coords(unit, p, eff, m0, nt, kb0, kb1)) continue;
@@ -405,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (elect_one()) {
+          if (lose) {
+            lose = false;   // the stage's full barrier never completes: its consumer's wait runs out
+          } else if (elect_one()) {
             uint8_t* sa = smem + s * S::STAGE_BYTES;
             uint8_t* sb = sa + S::A_BYTES;
             mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
@@ -614,6 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      bool lose = p.lose_first_load != 0;
       for (int unit = pair; unit < units && ok; unit += npairs) {
         int m0, nt, kb0, kb1;
         if (!unit_coords2(unit, p, eff, m0, nt, kb0, kb1)) continue;
@@ -624,7 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (elect_one()) {
+          if (lose) {
+            lose = false;   // the leader's full barrier never completes: the MMA issuer's wait runs out
+          } else if (elect_one()) {
             uint8_t* sa = smem + s * S::STAGE_BYTES;
             uint8_t* sb = sa + S::A_BYTES;
             const uint32_t fl = mapa_shared(smem_u32(&full[s]), 0);
@@ -769,6 +776,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+int g_lose_loads = 0;   // GEMM launches left whose first K block load is dropped (test setting)
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -892,6 +901,11 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   p.dyn_scale = g.dyn_scale;
   p.dyn_dim = g.dyn_dim;
   p.cells = g.cells;
+  p.lose_first_load = 0;
+  if (g_lose_loads > 0) {
+    --g_lose_loads;
+    p.lose_first_load = 1;
+  }
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
   bool launched;
   if (pair) {
@@ -923,6 +937,12 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
     else launched = launch_t<128, 6, true, true>(ta, tb, p, grid, st);
   }
   return launched ? FRNNT_OK : FRNNT_ERR_CUDA;
+}
+
+int lose_gemm_loads(int n) {
+  const int prev = g_lose_loads;
+  g_lose_loads = n < 0 ? 0 : n;
+  return prev;
 }
 
 }  // namespace frnnt

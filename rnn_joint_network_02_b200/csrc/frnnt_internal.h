@@ -198,6 +198,10 @@ struct GemmTcArgs {
                        // GEMM_EPI_DTANH_SEG: the same dpre summed into cells.dF / cells.dG, nothing stored
 };
 int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
+// Test setting: the next n gemm_tc launches each drop their CTAs' first K block
+// load (so a bounded wait expires and the status word gets FRNNT_STATUS_TIMEOUT);
+// returns the previous count.  Process-wide, not thread-safe.
+int lose_gemm_loads(int n);
 
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
                        uint32_t box_inner, uint32_t box_outer);

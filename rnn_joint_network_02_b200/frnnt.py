@@ -27,7 +27,7 @@ EXPORTED = ("frnnt_workspace_size", "frnnt_fwd_bwd", "frnnt_error_string", "frnn
             "frnnt_profile_read", "frnnt_fwd_bwd_noalloc", "frnnt_fwd_bwd_pruned", "frnnt_fwd_bwd_tdt")
 MAX_DURATIONS = 8
 NOALLOC_MAX_BYTES = 64 * 1024 * 1024
-TEST_HOOKS = ("frnnt_test_gemm_bf16", "frnnt_test_joint_variant")
+TEST_HOOKS = ("frnnt_test_gemm_bf16", "frnnt_test_joint_variant", "frnnt_test_lose_gemm_loads")
 
 
 class Dims(ctypes.Structure):
@@ -51,10 +51,11 @@ class FrnntError(RuntimeError):
 
 class FrnntStatusError(RuntimeError):
     def __init__(self, bits: int):
-        names = [n for n, v in (("length", STATUS_LENGTH), ("label", STATUS_LABEL), ("timeout", STATUS_TIMEOUT),
-                                ("bounds", STATUS_BOUNDS))
+        names = [n for n, v in (("invalid lengths", STATUS_LENGTH), ("invalid labels", STATUS_LABEL),
+                                ("a bounded device wait timed out", STATUS_TIMEOUT),
+                                ("invalid pruning bounds", STATUS_BOUNDS))
                  if bits & v]
-        super().__init__(f"frnnt device status {bits}: invalid {', '.join(names)}")
+        super().__init__(f"frnnt device status {bits}: {'; '.join(names)}")
         self.bits = bits
 
 
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.frnnt_test_gemm_bf16.restype = ctypes.c_int
         L.frnnt_test_joint_variant.argtypes = [ctypes.c_int]
         L.frnnt_test_joint_variant.restype = ctypes.c_int
+        L.frnnt_test_lose_gemm_loads.argtypes = [ctypes.c_int]
+        L.frnnt_test_lose_gemm_loads.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -250,7 +253,7 @@ def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=No
 
 
 def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: int = 0, k_splits: int = 1,
-                   out=None, stream=None, variant: int = -1):
+                   out=None, stream=None, variant: int = -1, status=None):
     """Test hook: the tensor-core GEMM D = A * B (see include/frnnt_testing.h).
     A is [M][K] (a_mn False) or [K][M]; B is [N][K] (b_mn False) or [K][N]."""
     if out is None:
@@ -258,11 +261,18 @@ def test_gemm_bf16(A, B, a_mn: bool, b_mn: bool, M: int, N: int, K: int, epi: in
     if stream is None:
         stream = torch.cuda.current_stream(A.device)
     rc = lib().frnnt_test_gemm_bf16(M, N, K, _ptr(A), int(a_mn), A.stride(0), _ptr(B), int(b_mn), B.stride(0), epi,
-                                    k_splits, _ptr(out), out.stride(0), variant, None,
+                                    k_splits, _ptr(out), out.stride(0), variant, _ptr(status),
                                     ctypes.c_void_p(stream.cuda_stream))
     if rc != OK:
         raise FrnntError(rc, error_string(rc))
     return out
+
+
+def lose_gemm_loads(n: int) -> int:
+    """Test setting (include/frnnt_testing.h): the next n tensor-core GEMM
+    launches drop their first K block load, so their bounded wait runs out and
+    the status word gets STATUS_TIMEOUT.  Returns the previous count."""
+    return int(lib().frnnt_test_lose_gemm_loads(int(n)))
 
 
 def set_joint_variant(variant: int) -> int:
