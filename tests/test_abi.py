@@ -154,3 +154,55 @@ def test_tdt_dims_rules():
     targs[0] = ctypes.byref(tdt)
     targs[7] = None                                     # missing W_d
     assert lib.frnnt_fwd_bwd_tdt(*targs) == 1
+
+
+C_USER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "frnnt.h"
+#include "frnnt_testing.h"
+
+int main(void) {
+  frnnt_dims d;
+  size_t tiled = 0, untiled = 0;
+  memset(&d, 0, sizeof d);
+  d.B = 16; d.T = 400; d.U = 80; d.D_enc = 512; d.D_pred = 640; d.H = 640; d.V = 1024; d.blank = 0;
+  d.dtype = FRNNT_BF16; d.mode = FRNNT_TILED; d.path = FRNNT_PATH_AUTO; d.loss = FRNNT_LOSS_MARGINAL;
+  if (frnnt_workspace_size(&d, &tiled) != FRNNT_OK) return 2;
+  d.mode = FRNNT_UNTILED;
+  if (frnnt_workspace_size(&d, &untiled) != FRNNT_OK) return 3;
+  d.blank = d.V;
+  if (frnnt_workspace_size(&d, &untiled) != FRNNT_ERR_DIMS) return 4;
+  if (frnnt_workspace_size(NULL, &untiled) != FRNNT_ERR_NULL) return 5;
+  printf("%zu %zu %s|%s\n", tiled, untiled, frnnt_version(), frnnt_error_string(FRNNT_ERR_ALIGN));
+  return 0;
+}
+"""
+
+
+def test_headers_are_plain_c_and_host_calls_link(tmp_path):
+    """The public headers compile as strict C11 (no C++ or CUDA types in the
+    interface) and a C program linked against the library makes the host-only
+    calls: workspace sizing for both modes, argument errors, strings."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    frnnt.lib()      # the library exists (raises with a build hint otherwise)
+    src = tmp_path / "user.c"
+    src.write_text(C_USER)
+    exe = tmp_path / "user"
+    libdir = os.path.dirname(frnnt.LIB_PATH)
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Wpedantic", "-Wstrict-prototypes", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lfrnnt",
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    tiled, untiled = int(out[0]), int(out[1])
+    assert 0 < tiled < untiled, (tiled, untiled)
+    size = ctypes.c_size_t(0)
+    dims = frnnt.make_dims(16, 400, 80, 512, 640, 640, 1024, dtype="bf16", mode="untiled")
+    assert frnnt.lib().frnnt_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == frnnt.OK
+    assert size.value == untiled, "C and Python callers see the same struct layout"
+    assert out[2].startswith(frnnt.version()) and "aligned" in " ".join(out[2:])
