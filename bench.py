@@ -36,7 +36,7 @@ UNIT = "cells/s"
 L2_BYTES = 126 * 1024 * 1024
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--prune", type=int, default=0,
                    help="pruned lattice: S label positions per frame on a band along the diagonal (0: whole lattice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 # DRAM bytes (read + write) per launch of a stage's kernel, from one ncu
@@ -80,10 +80,16 @@ def peaks():
     return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
 
 
+def modes_of(args):
+    """Modes a run measures; the first is the headline."""
+    return ["untiled", "tiled"] if args.mode == "both" else [args.mode]
+
+
 def config_of(batch, args, n_gpus):
+    """The workload as both arms' JSON lines name it (the headline mode)."""
     d = batch.dims
     return {"workload": args.workload, "B": d["B"], "T": d["T"], "U": d["U"], "D_enc": d["D_enc"],
-            "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": args.mode, "path": args.path,
+            "D_pred": d["D_pred"], "H": d["H"], "V": d["V"], "mode": modes_of(args)[0], "path": args.path,
             "loss": args.loss, "prune_S": args.prune,
             "durations": list(synth.TDT_DURATIONS) if args.loss == "tdt" else None,
             "valid_cells": batch.valid_cells(), "padded_cells": batch.padded_cells(),
@@ -240,7 +246,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(batch, args, 1),
+            "config": config_of(batch, args, args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -413,7 +419,7 @@ def run_ours(args):
     footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
                  4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
 
-    modes = ["untiled", "tiled"] if args.mode == "both" else [args.mode]
+    modes = modes_of(args)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     results = {}
     for m in modes:
@@ -430,7 +436,6 @@ def run_ours(args):
 
     if rank == 0:
         cfg = config_of(batch, args, world)
-        cfg["mode"] = modes[0]
         line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes of the workload)",
