@@ -54,7 +54,7 @@ def test_tiled_workspace_bounded_by_chunk():
 
 
 @pytest.mark.parametrize("field,value,code", [("B", 0, 2), ("H", -1, 2), ("blank", 8, 2), ("U", 1024, 2),
-                                              ("dtype", 7, 4), ("mode", 3, 4), ("path", 9, 4)])
+                                              ("U", 1023, 0), ("dtype", 7, 4), ("mode", 3, 4), ("path", 9, 4)])
 def test_bad_dims_rejected(field, value, code):
     d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
     setattr(d, field, value)

@@ -197,3 +197,19 @@ def test_wide_label_lattice(cuda_ok, loss):
                              d["U_len"], mode=mode, chunk_cells=4096, blank=batch.blank, loss=loss)
         torch.cuda.synchronize()
         compare(l, g, ref, "bf16", extra_note=f"wide lattice {loss}/{mode}")
+
+
+@pytest.mark.parametrize("loss", ["marginal", "viterbi"])
+def test_maximum_label_positions(cuda_ok, loss):
+    """U+1 = 1024, the widest lattice the interface accepts (one DP thread per
+    label position, a full 1024-thread block), both modes."""
+    batch = synth.make(B=2, T=6, U=1023, D_enc=64, D_pred=64, H=128, V=128, dtype="bf16", seed=1023,
+                       T_range=(3, 6), U_range=(1000, 1023), bias_std=0.3)
+    batch.U_len[0] = 1023
+    ref = run_oracle(batch, loss=loss)
+    for mode in ("untiled", "tiled"):
+        d = to_device(batch)
+        l, g = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
+                             d["U_len"], mode=mode, chunk_cells=4096, blank=batch.blank, loss=loss)
+        torch.cuda.synchronize()
+        compare(l, g, ref, "bf16", extra_note=f"U+1 = 1024 {loss}/{mode}")
