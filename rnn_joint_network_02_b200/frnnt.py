@@ -167,6 +167,56 @@ def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", p
                      durations)
 
 
+def _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=None, W_d=None, b_d=None):
+    """Host-side checks before any pointer reaches the library: a tensor of the
+    wrong shape, dtype, layout or device would otherwise be read or written out
+    of bounds by the kernels.  Shapes and dtypes are checked first, then that
+    every tensor lives on the same CUDA device.  Raises ValueError."""
+    if f.dim() != 3 or g.dim() != 3 or W_o.dim() != 2:
+        raise ValueError("f must be [B, T, D_enc], g [B, U+1, D_pred] and W_o [V, H]")
+    B, T, D_enc = f.shape
+    Up1, D_pred = g.shape[1], g.shape[2]
+    V, H = W_o.shape
+    ft = f.dtype
+    if ft not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"f must be float32 or bfloat16, not {ft}")
+    want = [("f", f, (B, T, D_enc), ft), ("g", g, (B, Up1, D_pred), ft), ("W_f", W_f, (D_enc, H), ft),
+            ("W_g", W_g, (D_pred, H), ft), ("W_o", W_o, (V, H), ft), ("b_o", b_o, (V,), ft),
+            ("labels", labels, (B, Up1 - 1), torch.int32), ("T_len", T_len, (B,), torch.int32),
+            ("U_len", U_len, (B,), torch.int32)]
+    if grad_loss is not None:
+        want.append(("grad_loss", grad_loss, (B,), torch.float32))
+    if bounds is not None:
+        want.append(("bounds", bounds, (B, T), torch.int32))
+    if W_d is not None or b_d is not None:
+        if W_d is None or b_d is None or W_d.dim() != 2:
+            raise ValueError("the duration head needs W_d [n_dur, H] and b_d [n_dur]")
+        want += [("W_d", W_d, (W_d.shape[0], H), ft), ("b_d", b_d, (W_d.shape[0],), ft)]
+    if out is not None:
+        want += [("out.loss", out.loss, (B,), torch.float32), ("out.df", out.df, tuple(f.shape), ft),
+                 ("out.dg", out.dg, tuple(g.shape), ft), ("out.dW_f", out.dW_f, (D_enc, H), ft),
+                 ("out.dW_g", out.dW_g, (D_pred, H), ft), ("out.dW_o", out.dW_o, (V, H), ft),
+                 ("out.db_o", out.db_o, (V,), ft), ("out.status", out.status, (4,), torch.int32)]
+        if W_d is not None:
+            if out.dW_d is None or out.db_d is None:
+                raise ValueError("out has no duration-head gradients")
+            want += [("out.dW_d", out.dW_d, tuple(W_d.shape), ft), ("out.db_d", out.db_d, tuple(b_d.shape), ft)]
+    for name, t, shape, dt in want:
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != dt:
+            raise ValueError(f"{name} is {t.dtype}, expected {dt}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if f.device.type != "cuda":
+        raise ValueError("the library computes on the GPU: pass CUDA tensors")
+    for name, t, _, _ in want:
+        if t.device != f.device:
+            raise ValueError(f"{name} is on {t.device}, the call's tensors on {f.device}")
+    if out is not None and out.workspace is not None and out.workspace.device != f.device:
+        raise ValueError(f"the workspace is on {out.workspace.device}, the call's tensors on {f.device}")
+
+
 class Outputs:
     """Preallocated outputs and workspace of one call shape."""
 
@@ -202,6 +252,7 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode
     status word is read back (one 4-byte device-to-host copy, which
     synchronises the stream) and a non-zero status raises FrnntStatusError.
     """
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
     dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss)
     if out is None:
@@ -229,6 +280,7 @@ def fwd_bwd_noalloc(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=No
     array replaces the workspace (``out.workspace`` is not used).  Raises
     FrnntError(FRNNT_ERR_WORKSPACE) when these dims need more than
     NOALLOC_MAX_BYTES of scratch."""
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
     dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss)
     if out is None:
@@ -287,6 +339,7 @@ def fwd_bwd_pruned(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, S: in
     """frnnt_fwd_bwd_pruned: the loss and gradients on the pruned lattice that
     keeps, for frame t of utterance b, the S label positions
     bounds[b,t] <= u < bounds[b,t] + S (bounds: int32 [B, T] on the device)."""
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=bounds)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
     dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss, S)
     if out is None:
@@ -315,6 +368,7 @@ def fwd_bwd_tdt(f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, durati
     weights); ``durations`` is the duration set (frame counts, increasing,
     starting 0, 1).  Returns (loss [B] fp32, dict of gradients including dW_d
     and db_d)."""
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, W_d=W_d, b_d=b_d)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
     dims = dims_of(f, g, W_o, dtype, mode, "auto", chunk_cells, blank, "marginal", 0, tuple(durations))
     if out is None:

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from rnn_joint_network_02_b200 import frnnt
 
@@ -206,3 +207,48 @@ def test_headers_are_plain_c_and_host_calls_link(tmp_path):
     assert frnnt.lib().frnnt_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == frnnt.OK
     assert size.value == untiled, "C and Python callers see the same struct layout"
     assert out[2].startswith(frnnt.version()) and "aligned" in " ".join(out[2:])
+
+
+def _tiny_args():
+    from rnn_joint_network_02_b200 import synth
+    b = synth.workload("tiny")
+    return dict(f=b.f, g=b.g, W_f=b.W_f, W_g=b.W_g, W_o=b.W_o, b_o=b.b_o, labels=b.labels, T_len=b.T_len,
+                U_len=b.U_len)
+
+
+def _fwd_bwd(a, **kw):
+    return frnnt.fwd_bwd(a["f"], a["g"], a["W_f"], a["W_g"], a["W_o"], a["b_o"], a["labels"], a["T_len"],
+                         a["U_len"], **kw)
+
+
+@pytest.mark.parametrize("field,bad,msg", [
+    ("W_f", lambda t: t[:, :-1], "W_f has shape"),
+    ("W_o", lambda t: t.t().contiguous(), "W_o|b_o|W_f"),
+    ("labels", lambda t: t.long(), "labels is torch.int64"),
+    ("labels", lambda t: t[:, :-1], "labels has shape"),
+    ("T_len", lambda t: t[:1], "T_len has shape"),
+    ("W_g", lambda t: t.double(), "W_g is torch.float64"),
+    ("f", lambda t: t.transpose(0, 1).contiguous().transpose(0, 1), "f must be contiguous"),
+])
+def test_binding_rejects_bad_tensors_before_the_library(field, bad, msg):
+    """Shapes, dtypes and layouts are checked on the host before any pointer
+    reaches the library (a wrong one would be read out of bounds on the GPU)."""
+    a = _tiny_args()
+    a[field] = bad(a[field])
+    with pytest.raises(ValueError, match=msg):
+        _fwd_bwd(a)
+
+
+def test_binding_rejects_host_tensors_and_bad_extras():
+    a = _tiny_args()
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _fwd_bwd(a)
+    with pytest.raises(ValueError, match="grad_loss is torch.float64"):
+        _fwd_bwd(a, grad_loss=torch.ones(a["f"].shape[0], dtype=torch.float64))
+    with pytest.raises(ValueError, match="bounds has shape"):
+        frnnt.fwd_bwd_pruned(a["f"], a["g"], a["W_f"], a["W_g"], a["W_o"], a["b_o"], a["labels"], a["T_len"],
+                             a["U_len"], torch.zeros(2, 3, dtype=torch.int32), 4)
+    H = a["W_o"].shape[1]
+    with pytest.raises(ValueError, match="b_d has shape"):
+        frnnt.fwd_bwd_tdt(a["f"], a["g"], a["W_f"], a["W_g"], a["W_o"], a["b_o"], torch.zeros(5, H),
+                          torch.zeros(4), a["labels"], a["T_len"], a["U_len"], (0, 1, 2, 3, 4))
