@@ -918,12 +918,13 @@ void launch_tdt_dp_t(const Shape& s, const Lattice& L, const int32_t* T_len, con
                      int threads, cudaStream_t st) {
   dim3 grid(s.B, 2);
   const int smem = 2 * (DM + 2) * threads * (int)sizeof(float);   // <= 80 KB (DM 8, 1024 threads)
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kDeviceSlots] = {};
+  const int dev = current_device();
+  if (!attr[dev]) {
     cudaFuncSetAttribute(tdt_dp_kernel<DM, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 256 * 4);
     cudaFuncSetAttribute(tdt_dp_kernel<DM, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 512 * 4);
     cudaFuncSetAttribute(tdt_dp_kernel<DM, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * (DM + 2) * 1024 * 4);
-    attr = true;
+    attr[dev] = true;
   }
   if (threads <= 256)
     tdt_dp_kernel<DM, 256><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
@@ -979,10 +980,11 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
     // decision bits in shared memory when they fit in 96 KB
     const long long words = ((long long)s.T * s.Up1 + 31) / 32;
     const int smem = words * 4 <= 96 * 1024 ? (int)(words * 4) : 0;
-    static bool attr = false;
-    if (!attr) {
+    static bool attr[kDeviceSlots] = {};
+    const int dev = current_device();
+    if (!attr[dev]) {
       cudaFuncSetAttribute(dp_viterbi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-      attr = true;
+      attr[dev] = true;
     }
     dp_viterbi_kernel<<<s.B, threads, smem, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.path, T_len,
                                                   U_len, loss, smem > 0 ? 1 : 0);

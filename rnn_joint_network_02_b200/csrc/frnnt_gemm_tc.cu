@@ -793,11 +793,12 @@ template <int BN, int STAGES, bool A_MN, bool B_MN>
 bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
   auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN>;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kDeviceSlots] = {};
+  const int dev = current_device();
+  if (!attr[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) != cudaSuccess)
       return false;
-    attr = true;
+    attr[dev] = true;
   }
   kern<<<grid, kThreads, S::TOTAL, st>>>(ta, tb, p);
   note_launch();
@@ -808,11 +809,12 @@ template <int BN, int STAGES, bool A_MN, bool B_MN>
 bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = Gemm2Smem<BN, STAGES>;
   auto kern = gemm2_tc_kernel<BN, STAGES, A_MN, B_MN>;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kDeviceSlots] = {};
+  const int dev = current_device();
+  if (!attr[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) != cudaSuccess)
       return false;
-    attr = true;
+    attr[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);

@@ -233,6 +233,15 @@ struct JointLaunch {
 bool joint_tc_supported(int H, int V, int T, int U, int S);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the
 // dW_o GEMM's N is a whole number of its N tiles.
+// Per-device slots of the host-side state that CUDA keeps per device (kernel
+// attributes, occupancy answers): a process may drive several GPUs.
+constexpr int kDeviceSlots = 64;
+inline int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kDeviceSlots) d = 0;
+  return d;
+}
+
 inline int hidden_stride(int H) { return H >= 512 ? ((H + 1 + 255) / 256) * 256 : ((H + 1 + 127) / 128) * 128; }
 void tile_shape(int T, int U, int* TB, int* UB);
 // Cell tile of the shape: TB frames x UB label positions, or for a pruned

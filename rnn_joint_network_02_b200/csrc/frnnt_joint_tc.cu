@@ -1115,11 +1115,12 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
   if (p.stages < 2) return FRNNT_ERR_UNSUPPORTED;
   const int smem = smem_fixed(p.KB, p.Vx, p.TB, p.UB, p.srows, p.stage_fg != 0) + p.stages * stage_bytes;
   auto kern = joint_tc_kernel<MODE, PAIR>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[kDeviceSlots] = {};
+  const int dev = current_device();
+  if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return FRNNT_ERR_CUDA;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   if (!PAIR) {
     kern<<<sms(), kThreads, smem, st>>>(tm, p);
@@ -1138,19 +1139,19 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
     attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    static int resident = 0, resident_smem = -1;
-    if (resident_smem != smem) {
+    static int resident[kDeviceSlots] = {}, resident_smem[kDeviceSlots] = {};
+    if (resident_smem[dev] != smem) {
       cfg.gridDim = dim3(sms(), 1, 1);
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = sms() / 2;
       }
-      resident = n < sms() / 2 ? n : sms() / 2;
-      resident_smem = smem;
+      resident[dev] = n < sms() / 2 ? n : sms() / 2;
+      resident_smem[dev] = smem;
     }
     const int pairs = (ntiles_max + 1) / 2;
-    const int npairs = pairs < resident ? (pairs > 0 ? pairs : 1) : resident;
+    const int npairs = pairs < resident[dev] ? (pairs > 0 ? pairs : 1) : resident[dev];
     cfg.gridDim = dim3(2 * npairs, 1, 1);
     if (cudaLaunchKernelEx(&cfg, kern, tm, p) != cudaSuccess) {
       note_launch();
@@ -1449,10 +1450,11 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   if (j.s.S == 0) {
     // whole lattice: one block per cell tile, F and G rows read once per tile
     const int smem = (j.TB + j.UB) * j.s.H * 2;
-    static int smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
+    static int smem_set[kDeviceSlots] = {};
+    const int dev = current_device();
+    if (smem > 48 * 1024 && smem > smem_set[dev]) {
       cudaFuncSetAttribute(hidden_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      smem_set = smem;
+      smem_set[dev] = smem;
     }
     // up to 6 resident blocks per SM (measured best beside the DP on medium),
     // fewer when their shared memory does not fit: one full wave
