@@ -135,8 +135,13 @@ FRNNT_API int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes);
 /* One forward + backward pass over one batch (one call per batch).
  *
  * All pointers are DEVICE pointers on the current device, 16-byte aligned,
- * owned by the caller; the library allocates nothing and keeps no state
- * between calls.  Float tensors are fp32 (FRNNT_F32) or bf16 bit patterns
+ * owned by the caller; the library allocates no device memory and keeps no
+ * data between calls.  Host-side it caches, per device, kernel attributes and
+ * one internal stream with two events (created by the first call on that
+ * device, outside any stream capture), on which part of the work runs beside
+ * the caller's stream.  Calls on different devices may come from different
+ * host threads at the same time; calls on one device must not overlap on the
+ * host (they share that stream's events).  Float tensors are fp32 (FRNNT_F32) or bf16 bit patterns
  * (FRNNT_BF16); b_o and all gradients have that same element type.
  *   grad_loss   [B] fp32 weights w_b of d(sum_b w_b loss_b), or NULL (= 1)
  *   loss        [B] fp32 output, -log P(y_b | x_b) per utterance

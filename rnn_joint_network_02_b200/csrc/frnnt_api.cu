@@ -273,8 +273,9 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
 // occupies one block per utterance and direction), forked from and joined
 // back to the caller's stream with events, so stream order, graph capture and
 // the caller's synchronisation are unaffected.  Shared by all calls on the
-// device: concurrent calls from several host threads stay correct and
-// serialise their side work.
+// device, so calls on one device must not overlap on the host: between one
+// call's record of `fork` and its stream's wait on it, another call's record
+// would redirect that wait (calls on different devices use different slots).
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;     // hidden rows beside the lattice DP
