@@ -353,3 +353,18 @@ def test_validate_bits():
     assert oracle.validate(5, 3, 8, 0, labels, [5, 5], [4, 1]) == oracle.STATUS_LENGTH
     assert oracle.validate(5, 3, 8, 0, labels, [5, 5], [-1, 2]) == (oracle.STATUS_LENGTH
                                                                    | oracle.STATUS_LABEL)
+
+
+def test_golden_file_is_the_oracles_output():
+    """tests/golden/tiny_oracle.json (read by the GPU parity test) is exactly
+    what its generating script's oracle call produces today."""
+    import json
+    import os
+    gold = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_oracle.json")))
+    batch = synth.workload("tiny")
+    f, g, W_f, W_g, W_o, b_o = (t.numpy() for t in batch.float64())
+    res = oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy())
+    assert gold["status"] == res.status == 0
+    np.testing.assert_allclose(gold["loss"], res.loss, rtol=1e-12, atol=0)
+    for name in ("df", "dg", "dW_f", "dW_g", "dW_o", "db_o"):
+        np.testing.assert_allclose(gold[name], getattr(res, name).reshape(-1), rtol=1e-10, atol=1e-14)
