@@ -109,7 +109,113 @@ def test_the_oracle_as_written_passes_the_pins():
 
 
 @pytest.mark.parametrize("what,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")   # a mutant may produce inf - inf
 def test_every_planted_mistake_fails_a_pin(what, old, new):
     assert SOURCE.count(old) == 1, f"mutation site not unique or missing: {old!r}"
     mutant = _load(SOURCE.replace(old, new), "_oracle_mutant")
     assert not _pins_hold(mutant), f"the pins did not notice: {what}"
+
+
+# ---------------------------------------------------------------- maximum approximation and pruned band
+
+from tests.test_oracle_pruned import _band_alignment_scores, _random_bounds  # noqa: E402
+from tests.test_oracle_viterbi import _alignments, _score  # noqa: E402
+
+VITERBI_MUTANTS = [
+    ("ties to the label edge", "            if by_blank >= by_label:\n", "            if by_blank > by_label:\n"),
+    ("max-product label edge from the wrong cell",
+     "by_label = A[t, u - 1] + label_lp[t, u - 1] if u > 0 else NEG_INF",
+     "by_label = A[t, u - 1] + label_lp[t, u] if u > 0 else NEG_INF"),
+    ("final blank left off the best alignment",
+     "    bpath[t, u] = 1.0                      # the final blank", "    pass  # the final blank"),
+    ("backtrack marks the blank edge at the wrong frame", "            t -= 1\n            bpath[t, u] = 1.0\n",
+     "            bpath[t, u] = 1.0\n            t -= 1\n"),
+]
+
+BAND_MUTANTS = [
+    ("band one position short", "M[t, s:min(Ub + 1, s + S)] = True", "M[t, s:min(Ub + 1, s + S - 1)] = True"),
+    ("band start ignored", "        s = int(bounds_b[t])\n", "        s = 0\n"),
+]
+
+
+def _viterbi_pins_hold(mod) -> bool:
+    """Brute-force maximisation (loss and the best alignment's edges) on random
+    batches, and the tie rule on zero logits (every label at frame 0)."""
+    try:
+        for seed in range(3):
+            batch = _batch(10 + seed)
+            params = [t.numpy() for t in batch.float64()]
+            ints = (batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy())
+            res = mod.fwd_bwd(*params, *ints, loss="viterbi", keep_lattice=True)
+            for b in range(2):
+                Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
+                lp = _log_probs_torch(batch, b)
+                labels = batch.labels[b].tolist()
+                best, edges = max(((_score(lp, labels, e), e) for e in _alignments(Tb, Ub)), key=lambda x: x[0])
+                if not abs(-res.loss[b] - best) <= 1e-11 * max(1.0, abs(best)):
+                    return False
+                bp, lq = np.zeros((Tb, Ub + 1)), np.zeros((Tb, Ub + 1))
+                for (t, u), kind in edges:
+                    (bp if kind == "b" else lq)[t, u] = 1.0
+                if not (np.array_equal(res.lattice[b].bpost, bp) and np.array_equal(res.lattice[b].lpost, lq)):
+                    return False
+        batch = _batch(20)
+        params = [t.numpy() for t in batch.float64()]
+        params[4] = np.zeros_like(params[4])
+        params[5] = np.zeros_like(params[5])
+        res = mod.fwd_bwd(*params, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                          loss="viterbi", keep_lattice=True)
+        for b in range(2):
+            Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
+            lat = res.lattice[b]
+            want_l = np.zeros((Tb, Ub + 1))
+            want_l[0, :Ub] = 1.0
+            want_b = np.zeros((Tb, Ub + 1))
+            want_b[:, Ub] = 1.0
+            if not (np.array_equal(lat.lpost, want_l) and np.array_equal(lat.bpost, want_b)):
+                return False
+    except (AssertionError, ValueError, IndexError, FloatingPointError):
+        return False
+    return True
+
+
+def _band_pins_hold(mod) -> bool:
+    """Brute force over the alignments inside random valid bands."""
+    try:
+        for seed in range(3):
+            batch = _batch(30 + seed)
+            S = 2
+            bounds = _random_bounds(batch, S, np.random.default_rng(seed))
+            params = [t.numpy() for t in batch.float64()]
+            res = mod.fwd_bwd(*params, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                              bounds=bounds, S=S)
+            for b in range(2):
+                Tb, Ub = int(batch.T_len[b]), int(batch.U_len[b])
+                sc = _band_alignment_scores(_log_probs_torch(batch, b), batch.labels[b].tolist(), Tb, Ub,
+                                            bounds[b], S)
+                m = max(sc)
+                ref = -(m + np.log(np.sum(np.exp(np.array(sc) - m))))
+                if not abs(res.loss[b] - ref) <= 1e-9 * abs(ref):
+                    return False
+    except (AssertionError, ValueError, IndexError, FloatingPointError):
+        return False
+    return True
+
+
+def test_the_viterbi_and_band_paths_as_written_pass_their_pins():
+    clean = _load(SOURCE, "_oracle_clean2")
+    assert _viterbi_pins_hold(clean) and _band_pins_hold(clean)
+
+
+@pytest.mark.parametrize("what,old,new", VITERBI_MUTANTS, ids=[m[0] for m in VITERBI_MUTANTS])
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")   # a mutant may produce inf - inf
+def test_every_planted_viterbi_mistake_fails_a_pin(what, old, new):
+    assert SOURCE.count(old) == 1, f"mutation site not unique or missing: {old!r}"
+    assert not _viterbi_pins_hold(_load(SOURCE.replace(old, new), "_oracle_vmutant")), what
+
+
+@pytest.mark.parametrize("what,old,new", BAND_MUTANTS, ids=[m[0] for m in BAND_MUTANTS])
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")   # a mutant may produce inf - inf
+def test_every_planted_band_mistake_fails_a_pin(what, old, new):
+    assert SOURCE.count(old) == 1, f"mutation site not unique or missing: {old!r}"
+    assert not _band_pins_hold(_load(SOURCE.replace(old, new), "_oracle_bmutant")), what
