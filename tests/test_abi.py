@@ -252,3 +252,20 @@ def test_binding_rejects_host_tensors_and_bad_extras():
     with pytest.raises(ValueError, match="b_d has shape"):
         frnnt.fwd_bwd_tdt(a["f"], a["g"], a["W_f"], a["W_g"], a["W_o"], a["b_o"], torch.zeros(5, H),
                           torch.zeros(4), a["labels"], a["T_len"], a["U_len"], (0, 1, 2, 3, 4))
+
+
+def test_every_entry_point_is_documented_in_its_header():
+    """Each FRNNT_API declaration directly follows a comment block (what the
+    call computes, its arguments, ownership and errors)."""
+    inc = os.path.join(ROOT, "include")
+    seen = 0
+    for fn in sorted(os.listdir(inc)):
+        if not fn.endswith(".h"):
+            continue
+        lines = open(os.path.join(inc, fn)).read().splitlines()
+        for i, line in enumerate(lines):
+            m = re.search(r"FRNNT_API\s+[\w\s\*]*?\b(frnnt_\w+)\s*\(", line)
+            if m:
+                seen += 1
+                assert i > 0 and lines[i - 1].strip().endswith("*/"), f"{fn}: {m.group(1)} has no doc comment"
+    assert seen == len(_declared_functions())
