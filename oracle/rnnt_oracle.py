@@ -383,7 +383,8 @@ def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None,
 
 def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, loss: str = "marginal",
               bounds=None, S: int = 0):
-    """Per-utterance losses (forward only), used by finite-difference checks."""
+    """Per-utterance losses (forward only): finite-difference checks, and the
+    loss of every utterance of the full-size GPU parity checks."""
     f = np.asarray(f, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     W_f = np.asarray(W_f, dtype=np.float64)
@@ -391,16 +392,21 @@ def loss_only(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, blank: int = 0, lo
     W_o = np.asarray(W_o, dtype=np.float64)
     b_o = np.asarray(b_o, dtype=np.float64)
     B = f.shape[0]
+    V, H = W_o.shape
     out = np.empty(B)
     for b in range(B):
         Tb, Ub = int(T_len[b]), int(U_len[b])
         F, G = projections(f[b, :Tb], g[b, :Ub + 1], W_f, W_g)
-        _, z = joint_logits(F, G, W_o, b_o)
-        lse = log_sum_exp_last(z)
-        blank_lp = z[:, :, blank] - lse
+        blank_lp = np.empty((Tb, Ub + 1))
         label_lp = np.full((Tb, Ub + 1), NEG_INF)
-        for u in range(Ub):
-            label_lp[:, u] = z[:, u, int(labels[b, u])] - lse[:, u]
+        step = _frame_block(Ub, V, H)           # a block of frames at a time, only to bound memory
+        for t0 in range(0, Tb, step):
+            t1 = min(Tb, t0 + step)
+            _, z = joint_logits(F[t0:t1], G, W_o, b_o)
+            lse = log_sum_exp_last(z)
+            blank_lp[t0:t1] = z[:, :, blank] - lse
+            for u in range(Ub):
+                label_lp[t0:t1, u] = z[:, u, int(labels[b, u])] - lse[:, u]
         mask = None if bounds is None else band_mask(bounds[b], S, Tb, Ub)
         if loss == "viterbi":
             A, _ = viterbi_lattice(blank_lp, label_lp, Tb, Ub, mask)
