@@ -53,6 +53,9 @@ def parse(argv=None):
     p.add_argument("--prune", type=int, default=0,
                    help="pruned lattice: S label positions per frame on a band along the diagonal (0: whole lattice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the per-workload block (short, medium, long, large in both modes) and the "
+                        "chunk-size protocol that a one-GPU run adds after the headline")
     return p.parse_args(argv)
 
 
@@ -71,13 +74,25 @@ MEASURED_TRAFFIC = {
 }
 
 
+# Nominal dense bf16 tensor throughput of one B200 (NVIDIA's B200 datasheet
+# figure without 2:4 sparsity), for context beside the measured peaks.
+DATASHEET_BF16_TFLOPS = 2250.0
+# MUFU (tanh, exp2) results per clock per SM; 148 SMs.
+MUFU_PER_CLK_SM = 16
+SMS = 148
+
+
 def peaks():
+    """Roofline denominators: the measured copy bandwidth and the measured
+    dense bf16 GEMM throughput of this machine's B200s (burst: a GEMM timed alone
+    at full clocks, the right denominator for a stage of a millisecond-scale
+    step; sustained: seconds back to back under the power cap)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
         return dict(hbm=d["hbm_gbs"], tensor=d["bf16_tflops"], tensor_sustained=d["bf16_tflops_sustained"],
-                    source="measured")
-    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
 
 
 def modes_of(args):
@@ -197,26 +212,53 @@ def duration_head(batch):
     return synth.duration_head(batch, len(synth.TDT_DURATIONS), seed=5)
 
 
-def oracle_sample(batch, utterance=0, loss="marginal"):
-    """Times the fp64 oracle on one utterance; returns (seconds, metric units)."""
+def oracle_sample(batch, budget_s=10.0, loss="marginal", first=0):
+    """Times the fp64 oracle on utterances first, first+1, ... until ``budget_s``
+    seconds of CPU work (at least one utterance).  The metric's unit is the
+    batch's padded cells B*T*(U+1)*V per second; the oracle computes only
+    valid cells, so the sample stands for the batch in proportion to its valid
+    cells: value = padded units of the batch / (sample time * batch valid cells
+    / sample valid cells).  Also returns the plain valid-cell rate."""
     import numpy as np
 
     import oracle
     f, g, W_f, W_g, W_o, b_o = (t.numpy() for t in batch.float64())
-    w = np.zeros(batch.f.shape[0])
-    w[utterance] = 1.0
-    t0 = time.perf_counter()
+    B = batch.f.shape[0]
+    d = batch.dims
+    W_d = b_d = None
     if loss == "tdt":
         W_d, b_d = (t.double().numpy() for t in duration_head(batch))
-        oracle.tdt_fwd_bwd(f, g, W_f, W_g, W_o, b_o, W_d, b_d, batch.labels.numpy(), batch.T_len.numpy(),
-                           batch.U_len.numpy(), synth.TDT_DURATIONS, grad_loss=w, utterances=[utterance])
-    else:
-        oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
-                       grad_loss=w, utterances=[utterance], loss=loss)
-    dt = time.perf_counter() - t0
-    d = batch.dims
-    units = d["T"] * (d["U"] + 1) * d["V"]      # this utterance's share of B*T*(U+1)*V
-    return dt, units
+    done, secs, valid = [], 0.0, 0
+    for k in range(B):
+        b = (first + k) % B
+        w = np.zeros(B)
+        w[b] = 1.0
+        t0 = time.perf_counter()
+        if loss == "tdt":
+            oracle.tdt_fwd_bwd(f, g, W_f, W_g, W_o, b_o, W_d, b_d, batch.labels.numpy(), batch.T_len.numpy(),
+                               batch.U_len.numpy(), synth.TDT_DURATIONS, grad_loss=w, utterances=[b])
+        else:
+            oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                           grad_loss=w, utterances=[b], loss=loss)
+        secs += time.perf_counter() - t0
+        done.append(b)
+        valid += int(batch.T_len[b]) * (int(batch.U_len[b]) + 1)
+        if secs >= budget_s:
+            break
+    batch_secs = secs * batch.valid_cells() / valid
+    return {"seconds": secs, "utterances": done, "valid_cells": valid, "batch_seconds_est": batch_secs,
+            "value": batch.padded_cells() * d["V"] / batch_secs, "valid_cells_per_s": valid * d["V"] / secs}
+
+
+def oracle_line(batch, name, sample):
+    """The cpu_baseline object of a JSON line from one oracle sample."""
+    return {"value": sample["value"], "unit": UNIT, "cores": cores(), "kind": "oracle",
+            "valid_cells_per_s": sample["valid_cells_per_s"],
+            "sample": (f"{name}: utterances {sample['utterances']} ({sample['valid_cells']} valid cells of the "
+                       f"batch's {batch.valid_cells()}) in {sample['seconds']:.2f} s; value = the batch's "
+                       f"B*T*(U+1)*V over the sample time scaled to the batch's valid cells "
+                       f"({sample['batch_seconds_est']:.1f} s per batch); valid_cells_per_s = the sample's "
+                       f"T_len*(U_len+1)*V per second; numpy fp64, BLAS threads = all cores")}
 
 
 def cores():
@@ -231,37 +273,87 @@ def run_reference(args):
     if rank != 0:
         return
     batch = synth.workload(args.workload)
+    # each step: the oracle on utterance 0 of the workload (a bounded sample,
+    # scaled to the batch by its valid cells; see oracle_sample)
     for _ in range(args.warmup):
-        oracle_sample(batch, loss=args.loss)
-    times = []
-    units = 0
-    for _ in range(args.steps):
-        dt, units = oracle_sample(batch, loss=args.loss)
-        times.append(dt)
-    sec = sum(times) / len(times)
-    value = units / sec
-    Tb, Ub = int(batch.T_len[0]), int(batch.U_len[0])
-    sample = (f"utterance 0 of {args.workload} (T_len={Tb}, U_len={Ub}) per step; "
-              f"units = T*(U+1)*V of one utterance")
+        oracle_sample(batch, budget_s=0.0, loss=args.loss)
+    samples = [oracle_sample(batch, budget_s=0.0, loss=args.loss) for _ in range(args.steps)]
+    secs = sum(x["batch_seconds_est"] for x in samples) / len(samples)
+    value = batch.padded_cells() * batch.dims["V"] / secs
+    cpu = oracle_line(batch, args.workload, samples[-1])
+    cpu["value"] = value
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(batch, args, args.gpus),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores(), "kind": "oracle", "sample": sample},
+            "config": config_of(batch, args, args.gpus), "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ our arm
 
-def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
+def stage_rooflines(batch, mode, stages, steps, valid, n_dur, workload, loss, prune):
+    """Per stage: its algorithmic work over its device time against the peak
+    of its bound (tensor: measured burst dense bf16, also shown against the
+    sustained and datasheet figures; hbm: measured copy bandwidth)."""
+    pk = peaks()
+    out = {}
+    for name, st in stages.items():
+        kind, work = stage_work(batch, name, mode, valid, n_dur)
+        if kind is None or st["ms"] <= 0:
+            continue
+        per_call_ms = st["ms"] / steps
+        tr = None if prune else MEASURED_TRAFFIC.get((workload, mode, name, loss))
+        if kind == "tensor":
+            achieved = work / (per_call_ms / 1e3) / 1e12
+            out[name] = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["tensor"], "traffic": tr[0] if tr else None,
+                         "traffic_source": tr[1] if tr else None, "stage": name,
+                         "ms_per_step": per_call_ms, "launches_per_step": st["launches"] / steps,
+                         "frac_sustained": achieved / pk["tensor_sustained"],
+                         "frac_datasheet": achieved / DATASHEET_BF16_TFLOPS,
+                         "peak_source": pk["source"] + " burst dense bf16 (cuBLAS GEMM timed alone at full "
+                                                       "clocks); frac_sustained: against the power-capped "
+                                                       "sustained figure; frac_datasheet: against 2250 TFLOP/s"}
+        else:
+            achieved = work / (per_call_ms / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm"], "traffic": tr[0] if tr else None,
+                         "traffic_source": tr[1] if tr else None, "stage": name,
+                         "ms_per_step": per_call_ms, "launches_per_step": st["launches"] / steps,
+                         "peak_source": pk["source"] + " copy bandwidth"}
+    return out
+
+
+def mufu_roofline(batch, valid, ms, clocks):
+    """MUFU work of the path, 2H tanh + 2V exp per valid cell (forward and
+    backward), over the whole step against 16 results/clock/SM on 148 SMs at
+    the SM clock seen under load."""
+    d = batch.dims
+    ops = (2.0 * d["H"] + 2.0 * d["V"]) * valid
+    mhz = (clocks or {}).get("sm_mhz") or peaks()["sm_max_mhz"]
+    peak = MUFU_PER_CLK_SM * SMS * mhz * 1e6
+    achieved = ops / (ms / 1e3)
+    return {"bound": "alu", "unit": "MUFU results/s", "achieved": achieved, "peak": peak, "frac": achieved / peak,
+            "per_cell": "2H tanh + 2V exp", "peak_source": f"16/clk/SM x 148 SMs x {mhz:.0f} MHz"}
+
+
+def measure_mode(args, mode, batch, d, dev, world, rank, local, flush, workload=None, chunk_cells=None,
+                 steps=None, warmup=None, e2e=True):
     """Times one mode: warm-up, K timed steps (each after an L2 flush), the
     end-to-end variant with host buffers, per-stage device times."""
+    workload = args.workload if workload is None else workload
+    chunk_cells = args.chunk_cells if chunk_cells is None else chunk_cells
+    steps = args.steps if steps is None else steps
+    warmup = args.warmup if warmup is None else warmup
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
     tdt = args.loss == "tdt"
     durations = tuple(synth.TDT_DURATIONS) if tdt else ()
-    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, args.chunk_cells, batch.blank,
-                         "marginal" if tdt else args.loss, args.prune, durations)
+    # data parallelism: the weight gradients come back as fp32 accumulators
+    # (views of one flat buffer) so the exchange is one fp32 all-reduce
+    wf32 = world > 1
+    dims = frnnt.dims_of(d["f"], d["g"], d["W_o"], dtype, mode, args.path, chunk_cells, batch.blank,
+                         "marginal" if tdt else args.loss, args.prune, durations, wgrad_f32=wf32)
     bounds = None
     valid = batch.valid_cells()
     if args.prune:
@@ -277,20 +369,21 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         if tdt:
             res = frnnt.fwd_bwd_tdt(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["W_d"], d["b_d"],
                                     d["labels"], d["T_len"], d["U_len"], durations, mode=mode,
-                                    chunk_cells=args.chunk_cells, blank=batch.blank, out=out, check=check,
-                                    stream=stream)
+                                    chunk_cells=chunk_cells, blank=batch.blank, out=out, check=check,
+                                    stream=stream, wgrad_f32=wf32)
         elif bounds is not None:
             res = frnnt.fwd_bwd_pruned(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"],
                                        d["T_len"], d["U_len"], bounds, args.prune, mode=mode, path=args.path,
-                                       chunk_cells=args.chunk_cells, loss=args.loss, blank=batch.blank, out=out,
-                                       check=check, stream=stream)
+                                       chunk_cells=chunk_cells, loss=args.loss, blank=batch.blank, out=out,
+                                       check=check, stream=stream, wgrad_f32=wf32)
         else:
             res = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
-                                d["U_len"], mode=mode, path=args.path, chunk_cells=args.chunk_cells, loss=args.loss,
-                                blank=batch.blank, out=out, check=check, stream=stream)
+                                d["U_len"], mode=mode, path=args.path, chunk_cells=chunk_cells, loss=args.loss,
+                                blank=batch.blank, out=out, check=check, stream=stream, wgrad_f32=wf32)
         if world > 1:
-            # the data-parallel exchange: weight gradients summed over ranks
-            rdist.allreduce_weight_grads(res[1])
+            # the data-parallel exchange: one all-reduce of the flat fp32 weight
+            # gradients, each sum rounded once to the input dtype
+            rdist.allreduce_weight_grads(res[1], out_dtype=d["W_o"].dtype)
         return res
 
     # peak device memory of one call: the library allocates nothing, so the
@@ -303,7 +396,7 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     torch.cuda.synchronize()
     peak_bytes = torch.cuda.max_memory_allocated(dev) - flush_bytes
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         call()
     torch.cuda.synchronize()
     frnnt.profile_read()
@@ -312,10 +405,10 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local) if rank == 0 else None
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if sampler:
         sampler.mark_start()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         evs[i][0].record(stream)
         call()
@@ -328,71 +421,107 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush):
     clocks = sampler.stop() if sampler else None
     frnnt.profile(False)
     stages = frnnt.profile_read()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     if world > 1:
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
 
-    # end to end through the public API with host buffers: pinned H2D of the
-    # step's inputs, the call, D2H of the loss and status word
-    host = {k: v.cpu().pin_memory() for k, v in d.items()}
-    loss_h = torch.empty(batch.f.shape[0], dtype=torch.float32).pin_memory()
-    status_h = torch.empty(4, dtype=torch.int32).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = loss_h.numel() * 4 + status_h.numel() * 4
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for k, v in host.items():
-            d[k].copy_(v, non_blocking=True)
-        call()
-        loss_h.copy_(out.loss, non_blocking=True)
-        status_h.copy_(out.status, non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        if int(status_h[0]) != 0:
-            raise RuntimeError(f"device status {int(status_h[0])}")
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = float(t.item())
-
     # cells of the lattice that is computed: B*T*(U+1), or B*T*S when pruned
     units = (batch.dims["B"] * batch.dims["T"] * args.prune if args.prune else batch.padded_cells()) * batch.dims["V"]
-    launches = sum(v["launches"] for v in stages.values())
-    roofline = None
-    pk = peaks()
-    if stages:
-        dom = max(stages, key=lambda k: stages[k]["ms"])
-        kind, work = stage_work(batch, dom, mode, valid, len(durations))
-        per_call_ms = stages[dom]["ms"] / args.steps
-        tr = None if args.prune else MEASURED_TRAFFIC.get((args.workload, mode, dom, args.loss))
-        if kind == "tensor":
-            achieved = work / (per_call_ms / 1e3) / 1e12
-            roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["tensor_sustained"], "unit": "TFLOP/s",
-                        "frac": achieved / pk["tensor_sustained"], "traffic": tr[0] if tr else None,
-                        "traffic_source": tr[1] if tr else None, "stage": dom,
-                        "launches_per_step": stages[dom]["launches"] / args.steps,
-                        "peak_source": pk["source"] + " sustained dense bf16 (the stage runs inside a long step)"}
-        elif kind == "hbm":
-            achieved = work / (per_call_ms / 1e3) / 1e9
-            roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                        "frac": achieved / pk["hbm"], "traffic": tr[0] if tr else None,
-                        "traffic_source": tr[1] if tr else None, "stage": dom, "peak_source": pk["source"]}
-    return {"ms": ms, "value": world * units / (ms / 1e3), "peak_bytes": peak_bytes,
-            "valid_cells_per_s": world * valid * batch.dims["V"] / (ms / 1e3),
-            "e2e": {"value": world * units / (e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
-            "launches": launches, "roofline": roofline, "clocks": clocks,
-            "stages": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps}
-                       for k, v in stages.items()}}
+    res = {"ms": ms, "value": world * units / (ms / 1e3), "peak_bytes": peak_bytes,
+           "valid_cells_per_s": world * valid * batch.dims["V"] / (ms / 1e3), "clocks": clocks,
+           "launches": sum(v["launches"] for v in stages.values()),
+           "stages": {k: {"ms_per_step": v["ms"] / steps, "launches_per_step": v["launches"] / steps}
+                      for k, v in stages.items()}}
+    rl = stage_rooflines(batch, mode, stages, steps, valid, len(durations), workload, args.loss, args.prune)
+    res["rooflines"] = rl
+    res["roofline"] = rl[max(rl, key=lambda k: rl[k]["ms_per_step"])] if rl else None
+    res["mufu"] = mufu_roofline(batch, valid, ms, clocks)
+
+    if e2e:
+        # end to end through the public API with host buffers: pinned H2D of the
+        # step's inputs, the call, D2H of the loss and status word
+        host = {k: v.cpu().pin_memory() for k, v in d.items()}
+        loss_h = torch.empty(batch.f.shape[0], dtype=torch.float32).pin_memory()
+        status_h = torch.empty(4, dtype=torch.int32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = loss_h.numel() * 4 + status_h.numel() * 4
+        e2e_ms = []
+        for i in range(warmup + steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for k, v in host.items():
+                d[k].copy_(v, non_blocking=True)
+            call()
+            loss_h.copy_(out.loss, non_blocking=True)
+            status_h.copy_(out.status, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            if int(status_h[0]) != 0:
+                raise RuntimeError(f"device status {int(status_h[0])}")
+            if i >= warmup:
+                e2e_ms.append(a.elapsed_time(b))
+        e2e_t = sum(e2e_ms) / len(e2e_ms)
+        if world > 1:
+            t = torch.tensor([e2e_t], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_t = float(t.item())
+        res["e2e"] = {"value": world * units / (e2e_t / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_t}
+    del out
+    return res
+
+
+def inputs_on(batch, dev, loss):
+    d = {k: getattr(batch, k).to(dev).contiguous()
+         for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+    if loss == "tdt":
+        W_d, b_d = duration_head(batch)
+        d["W_d"], d["b_d"] = W_d.to(dev).contiguous(), b_d.to(dev).contiguous()
+    return d
+
+
+def footprint_bytes(batch):
+    """Inputs + weights + gradients (gradients in the input dtype) + the int arrays."""
+    elt = 2 if batch.dtype == "bf16" else 4
+    return (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
+            4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
+
+
+def mode_entry(r, footprint):
+    return {"value": r["value"], "ms_per_step": r["ms"], "valid_cells_per_s": r["valid_cells_per_s"],
+            "peak_gb": r["peak_bytes"] / 1e9, "peak_over_footprint": r["peak_bytes"] / footprint,
+            "e2e_value": r["e2e"]["value"] if "e2e" in r else None, "roofline": r["roofline"],
+            "rooflines": r["rooflines"], "mufu": r["mufu"], "stages": r["stages"], "clocks": r["clocks"]}
+
+
+WORKLOAD_BLOCK = ("short", "medium", "long", "large")
+PROTOCOL_CHUNKS = (8192, 16384, 32768, 65536, 131072, 262144)
+PROTOCOL_WORKLOADS = ("medium", "long")
+
+
+def protocol(args, name, batch, d, dev, flush, footprint, untiled):
+    """The comparison protocol of "Flash RNN-T" (abstract): each mode at its
+    lowest-memory setting whose throughput is within 95 % of that mode's peak.
+    Tiled mode's memory knob is the backward chunk (cells per chunk); untiled
+    mode has none (one setting)."""
+    pts = []
+    for c in PROTOCOL_CHUNKS:
+        r = measure_mode(args, "tiled", batch, d, dev, 1, 0, 0, flush, workload=name, chunk_cells=c,
+                         steps=min(args.steps, 5), warmup=3, e2e=False)
+        pts.append({"chunk_cells": c, "ms_per_step": r["ms"], "value": r["value"], "peak_gb": r["peak_bytes"] / 1e9,
+                    "peak_over_footprint": r["peak_bytes"] / footprint})
+    best = max(p["value"] for p in pts)
+    ok = [p for p in pts if p["value"] >= 0.95 * best]
+    pick = min(ok, key=lambda p: p["peak_gb"])
+    return {"tiled": {"points": pts, "peak_value": best, "lowest_memory_within_95pct": pick},
+            "untiled": {"points": [{"chunk_cells": None, "ms_per_step": untiled["ms"], "value": untiled["value"],
+                                    "peak_gb": untiled["peak_bytes"] / 1e9,
+                                    "peak_over_footprint": untiled["peak_bytes"] / footprint}],
+                        "note": "no memory knob: the logits of the whole lattice are stored"}}
 
 
 def run_ours(args):
@@ -409,15 +538,9 @@ def run_ours(args):
 
     idx = synth.WORKLOADS[args.workload]["index"]
     batch = synth.workload(args.workload, seed=1000 + idx + 7919 * rank)
-    d = {k: getattr(batch, k).to(dev).contiguous()
-         for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
-    if args.loss == "tdt":
-        W_d, b_d = duration_head(batch)
-        d["W_d"], d["b_d"] = W_d.to(dev).contiguous(), b_d.to(dev).contiguous()
+    d = inputs_on(batch, dev, args.loss)
     dtype = "bf16" if batch.dtype == "bf16" else "f32"
-    elt = 2 if dtype == "bf16" else 4
-    footprint = (2 * sum(getattr(batch, k).numel() for k in ("f", "g", "W_f", "W_g", "W_o", "b_o")) * elt +
-                 4 * (batch.labels.numel() + 2 * batch.T_len.numel()) + 4 * batch.T_len.numel())
+    footprint = footprint_bytes(batch)
 
     modes = modes_of(args)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -428,11 +551,33 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, u = oracle_sample(batch, loss=args.loss)
-        Tb, Ub = int(batch.T_len[0]), int(batch.U_len[0])
-        cpu = {"value": u / dt, "unit": UNIT, "cores": cores(), "kind": "oracle",
-               "sample": f"utterance 0 of {args.workload} (T_len={Tb}, U_len={Ub}); units = T*(U+1)*V of one "
-                         f"utterance; numpy fp64, BLAS threads = all cores"}
+        cpu = oracle_line(batch, args.workload, oracle_sample(batch, budget_s=10.0, loss=args.loss))
+
+    # one GPU, default criterion: every workload in both modes, and the
+    # chunk-size protocol, after the headline
+    workloads, proto = None, None
+    if world == 1 and not args.no_workloads and args.loss == "marginal" and not args.prune and args.path == "auto":
+        del d
+        workloads, proto = {}, {}
+        for name in WORKLOAD_BLOCK:
+            wb = batch if name == args.workload else synth.workload(name)
+            wd = inputs_on(wb, dev, args.loss)
+            fp = footprint_bytes(wb)
+            entry = {"footprint_gb": fp / 1e9, "valid_cells": wb.valid_cells(), "padded_cells": wb.padded_cells()}
+            measured = {}
+            for m in ("untiled", "tiled"):
+                r = results[m] if name == args.workload and m in results else measure_mode(
+                    args, m, wb, wd, dev, 1, 0, local, flush, workload=name, e2e=False)
+                measured[m] = r
+                entry[m] = mode_entry(r, fp)
+                torch.cuda.empty_cache()
+            if name in PROTOCOL_WORKLOADS:
+                proto[name] = protocol(args, name, wb, wd, dev, flush, fp, measured["untiled"])
+            if not args.no_cpu_baseline:
+                entry["oracle"] = oracle_line(wb, name, oracle_sample(wb, budget_s=3.0))
+            workloads[name] = entry
+            del wd
+            torch.cuda.empty_cache()
 
     if rank == 0:
         cfg = config_of(batch, args, world)
@@ -443,12 +588,12 @@ def run_ours(args):
                 "peak_gb": head["peak_bytes"] / 1e9, "footprint_gb": footprint / 1e9,
                 "peak_over_footprint": head["peak_bytes"] / footprint,
                 "valid_cells_per_s": head["valid_cells_per_s"], "e2e": head["e2e"], "gpu_launches": head["launches"],
-                "stages": head["stages"], "roofline": head["roofline"], "cpu_baseline": cpu,
-                "clocks": head["clocks"],
-                "modes": {m: {"value": r["value"], "ms_per_step": r["ms"], "peak_gb": r["peak_bytes"] / 1e9,
-                              "peak_over_footprint": r["peak_bytes"] / footprint, "e2e_value": r["e2e"]["value"],
-                              "roofline": r["roofline"], "stages": r["stages"], "clocks": r["clocks"]}
-                          for m, r in results.items()}}
+                "stages": head["stages"], "roofline": head["roofline"], "rooflines": head["rooflines"],
+                "mufu": head["mufu"], "cpu_baseline": cpu, "clocks": head["clocks"],
+                "modes": {m: mode_entry(r, footprint) for m, r in results.items()}}
+        if workloads is not None:
+            line["workloads"] = workloads
+            line["protocol"] = proto
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

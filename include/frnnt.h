@@ -104,6 +104,16 @@ typedef struct {
                           /* strictly increasing frame counts, durations[0] = 0,
                              durations[1] = 1, durations[n_dur-1] <=
                              FRNNT_MAX_DURATION; entries past n_dur unused    */
+  int wgrad_f32;          /* 0: every gradient in the input dtype.  1: the
+                             weight gradients dW_f, dW_g, dW_o, db_o (and the
+                             duration head's dW_d, db_d) are written as fp32
+                             arrays -- the library's fp32 accumulators, never
+                             rounded -- also for FRNNT_BF16; df and dg stay in
+                             the input dtype.  For data parallelism: partial
+                             weight gradients of several devices are summed in
+                             fp32 and rounded once (the loss is a sum over
+                             utterances, "Sequence Transduction with Recurrent
+                             Neural Networks", abstract).                     */
 } frnnt_dims;
 
 /* Host return codes. */
@@ -137,16 +147,21 @@ FRNNT_API int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes);
  * All pointers are DEVICE pointers on the current device, 16-byte aligned,
  * owned by the caller; the library allocates no device memory and keeps no
  * data between calls.  Host-side it caches, per device, kernel attributes and
- * one internal stream with two events (created by the first call on that
+ * one internal stream with its events (created by the first call on that
  * device, outside any stream capture), on which part of the work runs beside
- * the caller's stream.  Calls on different devices may come from different
- * host threads at the same time; calls on one device must not overlap on the
- * host (they share that stream's events).  Float tensors are fp32 (FRNNT_F32) or bf16 bit patterns
- * (FRNNT_BF16); b_o and all gradients have that same element type.
+ * the caller's stream.  Calls may come from several host threads at once, on
+ * one device or several, on any streams: a per-device lock serialises the
+ * host-side queuing of the calls that use the internal stream (each holds it
+ * from its first fork to its last join), so every call's joins wait for its
+ * own side work; on the GPU the calls still overlap, except that their side
+ * work runs in queue order on the one internal stream.  Float tensors are
+ * fp32 (FRNNT_F32) or bf16 bit patterns (FRNNT_BF16); b_o and all gradients
+ * have that same element type (weight gradients: fp32 with d->wgrad_f32).
  *   grad_loss   [B] fp32 weights w_b of d(sum_b w_b loss_b), or NULL (= 1)
  *   loss        [B] fp32 output, -log P(y_b | x_b) per utterance
  *   df, dg, dW_f, dW_g, dW_o, db_o   outputs, overwritten (not accumulated),
- *               same shapes as f, g, W_f, W_g, W_o, b_o
+ *               same shapes as f, g, W_f, W_g, W_o, b_o (dW_* and db_o fp32
+ *               when d->wgrad_f32 is 1)
  *   workspace   >= frnnt_workspace_size bytes, contents undefined on entry
  *   status      [1] int32 output: 0, or an OR of FRNNT_STATUS_* bits found by
  *               the device-side validation; when non-zero every other output
@@ -226,10 +241,19 @@ FRNNT_API int frnnt_fwd_bwd_tdt(const frnnt_dims* d,
  * the library, reserved on every GPU that loads the library until the process
  * exits; dims whose frnnt_workspace_size exceeds it return FRNNT_ERR_WORKSPACE
  * before any launch (a smaller chunk_cells lowers the need in tiled mode).
- * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Allocates nothing itself: no cudaMalloc, cudaFree or allocating library
+ * call.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    outside any stream capture.
+ *    outside any stream capture.  Under lazy module loading (the CUDA 12
+ *    default) that lookup is also when the driver loads the array's module
+ *    and reserves its FRNNT_NOALLOC_MAX_BYTES on the device: if the device's
+ *    memory is already taken by then, that first call fails with
+ *    FRNNT_ERR_CUDA (the CUDA error state is cleared).  So make one call
+ *    during start-up, before a framework allocator takes the device's memory
+ *    (or load modules eagerly, CUDA_MODULE_LOADING=EAGER).
+ *  - Two host threads making their first calls on different devices at once
+ *    are safe (each device's address is stored atomically).
  *  - All calls share the one array, which keeps the previous call's
  *    contents; each call clears on its stream what must start at zero.
  *    Calls that can overlap on the GPU (different streams, or different

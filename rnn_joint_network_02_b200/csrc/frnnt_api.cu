@@ -6,6 +6,8 @@
 // allocated and nothing is synchronised.
 #include <string.h>
 
+#include <mutex>
+
 #include "frnnt_common.cuh"
 #include "frnnt_internal.h"
 
@@ -34,6 +36,7 @@ bool dims_ok(const frnnt_dims* d) {
   if (d->U + 1 > 1024) return false;
   if (d->chunk_cells < 0) return false;
   if (d->prune_S < 0 || d->prune_S > 32) return false;
+  if (d->wgrad_f32 != 0 && d->wgrad_f32 != 1) return false;
   if (d->n_dur != 0) {
     // token-and-duration transducer: 0 and 1 frames first, strictly increasing, at most 8 frames
     if (d->n_dur < 2 || d->n_dur > FRNNT_MAX_DURATIONS) return false;
@@ -181,10 +184,11 @@ int run_simt(const frnnt_dims* d, const Shape& s, const void* f, const void* g, 
     launch_convert(p.df_tmp, df, s.BT * s.Dx, true, st);
     launch_convert(p.dg_tmp, dg, s.BU * s.Dy, true, st);
   }
-  launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, bf, st);
-  launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, bf, st);
-  launch_convert(p.accWo, dW_o, (long long)s.V * s.H, bf, st);
-  launch_convert(p.accbo, db_o, s.V, bf, st);
+  const bool wbf = bf && !d->wgrad_f32;   // weight gradients rounded to bf16, or the fp32 accumulators
+  launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, wbf, st);
+  launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, wbf, st);
+  launch_convert(p.accWo, dW_o, (long long)s.V * s.H, wbf, st);
+  launch_convert(p.accbo, db_o, s.V, wbf, st);
   return cudaGetLastError() == cudaSuccess ? FRNNT_OK : FRNNT_ERR_CUDA;
 }
 
@@ -273,21 +277,25 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
 // occupies one block per utterance and direction), forked from and joined
 // back to the caller's stream with events, so stream order, graph capture and
 // the caller's synchronisation are unaffected.  Shared by all calls on the
-// device, so calls on one device must not overlap on the host: between one
-// call's record of `fork` and its stream's wait on it, another call's record
-// would redirect that wait (calls on different devices use different slots).
+// device: between one call's record of `fork` and its stream's wait on it,
+// another call's record would redirect that wait.  So a call holds the
+// device's `mu` from before its first fork until after its last join wait
+// (host-side queuing only; calls on different devices use different slots).
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;     // hidden rows beside the lattice DP
   cudaEvent_t fork2 = nullptr, join2 = nullptr;   // the G-side projection backward beside the F side
   bool ok = false;
+  std::mutex mu;
 };
 
 SideStream* side_stream() {
   static SideStream sides[64];
+  static std::mutex init_mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   SideStream& x = sides[dev];
+  std::lock_guard<std::mutex> guard(init_mu);
   if (!x.ok && !x.s) {
     if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) == cudaSuccess &&
         cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
@@ -318,7 +326,13 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   TcPlan p = plan_tc(d, s, ws);
   const bool untiled = d->mode == FRNNT_UNTILED;
   const bool tdt = s.n_dur > 0;
+  const bool wf32 = d->wgrad_f32 != 0;
   int rc = FRNNT_OK;
+  // the side stream's fork / join events are shared by the device's calls:
+  // hold its lock while this call queues work (released on every return)
+  SideStream* side_lock = side_stream();
+  std::unique_lock<std::mutex> queue_lock;
+  if (side_lock) queue_lock = std::unique_lock<std::mutex>(side_lock->mu);
 #define FRNNT_TRY(x)            \
   do {                          \
     rc = (x);                   \
@@ -465,8 +479,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       cudaEventRecord(ps->fork2, st);
       cudaStreamWaitEvent(gs, ps->fork2, 0);
     }
-    launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st, p.db_part);
-    if (tdt) launch_wo_finalize(p.accWd, s.n_dur, s.H, dW_d, db_d, st);
+    launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st, p.db_part, wf32);
+    if (tdt) launch_wo_finalize(p.accWd, s.n_dur, s.H, dW_d, db_d, st, nullptr, wf32);
     launch_convert_bf16(p.dF, p.dFb, s.BT * s.H, st);
     launch_convert_bf16(p.dG, p.dGb, s.BU * s.H, gs);
     GemmTcArgs a{};
@@ -485,8 +499,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     w.M = s.Dy; w.K = (int)s.BU; w.A = g; w.lda = s.Dy; w.B = p.dGb; w.k_splits = splits_for(s.Dy, s.H, (int)s.BU);
     w.out_f32 = p.accWg;
     if (rc_g == FRNNT_OK) rc_g = gemm_tc(w, gs);
-    launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, true, st);
-    launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, true, gs);
+    launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, !wf32, st);
+    launch_convert(p.accWg, dW_g, (long long)s.Dy * s.H, !wf32, gs);
     if (ps) {   // joined on every path, so the caller's stream never runs ahead of the side work
       cudaEventRecord(ps->join2, gs);
       cudaStreamWaitEvent(st, ps->join2, 0);

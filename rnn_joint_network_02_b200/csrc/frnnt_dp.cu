@@ -11,11 +11,16 @@
 // only on diagonal d-1 (alpha) or d+1 (beta), so one thread owns one label
 // position u and walks the diagonals; the value it needs from its neighbour
 // u-1 (alpha) or u+1 (beta) is the neighbour's result on the previous
-// diagonal, passed by a warp shuffle, and across a warp boundary by a
-// parity-double-buffered shared-memory slot.  One block per (utterance,
-// direction): alpha and beta run concurrently.  The marginal kernel
-// (dp2_kernel) advances two diagonals per dependent step; the maximum
-// approximation and the pruned band keep one.
+// diagonal.  One block per (utterance, direction): alpha and beta run
+// concurrently.  How the neighbour's value travels depends on the kernel:
+//  * dp2_kernel (marginal loss) advances two diagonals per dependent step and
+//    exchanges every neighbour value through a parity-double-buffered
+//    shared-memory row (no shuffles, no warp-edge special cases);
+//  * dp_viterbi_kernel (maximum approximation) passes it by a warp shuffle
+//    inside a warp and by shared memory across warp boundaries;
+//  * dp_band_warp_kernel (pruned band, one warp per utterance and direction)
+//    scans the band with shuffles;
+//  * tdt_dp_kernel (token-and-duration lattice) uses shared memory only.
 #include "frnnt_common.cuh"
 #include "frnnt_internal.h"
 

@@ -275,7 +275,7 @@ void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const 
 void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, int blocks_per_sm = 8);
 // dW_o = acc[:, :H]; db_o = db (when non-null) or acc[:, H]; acc rows of hidden_stride(H)
 void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st,
-                        const float* db = nullptr);
+                        const float* db = nullptr, bool out_f32 = false);
 // Untiled dz pass that also sums db_o into db_acc [V] (cleared beforehand), for
 // dz_db_supported(V, H): the dW_o GEMM then runs on N = H.
 bool dz_db_supported(int V, int H);

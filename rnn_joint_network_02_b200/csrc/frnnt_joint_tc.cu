@@ -1040,15 +1040,22 @@ __global__ void __launch_bounds__(256) hidden_tiles_kernel(JointParams p, int ro
   }
 }
 
-// dW_o [V][H] and db_o [V] (bf16) out of the extended fp32 accumulator [V][HS]
-// whose column H is the sum of dz over cells.
+// dW_o [V][H] and db_o [V] (bf16, or fp32 when OUT_F32) out of the extended
+// fp32 accumulator [V][HS] whose column H is the sum of dz over cells.
+template <bool OUT_F32>
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, const float* __restrict__ db,
-                                   __nv_bfloat16* __restrict__ dW_o, __nv_bfloat16* __restrict__ db_o) {
+                                   void* __restrict__ dW_o, void* __restrict__ db_o) {
   const long long n = (long long)V * H;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const long long k = i / H, j = i % H;
-    dW_o[i] = __float2bfloat16_rn(acc[k * HS + j]);
-    if (j == 0) db_o[k] = __float2bfloat16_rn(db ? db[k] : acc[k * HS + H]);
+    const float w = acc[k * HS + j];
+    if (OUT_F32) ((float*)dW_o)[i] = w;
+    else ((__nv_bfloat16*)dW_o)[i] = __float2bfloat16_rn(w);
+    if (j == 0) {
+      const float bias = db ? db[k] : acc[k * HS + H];
+      if (OUT_F32) ((float*)db_o)[k] = bias;
+      else ((__nv_bfloat16*)db_o)[k] = __float2bfloat16_rn(bias);
+    }
   }
 }
 
@@ -1467,12 +1474,15 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
   note_launch();
 }
 
-void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st, const float* db) {
+void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, cudaStream_t st, const float* db,
+                        bool out_f32) {
   long long n = (long long)V * H;
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  wo_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, (__nv_bfloat16*)dW_o,
-                                                       (__nv_bfloat16*)db_o);
+  if (out_f32)
+    wo_finalize_kernel<true><<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, dW_o, db_o);
+  else
+    wo_finalize_kernel<false><<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, dW_o, db_o);
   note_launch();
 }
 

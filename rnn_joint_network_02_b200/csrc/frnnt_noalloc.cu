@@ -10,7 +10,12 @@
 // input and output buffer; only the scratch memory is supplied here.
 //
 // The scratch is one file-scope __device__ array of FRNNT_NOALLOC_MAX_BYTES.
-// Every GPU that loads this library reserves it until the process exits.
+// Every GPU that loads this file's module holds it until the process exits.
+// With lazy module loading (the CUDA 12 default) the driver loads the module,
+// and reserves the array, inside the first cudaGetSymbolAddress on a device,
+// i.e. during the first call there: callers make that call at start-up.
+#include <atomic>
+
 #include "frnnt_common.cuh"
 #include "frnnt_internal.h"
 
@@ -21,20 +26,28 @@ constexpr size_t kScratchBytes = (size_t)FRNNT_NOALLOC_MAX_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
+std::atomic<void*> g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address must come
 // from cudaGetSymbolAddress (once per device, with that device current).
+// Threads racing on a device's first call each look the address up (the
+// same value) and store it atomically.
 int scratch_for_current_device(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FRNNT_ERR_CUDA;
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FRNNT_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FRNNT_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();   // e.g. out of memory while the module loads: leave no sticky error behind
+      return FRNNT_ERR_CUDA;
+    }
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
   return FRNNT_OK;
 }
 

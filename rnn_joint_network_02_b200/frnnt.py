@@ -35,7 +35,7 @@ class Dims(ctypes.Structure):
                 ("D_pred", ctypes.c_int), ("H", ctypes.c_int), ("V", ctypes.c_int), ("blank", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("mode", ctypes.c_int), ("path", ctypes.c_int),
                 ("chunk_cells", ctypes.c_int), ("loss", ctypes.c_int), ("prune_S", ctypes.c_int),
-                ("n_dur", ctypes.c_int), ("durations", ctypes.c_int * 8)]
+                ("n_dur", ctypes.c_int), ("durations", ctypes.c_int * 8), ("wgrad_f32", ctypes.c_int)]
 
 
 class StageStat(ctypes.Structure):
@@ -137,14 +137,15 @@ LOSSES = {"marginal": 0, "viterbi": 1}
 
 
 def make_dims(B, T, U, D_enc, D_pred, H, V, dtype="bf16", mode="tiled", path="auto", chunk_cells=0,
-              blank=0, loss="marginal", prune_S=0, durations=()) -> Dims:
-    """``durations`` (token-and-duration transducer): the duration set, or () for the transducer."""
+              blank=0, loss="marginal", prune_S=0, durations=(), wgrad_f32=False) -> Dims:
+    """``durations`` (token-and-duration transducer): the duration set, or () for the transducer.
+    ``wgrad_f32``: weight gradients come back as the library's fp32 accumulators."""
     if len(durations) > MAX_DURATIONS:
         raise ValueError(f"at most {MAX_DURATIONS} durations")
     dur = (ctypes.c_int * 8)(*[int(x) for x in durations])
     return Dims(B, T, U, D_enc, D_pred, H, V, blank, BF16 if dtype == "bf16" else F32,
                 TILED if mode == "tiled" else UNTILED, PATH_SIMT if path == "simt" else PATH_AUTO,
-                chunk_cells, LOSSES[loss], prune_S, len(durations), dur)
+                chunk_cells, LOSSES[loss], prune_S, len(durations), dur, 1 if wgrad_f32 else 0)
 
 
 def workspace_size(dims: Dims) -> int:
@@ -159,15 +160,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", prune_S=0, durations=()) -> Dims:
+def dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss="marginal", prune_S=0, durations=(),
+            wgrad_f32=False) -> Dims:
     B, T, D_enc = f.shape
     U = g.shape[1] - 1
     V, H = W_o.shape
     return make_dims(B, T, U, D_enc, g.shape[2], H, V, dtype, mode, path, chunk_cells, blank, loss, prune_S,
-                     durations)
+                     durations, wgrad_f32)
 
 
-def _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=None, W_d=None, b_d=None):
+def _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=None, W_d=None, b_d=None,
+                wgrad_f32=False):
     """Host-side checks before any pointer reaches the library: a tensor of the
     wrong shape, dtype, layout or device would otherwise be read or written out
     of bounds by the kernels.  Shapes and dtypes are checked first, then that
@@ -193,14 +196,15 @@ def _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, 
             raise ValueError("the duration head needs W_d [n_dur, H] and b_d [n_dur]")
         want += [("W_d", W_d, (W_d.shape[0], H), ft), ("b_d", b_d, (W_d.shape[0],), ft)]
     if out is not None:
+        wt = torch.float32 if wgrad_f32 else ft     # dtype of the weight gradients
         want += [("out.loss", out.loss, (B,), torch.float32), ("out.df", out.df, tuple(f.shape), ft),
-                 ("out.dg", out.dg, tuple(g.shape), ft), ("out.dW_f", out.dW_f, (D_enc, H), ft),
-                 ("out.dW_g", out.dW_g, (D_pred, H), ft), ("out.dW_o", out.dW_o, (V, H), ft),
-                 ("out.db_o", out.db_o, (V,), ft), ("out.status", out.status, (4,), torch.int32)]
+                 ("out.dg", out.dg, tuple(g.shape), ft), ("out.dW_f", out.dW_f, (D_enc, H), wt),
+                 ("out.dW_g", out.dW_g, (D_pred, H), wt), ("out.dW_o", out.dW_o, (V, H), wt),
+                 ("out.db_o", out.db_o, (V,), wt), ("out.status", out.status, (4,), torch.int32)]
         if W_d is not None:
             if out.dW_d is None or out.db_d is None:
                 raise ValueError("out has no duration-head gradients")
-            want += [("out.dW_d", out.dW_d, tuple(W_d.shape), ft), ("out.db_d", out.db_d, tuple(b_d.shape), ft)]
+            want += [("out.dW_d", out.dW_d, tuple(W_d.shape), wt), ("out.db_d", out.db_d, tuple(b_d.shape), wt)]
     for name, t, shape, dt in want:
         if tuple(t.shape) != tuple(shape):
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
@@ -218,19 +222,33 @@ def _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, 
 
 
 class Outputs:
-    """Preallocated outputs and workspace of one call shape."""
+    """Preallocated outputs and workspace of one call shape.
+
+    With ``dims.wgrad_f32`` the weight gradients (dW_f, dW_g, dW_o, db_o and
+    the duration head's dW_d, db_d) are fp32 views into one flat buffer,
+    ``wflat``, so a data-parallel exchange sums them with one all-reduce."""
 
     def __init__(self, f, g, W_f, W_g, W_o, b_o, dims: Dims, with_workspace: bool = True, W_d=None, b_d=None):
         dev = f.device
-        self.dW_d = None if W_d is None else torch.empty_like(W_d)
-        self.db_d = None if b_d is None else torch.empty_like(b_d)
         self.loss = torch.empty(f.shape[0], dtype=torch.float32, device=dev)
         self.df = torch.empty_like(f)
         self.dg = torch.empty_like(g)
-        self.dW_f = torch.empty_like(W_f)
-        self.dW_g = torch.empty_like(W_g)
-        self.dW_o = torch.empty_like(W_o)
-        self.db_o = torch.empty_like(b_o)
+        weights = [("dW_f", W_f), ("dW_g", W_g), ("dW_o", W_o), ("db_o", b_o)]
+        if W_d is not None:
+            weights += [("dW_d", W_d), ("db_d", b_d)]
+        self.dW_d = self.db_d = None
+        self.wflat = None
+        if dims.wgrad_f32:
+            # segments start on 16-byte boundaries (the library's alignment rule)
+            sizes = [(t.numel() + 3) // 4 * 4 for _, t in weights]
+            self.wflat = torch.zeros(sum(sizes), dtype=torch.float32, device=dev)
+            off = 0
+            for (name, t), n in zip(weights, sizes):
+                setattr(self, name, self.wflat[off:off + t.numel()].view(t.shape))
+                off += n
+        else:
+            for name, t in weights:
+                setattr(self, name, torch.empty_like(t))
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         n = max(workspace_size(dims), 16) if with_workspace else 16
         self.workspace = torch.empty(n, dtype=torch.uint8, device=dev)
@@ -243,18 +261,20 @@ class Outputs:
 
 
 def fwd_bwd(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss=None, mode="tiled", path="auto",
-            chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None, loss="marginal"):
+            chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None, loss="marginal",
+            wgrad_f32=False):
     """One call of frnnt_fwd_bwd on CUDA tensors.
 
     Float tensors are all float32 or all bfloat16; labels/T_len/U_len int32.
     ``loss`` is "marginal" (every alignment) or "viterbi" (the best one).
+    ``wgrad_f32``: the weight gradients come back in fp32 (unrounded).
     Returns (loss [B] fp32, dict of gradients).  With ``check`` the device
     status word is read back (one 4-byte device-to-host copy, which
     synchronises the stream) and a non-zero status raises FrnntStatusError.
     """
-    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out)
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, wgrad_f32=wgrad_f32)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
-    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss)
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss, wgrad_f32=wgrad_f32)
     if out is None:
         out = Outputs(f, g, W_f, W_g, W_o, b_o, dims)
     if stream is None:
@@ -335,13 +355,13 @@ def set_joint_variant(variant: int) -> int:
 
 def fwd_bwd_pruned(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, S: int, grad_loss=None, mode="tiled",
                    path="auto", chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None,
-                   loss="marginal"):
+                   loss="marginal", wgrad_f32=False):
     """frnnt_fwd_bwd_pruned: the loss and gradients on the pruned lattice that
     keeps, for frame t of utterance b, the S label positions
     bounds[b,t] <= u < bounds[b,t] + S (bounds: int32 [B, T] on the device)."""
-    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=bounds)
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, bounds=bounds, wgrad_f32=wgrad_f32)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
-    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss, S)
+    dims = dims_of(f, g, W_o, dtype, mode, path, chunk_cells, blank, loss, S, wgrad_f32=wgrad_f32)
     if out is None:
         out = Outputs(f, g, W_f, W_g, W_o, b_o, dims)
     if stream is None:
@@ -361,16 +381,19 @@ def fwd_bwd_pruned(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, bounds, S: in
 
 
 def fwd_bwd_tdt(f, g, W_f, W_g, W_o, b_o, W_d, b_d, labels, T_len, U_len, durations, grad_loss=None,
-                mode="tiled", chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None):
+                mode="tiled", chunk_cells=0, blank=0, out: Outputs | None = None, check=True, stream=None,
+                wgrad_f32=False):
     """frnnt_fwd_bwd_tdt: the token-and-duration transducer loss and gradients.
 
     W_d [n_dur, H] and b_d [n_dur] are the duration head (bf16, like the other
     weights); ``durations`` is the duration set (frame counts, increasing,
     starting 0, 1).  Returns (loss [B] fp32, dict of gradients including dW_d
     and db_d)."""
-    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, W_d=W_d, b_d=b_d)
+    _check_call(f, g, W_f, W_g, W_o, b_o, labels, T_len, U_len, grad_loss, out, W_d=W_d, b_d=b_d,
+                wgrad_f32=wgrad_f32)
     dtype = "bf16" if f.dtype == torch.bfloat16 else "f32"
-    dims = dims_of(f, g, W_o, dtype, mode, "auto", chunk_cells, blank, "marginal", 0, tuple(durations))
+    dims = dims_of(f, g, W_o, dtype, mode, "auto", chunk_cells, blank, "marginal", 0, tuple(durations),
+                   wgrad_f32=wgrad_f32)
     if out is None:
         out = Outputs(f, g, W_f, W_g, W_o, b_o, dims, W_d=W_d, b_d=b_d)
     if stream is None:

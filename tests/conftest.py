@@ -19,3 +19,17 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The parity margins: for each compared tensor, the worst measured error
+    of the session against the tolerance of its dtype."""
+    try:
+        from tests.helpers import margin_report
+    except Exception:       # the helpers failed to import: their tests report it
+        return
+    lines = margin_report()
+    if lines:
+        terminalreporter.write_sep("-", "parity margins (worst error per tensor / tolerance)")
+        for line in lines:
+            terminalreporter.write_line(line)

@@ -13,6 +13,29 @@ import oracle
 TOL = {"f32": dict(loss=1e-4, grad=1e-4), "bf16": dict(loss=5e-3, grad=2e-2)}
 GRADS = ("df", "dg", "dW_f", "dW_g", "dW_o", "db_o")
 
+# Every comparison's measured errors, (note, dtype, {name: error}); the test
+# session's summary prints the worst error of each tensor against its tolerance.
+MARGINS: list = []
+
+
+def record(note: str, dtype: str, errs: dict) -> None:
+    MARGINS.append((note, dtype, dict(errs)))
+
+
+def margin_report() -> list:
+    """Lines: per (dtype, tensor), the largest error / tolerance and where."""
+    worst = {}
+    for note, dtype, errs in MARGINS:
+        for name, err in errs.items():
+            tol = TOL[dtype]["loss" if name == "loss" else "grad"]
+            key = (dtype, name)
+            if key not in worst or err / tol > worst[key][0]:
+                worst[key] = (err / tol, err, tol, note)
+    lines = []
+    for (dtype, name), (frac, err, tol, note) in sorted(worst.items()):
+        lines.append(f"{dtype:5s} {name:6s} worst {err:.3e} = {frac:6.1%} of tolerance {tol:.0e}  ({note})")
+    return lines
+
 
 def to_device(batch, device="cuda"):
     d = {k: getattr(batch, k).to(device).contiguous()
@@ -50,6 +73,7 @@ def compare(loss, grads, ref, dtype, utterances=None, extra_note=""):
             gpu = gpu[idx]
             r = r[idx]
         errs[name] = rel_l2(gpu, r)
+    record(extra_note, dtype, errs)
     bad = {k: v for k, v in errs.items() if v > (tol["loss"] if k == "loss" else tol["grad"])}
     assert not bad, f"{extra_note} tolerance exceeded: {bad} (all: {errs})"
     return errs

@@ -160,3 +160,87 @@ def test_two_gloo_ranks_tdt_duration_head_grads_summed(tmp_path):
         for k in ("dW_f", "dW_g", "dW_o", "db_o", "dW_d", "db_d"):
             np.testing.assert_allclose(d["grads"][k].numpy(), getattr(ref, k), rtol=1e-10, atol=1e-12)
     assert sorted(seen) == list(range(5))
+
+
+def _flat_fp32_compute(shard, w):
+    """The oracle as the per-rank compute, returning what the library returns
+    with wgrad_f32: fp32 weight gradients (here the fp64 values rounded to
+    fp32 once) as views of one flat fp32 buffer with 16-byte-aligned segments."""
+    loss, grads = _oracle_compute(shard, w)
+    keys = ("dW_f", "dW_g", "dW_o", "db_o")
+    sizes = [(grads[k].numel() + 3) // 4 * 4 for k in keys]
+    flat = torch.zeros(sum(sizes), dtype=torch.float32)
+    off = 0
+    out = dict(grads)
+    for k, n in zip(keys, sizes):
+        v = flat[off:off + grads[k].numel()].view(grads[k].shape)
+        v.copy_(grads[k].float())
+        out[k] = v
+        off += n
+    return loss, out
+
+
+def _fp32_worker(rank, world, port, out_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    calls = []
+    real = dist.all_reduce
+
+    def counting(*a, **k):
+        calls.append(1)
+        return real(*a, **k)
+
+    dist.all_reduce = counting
+    try:
+        batch = synth.make(B=5, T=7, U=4, D_enc=4, D_pred=3, H=6, V=7, dtype="f32", seed=77, T_range=(2, 7),
+                           U_range=(0, 4), bias_std=0.3)
+        t = {k: getattr(batch, k) for k in ("f", "g", "W_f", "W_g", "W_o", "b_o", "labels", "T_len", "U_len")}
+        w = torch.linspace(0.5, 1.5, 5)
+        # fp32 partials reduced in place: one all-reduce, the sum kept in fp32
+        idx, _, g32 = rdist.fwd_bwd_sharded(t, _flat_fp32_compute, rank, world, grad_loss=w)
+        n_flat = len(calls)
+        # separate fp32 partials: packed into one buffer, one all-reduce, the sum rounded once to bf16
+        def fp32_compute(shard, ww):
+            loss, grads = _oracle_compute(shard, ww)
+            return loss, {k: v.float() for k, v in grads.items()}
+        _, _, g16 = rdist.fwd_bwd_sharded(t, fp32_compute, rank, world, grad_loss=w, out_dtype=torch.bfloat16)
+        n_packed = len(calls) - n_flat
+        torch.save({"idx": idx, "g32": g32, "g16": g16, "n_flat": n_flat, "n_packed": n_packed},
+                   f"{out_path}.{rank}")
+    finally:
+        dist.all_reduce = real
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_fp32_partials_one_allreduce(tmp_path):
+    """The exchange is one all-reduce of one flat fp32 buffer.  Summing the
+    ranks' fp32 partial weight gradients gives the single-device result at fp32
+    accumulation (the loss is a sum over utterances, "Sequence Transduction
+    with Recurrent Neural Networks", abstract): within fp32 reassociation of
+    the single-device gradient rounded to fp32."""
+    world = 2
+    out = str(tmp_path / "f32")
+    mp.start_processes(_fp32_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
+    import oracle
+    batch = synth.make(B=5, T=7, U=4, D_enc=4, D_pred=3, H=6, V=7, dtype="f32", seed=77, T_range=(2, 7),
+                       U_range=(0, 4), bias_std=0.3)
+    f, g, W_f, W_g, W_o, b_o = (x.numpy() for x in batch.float64())
+    ref = oracle.fwd_bwd(f, g, W_f, W_g, W_o, b_o, batch.labels.numpy(), batch.T_len.numpy(), batch.U_len.numpy(),
+                         grad_loss=np.linspace(0.5, 1.5, 5))
+    for r in range(world):
+        d = torch.load(f"{out}.{r}")
+        assert d["n_flat"] == 1 and d["n_packed"] == 1, (d["n_flat"], d["n_packed"])
+        for k in ("dW_f", "dW_g", "dW_o", "db_o"):
+            single = getattr(ref, k).astype(np.float32)        # the single-device fp32 accumulator
+            got = d["g32"][k]
+            assert got.dtype == torch.float32
+            scale = np.abs(single).max()
+            np.testing.assert_allclose(got.numpy(), single, rtol=1e-6, atol=1e-6 * scale)
+            # summed in fp32, rounded once to bf16: within one bf16 rounding (half a step, 2^-8
+            # relative) of the exact sum, plus the fp32 sum's own error
+            got16 = d["g16"][k]
+            assert got16.dtype == torch.bfloat16
+            exact = getattr(ref, k)
+            err = np.abs(got16.double().numpy() - exact)
+            assert np.all(err <= np.abs(exact) * 2.0 ** -8 + 1e-6 * scale), k

@@ -16,12 +16,12 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def _call(batch, mode="tiled", path="auto", grad_loss=None, chunk_cells=0, check=True):
+def _call(batch, mode="tiled", path="auto", grad_loss=None, chunk_cells=0, check=True, wgrad_f32=False):
     d = to_device(batch)
     w = None if grad_loss is None else torch.as_tensor(grad_loss, dtype=torch.float32).cuda()
     loss, grads = frnnt.fwd_bwd(d["f"], d["g"], d["W_f"], d["W_g"], d["W_o"], d["b_o"], d["labels"], d["T_len"],
                                 d["U_len"], grad_loss=w, mode=mode, path=path, chunk_cells=chunk_cells,
-                                blank=batch.blank, check=check)
+                                blank=batch.blank, check=check, wgrad_f32=wgrad_f32)
     torch.cuda.synchronize()
     return loss, grads
 
@@ -123,21 +123,30 @@ def test_padding_labels_are_not_validated(cuda_ok):
     _call(batch)                     # must not raise
 
 
-# ---------------------------------------------------------------- full-size, sampled utterances
+# ---------------------------------------------------------------- fp32 weight gradients
 
 @pytest.mark.parametrize("mode", ["tiled", "untiled"])
-@pytest.mark.parametrize("name", ["medium", "large", "long"])
-def test_full_size_sampled_utterances(cuda_ok, name, mode):
-    """Full-size workloads in the bench's launch configuration: the gradient
-    weights select two utterances, so every output is the oracle's on those two
-    (the other utterances still run through every kernel)."""
-    batch = synth.workload(name)
-    B = batch.f.shape[0]
-    pick = [0, B - 1]
-    w = weights_for(B, pick, device="cpu").numpy()
-    loss, grads = _call(batch, mode=mode, grad_loss=w)
-    ref = run_oracle(batch, grad_loss=w, utterances=pick)
-    compare(loss, grads, ref, "bf16", utterances=pick, extra_note=f"{name}/{mode}")
+@pytest.mark.parametrize("path", ["auto", "simt"])
+def test_fp32_weight_gradients(cuda_ok, mode, path):
+    """wgrad_f32: the weight gradients come back as the fp32 accumulators (df /
+    dg stay bf16); they match the oracle, and rounding them to bf16 gives the
+    default call's bf16 weight gradients up to the reassociation of the fp32
+    atomics (at most one bf16 step apart)."""
+    batch = synth.workload("short")
+    w = np.linspace(0.5, 1.5, batch.f.shape[0])
+    l32, g32 = _call(batch, mode=mode, path=path, grad_loss=w, wgrad_f32=True)
+    l32, g32 = l32.clone(), {k: v.clone() for k, v in g32.items()}
+    for k in ("dW_f", "dW_g", "dW_o", "db_o"):
+        assert g32[k].dtype == torch.float32, k
+    for k in ("df", "dg"):
+        assert g32[k].dtype == torch.bfloat16, k
+    compare(l32, g32, run_oracle(batch, grad_loss=w), "bf16", extra_note=f"short fp32 weight grads/{mode}/{path}")
+    l16, g16 = _call(batch, mode=mode, path=path, grad_loss=w)
+    for k in ("dW_f", "dW_g", "dW_o", "db_o"):
+        a = g32[k].to(torch.bfloat16).float()
+        b = g16[k].float()
+        step = a.abs().clamp_min(1e-30) * 2.0 ** -7
+        assert bool(((a - b).abs() <= step + 1e-6 * a.abs().max()).all()), k
 
 
 def test_tiled_small_chunks_match_untiled(cuda_ok):

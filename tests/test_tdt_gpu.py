@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from rnn_joint_network_02_b200 import frnnt, synth
-from tests.helpers import GRADS, TOL, rel_l2, to_device, weights_for
+from tests.helpers import GRADS, TOL, record, rel_l2, to_device, weights_for
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +43,7 @@ def _compare(loss, grads, ref, note, utterances=None):
         if utterances is not None and name in ("df", "dg"):
             gpu, r = gpu[idx], r[idx]
         errs[name] = rel_l2(gpu, r)
+    record(note, "bf16", errs)
     bad = {k: v for k, v in errs.items() if v > (tol["loss"] if k == "loss" else tol["grad"])}
     assert not bad, f"{note}: tolerance exceeded {bad} (all {errs})"
     return errs
