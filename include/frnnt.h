@@ -86,7 +86,11 @@ typedef struct {
   frnnt_mode mode;
   frnnt_path path;
   int chunk_cells;        /* FRNNT_TILED: lattice cells per backward chunk;
-                             0 = default (65536).  Rounded up to whole tiles. */
+                             0 = default (75776 = 592 tiles of 128 cells, four
+                             waves over 148 SMs, on the tensor-core kernels;
+                             65536 on the CUDA-core kernels).  Rounded up to
+                             whole tiles (whole frame rows on the CUDA-core
+                             kernels). */
   frnnt_loss loss;        /* training criterion (MARGINAL unless set)         */
   int prune_S;            /* 0: the whole lattice.  S > 0 (S <= 32): pruned
                              lattice, frame t of utterance b keeps only the S

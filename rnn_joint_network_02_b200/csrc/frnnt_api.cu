@@ -15,6 +15,10 @@ namespace frnnt {
 namespace {
 
 constexpr int kDefaultChunkCells = 65536;
+// Tensor-core tiled mode, default chunk: four waves of 128-cell tiles over the
+// 148 SMs of a B200 (the backward joint pass runs one CTA per SM, so a chunk of
+// whole waves leaves no SM idle in its last wave).
+constexpr int kDefaultChunkTiles = 4 * 148;
 
 // Bump allocator over the caller's workspace (256-byte aligned slices).
 struct Carver {
@@ -231,16 +235,13 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   Carver c(ws);
   tile_shape_of(s, &p.TB, &p.UB);
   p.maxT = max_tiles(s, p.TB, p.UB);
-  const long long cells = d->chunk_cells > 0 ? d->chunk_cells : kDefaultChunkCells;
-  p.chunkT = (cells + 127) / 128;
+  p.chunkT = d->chunk_cells > 0 ? (d->chunk_cells + 127) / 128 : kDefaultChunkTiles;
   if (p.chunkT > p.maxT) p.chunkT = p.maxT;
   if (d->mode == FRNNT_UNTILED) p.chunkT = p.maxT;
   p.F = c.take<__nv_bfloat16>(s.BT * s.H);
   p.G = c.take<__nv_bfloat16>(s.BU * s.H);
   p.dF = c.take<float>(s.BT * s.H);
   p.dG = c.take<float>(s.BU * s.H);
-  p.dFb = c.take<__nv_bfloat16>(s.BT * s.H);
-  p.dGb = c.take<__nv_bfloat16>(s.BU * s.H);
   p.tiles = c.take<int4>(p.maxT);
   p.ntiles = c.take<int>(4);
   p.L.lse = c.take<float>(s.Nlat);
@@ -249,8 +250,11 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.alpha = c.take<float>(s.Nlat);
   p.L.beta = c.take<float>(s.Nlat);
   p.L.path = s.viterbi ? c.take<uint8_t>(s.Nlat) : nullptr;
-  // the two-diagonal DP's step weights (marginal loss, whole lattice, no durations)
-  p.L.dpw = (!s.viterbi && s.S == 0 && s.n_dur == 0) ? c.take<float>(dp2_weight_floats(s.B, s.T, s.U)) : nullptr;
+  // the two-diagonal DP's step weights (marginal loss, whole lattice, no
+  // durations), precomputed by a parallel pass in untiled mode; tiled mode
+  // keeps its memory down and has the DP form them step by step
+  p.L.dpw = (!s.viterbi && s.S == 0 && s.n_dur == 0 && d->mode == FRNNT_UNTILED)
+                ? c.take<float>(dp2_weight_floats(s.B, s.T, s.U)) : nullptr;
   if (s.n_dur > 0) {
     p.L.beta_l = c.take<float>(s.Nlat);
     p.L.dur_lp = c.take<float>((size_t)s.n_dur * s.Nlat);
@@ -267,8 +271,19 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.row_params = p.db_part ? c.take<float4>((size_t)p.maxT * 128) : nullptr;
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
-  p.zbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * s.Vx);
-  p.hbuf = c.take<__nv_bfloat16>((size_t)p.chunkT * 128 * hidden_stride(s.H));
+  const size_t zb = (size_t)p.chunkT * 128 * s.Vx, hb = (size_t)p.chunkT * 128 * hidden_stride(s.H);
+  p.zbuf = c.take<__nv_bfloat16>(zb);
+  p.hbuf = c.take<__nv_bfloat16>(hb);
+  // bf16 copies of dF and dG for the projection backward, made after the last
+  // chunk: they reuse the chunk buffers when those are large enough
+  const size_t fb = (size_t)s.BT * s.H, gb = (size_t)s.BU * s.H;
+  if ((((fb + 127) & ~(size_t)127) + gb) <= zb + hb) {
+    p.dFb = p.zbuf;
+    p.dGb = p.zbuf ? p.zbuf + ((fb + 127) & ~(size_t)127) : nullptr;
+  } else {
+    p.dFb = c.take<__nv_bfloat16>(fb);
+    p.dGb = c.take<__nv_bfloat16>(gb);
+  }
   p.bytes = c.off + 256;
   return p;
 }

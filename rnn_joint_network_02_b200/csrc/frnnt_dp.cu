@@ -162,6 +162,31 @@ __device__ __forceinline__ DpOps dp2_operands(bool is_beta, int step, int nsteps
   return o;
 }
 
+// The five weights of a step (below) from its six log-probabilities.
+__device__ __forceinline__ void dp2_step_weights(bool is_beta, int step, int nsteps, int last, int u, int Tb, int Ub,
+                                                 const DpOps& o, float (&wv)[5]) {
+  const bool live = step < nsteps && u <= Ub;
+  if (!is_beta) {
+    const int t = 2 * step + 2 - u;
+    const bool mid = live && t - 1 >= 0 && t - 1 < Tb;
+    const bool far = live && 2 * step + 2 <= last && t >= 0 && t < Tb;
+    wv[0] = mid ? o.bA : -INFINITY;
+    wv[1] = mid ? o.lB : -INFINITY;
+    wv[2] = far ? o.bA + o.bB : -INFINITY;
+    wv[3] = far ? log_add_exp(o.bC + o.lA, o.lB + o.bB) : -INFINITY;
+    wv[4] = far ? o.lC + o.lA : -INFINITY;
+  } else {
+    const int t = last - 2 * step - 2 - u;
+    const bool mid = live && t + 1 >= 0 && t + 1 < Tb;
+    const bool far = live && last - 2 * step - 2 >= 0 && t >= 0 && t < Tb;
+    wv[0] = mid ? o.bB : -INFINITY;
+    wv[1] = mid ? o.lA : -INFINITY;
+    wv[2] = far ? o.bA + o.bB : -INFINITY;
+    wv[3] = far ? log_add_exp(o.bA + o.lA, o.lB + o.bC) : -INFINITY;
+    wv[4] = far ? o.lB + o.lC : -INFINITY;
+  }
+}
+
 // The step's weights, precomputed for every (utterance, direction, step, label
 // position) by a parallel kernel, so that the serial wavefront loads five
 // numbers per step with no index arithmetic or bounds checks on them:
@@ -194,37 +219,20 @@ __global__ void dp2_weights_kernel(int B, int T, int U, int NS, int UP, const fl
     const int nsteps = (last + 1) / 2;
     const size_t base = (size_t)b * T * Up1;
     const DpOps o = dp2_operands(is_beta, step, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
-    const bool live = step < nsteps && u <= Ub;
-    float m1, m2, w1, w2, w3;
-    if (!is_beta) {
-      const int t = 2 * step + 2 - u;
-      const bool mid = live && t - 1 >= 0 && t - 1 < Tb;
-      const bool far = live && 2 * step + 2 <= last && t >= 0 && t < Tb;
-      m1 = mid ? o.bA : -INFINITY;
-      m2 = mid ? o.lB : -INFINITY;
-      w1 = far ? o.bA + o.bB : -INFINITY;
-      w2 = far ? log_add_exp(o.bC + o.lA, o.lB + o.bB) : -INFINITY;
-      w3 = far ? o.lC + o.lA : -INFINITY;
-    } else {
-      const int t = last - 2 * step - 2 - u;
-      const bool mid = live && t + 1 >= 0 && t + 1 < Tb;
-      const bool far = live && last - 2 * step - 2 >= 0 && t >= 0 && t < Tb;
-      m1 = mid ? o.bB : -INFINITY;
-      m2 = mid ? o.lA : -INFINITY;
-      w1 = far ? o.bA + o.bB : -INFINITY;
-      w2 = far ? log_add_exp(o.bA + o.lA, o.lB + o.bC) : -INFINITY;
-      w3 = far ? o.lB + o.lC : -INFINITY;
-    }
+    float wv[5];
+    dp2_step_weights(is_beta, step, nsteps, last, u, Tb, Ub, o, wv);
     float* dst = w + ((size_t)(((long long)b * 2 + (is_beta ? 1 : 0)) * NS + step) * 5) * UP + u;
-    dst[0] = m1;
-    dst[UP] = m2;
-    dst[2 * UP] = w1;
-    dst[3 * UP] = w2;
-    dst[4 * UP] = w3;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) dst[k * UP] = wv[k];
   }
 }
 
-__global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank_lp, const float* __restrict__ wts,
+// PRE: the step weights come from dp2_weights_kernel (wts); otherwise each
+// thread forms its own from the six log-probabilities of the step, fetched
+// kPrefetch2 steps ahead (no weight array: the tiled mode's memory budget).
+template <bool PRE>
+__global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank_lp,
+                           const float* __restrict__ label_lp, const float* __restrict__ wts,
                            float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
                            const int32_t* __restrict__ U_len, float* __restrict__ loss) {
   __shared__ float xa[2][1024];     // [parity][thread]: each thread's value on the last far diagonal
@@ -239,7 +247,7 @@ __global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank
   const int last = Tb - 1 + Ub;             // the last diagonal
   const int nsteps = (last + 1) / 2;        // steps of two diagonals after diagonal 0 (alpha) / `last` (beta)
   const bool in_u = u <= Ub;
-  const float* wp = wts + (size_t)((long long)b * 2 + (is_beta ? 1 : 0)) * NS * 5 * nth + u;
+  const float* wp = PRE ? wts + (size_t)((long long)b * 2 + (is_beta ? 1 : 0)) * NS * 5 * nth + u : nullptr;
 
   // the first diagonal: (0,0) for alpha, (Tb-1, Ub) for beta
   float cur = -INFINITY;
@@ -256,10 +264,17 @@ __global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank
   }
 
   float q[kPrefetch2][5];
+  DpOps qo[PRE ? 1 : kPrefetch2];
+  if constexpr (PRE) {
 #pragma unroll
-  for (int i = 0; i < kPrefetch2; ++i)
+    for (int i = 0; i < kPrefetch2; ++i)
 #pragma unroll
-    for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)(i * 5 + k) * nth);
+      for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)(i * 5 + k) * nth);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPrefetch2; ++i)
+      qo[i] = dp2_operands(is_beta, i, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+  }
 
   // parity 1 holds the first diagonal
   xa[1][u] = cur;
@@ -270,10 +285,18 @@ __global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank
     for (int i = 0; i < kPrefetch2; ++i) {
       const int step = step0 + i;
       if (step >= nsteps) break;    // uniform across the block
-      const float m1 = q[i][0], m2 = q[i][1], w1 = q[i][2], w2 = q[i][3], w3 = q[i][4];
-      // (NS covers nsteps + kPrefetch2 steps: no bound on the prefetch)
+      float m1, m2, w1, w2, w3;
+      if constexpr (PRE) {
+        m1 = q[i][0]; m2 = q[i][1]; w1 = q[i][2]; w2 = q[i][3]; w3 = q[i][4];
+        // (NS covers nsteps + kPrefetch2 steps: no bound on the prefetch)
 #pragma unroll
-      for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)((step + kPrefetch2) * 5 + k) * nth);
+        for (int k = 0; k < 5; ++k) q[i][k] = __ldg(wp + (size_t)((step + kPrefetch2) * 5 + k) * nth);
+      } else {
+        float wv[5];
+        dp2_step_weights(is_beta, step, nsteps, last, u, Tb, Ub, qo[i], wv);
+        m1 = wv[0]; m2 = wv[1]; w1 = wv[2]; w2 = wv[3]; w3 = wv[4];
+        qo[i] = dp2_operands(is_beta, step + kPrefetch2, nsteps, u, Tb, Ub, Up1, last, base, blank_lp, label_lp);
+      }
       const int par = (step + 1) & 1;       // parity holding the previous pair's far values
       float n1, n2;                          // neighbours at distance 1 and 2 on the previous far diagonal
       if (!is_beta) {
@@ -995,8 +1018,12 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
                                                   U_len, loss, smem > 0 ? 1 : 0);
   } else {
     dim3 grid(s.B, 2);
-    dp2_kernel<<<grid, threads, 0, st>>>(s.T, s.U, dp2_weight_steps(s.T, s.U), L.blank_lp, L.dpw, L.alpha, L.beta,
-                                         T_len, U_len, loss);
+    if (L.dpw)
+      dp2_kernel<true><<<grid, threads, 0, st>>>(s.T, s.U, dp2_weight_steps(s.T, s.U), L.blank_lp, L.label_lp, L.dpw,
+                                                 L.alpha, L.beta, T_len, U_len, loss);
+    else
+      dp2_kernel<false><<<grid, threads, 0, st>>>(s.T, s.U, 0, L.blank_lp, L.label_lp, nullptr, L.alpha, L.beta,
+                                                  T_len, U_len, loss);
   }
   note_launch();
 }

@@ -282,19 +282,20 @@ __device__ __forceinline__ void seg_chunk_g(const CellMap& m, const SegRow& sr, 
   }
   if (sr.dg) red_add_n<32>(sr.dg + col0, d);
 }
-// dpre = acc (1 - h^2) of the lane's row (0 when it is no cell), then the sums.
-// Every lane of the warp calls this for the same chunk (the shuffles need all).
+// dpre = acc * tanh'(F + G) of the lane's row (0 when it is no cell), then the
+// sums; sv4 holds the derivative (bf16, from dtanh_from_fg).  Every lane of the
+// warp calls this for the same chunk (the shuffles need all).
 __device__ __forceinline__ void seg_chunk(const CellMap& m, const SegRow& sr, int col0, const uint32_t (&r)[32],
-                                          const uint4 (&hv4)[4], int lane) {
+                                          const uint4 (&sv4)[4], int lane) {
   float d[32];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t hw[4] = {hv4[j].x, hv4[j].y, hv4[j].z, hv4[j].w};
+    const uint32_t sw[4] = {sv4[j].x, sv4[j].y, sv4[j].z, sv4[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[q]));
-      d[8 * j + 2 * q] = sr.f ? __uint_as_float(r[8 * j + 2 * q]) * (1.f - hf.x * hf.x) : 0.f;
-      d[8 * j + 2 * q + 1] = sr.f ? __uint_as_float(r[8 * j + 2 * q + 1]) * (1.f - hf.y * hf.y) : 0.f;
+      const float2 sf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sw[q]));
+      d[8 * j + 2 * q] = sr.f ? __uint_as_float(r[8 * j + 2 * q]) * sf.x : 0.f;
+      d[8 * j + 2 * q + 1] = sr.f ? __uint_as_float(r[8 * j + 2 * q + 1]) * sf.y : 0.f;
     }
   }
   switch (m.UB) {
@@ -342,6 +343,56 @@ __device__ __forceinline__ void h_from_fg(const FgRows& fr, int col0, uint4 (&hv
   }
 }
 
+__device__ __forceinline__ float ex2_approx_g(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx_g(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// tanh'(x) = 1 - tanh(x)^2 = sech(x)^2 = 4e / (1 + e)^2 with e = exp(-2|x|) in
+// (0, 1], in fp32 (two MUFU operations: exp2 and reciprocal, each within a few
+// ulp).  Formed this way it keeps its relative accuracy where tanh saturates,
+// which 1 - h^2 of a rounded h loses (h = 0.995 rounded to bf16 is off by up
+// to 2^-9, the derivative there is 0.01).
+__device__ __forceinline__ float sech2_f32(float x) {
+  const float e = ex2_approx_g(-2.8853900817779268f * fabsf(x));   // 2 log2(e) |x|
+  const float r2 = 2.f * rcp_approx_g(1.f + e);
+  return e * r2 * r2;
+}
+// tanh'(F + G) of 32 columns from col0 in bf16 pairs (F and G added in fp32),
+// into sv (the layout of h_from_fg's output); zero when the row is no cell
+__device__ __forceinline__ void dtanh_from_fg(const FgRows& fr, int col0, uint4 (&sv)[4]) {
+  if (!fr.f) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sv[j] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* fp = (const uint4*)(fr.f + col0);
+  const uint4* gp = (const uint4*)(fr.g + col0);
+  uint4 fv[4], gv[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    fv[j] = __ldg(fp + j);
+    gv[j] = __ldg(gp + j);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t o[4];
+    const uint32_t fw[4] = {fv[j].x, fv[j].y, fv[j].z, fv[j].w}, gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&fw[q]));
+      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[q]));
+      o[q] = pack_bf16x2(sech2_f32(a.x + c.x), sech2_f32(a.y + c.y));
+    }
+    sv[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // dtanh epilogue: pull this thread's h row segment of a coming tile into L2
 // while the tile's MMAs run, so the epilogue's reads do not wait on HBM.
 __device__ __forceinline__ void dtanh_prefetch(const GemmParams& p, int row, int n0, int bn, int M) {
@@ -366,6 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
   const Eff eff = eff_of(p);
+  // nothing to do anywhere in the grid (a chunk past the device-built tile
+  // list): leave before any set-up; every CTA sees the same limits
+  if (eff.M <= 0 || eff.kblocks <= 0) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -504,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) h_from_fg(FgRows{sr.f, sr.g}, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg(FgRows{sr.f, sr.g}, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (p.epi == GEMM_EPI_DTANH_SEG) {
@@ -587,6 +641,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
   const Eff eff = eff_of(p);
+  // nothing to do anywhere in the grid: both CTAs of every pair leave alike,
+  // before any set-up or cluster barrier
+  if (eff.M <= 0 || eff.kblocks <= 0) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -727,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hv[4];
         if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
         if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) h_from_fg(FgRows{sr.f, sr.g}, col0, hv);
+        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg(FgRows{sr.f, sr.g}, col0, hv);
         tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
         tmem_wait_ld();
         if (p.epi == GEMM_EPI_DTANH_SEG) {

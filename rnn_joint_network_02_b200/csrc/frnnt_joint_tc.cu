@@ -237,6 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   const int span = ntiles - p.tile_begin;
   const int niter = span <= 0 ? 0 : (PAIR ? (span + 1) / 2 : span);
   auto tile_of = [&](int i) { return p.tile_begin + (PAIR ? 2 * i + (int)rank : i); };
+  // an empty tile range (a chunk past the device-built tile list): every CTA
+  // of the grid computes the same niter, so all leave here, before any set-up
+  // or cluster barrier
+  if (niter == 0) return;
   // arrivals on barriers the (leader's) MMA thread waits for
   auto arrive_leader = [&](uint64_t* bar) {
     if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
@@ -646,12 +650,23 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
             }
           } else if (real) {
+            if (ri.valid) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float d = occ * ex2(fmaf(v[j], kLog2e, -lk));
-              if (col0 + j == p.blank) d -= bpost;
-              if (col0 + j == ri.y) d -= lpost;
-              v[j] = ri.valid ? d : 0.f;
+              for (int j = 0; j < 32; ++j) v[j] = occ * ex2(fmaf(v[j], kLog2e, -lk));
+              // the blank and label columns fall in one 32-column chunk each
+              if (p.blank >= col0 && p.blank < col0 + 32) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (col0 + j == p.blank) v[j] -= bpost;
+              }
+              if (ri.y >= col0 && ri.y < col0 + 32) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (col0 + j == ri.y) v[j] -= lpost;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.f;
             }
             uint32_t w[16];
 #pragma unroll

@@ -131,7 +131,7 @@ def test_fp32_weight_gradients(cuda_ok, mode, path):
     """wgrad_f32: the weight gradients come back as the fp32 accumulators (df /
     dg stay bf16); they match the oracle, and rounding them to bf16 gives the
     default call's bf16 weight gradients up to the reassociation of the fp32
-    atomics (at most one bf16 step apart)."""
+    atomics (bias sums cancel heavily, so this is checked in relative L2)."""
     batch = synth.workload("short")
     w = np.linspace(0.5, 1.5, batch.f.shape[0])
     l32, g32 = _call(batch, mode=mode, path=path, grad_loss=w, wgrad_f32=True)
@@ -143,10 +143,9 @@ def test_fp32_weight_gradients(cuda_ok, mode, path):
     compare(l32, g32, run_oracle(batch, grad_loss=w), "bf16", extra_note=f"short fp32 weight grads/{mode}/{path}")
     l16, g16 = _call(batch, mode=mode, path=path, grad_loss=w)
     for k in ("dW_f", "dW_g", "dW_o", "db_o"):
-        a = g32[k].to(torch.bfloat16).float()
-        b = g16[k].float()
-        step = a.abs().clamp_min(1e-30) * 2.0 ** -7
-        assert bool(((a - b).abs() <= step + 1e-6 * a.abs().max()).all()), k
+        a = g32[k].to(torch.bfloat16).float().cpu().numpy()
+        b = g16[k].float().cpu().numpy()
+        assert rel_l2(a, b) <= 5e-3, (k, rel_l2(a, b))
 
 
 def test_tiled_small_chunks_match_untiled(cuda_ok):
