@@ -268,7 +268,10 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   // untiled with H a multiple of 256: db_o is summed by the dz pass, so the
   // dW_o GEMM runs on N = H (whole 256-wide tiles) without the ones column
   p.db_part = (d->mode == FRNNT_UNTILED && dz_db_supported(s.V, s.H)) ? c.take<float>(s.V) : nullptr;
-  p.row_params = p.db_part ? c.take<float4>((size_t)p.maxT * 128) : nullptr;
+  // per-row scalars of the dz pass: the whole lattice (untiled, with db_o
+  // sums) or one chunk (tiled)
+  p.row_params = p.db_part ? c.take<float4>((size_t)p.maxT * 128)
+                           : (d->mode == FRNNT_TILED ? c.take<float4>((size_t)p.chunkT * 128) : nullptr);
   p.accWf = c.take<float>((size_t)s.Dx * s.H);
   p.accWg = c.take<float>((size_t)s.Dy * s.H);
   const size_t zb = (size_t)p.chunkT * 128 * s.Vx, hb = (size_t)p.chunkT * 128 * hidden_stride(s.H);
@@ -438,6 +441,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       } else {
         j.mode = 2;
         j.store_h = 1;
+        j.row_params = p.row_params;
+        launch_row_params(j, p.row_params, st);
         FRNNT_TRY(launch_joint_tc(j, st));
         if (tdt) launch_tdt_dzd(j, st);
       }

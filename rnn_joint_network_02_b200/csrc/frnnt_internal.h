@@ -229,6 +229,7 @@ struct JointLaunch {
   int32_t* status;
   const int32_t* bounds;        // pruned lattice (s.S > 0): [B][T] first label position of each frame's band
   int store_h = 0;              // modes 1 and 2: the generators also write the h rows of hbuf
+  const float4* row_params = nullptr;   // mode 2: per-row scalars of the launch's tiles (launch_row_params)
 };
 bool joint_tc_supported(int H, int V, int T, int U, int S);
 // Row stride of the h buffer (H hidden columns, then the [1, 0, ...] column block), padded so the
@@ -279,6 +280,9 @@ void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, 
 // Untiled dz pass that also sums db_o into db_acc [V] (cleared beforehand), for
 // dz_db_supported(V, H): the dW_o GEMM then runs on N = H.
 bool dz_db_supported(int V, int H);
+// Per-row scalars (lse log2 e, w bpost, w lpost, label or -2 for no cell) of
+// the tiles [j.tile_begin, j.tile_end), rows (tile - tile_begin) * 128 + r.
+void launch_row_params(const JointLaunch& j, float4* row_params, cudaStream_t st);
 // row_params: scratch of one float4 per row of the launch's tiles.
 void launch_dz_db(const JointLaunch& j, float* db_acc, float4* row_params, cudaStream_t st);
 

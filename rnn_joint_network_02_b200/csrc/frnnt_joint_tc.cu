@@ -80,8 +80,12 @@ struct JointParams {
   __nv_bfloat16* zbuf;    // FWD_STORE: z [tile*128 + r][V]; BWD_DZ: dz [(tile-tile_begin)*128 + r][V]
   __nv_bfloat16* hbuf;    // FWD_STORE / BWD_DZ: h rows [.][HS], same row indexing as zbuf; column H holds 1
   int HS;                 // row stride of hbuf (hidden_stride(H))
-  int srows;              // rows per epilogue store-staging pass (8 or 32)
+  int srows;              // epilogue store-staging rows per warp (0: stores go straight from registers)
   float* db_part;         // dz_db_kernel: db_o accumulator [V] (column sums of dz), else unused
+  // BWD_DZ: per-row scalars of this launch's tiles (row_params_kernel), row
+  // (tile - tile_begin) * 128 + r: (lse log2 e, w bpost, w lpost, label or -2
+  // for no cell), so the epilogue needs one independent load per tile row
+  const float4* rp;
   int32_t* status;
   const int32_t* bounds;  // pruned lattice: [B][T] band starts; S = band width (0: whole lattice)
   int S;
@@ -170,29 +174,17 @@ __device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Store this warp's 32 rows x 32 bf16 (each lane holds its row's 64 bytes in
-// w[16]) to global rows grow0 + i, columns col0.., through a shared staging
-// block of srows rows (80-byte padded rows, bank-conflict-free on both sides),
-// so every global store instruction writes 8 rows x 64 contiguous bytes.
-__device__ __forceinline__ void staged_store_rows(uint8_t* stage, int srows, const uint32_t (&w)[16],
-                                                  __nv_bfloat16* gbase, size_t grow0, size_t ld, int col0) {
-  const int lane = threadIdx.x & 31;
-  for (int pass = 0; pass < 32 / srows; ++pass) {
-    if (lane / srows == pass) {
-      uint4* d = (uint4*)(stage + (lane % srows) * 80);
-      d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      d[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      d[2] = make_uint4(w[8], w[9], w[10], w[11]);
-      d[3] = make_uint4(w[12], w[13], w[14], w[15]);
-    }
-    __syncwarp();
-    for (int k = 0; k < srows / 8; ++k) {
-      const int rr = 8 * k + lane / 4, ch = lane % 4;
-      const uint4 v = *(const uint4*)(stage + rr * 80 + ch * 16);
-      *(uint4*)(gbase + (grow0 + pass * srows + rr) * ld + col0 + ch * 8) = v;
-    }
-    __syncwarp();
-  }
+// Store one row's 32 bf16 (64 bytes, this lane's row of the tile) straight
+// from registers with two 256-bit stores: every store fills one 32-byte
+// sector, so no shared-memory staging is needed to write whole sectors (the
+// staging's shared-memory traffic competed with the W_o operand stream).
+__device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint32_t (&w)[16]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16), "r"(w[8]), "r"(w[9]),
+               "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+               : "memory");
 }
 
 // PAIR: the CTAs of a 2-CTA cluster each own a cell tile (h, epilogue, F/G
@@ -489,9 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               for (int w = 0; w < 8; ++w) pk[kk][j][w] = 0u;
             }
             if (hrow && kk < nk) {
-              uint4* dst = (uint4*)(hrow + seg * 16);
-              dst[0] = make_uint4(pk[kk][j][0], pk[kk][j][1], pk[kk][j][2], pk[kk][j][3]);
-              dst[1] = make_uint4(pk[kk][j][4], pk[kk][j][5], pk[kk][j][6], pk[kk][j][7]);
+              // one 256-bit store: the row segment's whole 32-byte sector
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(hrow + seg * 16),
+                           "r"(pk[kk][j][0]), "r"(pk[kk][j][1]), "r"(pk[kk][j][2]), "r"(pk[kk][j][3]),
+                           "r"(pk[kk][j][4]), "r"(pk[kk][j][5]), "r"(pk[kk][j][6]), "r"(pk[kk][j][7])
+                           : "memory");
             }
           }
         }
@@ -548,26 +542,31 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     const int V = p.Vx;                       // row stride of zbuf
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     int acc_i = 0;
+    // BWD_DZ: the row's scalars, loaded one tile ahead
+    auto load_rp = [&](int i) {
+      const int tl = tile_of(i);
+      return tl < ntiles ? p.rp[(size_t)(tl - p.tile_begin) * 128 + r] : make_float4(0.f, 0.f, 0.f, __int_as_float(-2));
+    };
+    float4 rp_next = make_float4(0.f, 0.f, 0.f, __int_as_float(-2));
+    if (MODE == MODE_BWD_DZ && slot < niter) rp_next = load_rp(slot);
     for (int it = slot; it < niter; it += nslots) {
       const int tile = tile_of(it);
       const bool real = tile < ntiles;   // else the dummy of a pair: consume the accumulators, store nothing
-      const int4 td = real ? p.tiles[tile] : make_int4(0, p.T, 0, 0);
       const size_t row_base = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
-      const RowInfo ri = row_info(p, td, r);
+      RowInfo ri;
       float m = -INFINITY, ssum = 0.f, zb = 0.f, zy = 0.f;
       float lk = 0.f, bpost = 0.f, lpost = 0.f, occ = 0.f;
-      if (MODE == MODE_BWD_DZ && ri.valid) {
-        const size_t c = ri.cell;
-        lk = p.L.lse[c] * kLog2e;
-        const float w = p.grad_loss ? p.grad_loss[ri.b] : 1.f;
-        size_t c0;
-        long long c_t1, c_u1;
-        bool last;
-        lattice_neighbors(p, ri, c0, c_t1, c_u1, last);
-        edge_posteriors(p.L, c, c0, c_t1, c_u1, last, bpost, lpost);
-        bpost *= w;
-        lpost *= w;
+      if (MODE == MODE_BWD_DZ) {
+        const float4 rv = rp_next;
+        if (it + nslots < niter) rp_next = load_rp(it + nslots);
+        ri.y = __float_as_int(rv.w);
+        ri.valid = ri.y != -2;
+        lk = rv.x;
+        bpost = rv.y;
+        lpost = rv.z;
         occ = bpost + lpost;
+      } else {
+        ri = row_info(p, real ? p.tiles[tile] : make_int4(0, p.T, 0, 0), r);
       }
       bool ok = true;
       for (int n = 0; n < p.nV; ++n, ++acc_i) {
@@ -647,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
               uint32_t w[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-              staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
+              store_row64(p.zbuf + (row_base + r) * V + col0, w);
             }
           } else if (real) {
             if (ri.valid) {
@@ -671,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-            staged_store_rows(stage_s + warp * p.srows * 80, p.srows, w, p.zbuf, row_base + q * 32, V, col0);
+            store_row64(p.zbuf + (row_base + r) * V + col0, w);
           }
         }
         tc_fence_before();
@@ -1095,9 +1094,8 @@ int smem_fixed(int KB, int V, int TB, int UB, int srows, bool stage_fg = true) {
 }
 
 // Staging rows: 32 when that still leaves at least 6 full W_o tiles of ring, else 8.
-int staging_rows(int KB, int V, int TB, int UB, bool stage_fg = true) {
-  return (kSmemLimit - smem_fixed(KB, V, TB, UB, 32, stage_fg)) / kStageBytes >= 6 ? 32 : 8;
-}
+// (the epilogue stores straight from registers: no staging rows)
+int staging_rows(int, int, int, int, bool = true) { return 0; }
 
 // Ring stages of stage_bytes each (a full W_o tile, or half of one per CTA of a pair).
 int stages_for(int KB, int V, int TB, int UB, int stage_bytes = kStageBytes, bool stage_fg = true) {
@@ -1321,6 +1319,8 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   p.Vx = j.s.Vx;
   p.n_dur = j.s.n_dur;
   p.store_h = j.store_h;
+  p.rp = j.row_params;
+  if (j.mode == MODE_BWD_DZ && !p.rp) return FRNNT_ERR_CUDA;   // launch_row_params first
   // the backward dz pass covers the label tiles only (the duration head's
   // gradient comes from the stored duration log-probs)
   p.nV = (j.mode == MODE_BWD_DZ ? p.V : p.Vx) / BN;
@@ -1414,6 +1414,36 @@ void launch_dz_db(const JointLaunch& j, float* db_acc, float4* row_params, cudaS
 }
 
 bool dz_db_supported(int V, int H) { return V % 256 == 0 && V <= 4096 && H % 256 == 0; }
+
+void launch_row_params(const JointLaunch& j, float4* row_params, cudaStream_t st) {
+  JointParams p{};
+  p.T = j.s.T;
+  p.U = j.s.U;
+  p.H = j.s.H;
+  p.V = j.s.V;
+  p.blank = j.s.blank;
+  p.TB = j.TB;
+  p.UB = j.UB;
+  p.labels = j.labels;
+  p.T_len = j.T_len;
+  p.U_len = j.U_len;
+  p.grad_loss = j.grad_loss;
+  p.tiles = j.tiles;
+  p.ntiles = j.ntiles;
+  p.tile_begin = j.tile_begin;
+  p.tile_end = j.tile_end;
+  p.bounds = j.bounds;
+  p.S = j.s.S;
+  p.L = j.L;
+  p.Vx = j.s.Vx;
+  p.n_dur = j.s.n_dur;
+  const long long rows = (long long)(j.tile_end - j.tile_begin) * 128;
+  long long blocks = (rows + 255) / 256;
+  if (blocks > sms() * 8) blocks = sms() * 8;
+  if (blocks < 1) blocks = 1;
+  row_params_kernel<<<(unsigned)blocks, 256, 0, st>>>(p, row_params);
+  note_launch();
+}
 
 void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st) {
   JointParams p{};
