@@ -65,12 +65,15 @@ def parse(argv=None):
 # An entry is removed whenever its kernel changes, so the roofline's traffic is
 # null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dWo", "marginal"): (1.204969e9 + 0.008939e9,
+    ("medium", "untiled", "bwd_dWo", "marginal"): (1.147724e9 + 0.008613e9,
                                                    "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "bwd_dh", "marginal"): (0.628156e9 + 0.015830e9,
+    ("medium", "untiled", "bwd_dh", "marginal"): (0.628054e9 + 0.016244e9,
                                                   "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd", "marginal"): (0.009181e9 + 0.556763e9,
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009147e9 + 0.555135e9,
                                                      "profiles/ncu_joint_tc_medium_untiled.md"),
+    # one full 592-tile chunk launch (the stage has four real launches per call)
+    ("medium", "tiled", "joint_bwd_dz", "marginal"): (0.005221e9 + 0.217778e9,
+                                                      "profiles/ncu_joint_bwd_dz_medium_tiled.md (per 592-tile launch)"),
 }
 
 
