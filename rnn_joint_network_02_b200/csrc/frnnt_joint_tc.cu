@@ -1327,10 +1327,13 @@ int launch_joint_tc(const JointLaunch& j, cudaStream_t st) {
   // upper bound of this launch's tile count (the exact count is on the device)
   const long long span = (long long)std::min<long long>(j.tile_end, max_tiles(j.s, j.TB, j.UB)) - j.tile_begin;
   const int ntiles_max = (int)std::max<long long>(0, span);
-  // CTA pairs pay off when W_o is large (each CTA then streams half of it);
-  // for small W_o the coupling of the two CTAs' h generation costs more
+  // CTA pairs pay off when W_o is large (each CTA then streams half of it
+  // through its shared memory, whose bandwidth bounds the one-CTA kernel); for
+  // small W_o the coupling of the two CTAs' h generation costs more (measured:
+  // pairs win from V H = 655k, medium, by 3-5 % in the forward and the
+  // recompute pass, and by 25 % at 4.2M, large)
   const bool pair = g_joint_variant == 1 ||
-                    (g_joint_variant < 0 && ntiles_max >= sms() && (long long)p.Vx * p.H >= (1LL << 21));
+                    (g_joint_variant < 0 && ntiles_max >= sms() && (long long)p.Vx * p.H >= (1LL << 19));
   CUtensorMap tm;
   // a pair CTA stages 64 of the BN rows of every W_o tile
   if (!make_tmap_bf16_2d(&tm, j.W_o, p.H, p.Vx, p.H, 64, pair ? BN / 2 : BN)) return FRNNT_ERR_CUDA;
