@@ -250,11 +250,10 @@ TcPlan plan_tc(const frnnt_dims* d, const Shape& s, void* ws) {
   p.L.alpha = c.take<float>(s.Nlat);
   p.L.beta = c.take<float>(s.Nlat);
   p.L.path = s.viterbi ? c.take<uint8_t>(s.Nlat) : nullptr;
-  // the two-diagonal DP's step weights (marginal loss, whole lattice, no
-  // durations), precomputed by a parallel pass in untiled mode; tiled mode
-  // keeps its memory down and has the DP form them step by step
-  p.L.dpw = (!s.viterbi && s.S == 0 && s.n_dur == 0 && d->mode == FRNNT_UNTILED)
-                ? c.take<float>(dp2_weight_floats(s.B, s.T, s.U)) : nullptr;
+  // the two-diagonal DP forms its step weights step by step (no weight
+  // array: measured as fast as precomputing them by a parallel pass, which
+  // competes with the hidden rows beside the DP in untiled mode)
+  p.L.dpw = nullptr;
   if (s.n_dur > 0) {
     p.L.beta_l = c.take<float>(s.Nlat);
     p.L.dur_lp = c.take<float>((size_t)s.n_dur * s.Nlat);

@@ -30,8 +30,14 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 // warps 0-7 epilogue (two per TMEM lane quadrant, each half of the tile's
 // columns), warp 8 TMA producer, warp 9 MMA issuer
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8, kProdWarp = 8, kMmaWarp = 9;
+// Warp roles (EW = epilogue warps, 8 or 16): warps 0 .. EW-1 epilogue (EW/4
+// per TMEM lane quadrant, each a 4/EW share of a tile's columns), warp EW the
+// TMA producer, warp EW+1 the MMA issuer.  The d_hidden GEMM, whose epilogue
+// (tanh' from F and G, segment sums) outweighs its MMAs, runs with 16
+// epilogue warps so that each scheduler has four to hide the epilogue's load,
+// MUFU and shuffle latencies (medium: 0.406 -> 0.390 ms); the other epilogues
+// keep 8 (more registers per thread).
+constexpr int threads_of(int EW) { return EW * 32 + 64; }
 
 struct GemmParams {
   int M, N, K;
@@ -401,10 +407,11 @@ __device__ __forceinline__ void dtanh_prefetch(const GemmParams& p, int row, int
   for (int c = n0; c < n0 + bn && c < p.N; c += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + c));
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EW>
+__global__ void __launch_bounds__(threads_of(EW), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
   using S = GemmSmem<BN, STAGES>;
+  constexpr int kEpiWarps = EW, kProdWarp = EW, kMmaWarp = EW + 1, kEpiParts = EW / 4;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + S::TILES_BYTES);
@@ -542,16 +549,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column half
+      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column part
       const int row = m0 + q * 32 + lane;
       const bool row_ok = row < eff.M;
-      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0)
+        dtanh_prefetch(p, row, n0 + half * (BN / kEpiParts), BN / kEpiParts, eff.M);
       const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
       const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
       if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
 #pragma unroll 1
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+      for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
         uint32_t r[32];
         const int col0 = n0 + c * 32;
         const bool st = row_ok && col0 < p.N;
@@ -576,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.epi == GEMM_EPI_DTANH) {
         int nm0, nnt, nkb0, nkb1;
         if (unit + (int)gridDim.x < units && unit_coords(unit + gridDim.x, p, eff, nm0, nnt, nkb0, nkb1))
-          dtanh_prefetch(p, nm0 + q * 32 + lane, nnt * BN + half * (BN / 2), BN / 2, eff.M);
+          dtanh_prefetch(p, nm0 + q * 32 + lane, nnt * BN + half * (BN / kEpiParts), BN / kEpiParts, eff.M);
       }
     }
   }
@@ -622,10 +630,11 @@ __device__ __forceinline__ bool unit_coords2(int unit, const GemmParams& p, cons
   return m0 < e.M && kb0 < kb1;
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EW>
+__global__ void __launch_bounds__(threads_of(EW), 1)
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
   using S = Gemm2Smem<BN, STAGES>;
+  constexpr int kEpiWarps = EW, kProdWarp = EW, kMmaWarp = EW + 1, kEpiParts = EW / 4;
   constexpr int HB = BN / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -768,16 +777,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = nt * BN;
       const int a = acc_i & 1;
       const uint32_t aph = (acc_i >> 1) & 1;
-      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column half
+      const int q = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column part
       const int row = m0 + (int)rank * 128 + q * 32 + lane;
       const bool row_ok = row < eff.M;
-      if (p.epi == GEMM_EPI_DTANH && acc_i == 0) dtanh_prefetch(p, row, n0 + half * (BN / 2), BN / 2, eff.M);
+      if (p.epi == GEMM_EPI_DTANH && acc_i == 0)
+        dtanh_prefetch(p, row, n0 + half * (BN / kEpiParts), BN / kEpiParts, eff.M);
       const FgRows fr = (p.epi == GEMM_EPI_DTANH_FG && row_ok) ? fg_rows(p.cells, row) : FgRows{nullptr, nullptr};
       const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
       if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
 #pragma unroll 1
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+      for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
         uint32_t r[32];
         const int col0 = n0 + c * 32;
         const bool st = row_ok && col0 < p.N;
@@ -802,7 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.epi == GEMM_EPI_DTANH) {
         int nm0, nnt, nkb0, nkb1;
         if (unit + npairs < units && unit_coords2(unit + npairs, p, eff, nm0, nnt, nkb0, nkb1))
-          dtanh_prefetch(p, nm0 + (int)rank * 128 + q * 32 + lane, nnt * BN + half * (BN / 2), BN / 2, eff.M);
+          dtanh_prefetch(p, nm0 + (int)rank * 128 + q * 32 + lane, nnt * BN + half * (BN / kEpiParts),
+                         BN / kEpiParts, eff.M);
       }
     }
   }
@@ -846,10 +857,10 @@ int sm_count() {
   return n;
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN>
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EW = 8>
 bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
-  auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN>;
+  auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN, EW>;
   static bool attr[kDeviceSlots] = {};
   const int dev = current_device();
   if (!attr[dev]) {
@@ -857,15 +868,15 @@ bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
       return false;
     attr[dev] = true;
   }
-  kern<<<grid, kThreads, S::TOTAL, st>>>(ta, tb, p);
+  kern<<<grid, threads_of(EW), S::TOTAL, st>>>(ta, tb, p);
   note_launch();
   return cudaPeekAtLastError() == cudaSuccess;
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN>
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EW = 8>
 bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = Gemm2Smem<BN, STAGES>;
-  auto kern = gemm2_tc_kernel<BN, STAGES, A_MN, B_MN>;
+  auto kern = gemm2_tc_kernel<BN, STAGES, A_MN, B_MN, EW>;
   static bool attr[kDeviceSlots] = {};
   const int dev = current_device();
   if (!attr[dev]) {
@@ -875,7 +886,7 @@ bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads_of(EW), 1, 1);
   cfg.dynamicSmemBytes = S::TOTAL;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
@@ -966,18 +977,23 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
     p.lose_first_load = 1;
   }
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  const bool seg = g.epi == GEMM_EPI_DTANH_SEG;   // 16 epilogue warps
   bool launched;
   if (pair) {
     const int npairs = units < sm_count() / 2 ? units : sm_count() / 2;
     const int grid = 2 * npairs;
     if (BN == 256) {
       if (!g.a_mn && !g.b_mn) launched = launch2_t<256, 6, false, false>(ta, tb, p, grid, st);
-      else if (!g.a_mn && g.b_mn) launched = launch2_t<256, 6, false, true>(ta, tb, p, grid, st);
+      else if (!g.a_mn && g.b_mn)
+        launched = seg ? launch2_t<256, 6, false, true, 16>(ta, tb, p, grid, st)
+                       : launch2_t<256, 6, false, true>(ta, tb, p, grid, st);
       else if (g.a_mn && !g.b_mn) launched = launch2_t<256, 6, true, false>(ta, tb, p, grid, st);
       else launched = launch2_t<256, 6, true, true>(ta, tb, p, grid, st);
     } else {
       if (!g.a_mn && !g.b_mn) launched = launch2_t<128, 8, false, false>(ta, tb, p, grid, st);
-      else if (!g.a_mn && g.b_mn) launched = launch2_t<128, 8, false, true>(ta, tb, p, grid, st);
+      else if (!g.a_mn && g.b_mn)
+        launched = seg ? launch2_t<128, 8, false, true, 16>(ta, tb, p, grid, st)
+                       : launch2_t<128, 8, false, true>(ta, tb, p, grid, st);
       else if (g.a_mn && !g.b_mn) launched = launch2_t<128, 8, true, false>(ta, tb, p, grid, st);
       else launched = launch2_t<128, 8, true, true>(ta, tb, p, grid, st);
     }
@@ -986,12 +1002,16 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   const int grid = units < sm_count() ? units : sm_count();
   if (BN == 256) {
     if (!g.a_mn && !g.b_mn) launched = launch_t<256, 4, false, false>(ta, tb, p, grid, st);
-    else if (!g.a_mn && g.b_mn) launched = launch_t<256, 4, false, true>(ta, tb, p, grid, st);
+    else if (!g.a_mn && g.b_mn)
+      launched = seg ? launch_t<256, 4, false, true, 16>(ta, tb, p, grid, st)
+                     : launch_t<256, 4, false, true>(ta, tb, p, grid, st);
     else if (g.a_mn && !g.b_mn) launched = launch_t<256, 4, true, false>(ta, tb, p, grid, st);
     else launched = launch_t<256, 4, true, true>(ta, tb, p, grid, st);
   } else {
     if (!g.a_mn && !g.b_mn) launched = launch_t<128, 6, false, false>(ta, tb, p, grid, st);
-    else if (!g.a_mn && g.b_mn) launched = launch_t<128, 6, false, true>(ta, tb, p, grid, st);
+    else if (!g.a_mn && g.b_mn)
+      launched = seg ? launch_t<128, 6, false, true, 16>(ta, tb, p, grid, st)
+                     : launch_t<128, 6, false, true>(ta, tb, p, grid, st);
     else if (g.a_mn && !g.b_mn) launched = launch_t<128, 6, true, false>(ta, tb, p, grid, st);
     else launched = launch_t<128, 6, true, true>(ta, tb, p, grid, st);
   }
