@@ -799,20 +799,26 @@ __global__ void __launch_bounds__(256, 4) dz_from_z_kernel(JointParams p) {
         const int k = k0 + i * 256 + lane * 8;
         if (k >= V) break;
         const uint32_t zw[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
-        uint32_t o[4];
+        float d[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[q]));
-          float d0 = occ * ex2(fmaf(zf.x, kLog2e, -lk));
-          float d1 = occ * ex2(fmaf(zf.y, kLog2e, -lk));
-          const int k2 = k + 2 * q;
-          if (k2 == p.blank) d0 -= bpost;
-          if (k2 + 1 == p.blank) d1 -= bpost;
-          if (k2 == ri.y) d0 -= lpost;
-          if (k2 + 1 == ri.y) d1 -= lpost;
-          o[q] = pack_bf16x2(d0, d1);
+          d[2 * q] = occ * ex2(fmaf(zf.x, kLog2e, -lk));
+          d[2 * q + 1] = occ * ex2(fmaf(zf.y, kLog2e, -lk));
         }
-        *(uint4*)(zr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+        // the blank and label columns fall in one 8-column group each
+        if ((unsigned)(p.blank - k) < 8u) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (k + j == p.blank) d[j] -= bpost;
+        }
+        if ((unsigned)(ri.y - k) < 8u) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (k + j == ri.y) d[j] -= lpost;
+        }
+        *(uint4*)(zr + k) = make_uint4(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]), pack_bf16x2(d[4], d[5]),
+                                       pack_bf16x2(d[6], d[7]));
       }
     }
   }
@@ -899,18 +905,28 @@ __global__ void __launch_bounds__(256, 3) dz_db_kernel(JointParams p, const floa
       const int k = k0 + i * 256 + lane * 8;
       if (k >= V) break;
       const uint32_t zw[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
-      uint32_t o[4];
+      float d[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[q]));
-        float d0 = occ * ex2(fmaf(zf.x, kLog2e, -lk));
-        float d1 = occ * ex2(fmaf(zf.y, kLog2e, -lk));
-        const int k2 = k + 2 * q;
-        if (k2 == p.blank) d0 -= bpost;
-        if (k2 + 1 == p.blank) d1 -= bpost;
-        if (k2 == y) d0 -= lpost;
-        if (k2 + 1 == y) d1 -= lpost;
-        o[q] = pack_bf16x2(d0, d1);
+        d[2 * q] = occ * ex2(fmaf(zf.x, kLog2e, -lk));
+        d[2 * q + 1] = occ * ex2(fmaf(zf.y, kLog2e, -lk));
+      }
+      // the blank and label columns fall in one 8-column group each
+      if ((unsigned)(p.blank - k) < 8u) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (k + j == p.blank) d[j] -= bpost;
+      }
+      if ((unsigned)(y - k) < 8u) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (k + j == y) d[j] -= lpost;
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        o[q] = pack_bf16x2(d[2 * q], d[2 * q + 1]);
         // the bias gradient sums what the GEMMs read: the bf16-rounded dz
         const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o[q]));
         acc[i][2 * q] += r.x;

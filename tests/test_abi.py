@@ -55,7 +55,8 @@ def test_tiled_workspace_bounded_by_chunk():
 
 
 @pytest.mark.parametrize("field,value,code", [("B", 0, 2), ("H", -1, 2), ("blank", 8, 2), ("U", 1024, 2),
-                                              ("U", 1023, 0), ("dtype", 7, 4), ("mode", 3, 4), ("path", 9, 4)])
+                                              ("U", 1023, 0), ("dtype", 7, 4), ("mode", 3, 4), ("path", 9, 4),
+                                              ("wgrad_f32", 2, 2), ("wgrad_f32", 1, 0)])
 def test_bad_dims_rejected(field, value, code):
     d = frnnt.make_dims(2, 12, 5, 16, 16, 32, 8, dtype="f32")
     setattr(d, field, value)
@@ -269,3 +270,23 @@ def test_every_entry_point_is_documented_in_its_header():
                 seen += 1
                 assert i > 0 and lines[i - 1].strip().endswith("*/"), f"{fn}: {m.group(1)} has no doc comment"
     assert seen == len(_declared_functions())
+
+
+def test_fp32_weight_gradient_outputs_are_one_flat_buffer():
+    """With wgrad_f32 the binding lays dW_f, dW_g, dW_o, db_o out as fp32 views
+    of one flat buffer, each segment on a 16-byte boundary (the library's
+    alignment rule), so the data-parallel exchange reduces them in place."""
+    import torch
+    B, T, U, De, Dp, H, V = 2, 5, 3, 6, 5, 7, 9
+    f = torch.zeros(B, T, De, dtype=torch.bfloat16)
+    g = torch.zeros(B, U + 1, Dp, dtype=torch.bfloat16)
+    W_f, W_g = torch.zeros(De, H, dtype=torch.bfloat16), torch.zeros(Dp, H, dtype=torch.bfloat16)
+    W_o, b_o = torch.zeros(V, H, dtype=torch.bfloat16), torch.zeros(V, dtype=torch.bfloat16)
+    dims = frnnt.make_dims(B, T, U, De, Dp, H, V, wgrad_f32=True)
+    out = frnnt.Outputs(f, g, W_f, W_g, W_o, b_o, dims, with_workspace=False)
+    assert out.df.dtype == torch.bfloat16 and out.dg.dtype == torch.bfloat16
+    for name, ref in (("dW_f", W_f), ("dW_g", W_g), ("dW_o", W_o), ("db_o", b_o)):
+        t = getattr(out, name)
+        assert t.dtype == torch.float32 and tuple(t.shape) == tuple(ref.shape)
+        assert t._base is out.wflat
+        assert (t.data_ptr() - out.wflat.data_ptr()) % 16 == 0
