@@ -403,7 +403,6 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush, workload=
         call()
     torch.cuda.synchronize()
     frnnt.profile_read()
-    frnnt.profile(True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -422,8 +421,21 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush, workload=
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
+    launches = frnnt.profile_read()           # launch counts of the timed steps (always kept)
+    # per-stage device times from separate steps: the library's stage events
+    # sit between kernels that otherwise start while the previous one drains,
+    # so they are kept out of the timed steps
+    prof_steps = min(steps, 5)
+    frnnt.profile(True)
+    for _ in range(prof_steps):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
     frnnt.profile(False)
     stages = frnnt.profile_read()
+    for k, v in stages.items():           # as totals over the timed steps, like the launch counts
+        v["ms"] *= steps / prof_steps
+        v["launches"] = launches[k]["launches"] if k in launches else v["launches"] * steps / prof_steps
     ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     if world > 1:
         t = torch.tensor([ms], device=dev)

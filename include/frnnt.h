@@ -173,7 +173,11 @@ FRNNT_API int frnnt_workspace_size(const frnnt_dims* d, size_t* bytes);
  *               lengths and labels are clamped before use)
  *   stream      cudaStream_t the work is queued on (NULL = legacy stream)
  * The call is stream-ordered and returns without synchronising.  Host-side
- * errors (return value != FRNNT_OK) are detected before any launch. */
+ * errors (return value != FRNNT_OK) are detected before any launch.  Its
+ * consecutive kernels on `stream` are chained by programmatic dependent launch
+ * (each is launched as the previous one's last CTA exits and waits for that
+ * grid's results before touching memory); FRNNT_CHAIN=0 in the environment
+ * turns that off, for tools that do not follow such launches. */
 FRNNT_API int frnnt_fwd_bwd(const frnnt_dims* d,
                   const void* f, const void* g, const void* W_f, const void* W_g,
                   const void* W_o, const void* b_o,

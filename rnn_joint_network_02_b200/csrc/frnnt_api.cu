@@ -326,15 +326,6 @@ SideStream* side_stream() {
   return x.ok ? &x : nullptr;
 }
 
-int splits_for(int M, int N, int K) {
-  const int BN = (N % 256 == 0 && N >= 256) ? 256 : 128;
-  const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
-  const int kb = (K + 63) / 64;
-  int want = (2 * 148 + tiles - 1) / tiles;
-  if (want > kb) want = kb;
-  return want < 1 ? 1 : want;
-}
-
 int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, const void* W_f, const void* W_g,
            const void* W_o, const void* b_o, const void* W_d, const void* b_d, const int32_t* labels,
            const int32_t* T_len, const int32_t* U_len, const int32_t* bounds, const float* grad_loss, float* loss,
@@ -350,6 +341,12 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
   SideStream* side_lock = side_stream();
   std::unique_lock<std::mutex> queue_lock;
   if (side_lock) queue_lock = std::unique_lock<std::mutex>(side_lock->mu);
+  // consecutive kernels of this call on st are chained (each may start while
+  // the one before drains); ended on every return
+  struct ChainScope {
+    explicit ChainScope(cudaStream_t s) { chain_begin(s); }
+    ~ChainScope() { chain_end(); }
+  } chain_scope(st);
 #define FRNNT_TRY(x)            \
   do {                          \
     rc = (x);                   \
@@ -414,6 +411,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     j.tile_begin = 0;
     j.tile_end = (int)p.maxT;
     cudaEventRecord(side->fork, st);
+    chain_break(st);
     cudaStreamWaitEvent(side->s, side->fork, 0);
     {
       StageScope sc("bwd_hidden", side->s);
@@ -448,6 +446,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     }
     if (side) {
       cudaStreamWaitEvent(st, side->join, 0);
+      chain_break(st);
     } else if (untiled) {   // no side stream could be created: build the h rows here
       StageScope sc("bwd_hidden", st);
       launch_hidden_rows(j, 0, st);
@@ -459,14 +458,14 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias
       // gradient, unless the dz pass summed it (then N = H)
       a.M = s.V; a.N = p.db_part ? s.H : HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.Vx; a.B = hrows;
-      a.b_mn = true; a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = splits_for(s.V, a.N, rows);
+      a.b_mn = true; a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = 0;
       a.out_f32 = p.accWo;
       a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;
       FRNNT_TRY(gemm_tc(a, st));
       if (tdt) {
         // dW_d | db_d from the duration columns (64 of them, zero past n_dur)
-        a.M = 64; a.N = HS; a.A = zrows + s.V; a.k_splits = splits_for(64, HS, rows); a.out_f32 = p.accWd;
+        a.M = 64; a.N = HS; a.A = zrows + s.V; a.k_splits = 0; a.out_f32 = p.accWd;
         FRNNT_TRY(gemm_tc(a, st));
       }
     }
@@ -496,6 +495,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     cudaStream_t gs = ps ? ps->s : st;
     if (ps) {
       cudaEventRecord(ps->fork2, st);
+      chain_break(st);
       cudaStreamWaitEvent(gs, ps->fork2, 0);
     }
     launch_wo_finalize(p.accWo, s.V, s.H, dW_o, db_o, st, p.db_part, wf32);
@@ -512,10 +512,10 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     // dW_f = f^T dF : A = f read as MN-major [BT][D_enc], B = dF MN-major [BT][H]
     GemmTcArgs w{};
     w.M = s.Dx; w.N = s.H; w.K = (int)s.BT; w.A = f; w.a_mn = true; w.lda = s.Dx; w.B = p.dFb; w.b_mn = true;
-    w.ldb = s.H; w.epi = GEMM_EPI_RED_F32; w.k_splits = splits_for(s.Dx, s.H, (int)s.BT); w.out_f32 = p.accWf;
+    w.ldb = s.H; w.epi = GEMM_EPI_RED_F32; w.k_splits = 0; w.out_f32 = p.accWf;
     w.ldo = s.H; w.status = status;
     if (rc_f == FRNNT_OK) rc_f = gemm_tc(w, st);
-    w.M = s.Dy; w.K = (int)s.BU; w.A = g; w.lda = s.Dy; w.B = p.dGb; w.k_splits = splits_for(s.Dy, s.H, (int)s.BU);
+    w.M = s.Dy; w.K = (int)s.BU; w.A = g; w.lda = s.Dy; w.B = p.dGb; w.k_splits = 0;
     w.out_f32 = p.accWg;
     if (rc_g == FRNNT_OK) rc_g = gemm_tc(w, gs);
     launch_convert(p.accWf, dW_f, (long long)s.Dx * s.H, !wf32, st);
@@ -523,6 +523,7 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
     if (ps) {   // joined on every path, so the caller's stream never runs ahead of the side work
       cudaEventRecord(ps->join2, gs);
       cudaStreamWaitEvent(st, ps->join2, 0);
+      chain_break(st);
     }
     FRNNT_TRY(rc_f);
     FRNNT_TRY(rc_g);

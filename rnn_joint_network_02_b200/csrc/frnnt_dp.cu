@@ -29,6 +29,7 @@ namespace frnnt {
 __global__ void validate_kernel(int B, int T, int U, int V, int blank, const int32_t* __restrict__ labels,
                                 const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
                                 int32_t* __restrict__ status) {
+  chain_wait();
   int bits = validate_bits(B, T, U, V, blank, labels, T_len, U_len, threadIdx.x, blockDim.x);
   bits = __reduce_or_sync(0xffffffffu, bits);
   if ((threadIdx.x & 31) == 0 && bits) atomicOr(status, bits);
@@ -40,6 +41,7 @@ __global__ void validate_kernel(int B, int T, int U, int V, int blank, const int
 __global__ void validate_bounds_kernel(int B, int T, int U, int S, const int32_t* __restrict__ bounds,
                                        const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
                                        int32_t* __restrict__ status) {
+  chain_wait();
   int bad = 0;
   const long long n = (long long)B * T;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -65,18 +67,18 @@ void launch_validate_bounds(const Shape& s, const int32_t* bounds, const int32_t
                             int32_t* status, cudaStream_t st) {
   const long long n = (long long)s.B * s.T;
   const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
-  validate_bounds_kernel<<<blocks, 256, 0, st>>>(s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
+  launch_k(validate_bounds_kernel, dim3(blocks), dim3(256), 0, st, 1, s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
   note_launch();
 }
 
 void launch_validate(const Shape& s, const int32_t* labels, const int32_t* T_len, const int32_t* U_len,
                      const int32_t* bounds, int32_t* status, cudaStream_t st) {
-  validate_kernel<<<1, 256, 0, st>>>(s.B, s.T, s.U, s.V, s.blank, labels, T_len, U_len, status);
+  launch_k(validate_kernel, dim3(1), dim3(256), 0, st, 1, s.B, s.T, s.U, s.V, s.blank, labels, T_len, U_len, status);
   note_launch();
   if (s.S > 0) {
     const long long n = (long long)s.B * s.T;
     const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
-    validate_bounds_kernel<<<blocks, 256, 0, st>>>(s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
+    launch_k(validate_bounds_kernel, dim3(blocks), dim3(256), 0, st, 1, s.B, s.T, s.U, s.S, bounds, T_len, U_len, status);
     note_launch();
   }
 }
@@ -204,6 +206,7 @@ __device__ __forceinline__ void dp2_step_weights(bool is_beta, int step, int nst
 __global__ void dp2_weights_kernel(int B, int T, int U, int NS, int UP, const float* __restrict__ blank_lp,
                                    const float* __restrict__ label_lp, const int32_t* __restrict__ T_len,
                                    const int32_t* __restrict__ U_len, float* __restrict__ w) {
+  chain_wait();
   const long long n = (long long)B * 2 * NS * UP;
   const int Up1 = U + 1;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -235,6 +238,7 @@ __global__ void dp2_kernel(int T, int U, int NS, const float* __restrict__ blank
                            const float* __restrict__ label_lp, const float* __restrict__ wts,
                            float* __restrict__ alpha, float* __restrict__ beta, const int32_t* __restrict__ T_len,
                            const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  chain_wait();
   __shared__ float xa[2][1024];     // [parity][thread]: each thread's value on the last far diagonal
   const int b = blockIdx.x;
   const bool is_beta = blockIdx.y == 1;
@@ -346,6 +350,7 @@ __global__ void dp_viterbi_kernel(int T, int U, const float* __restrict__ blank_
                                   const float* __restrict__ label_lp, float* __restrict__ alpha,
                                   uint8_t* __restrict__ path, const int32_t* __restrict__ T_len,
                                   const int32_t* __restrict__ U_len, float* __restrict__ loss, int smem_bits) {
+  chain_wait();
   __shared__ float xs[2][32];
   extern __shared__ uint32_t dec_bits[];   // smem_bits: ceil(T (U+1) / 32) words
   const int b = blockIdx.x;
@@ -453,6 +458,7 @@ __global__ void dp_band_kernel(int T, int U, int S, const int32_t* __restrict__ 
                                float* __restrict__ alpha, float* __restrict__ beta, uint8_t* __restrict__ path,
                                const int32_t* __restrict__ T_len, const int32_t* __restrict__ U_len,
                                float* __restrict__ loss) {
+  chain_wait();
   __shared__ float row[2][32];      // [direction][j] of the neighbouring row
   const int b = blockIdx.x;
   const int dir = threadIdx.x;      // 0 alpha, 1 beta
@@ -580,6 +586,7 @@ __global__ void __launch_bounds__(32) dp_band_warp_kernel(int T, int U, int S, c
                                                           float* __restrict__ beta, uint8_t* __restrict__ path,
                                                           const int32_t* __restrict__ T_len,
                                                           const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  chain_wait();
   // shared memory: the utterance's band starts (T ints), then (viterbi) one
   // ballot of decisions per frame (T words)
   extern __shared__ int32_t dsm[];
@@ -811,6 +818,7 @@ __global__ void __launch_bounds__(MAXT) tdt_dp_kernel(int T, int U, uint32_t dma
                                                       float* __restrict__ beta_b, float* __restrict__ beta_l,
                                                       float* __restrict__ q, const int32_t* __restrict__ T_len,
                                                       const int32_t* __restrict__ U_len, float* __restrict__ loss) {
+  chain_wait();
   constexpr int P = tdt_prefetch(DM);
   extern __shared__ float xa[];           // [2][DM+2][blockDim]
   const int b = blockIdx.x;
@@ -955,13 +963,13 @@ void launch_tdt_dp_t(const Shape& s, const Lattice& L, const int32_t* T_len, con
     attr[dev] = true;
   }
   if (threads <= 256)
-    tdt_dp_kernel<DM, 256><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+    launch_k(tdt_dp_kernel<DM, 256>, dim3(grid), dim3(threads), smem, st, 1, s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
                                                         L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
   else if (threads <= 512)
-    tdt_dp_kernel<DM, 512><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
+    launch_k(tdt_dp_kernel<DM, 512>, dim3(grid), dim3(threads), smem, st, 1, s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp, L.dur_lp,
                                                         L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len, loss);
   else
-    tdt_dp_kernel<DM, 1024><<<grid, threads, smem, st>>>(s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp,
+    launch_k(tdt_dp_kernel<DM, 1024>, dim3(grid), dim3(threads), smem, st, 1, s.T, s.U, s.dmask, L.plane, L.blank_lp, L.label_lp,
                                                          L.dur_lp, L.alpha, L.beta, L.beta_l, L.tdt_q, T_len, U_len,
                                                          loss);
 }
@@ -973,7 +981,7 @@ void launch_dp_weights(const Shape& s, const Lattice& L, const int32_t* T_len, c
   const int NS = dp2_weight_steps(s.T, s.U);
   const long long n = (long long)s.B * 2 * NS * threads;
   const int wb = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
-  dp2_weights_kernel<<<wb, 256, 0, st>>>(s.B, s.T, s.U, NS, threads, L.blank_lp, L.label_lp, T_len, U_len, L.dpw);
+  launch_k(dp2_weights_kernel, dim3(wb), dim3(256), 0, st, 1, s.B, s.T, s.U, NS, threads, L.blank_lp, L.label_lp, T_len, U_len, L.dpw);
   note_launch();
 }
 
@@ -998,10 +1006,10 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
       const int sp = s.S <= 4 ? 4 : s.S <= 8 ? 8 : s.S <= 16 ? 16 : 32;
       auto kern = sp == 4 ? dp_band_warp_kernel<4> : sp == 8 ? dp_band_warp_kernel<8>
                 : sp == 16 ? dp_band_warp_kernel<16> : dp_band_warp_kernel<32>;
-      kern<<<grid, 32, smem, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
+      launch_k(kern, dim3(grid), dim3(32), smem, st, 1, s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta,
                                                   L.path, T_len, U_len, loss);
     } else {
-      dp_band_kernel<<<s.B, 32, 0, st>>>(s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta, L.path,
+      launch_k(dp_band_kernel, dim3(s.B), dim3(32), 0, st, 1, s.T, s.U, s.S, bounds, L.blank_lp, L.label_lp, L.alpha, L.beta, L.path,
                                          T_len, U_len, loss);
     }
   } else if (L.path) {
@@ -1014,15 +1022,15 @@ void launch_dp(const Shape& s, const Lattice& L, const int32_t* T_len, const int
       cudaFuncSetAttribute(dp_viterbi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
       attr[dev] = true;
     }
-    dp_viterbi_kernel<<<s.B, threads, smem, st>>>(s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.path, T_len,
+    launch_k(dp_viterbi_kernel, dim3(s.B), dim3(threads), smem, st, 1, s.T, s.U, L.blank_lp, L.label_lp, L.alpha, L.path, T_len,
                                                   U_len, loss, smem > 0 ? 1 : 0);
   } else {
     dim3 grid(s.B, 2);
     if (L.dpw)
-      dp2_kernel<true><<<grid, threads, 0, st>>>(s.T, s.U, dp2_weight_steps(s.T, s.U), L.blank_lp, L.label_lp, L.dpw,
+      launch_k(dp2_kernel<true>, dim3(grid), dim3(threads), 0, st, 1, s.T, s.U, dp2_weight_steps(s.T, s.U), L.blank_lp, L.label_lp, L.dpw,
                                                  L.alpha, L.beta, T_len, U_len, loss);
     else
-      dp2_kernel<false><<<grid, threads, 0, st>>>(s.T, s.U, 0, L.blank_lp, L.label_lp, nullptr, L.alpha, L.beta,
+      launch_k(dp2_kernel<false>, dim3(grid), dim3(threads), 0, st, 1, s.T, s.U, 0, L.blank_lp, L.label_lp, nullptr, L.alpha, L.beta,
                                                   T_len, U_len, loss);
   }
   note_launch();

@@ -423,10 +423,6 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
-  const Eff eff = eff_of(p);
-  // nothing to do anywhere in the grid (a chunk past the device-built tile
-  // list): leave before any set-up; every CTA sees the same limits
-  if (eff.M <= 0 || eff.kblocks <= 0) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -451,6 +447,11 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
+  // set-up done: from here on the previous launches' results are read.  A
+  // device-side limit that leaves no work (a chunk past the device-built tile
+  // list) makes every unit of every role empty.
+  chain_wait();
+  const Eff eff = eff_of(p);
 
   if (warp == kProdWarp) {
     // ---------------------------------------------------------------- producer (warp polls, one lane issues)
@@ -649,10 +650,6 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
-  const Eff eff = eff_of(p);
-  // nothing to do anywhere in the grid: both CTAs of every pair leave alike,
-  // before any set-up or cluster barrier
-  if (eff.M <= 0 || eff.kblocks <= 0) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -677,6 +674,9 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
+  // as in the one-CTA kernel: the previous launches' results are read from here on
+  chain_wait();
+  const Eff eff = eff_of(p);
 
   if (warp == kProdWarp) {
     // ---------------------------------------------------------------- producer (both CTAs; warp polls, one lane issues)
@@ -857,6 +857,36 @@ int sm_count() {
   return n;
 }
 
+// K slices of a split-K GEMM with mn output tiles on `workers` persistent CTAs
+// (or CTA pairs), each taking units workers apart.  The launch lasts about
+// rounds x (k blocks per unit + a unit's fixed cost: pipeline fill and the
+// atomic epilogue), so the slice count minimising that is taken, the fewest on
+// a tie.  A round that only a few workers reach costs as much as a full one:
+// 12 tiles x 13 slices = 156 units on 74 pairs keep 8 pairs busy for a third
+// round, where 6 slices fit one.  The fixed cost is taken as 64 k blocks, which
+// favours fewer slices (fewer atomic epilogues) where the fill is about equal:
+// on 40000 k blocks, 6 slices (one round) and 37 (six) measured the same.
+int auto_splits(int mn, int workers, int kblocks) {
+  if (mn <= 0 || workers <= 0 || kblocks <= 1) return 1;
+  constexpr long long kUnitCost = 64;
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= kblocks; ++s) {
+    const int per = (kblocks + s - 1) / s;
+    const int real = (kblocks + per - 1) / per;   // slices after rounding each to whole k blocks
+    if (real != s) continue;
+    const long long units = (long long)mn * real;
+    const long long rounds = (units + workers - 1) / workers;
+    const long long cost = rounds * (per + kUnitCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = real;
+    }
+    if (rounds > 16) break;   // more slices only add rounds
+  }
+  return best;
+}
+
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EW = 8>
 bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
@@ -868,7 +898,7 @@ bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
       return false;
     attr[dev] = true;
   }
-  kern<<<grid, threads_of(EW), S::TOTAL, st>>>(ta, tb, p);
+  launch_k(kern, dim3(grid), dim3(threads_of(EW)), S::TOTAL, st, 1, ta, tb, p);
   note_launch();
   return cudaPeekAtLastError() == cudaSuccess;
 }
@@ -884,19 +914,7 @@ bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p
       return false;
     attr[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(threads_of(EW), 1, 1);
-  cfg.dynamicSmemBytes = S::TOTAL;
-  cfg.stream = st;
-  cudaLaunchAttribute attrs[1];
-  attrs[0].id = cudaLaunchAttributeClusterDimension;
-  attrs[0].val.clusterDim.x = 2;
-  attrs[0].val.clusterDim.y = 1;
-  attrs[0].val.clusterDim.z = 1;
-  cfg.attrs = attrs;
-  cfg.numAttrs = 1;
-  const bool ok = cudaLaunchKernelEx(&cfg, kern, ta, tb, p) == cudaSuccess;
+  const bool ok = launch_k(kern, dim3(grid), dim3(threads_of(EW)), S::TOTAL, st, 2, ta, tb, p) == cudaSuccess;
   note_launch();
   return ok && cudaPeekAtLastError() == cudaSuccess;
 }
@@ -954,7 +972,10 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   p.m_tiles = (g.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
   p.n_tiles = (g.N + BN - 1) / BN;
   p.kblocks = (g.K + BK - 1) / BK;
-  int splits = g.k_splits < 1 ? 1 : g.k_splits;
+  int splits = g.k_splits;
+  if (splits == 0 && g.epi == GEMM_EPI_RED_F32)
+    splits = auto_splits(p.m_tiles * p.n_tiles, pair ? sm_count() / 2 : sm_count(), p.kblocks);
+  if (splits < 1) splits = 1;
   if (splits > p.kblocks) splits = p.kblocks;
   if (splits > 1 && g.epi != GEMM_EPI_RED_F32) return FRNNT_ERR_UNSUPPORTED;
   // every split must own at least one k block

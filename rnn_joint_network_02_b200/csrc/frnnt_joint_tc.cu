@@ -220,19 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   float* lse_x = (float*)(tmem_base_p + 4);       // [128][4] half-1 epilogue state for the combine
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = min(p.tile_end, *p.ntiles);
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   // iteration i of the persistent loop covers tile tile_begin + i (one CTA) or
   // tiles tile_begin + 2i and 2i + 1 (a pair; a missing odd tile is a dummy)
   const int slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nslots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int span = ntiles - p.tile_begin;
-  const int niter = span <= 0 ? 0 : (PAIR ? (span + 1) / 2 : span);
   auto tile_of = [&](int i) { return p.tile_begin + (PAIR ? 2 * i + (int)rank : i); };
-  // an empty tile range (a chunk past the device-built tile list): every CTA
-  // of the grid computes the same niter, so all leave here, before any set-up
-  // or cluster barrier
-  if (niter == 0) return;
   // arrivals on barriers the (leader's) MMA thread waits for
   auto arrive_leader = [&](uint64_t* bar) {
     if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
@@ -261,7 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int k = threadIdx.x; k < p.Vx; k += blockDim.x) bias_s[k] = p.b_o[k];
   if (warp == kMmaWarp) {
     if (PAIR) {
       tmem_alloc_pair(tmem_base_p, 512);
@@ -276,6 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   else __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
+  // set-up done: from here on the previous launches' results are read
+  chain_wait();
+  const int ntiles = min(p.tile_end, *p.ntiles);
+  const int span = ntiles - p.tile_begin;
+  // an empty tile range (a chunk past the device-built tile list) gives every
+  // CTA of the grid niter = 0: all skip to the teardown alike
+  const int niter = span <= 0 ? 0 : (PAIR ? (span + 1) / 2 : span);
+  for (int k = threadIdx.x; k < p.Vx; k += blockDim.x) bias_s[k] = p.b_o[k];
+  __syncthreads();
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer: W_o tiles
@@ -756,6 +757,7 @@ __device__ __forceinline__ void tdt_dzd_row(const JointParams& p, const RowInfo&
 // transducer's kernel keeps its register count and occupancy).
 template <bool TDT>
 __global__ void __launch_bounds__(256, 4) dz_from_z_kernel(JointParams p) {
+  chain_wait();
   // one warp per row; rows of tiles [tile_begin, ntiles).  A row's z is read
   // in batches of four 16-byte chunks per lane, all loads of a batch issued
   // before any store (the row is rewritten in place).
@@ -836,6 +838,7 @@ __global__ void __launch_bounds__(256, 4) dz_from_z_kernel(JointParams p) {
 // with the label -2 for a row that is no lattice cell (-1: a cell without a
 // label edge).
 __global__ void row_params_kernel(JointParams p, float4* __restrict__ rp) {
+  chain_wait();
   const int ntiles = min(p.tile_end, *p.ntiles);
   const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
   for (long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x; row < nrows;
@@ -859,6 +862,7 @@ __global__ void row_params_kernel(JointParams p, float4* __restrict__ rp) {
 
 template <bool TDT>
 __global__ void __launch_bounds__(256, 3) dz_db_kernel(JointParams p, const float4* __restrict__ rp) {
+  chain_wait();
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int V = p.V, ldz = p.Vx;
   const int lane = threadIdx.x & 31;
@@ -948,6 +952,7 @@ __global__ void __launch_bounds__(256, 3) dz_db_kernel(JointParams p, const floa
 // Tiled backward of the token-and-duration transducer: the duration columns of
 // the chunk's dz rows (the label columns come from the joint kernel's dz pass).
 __global__ void tdt_dzd_kernel(JointParams p) {
+  chain_wait();
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)max(0, ntiles - p.tile_begin) * 128;
@@ -964,6 +969,7 @@ __global__ void tdt_weights_kernel(int V, int H, int n_dur, int Vx, const __nv_b
                                    const __nv_bfloat16* __restrict__ b_o, const __nv_bfloat16* __restrict__ W_d,
                                    const __nv_bfloat16* __restrict__ b_d, __nv_bfloat16* __restrict__ W_x,
                                    __nv_bfloat16* __restrict__ b_x) {
+  chain_wait();
   const int cpr = H / 8;                          // 16-byte chunks per row
   const long long n = (long long)Vx * cpr;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -985,6 +991,7 @@ __global__ void tdt_weights_kernel(int V, int H, int n_dur, int Vx, const __nv_b
 // kernel, plus the extra column block [1, 0, ..., 0] (0 for cells outside the
 // lattice) whose dz-weighted sum is db_o.  One warp per row, coalesced.
 __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
+  chain_wait();
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int H = p.H, HS = p.HS, Up1 = p.U + 1;
   const int lane = threadIdx.x & 31;
@@ -1031,6 +1038,7 @@ __global__ void hidden_rows_kernel(JointParams p, int row_tile0) {
 // each F row serves UB rows, each G row TB rows), then 8 warps write the
 // tile's 128 rows, 16-byte stores.  Dynamic shared memory (TB + UB) H bf16.
 __global__ void __launch_bounds__(256) hidden_tiles_kernel(JointParams p, int row_tile0) {
+  chain_wait();
   extern __shared__ __align__(16) __nv_bfloat16 fg_s[];   // [TB][H] F rows, then [UB][H] G rows
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int H = p.H, HS = p.HS, Up1 = p.U + 1, TB = p.TB, UB = p.UB;
@@ -1075,6 +1083,7 @@ __global__ void __launch_bounds__(256) hidden_tiles_kernel(JointParams p, int ro
 template <bool OUT_F32>
 __global__ void wo_finalize_kernel(const float* __restrict__ acc, int V, int H, int HS, const float* __restrict__ db,
                                    void* __restrict__ dW_o, void* __restrict__ db_o) {
+  chain_wait();
   const long long n = (long long)V * H;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const long long k = i / H, j = i % H;
@@ -1159,7 +1168,7 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
     attr_set[dev] = true;
   }
   if (!PAIR) {
-    kern<<<sms(), kThreads, smem, st>>>(tm, p);
+    launch_k(kern, dim3(sms()), dim3(kThreads), smem, st, 1, tm, p);
   } else {
     // one cluster of two CTAs per pair of tiles; persistent, so no more
     // clusters than can be resident at once (an SM left without a partner in
@@ -1188,8 +1197,7 @@ int launch_joint_t(const CUtensorMap& tm, JointParams p, int ntiles_max, cudaStr
     }
     const int pairs = (ntiles_max + 1) / 2;
     const int npairs = pairs < resident[dev] ? (pairs > 0 ? pairs : 1) : resident[dev];
-    cfg.gridDim = dim3(2 * npairs, 1, 1);
-    if (cudaLaunchKernelEx(&cfg, kern, tm, p) != cudaSuccess) {
+    if (launch_k(kern, dim3(2 * npairs), dim3(kThreads), smem, st, 2, tm, p) != cudaSuccess) {
       note_launch();
       return FRNNT_ERR_CUDA;
     }
@@ -1250,6 +1258,7 @@ __global__ void __launch_bounds__(1024) prologue_kernel(int B, int T, int U, int
                                                         const int32_t* __restrict__ U_len, int32_t* status,
                                                         int4* __restrict__ tiles, int* __restrict__ ntiles,
                                                         ZeroList z) {
+  chain_wait();
   if (blockIdx.x > 0) {
     const long long stride = (long long)(gridDim.x - 1) * blockDim.x;
     const long long tid = (long long)(blockIdx.x - 1) * blockDim.x + threadIdx.x;
@@ -1298,7 +1307,7 @@ void launch_prologue(const Shape& s, int TB, int UB, const int32_t* labels, cons
   int zb = (int)((total / 4 + 1023) / 1024);
   if (zb > 2 * sms()) zb = 2 * sms();
   if (zb < 1) zb = 1;
-  prologue_kernel<<<1 + zb, 1024, 0, st>>>(s.B, s.T, s.U, s.V, s.blank, TB, UB, s.S > 0 ? 1 : 0, labels, T_len,
+  launch_k(prologue_kernel, dim3(1 + zb), dim3(1024), 0, st, 1, s.B, s.T, s.U, s.V, s.blank, TB, UB, s.S > 0 ? 1 : 0, labels, T_len,
                                            U_len, status, tiles, ntiles, z);
   note_launch();
 }
@@ -1392,8 +1401,8 @@ void launch_dz_from_z(const JointLaunch& j, cudaStream_t st) {
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.Vx = j.s.Vx;
   p.n_dur = j.s.n_dur;
-  if (p.n_dur > 0) dz_from_z_kernel<true><<<sms() * 4, 256, 0, st>>>(p);
-  else dz_from_z_kernel<false><<<sms() * 4, 256, 0, st>>>(p);
+  if (p.n_dur > 0) launch_k(dz_from_z_kernel<true>, dim3(sms() * 4), dim3(256), 0, st, 1, p);
+  else launch_k(dz_from_z_kernel<false>, dim3(sms() * 4), dim3(256), 0, st, 1, p);
   note_launch();
 }
 
@@ -1425,10 +1434,10 @@ void launch_dz_db(const JointLaunch& j, float* db_acc, float4* row_params, cudaS
   const int ncr = (j.s.V + 1023) / 1024;
   int blocks = sms() * 3;
   blocks -= blocks % (ncr == 3 ? 3 : 1);
-  row_params_kernel<<<sms() * 8, 256, 0, st>>>(p, row_params);
+  launch_k(row_params_kernel, dim3(sms() * 8), dim3(256), 0, st, 1, p, row_params);
   note_launch();
-  if (p.n_dur > 0) dz_db_kernel<true><<<blocks, 256, 0, st>>>(p, row_params);
-  else dz_db_kernel<false><<<blocks, 256, 0, st>>>(p, row_params);
+  if (p.n_dur > 0) launch_k(dz_db_kernel<true>, dim3(blocks), dim3(256), 0, st, 1, p, row_params);
+  else launch_k(dz_db_kernel<false>, dim3(blocks), dim3(256), 0, st, 1, p, row_params);
   note_launch();
 }
 
@@ -1460,7 +1469,7 @@ void launch_row_params(const JointLaunch& j, float4* row_params, cudaStream_t st
   long long blocks = (rows + 255) / 256;
   if (blocks > sms() * 8) blocks = sms() * 8;
   if (blocks < 1) blocks = 1;
-  row_params_kernel<<<(unsigned)blocks, 256, 0, st>>>(p, row_params);
+  launch_k(row_params_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, p, row_params);
   note_launch();
 }
 
@@ -1485,13 +1494,13 @@ void launch_tdt_dzd(const JointLaunch& j, cudaStream_t st) {
   p.zbuf = (__nv_bfloat16*)j.zbuf;
   p.Vx = j.s.Vx;
   p.n_dur = j.s.n_dur;
-  tdt_dzd_kernel<<<sms() * 4, 256, 0, st>>>(p);
+  launch_k(tdt_dzd_kernel, dim3(sms() * 4), dim3(256), 0, st, 1, p);
   note_launch();
 }
 
 void launch_tdt_weights(const Shape& s, const void* W_o, const void* b_o, const void* W_d, const void* b_d, void* W_x,
                         void* b_x, cudaStream_t st) {
-  tdt_weights_kernel<<<sms() * 2, 256, 0, st>>>(s.V, s.H, s.n_dur, s.Vx, (const __nv_bfloat16*)W_o,
+  launch_k(tdt_weights_kernel, dim3(sms() * 2), dim3(256), 0, st, 1, s.V, s.H, s.n_dur, s.Vx, (const __nv_bfloat16*)W_o,
                                                 (const __nv_bfloat16*)b_o, (const __nv_bfloat16*)W_d,
                                                 (const __nv_bfloat16*)b_d, (__nv_bfloat16*)W_x, (__nv_bfloat16*)b_x);
   note_launch();
@@ -1531,9 +1540,9 @@ void launch_hidden_rows(const JointLaunch& j, int row_tile0, cudaStream_t st, in
     // fewer when their shared memory does not fit: one full wave
     int hb = (220 * 1024) / smem;
     hb = hb < 1 ? 1 : (hb > 6 ? 6 : hb);
-    hidden_tiles_kernel<<<sms() * hb, 256, smem, st>>>(p, row_tile0);
+    launch_k(hidden_tiles_kernel, dim3(sms() * hb), dim3(256), smem, st, 1, p, row_tile0);
   } else {
-    hidden_rows_kernel<<<sms() * blocks_per_sm, 256, 0, st>>>(p, row_tile0);
+    launch_k(hidden_rows_kernel, dim3(sms() * blocks_per_sm), dim3(256), 0, st, 1, p, row_tile0);
   }
   note_launch();
 }
@@ -1544,9 +1553,9 @@ void launch_wo_finalize(const float* acc, int V, int H, void* dW_o, void* db_o, 
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (out_f32)
-    wo_finalize_kernel<true><<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, dW_o, db_o);
+    launch_k(wo_finalize_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, st, 1, acc, V, H, hidden_stride(H), db, dW_o, db_o);
   else
-    wo_finalize_kernel<false><<<(unsigned)blocks, 256, 0, st>>>(acc, V, H, hidden_stride(H), db, dW_o, db_o);
+    launch_k(wo_finalize_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, st, 1, acc, V, H, hidden_stride(H), db, dW_o, db_o);
   note_launch();
 }
 

@@ -1,4 +1,5 @@
 // Stage tracing: launch counts (always on) and optional CUDA-event timing.
+#include <stdlib.h>
 #include <string.h>
 
 #include <vector>
@@ -51,11 +52,45 @@ cudaEvent_t take_event() {
 
 void note_launch(int n) { g_launches += n; }
 
+// ---------------------------------------------------------------- launch chaining (per host thread)
+namespace {
+struct Chain {
+  cudaStream_t st = nullptr;
+  bool active = false;   // a call is queueing on st
+  bool armed = false;    // the last operation queued on st was one of the call's kernels
+};
+thread_local Chain t_chain;
+bool chain_enabled() {
+  // FRNNT_CHAIN=0 in the environment turns chaining off (every launch then
+  // waits for the previous one in the plain stream order)
+  static const bool on = [] {
+    const char* e = getenv("FRNNT_CHAIN");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+}  // namespace
+
+void chain_begin(cudaStream_t st) {
+  t_chain.st = st;
+  t_chain.active = chain_enabled();
+  t_chain.armed = false;
+}
+void chain_break(cudaStream_t st) {
+  if (t_chain.active && st == t_chain.st) t_chain.armed = false;
+}
+void chain_end() { t_chain = Chain{}; }
+bool chain_take(cudaStream_t st) { return t_chain.active && t_chain.armed && st == t_chain.st; }
+void chain_note(cudaStream_t st) {
+  if (t_chain.active && st == t_chain.st) t_chain.armed = true;
+}
+
 StageScope::StageScope(const char* name, cudaStream_t st) : st_(st), launches0_(g_launches) {
   stage_ = stage_index(name);
   if (g_timing) {
     start_ = take_event();
     if (start_) cudaEventRecord(start_, st_);
+    chain_break(st_);
   }
 }
 
@@ -67,6 +102,7 @@ StageScope::~StageScope() {
     cudaEvent_t stop = take_event();
     if (stop) {
       cudaEventRecord(stop, st_);
+      chain_break(st_);
       g_pending.push_back({stage_, (cudaEvent_t)start_, stop});
     } else {
       g_free_events.push_back((cudaEvent_t)start_);

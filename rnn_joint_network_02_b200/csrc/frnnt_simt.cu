@@ -309,6 +309,7 @@ void launch_dtanh_reduce_simt(const Shape& s, const float* dh, const float* h, l
 
 // ------------------------------------------------------------------ convert
 __global__ void convert_kernel(const float* __restrict__ in, void* __restrict__ out, long long n, int to_bf16) {
+  chain_wait();
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     if (to_bf16) ((__nv_bfloat16*)out)[i] = __float2bfloat16_rn(in[i]);
     else ((float*)out)[i] = in[i];
@@ -319,7 +320,7 @@ void launch_convert(const float* in, void* out, long long n, bool to_bf16, cudaS
   if (n <= 0) return;
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  convert_kernel<<<(unsigned)blocks, 256, 0, st>>>(in, out, n, to_bf16);
+  launch_k(convert_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, in, out, n, to_bf16);
   note_launch();
 }
 
