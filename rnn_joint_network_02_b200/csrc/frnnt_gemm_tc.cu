@@ -232,8 +232,8 @@ __device__ __forceinline__ SegRow seg_row(const CellMap& m, int row, bool row_ok
 // One recursive-halving level over lanes s apart: of the first N values a
 // lane keeps the upper half when (lane & s), the lower one otherwise, plus
 // its partner's copy of that half.
-template <int N>
-__device__ __forceinline__ void rs_level(float (&v)[32], int s, bool upper) {
+template <int N, int A>
+__device__ __forceinline__ void rs_level(float (&v)[A], int s, bool upper) {
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
     const float give = upper ? v[i] : v[i + N / 2];
@@ -241,25 +241,26 @@ __device__ __forceinline__ void rs_level(float (&v)[32], int s, bool upper) {
     v[i] = keep + __shfl_xor_sync(0xffffffffu, give, s);
   }
 }
-// Sum over each group of G consecutive lanes: v[0 .. 32/G) becomes the sum of
-// columns (32/G) (lane % G) + i.
-template <int G, int N = 32>
-__device__ __forceinline__ void rs_within(float (&v)[32], int lane) {
+// Sum over each group of G consecutive lanes (G <= N): v[0 .. N/G) becomes the
+// sum of columns (N/G) (lane % G) + i.
+template <int G, int N, int A>
+__device__ __forceinline__ void rs_within(float (&v)[A], int lane) {
   if constexpr (G > 1) {
     rs_level<N>(v, G / 2, (lane & (G / 2)) != 0);
     rs_within<G / 2, N / 2>(v, lane);
   }
 }
-// Sum over the lanes congruent modulo G: v[0 .. G) becomes the sum of columns G (lane / G) + i.
-template <int G, int S = 16, int N = 32>
-__device__ __forceinline__ void rs_across(float (&v)[32], int lane) {
+// Sum over the lanes congruent modulo G: v[0 .. N G/32) becomes the sum of
+// columns (N G/32) (lane / G) + i.
+template <int G, int N, int A, int S = 16>
+__device__ __forceinline__ void rs_across(float (&v)[A], int lane) {
   if constexpr (S >= G) {
     rs_level<N>(v, S, (lane & S) != 0);
-    rs_across<G, S / 2, N / 2>(v, lane);
+    rs_across<G, N / 2, A, S / 2>(v, lane);
   }
 }
-template <int NV>
-__device__ __forceinline__ void red_add_n(float* dst, const float (&v)[32]) {
+template <int NV, int A>
+__device__ __forceinline__ void red_add_n(float* dst, const float (&v)[A]) {
   if constexpr (NV == 1) {
     red_add_f32(dst, v[0]);
   } else if constexpr (NV == 2) {
@@ -269,33 +270,43 @@ __device__ __forceinline__ void red_add_n(float* dst, const float (&v)[32]) {
     for (int i = 0; i < NV; i += 4) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
   }
 }
-template <int G>
-__device__ __forceinline__ void seg_chunk_g(const CellMap& m, const SegRow& sr, int col0, const float (&d)[32],
+// The sums of one chunk of N columns (N = 16 or 32) of dpre: into dF over the
+// G lanes of a frame (G = the tile's label positions), into dG over the lanes
+// of a label position (pruned lattice: each lane its own dG row).
+template <int G, int N>
+__device__ __forceinline__ void seg_chunk_g(const CellMap& m, const SegRow& sr, int col0, const float (&d)[N],
                                             int lane) {
-  float v[32];
+  float v[N];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = d[i];
-  rs_within<G>(v, lane);
-  if (sr.df) red_add_n<32 / G>(sr.df + col0 + (32 / G) * (lane & (G - 1)), v);
+  for (int i = 0; i < N; ++i) v[i] = d[i];
+  if constexpr (G <= N) {
+    rs_within<G, N>(v, lane);
+    if (sr.df) red_add_n<N / G>(sr.df + col0 + (N / G) * (lane & (G - 1)), v);
+  } else {   // a 32-lane frame and 16 columns: sum each half-warp, then the halves
+    rs_within<N, N>(v, lane);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+    if (sr.df && lane < N) red_add_f32(sr.df + col0 + lane, v[0]);
+  }
   if constexpr (G < 32) {
     if (m.S == 0) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = d[i];
-      rs_across<G>(v, lane);
-      if (sr.dg) red_add_n<G>(sr.dg + col0 + G * (lane / G), v);
+      for (int i = 0; i < N; ++i) v[i] = d[i];
+      rs_across<G, N>(v, lane);
+      if (sr.dg) red_add_n<N * G / 32>(sr.dg + col0 + (N * G / 32) * (lane / G), v);
       return;
     }
   }
-  if (sr.dg) red_add_n<32>(sr.dg + col0, d);
+  if (sr.dg) red_add_n<N>(sr.dg + col0, d);
 }
 // dpre = acc * tanh'(F + G) of the lane's row (0 when it is no cell), then the
 // sums; sv4 holds the derivative (bf16, from dtanh_from_fg).  Every lane of the
 // warp calls this for the same chunk (the shuffles need all).
-__device__ __forceinline__ void seg_chunk(const CellMap& m, const SegRow& sr, int col0, const uint32_t (&r)[32],
-                                          const uint4 (&sv4)[4], int lane) {
-  float d[32];
+template <int N>
+__device__ __forceinline__ void seg_chunk(const CellMap& m, const SegRow& sr, int col0, const uint32_t (&r)[N],
+                                          const uint4 (&sv4)[N / 8], int lane) {
+  float d[N];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < N / 8; ++j) {
     const uint32_t sw[4] = {sv4[j].x, sv4[j].y, sv4[j].z, sv4[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -305,10 +316,10 @@ __device__ __forceinline__ void seg_chunk(const CellMap& m, const SegRow& sr, in
     }
   }
   switch (m.UB) {
-    case 4: seg_chunk_g<4>(m, sr, col0, d, lane); break;
-    case 8: seg_chunk_g<8>(m, sr, col0, d, lane); break;
-    case 16: seg_chunk_g<16>(m, sr, col0, d, lane); break;
-    default: seg_chunk_g<32>(m, sr, col0, d, lane); break;
+    case 4: seg_chunk_g<4, N>(m, sr, col0, d, lane); break;
+    case 8: seg_chunk_g<8, N>(m, sr, col0, d, lane); break;
+    case 16: seg_chunk_g<16, N>(m, sr, col0, d, lane); break;
+    default: seg_chunk_g<32, N>(m, sr, col0, d, lane); break;
   }
 }
 
@@ -369,24 +380,25 @@ __device__ __forceinline__ float sech2_f32(float x) {
   const float r2 = 2.f * rcp_approx_g(1.f + e);
   return e * r2 * r2;
 }
-// tanh'(F + G) of 32 columns from col0 in bf16 pairs (F and G added in fp32),
-// into sv (the layout of h_from_fg's output); zero when the row is no cell
-__device__ __forceinline__ void dtanh_from_fg(const FgRows& fr, int col0, uint4 (&sv)[4]) {
+// tanh'(F + G) of N columns (16 or 32) from col0 in bf16 pairs (F and G added
+// in fp32), into sv (the layout of h_from_fg's output); zero when the row is no cell
+template <int N>
+__device__ __forceinline__ void dtanh_from_fg(const FgRows& fr, int col0, uint4 (&sv)[N / 8]) {
   if (!fr.f) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) sv[j] = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < N / 8; ++j) sv[j] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   const uint4* fp = (const uint4*)(fr.f + col0);
   const uint4* gp = (const uint4*)(fr.g + col0);
-  uint4 fv[4], gv[4];
+  uint4 fv[N / 8], gv[N / 8];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < N / 8; ++j) {
     fv[j] = __ldg(fp + j);
     gv[j] = __ldg(gp + j);
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < N / 8; ++j) {
     uint32_t o[4];
     const uint32_t fw[4] = {fv[j].x, fv[j].y, fv[j].z, fv[j].w}, gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
 #pragma unroll
@@ -559,24 +571,41 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
       const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
       if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
+      if constexpr (EW == 16) {
+        // the d_hidden epilogue (the one launched with 16 epilogue warps) in
+        // 16-column chunks: half the registers of 32-column ones, so the 96 a
+        // thread gets at 576 threads hold it without spilling
 #pragma unroll 1
-      for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
-        uint32_t r[32];
-        const int col0 = n0 + c * 32;
-        const bool st = row_ok && col0 < p.N;
-        uint4 hv[4];
-        if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg(FgRows{sr.f, sr.g}, col0, hv);
-        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
-        tmem_wait_ld();
-        if (p.epi == GEMM_EPI_DTANH_SEG) {
-          if (col0 < p.N) seg_chunk(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
-          continue;
+        for (int c = half * (BN / (16 * kEpiParts)); c < (half + 1) * (BN / (16 * kEpiParts)); ++c) {
+          const int col0 = n0 + c * 16;
+          if (col0 >= p.N) break;   // the same for the whole warp; later chunks lie further right
+          uint4 hv[2];
+          dtanh_from_fg<16>(FgRows{sr.f, sr.g}, col0, hv);
+          uint32_t r[16];
+          tmem_ld16(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 16, r);
+          tmem_wait_ld();
+          seg_chunk<16>(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
         }
-        if (!st) continue;
-        if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
-        else epilogue_store(p, row, col0, r);
+      } else {
+#pragma unroll 1
+        for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
+          uint32_t r[32];
+          const int col0 = n0 + c * 32;
+          const bool st = row_ok && col0 < p.N;
+          uint4 hv[4];
+          if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
+          if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
+          if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg<32>(FgRows{sr.f, sr.g}, col0, hv);
+          tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
+          tmem_wait_ld();
+          if (p.epi == GEMM_EPI_DTANH_SEG) {
+            if (col0 < p.N) seg_chunk<32>(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
+            continue;
+          }
+          if (!st) continue;
+          if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
+          else epilogue_store(p, row, col0, r);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -786,24 +815,41 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
       const SegRow sr = p.epi == GEMM_EPI_DTANH_SEG ? seg_row(p.cells, row, row_ok) : SegRow{};
       if (!warp_wait(&tfull[a], aph, abort_flag)) break;   // warp-uniform: the epilogue uses warp-collective ops
       tc_fence_after();
+      if constexpr (EW == 16) {
+        // the d_hidden epilogue (the one launched with 16 epilogue warps) in
+        // 16-column chunks: half the registers of 32-column ones, so the 96 a
+        // thread gets at 576 threads hold it without spilling
 #pragma unroll 1
-      for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
-        uint32_t r[32];
-        const int col0 = n0 + c * 32;
-        const bool st = row_ok && col0 < p.N;
-        uint4 hv[4];
-        if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
-        if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg(FgRows{sr.f, sr.g}, col0, hv);
-        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
-        tmem_wait_ld();
-        if (p.epi == GEMM_EPI_DTANH_SEG) {
-          if (col0 < p.N) seg_chunk(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
-          continue;
+        for (int c = half * (BN / (16 * kEpiParts)); c < (half + 1) * (BN / (16 * kEpiParts)); ++c) {
+          const int col0 = n0 + c * 16;
+          if (col0 >= p.N) break;   // the same for the whole warp; later chunks lie further right
+          uint4 hv[2];
+          dtanh_from_fg<16>(FgRows{sr.f, sr.g}, col0, hv);
+          uint32_t r[16];
+          tmem_ld16(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 16, r);
+          tmem_wait_ld();
+          seg_chunk<16>(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
         }
-        if (!st) continue;
-        if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
-        else epilogue_store(p, row, col0, r);
+      } else {
+#pragma unroll 1
+        for (int c = half * (BN / (32 * kEpiParts)); c < (half + 1) * (BN / (32 * kEpiParts)); ++c) {
+          uint32_t r[32];
+          const int col0 = n0 + c * 32;
+          const bool st = row_ok && col0 < p.N;
+          uint4 hv[4];
+          if (p.epi == GEMM_EPI_DTANH && st) dtanh_load(p, row, col0, hv);
+          if (p.epi == GEMM_EPI_DTANH_FG && st) h_from_fg(fr, col0, hv);
+          if (p.epi == GEMM_EPI_DTANH_SEG && col0 < p.N) dtanh_from_fg<32>(FgRows{sr.f, sr.g}, col0, hv);
+          tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
+          tmem_wait_ld();
+          if (p.epi == GEMM_EPI_DTANH_SEG) {
+            if (col0 < p.N) seg_chunk<32>(p.cells, sr, col0, r, hv, lane);   // whole warp, same chunk
+            continue;
+          }
+          if (!st) continue;
+          if (p.epi == GEMM_EPI_DTANH || p.epi == GEMM_EPI_DTANH_FG) dtanh_store(p, row, col0, r, hv);
+          else epilogue_store(p, row, col0, r);
+        }
       }
       tc_fence_before();
       __syncwarp();

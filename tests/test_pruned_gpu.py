@@ -55,6 +55,19 @@ def test_ragged_random_bounds(cuda_ok, mode, S):
 
 
 @pytest.mark.parametrize("mode", ["tiled", "untiled"])
+def test_wide_band_32_lane_tiles(cuda_ok, mode):
+    """S = 20 rounds up to 32 band positions per tile row: a frame's cells fill
+    a whole warp, the one layout where the frame sums run over all 32 lanes."""
+    S = 20
+    batch = synth.make(B=3, T=24, U=48, D_enc=64, D_pred=32, H=128, V=256, dtype="bf16", seed=620,
+                       T_range=(6, 24), U_range=(10, 48), bias_std=0.3)
+    bounds = _random_bounds(batch, S, seed=S)
+    w = np.linspace(0.5, 1.5, 3)
+    l, g = _call(batch, bounds, S, mode=mode, grad_loss=w, chunk_cells=1024)
+    compare(l, g, run_oracle(batch, grad_loss=w, bounds=bounds, S=S), "bf16", extra_note=f"pruned S{S}/{mode}")
+
+
+@pytest.mark.parametrize("mode", ["tiled", "untiled"])
 def test_short_diagonal_band(cuda_ok, mode):
     batch = synth.workload("short")
     S = 6
