@@ -444,15 +444,8 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
         if (tdt) launch_tdt_dzd(j, st);
       }
     }
-    if (side) {
-      cudaStreamWaitEvent(st, side->join, 0);
-      chain_break(st);
-    } else if (untiled) {   // no side stream could be created: build the h rows here
-      StageScope sc("bwd_hidden", st);
-      launch_hidden_rows(j, 0, st);
-    }
     const int rows = (int)((c1 - c0) * 128);
-    {
+    auto run_dWo = [&]() -> int {
       StageScope sc("bwd_dWo", st);
       GemmTcArgs a{};
       // dW_o | db_o = dz^T [h | 1]: the extra column block of h yields the bias
@@ -462,14 +455,13 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       a.out_f32 = p.accWo;
       a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;
-      FRNNT_TRY(gemm_tc(a, st));
-      if (tdt) {
-        // dW_d | db_d from the duration columns (64 of them, zero past n_dur)
-        a.M = 64; a.N = HS; a.A = zrows + s.V; a.k_splits = 0; a.out_f32 = p.accWd;
-        FRNNT_TRY(gemm_tc(a, st));
-      }
-    }
-    {
+      const int r = gemm_tc(a, st);
+      if (r != FRNNT_OK || !tdt) return r;
+      // dW_d | db_d from the duration columns (64 of them, zero past n_dur)
+      a.M = 64; a.N = HS; a.A = zrows + s.V; a.k_splits = 0; a.out_f32 = p.accWd;
+      return gemm_tc(a, st);
+    };
+    auto run_dh = [&]() -> int {
       StageScope sc("bwd_dh", st);
       GemmTcArgs a{};
       // d_hidden = dz W_o; the epilogue forms dpre = d_hidden (1 - h^2), with h
@@ -484,8 +476,22 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       a.cells.UB = p.UB; a.cells.S = s.S; a.cells.bounds = bounds; a.cells.T_len = T_len; a.cells.U_len = U_len;
       a.cells.F = p.F; a.cells.G = p.G; a.cells.dF = p.dF; a.cells.dG = p.dG;
       a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128; a.dyn_dim = 1;
-      FRNNT_TRY(gemm_tc(a, st));
+      return gemm_tc(a, st);
+    };
+    // untiled: d_hidden first (it does not read the h rows, so it need not wait
+    // for the side stream; measured 0.03 ms faster on medium and 0.3 ms on
+    // long than after dW_o); tiled: dW_o first, while the chunk's last-written
+    // dz and h rows are still in L2 (measured 0.01-0.14 ms faster)
+    if (untiled) FRNNT_TRY(run_dh());
+    if (side) {   // the h rows of the side stream, for dW_o
+      cudaStreamWaitEvent(st, side->join, 0);
+      chain_break(st);
+    } else if (untiled) {   // no side stream could be created: build the h rows here
+      StageScope sc("bwd_hidden", st);
+      launch_hidden_rows(j, 0, st);
     }
+    FRNNT_TRY(run_dWo());
+    if (!untiled) FRNNT_TRY(run_dh());
   }
   {
     StageScope sc("projection_bwd", st);
