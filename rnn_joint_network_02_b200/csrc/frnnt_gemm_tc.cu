@@ -58,12 +58,13 @@ struct Eff {
   int M, m_tiles, kblocks, per;
 };
 
-__device__ __forceinline__ Eff eff_of(const GemmParams& p) {
+__device__ __forceinline__ Eff eff_of(const GemmParams& p, bool early = false) {
   Eff e;
   e.M = p.M;
   e.kblocks = p.kblocks;
   if (p.dyn_count) {
-    long long v = ((long long)__ldg(p.dyn_count) - p.dyn_base) * p.dyn_scale;
+    const int cnt = early ? tile_count_early(p.dyn_count) : __ldg(p.dyn_count);
+    long long v = ((long long)cnt - p.dyn_base) * p.dyn_scale;
     if (v < 0) v = 0;
     if (p.dyn_dim == 1) e.M = (int)min((long long)p.M, v);
     else e.kblocks = (int)min((long long)p.kblocks, (v + 63) / 64);
@@ -435,6 +436,16 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  {
+    // no work anywhere in the grid (a chunk past the device-built tile list):
+    // every CTA sees the same limits and leaves before any set-up, after
+    // waiting for the previous launch like every other launch of the call
+    const Eff e0 = eff_of(p, true);
+    if (e0.M <= 0 || e0.kblocks <= 0) {
+      chain_wait();
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -459,9 +470,7 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_p;
-  // set-up done: from here on the previous launches' results are read.  A
-  // device-side limit that leaves no work (a chunk past the device-built tile
-  // list) makes every unit of every role empty.
+  // set-up done: from here on the previous launches' results are read
   chain_wait();
   const Eff eff = eff_of(p);
 
@@ -679,6 +688,15 @@ __global__ void __launch_bounds__(threads_of(EW), 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int units = p.m_tiles * p.n_tiles * p.k_splits;
+  {
+    // as in the one-CTA kernel: an empty launch leaves before any set-up or
+    // cluster barrier (both CTAs of every pair alike)
+    const Eff e0 = eff_of(p, true);
+    if (e0.M <= 0 || e0.kblocks <= 0) {
+      chain_wait();
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {

@@ -42,6 +42,17 @@ class StageScope {
 // kernel triggers its dependents early: a dependent whose CTAs sat resident
 // beside a running GEMM, waiting, slowed the tiled call by 30 %.)
 __device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// The call's device-built tile count, read before chain_wait, from L2 (the
+// point of coherence), only so that a launch with no tiles in its range can
+// skip its set-up.  The prologue that writes the count is complete by then:
+// every launch waits for the one before it, also when it has no work, so when
+// a launch starts all launches but the previous one have completed, and the
+// prologue is at least three launches before any reader of the count.
+__device__ __forceinline__ int tile_count_early(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 // Host side (per host thread): a call names its stream (chain_begin); a kernel
 // launched there right after another of the call's kernels gets the attribute;

@@ -226,6 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   const int slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int nslots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   auto tile_of = [&](int i) { return p.tile_begin + (PAIR ? 2 * i + (int)rank : i); };
+  // an empty tile range (a chunk past the device-built tile list): every CTA
+  // of the grid sees the same count and leaves before any set-up or cluster
+  // barrier, after waiting for the previous launch like every other launch
+  if (min(p.tile_end, tile_count_early(p.ntiles)) <= p.tile_begin) {
+    chain_wait();
+    return;
+  }
   // arrivals on barriers the (leader's) MMA thread waits for
   auto arrive_leader = [&](uint64_t* bar) {
     if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
@@ -272,8 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
   chain_wait();
   const int ntiles = min(p.tile_end, *p.ntiles);
   const int span = ntiles - p.tile_begin;
-  // an empty tile range (a chunk past the device-built tile list) gives every
-  // CTA of the grid niter = 0: all skip to the teardown alike
   const int niter = span <= 0 ? 0 : (PAIR ? (span + 1) / 2 : span);
   for (int k = threadIdx.x; k < p.Vx; k += blockDim.x) bias_s[k] = p.b_o[k];
   __syncthreads();
