@@ -65,14 +65,14 @@ def parse(argv=None):
 # An entry is removed whenever its kernel changes, so the roofline's traffic is
 # null rather than stale.
 MEASURED_TRAFFIC = {
-    ("medium", "untiled", "bwd_dWo", "marginal"): (1.087124e9 + 0.003500e9,
+    ("medium", "untiled", "bwd_dWo", "marginal"): (1.111446e9 + 0.003530e9,
                                                    "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "bwd_dh", "marginal"): (0.630031e9 + 0.016449e9,
+    ("medium", "untiled", "bwd_dh", "marginal"): (0.628257e9 + 0.015802e9,
                                                   "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd", "marginal"): (0.009156e9 + 0.555447e9,
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009147e9 + 0.555396e9,
                                                      "profiles/ncu_joint_tc_medium_untiled.md"),
     # one full 592-tile chunk launch (the stage has four real launches per call)
-    ("medium", "tiled", "joint_bwd_dz", "marginal"): (0.005016e9 + 0.217656e9,
+    ("medium", "tiled", "joint_bwd_dz", "marginal"): (0.005075e9 + 0.217644e9,
                                                       "profiles/ncu_joint_bwd_dz_medium_tiled.md (per 592-tile launch)"),
 }
 
