@@ -455,47 +455,59 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush, workload=
     res["mufu"] = mufu_roofline(batch, valid, ms, clocks)
 
     if e2e:
-        # end to end through the public API with host buffers: pinned H2D of the
-        # step's inputs (packed in one pinned buffer, one copy), the call, D2H of
-        # the loss and status word
-        d = dict(d)   # the call's inputs become views of one device buffer (the caller's dict is kept)
+        # end to end through the public API with host buffers, as a training
+        # loop feeds it: every step's inputs come from pinned host memory (one
+        # packed H2D copy into one of two device buffers, on a copy stream, so
+        # that step i+1's inputs arrive while step i computes), then the call,
+        # then the D2H of its loss and status word.  The steps are queued back to
+        # back; the time per step is the device time from the end of the last
+        # warm-up step to the end of the last step, over the timed steps, so
+        # every timed step's copies lie inside it.  Results are checked after
+        # the last step.
+        d = dict(d)   # the call's inputs become views of the device buffers (the caller's dict is kept)
         keys = list(d.keys())
         sizes = [(d[k].numel() * d[k].element_size() + 255) // 256 * 256 for k in keys]
         host_buf = torch.empty(sum(sizes), dtype=torch.uint8).pin_memory()
-        dev_buf = torch.empty(sum(sizes), dtype=torch.uint8, device=dev)
+        dev_bufs = [torch.empty(sum(sizes), dtype=torch.uint8, device=dev) for _ in range(2)]
+        views = [{}, {}]
         off = 0
         for k, n in zip(keys, sizes):
             nb = d[k].numel() * d[k].element_size()
             host_buf[off:off + nb].copy_(d[k].cpu().contiguous().view(-1).view(torch.uint8))
-            d[k] = dev_buf[off:off + nb].view(d[k].dtype).view(d[k].shape)   # the call reads its inputs here
+            for b in range(2):
+                views[b][k] = dev_bufs[b][off:off + nb].view(d[k].dtype).view(d[k].shape)
             off += n
         n = warmup + steps
         loss_h = torch.empty(n, batch.f.shape[0], dtype=torch.float32).pin_memory()
         status_h = torch.zeros(n, 4, dtype=torch.int32).pin_memory()
         h2d = sum(d[k].numel() * d[k].element_size() for k in keys)
         d2h = loss_h[0].numel() * 4 + status_h[0].numel() * 4
-        # every step: H2D of its inputs, the call, D2H of its loss and status
-        # word, bracketed by events on the stream; the host queues step after
-        # step without waiting for each result (as a training loop does), so the
-        # device-timed region holds the step's copies and kernels, not host
-        # scheduling delays; the results are checked after the last step
-        evs_e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(n)]
+        used = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         torch.cuda.synchronize()
         t_host = time.perf_counter()
         for i in range(n):
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(used[i - 2])   # the buffer's previous step is done with it
+                dev_bufs[i % 2].copy_(host_buf, non_blocking=True)
+                copied[i].record(copy_stream)
             flush.zero_()
-            evs_e[i][0].record(stream)
-            dev_buf.copy_(host_buf, non_blocking=True)
+            stream.wait_event(copied[i])
+            d.update(views[i % 2])
             call()
+            used[i].record(stream)
             loss_h[i].copy_(out.loss, non_blocking=True)
             status_h[i].copy_(out.status, non_blocking=True)
-            evs_e[i][1].record(stream)
+            done[i].record(stream)
         t_host = (time.perf_counter() - t_host) / n
         torch.cuda.synchronize()
         if int(status_h[:, 0].abs().sum()) != 0:
             raise RuntimeError(f"device status {status_h[:, 0].tolist()}")
-        e2e_ms = [evs_e[i][0].elapsed_time(evs_e[i][1]) for i in range(warmup, n)]
-        e2e_t = sum(e2e_ms) / len(e2e_ms)
+        w0 = max(warmup, 1)   # the first step has no predecessor to be timed from
+        e2e_t = done[w0 - 1].elapsed_time(done[n - 1]) / (n - w0)
         if world > 1:
             t = torch.tensor([e2e_t], device=dev)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -503,8 +515,10 @@ def measure_mode(args, mode, batch, d, dev, world, rank, local, flush, workload=
         res["e2e"] = {"value": world * units / (e2e_t / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_t,
                       "host_queue_ms_per_step": t_host * 1e3,
-                      "how": "per step: pinned H2D of the inputs (one packed copy), the public call, D2H of loss and "
-                             "status; device-timed with events around each step, steps queued back to back"}
+                      "how": "per step: pinned H2D of the inputs (one packed copy, on a copy stream into one of two "
+                             "device buffers, so the next step's inputs arrive during this step), the public call, "
+                             "D2H of loss and status; steps queued back to back; device time from the end of the "
+                             "warm-up to the end of the last step, per step"}
     del out
     return res
 
