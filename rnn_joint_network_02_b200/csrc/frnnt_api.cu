@@ -452,6 +452,9 @@ int run_tc(const frnnt_dims* d, const Shape& s, const void* f, const void* g, co
       // gradient, unless the dz pass summed it (then N = H)
       a.M = s.V; a.N = p.db_part ? s.H : HS; a.K = rows; a.A = zrows; a.a_mn = true; a.lda = s.Vx; a.B = hrows;
       a.b_mn = true; a.ldb = HS; a.epi = GEMM_EPI_RED_F32; a.k_splits = 0;
+      // tiled: the recompute pass writes h rows up to the column block that
+      // holds the 1 of column H; the columns past it are read as zeros
+      a.b_inner = untiled ? 0 : s.H + 8;
       a.out_f32 = p.accWo;
       a.ldo = HS; a.status = status; a.dyn_count = p.ntiles; a.dyn_base = (int)c0; a.dyn_scale = 128;
       a.dyn_dim = 2;

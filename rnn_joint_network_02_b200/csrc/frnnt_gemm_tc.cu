@@ -1027,7 +1027,8 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st) {
   if (!ok) return FRNNT_ERR_CUDA;
   const int b_rows = pair ? BN / 2 : BN;
   if (!g.b_mn) ok = make_tmap_bf16_2d(&tb, g.B, g.K, g.N, (uint64_t)g.ldb, 64, b_rows);
-  else ok = make_tmap_bf16_2d(&tb, g.B, g.N, g.K, (uint64_t)g.ldb, 64, 64);
+  else ok = make_tmap_bf16_2d(&tb, g.B, g.b_inner > 0 && g.b_inner < g.N ? g.b_inner : g.N, g.K, (uint64_t)g.ldb,
+                              64, 64);
   if (!ok) return FRNNT_ERR_CUDA;
   GemmParams p;
   p.M = g.M;

@@ -248,6 +248,7 @@ struct GemmTcArgs {
   const void* B;
   bool b_mn;
   long long ldb;
+  long long b_inner;   // MN-major B: columns of B that hold data (0: N); TMA reads the rest as zeros
   int epi;             // GemmEpilogue
   int k_splits;        // > 1 only with GEMM_EPI_RED_F32; 0 with it: chosen for the launch's rounds
   float* out_f32;      // STORE_F32 / RED_F32 output [M][ldo]

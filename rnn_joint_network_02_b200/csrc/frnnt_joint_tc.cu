@@ -455,10 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_tc_kernel(const __grid_cons
       if (MODE != MODE_FWD && p.store_h && tile < ntiles) {
         const size_t row0 = (MODE == MODE_BWD_DZ) ? (size_t)(tile - p.tile_begin) * 128 : (size_t)tile * 128;
         hrow = p.hbuf + (row0 + r) * p.HS;
-        if (half == 0) {
-          const uint4 one = make_uint4(ri.valid ? 0x3F80u : 0u, 0u, 0u, 0u);   // bf16 1.0 in column H
-          for (int c = H; c < p.HS; c += 8) *(uint4*)(hrow + c) = c == H ? one : make_uint4(0u, 0u, 0u, 0u);
-        }
+        // bf16 1.0 in column H, zeros to H + 7; the dW_o GEMM reads the
+        // columns past those as zeros (its operand's extent ends there)
+        if (half == 0) *(uint4*)(hrow + H) = make_uint4(ri.valid ? 0x3F80u : 0u, 0u, 0u, 0u);
       }
       for (int g = 0; g < ngrp; ++g) {
         const int kb0 = g * p.ks, nk = min(p.ks, p.KB - kb0);
