@@ -69,10 +69,10 @@ MEASURED_TRAFFIC = {
                                                    "profiles/ncu_gemm2_backward_medium_untiled.md"),
     ("medium", "untiled", "bwd_dh", "marginal"): (0.628257e9 + 0.015802e9,
                                                   "profiles/ncu_gemm2_backward_medium_untiled.md"),
-    ("medium", "untiled", "joint_fwd", "marginal"): (0.009147e9 + 0.555396e9,
+    ("medium", "untiled", "joint_fwd", "marginal"): (0.009422e9 + 0.555290e9,
                                                      "profiles/ncu_joint_tc_medium_untiled.md"),
     # one full 592-tile chunk launch (the stage has four real launches per call)
-    ("medium", "tiled", "joint_bwd_dz", "marginal"): (0.005075e9 + 0.217644e9,
+    ("medium", "tiled", "joint_bwd_dz", "marginal"): (0.007356e9 + 0.200818e9,
                                                       "profiles/ncu_joint_bwd_dz_medium_tiled.md (per 592-tile launch)"),
 }
 
