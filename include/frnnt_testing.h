@@ -48,6 +48,13 @@ FRNNT_API int frnnt_test_joint_variant(int variant);
  * (set it between calls).  Returns the previous count. */
 FRNNT_API int frnnt_test_lose_gemm_loads(int n);
 
+/* The K-slice count the tensor-core GEMM takes for a split-K launch (host
+ * only, no GPU needed): mn output tiles on `workers` persistent CTAs (or CTA
+ * pairs), kblocks K blocks of 64.  It minimises rounds x (K blocks per unit +
+ * a fixed 64-block unit cost), the fewest slices on a tie; always in
+ * [1, max(kblocks, 1)]. */
+FRNNT_API int frnnt_test_auto_splits(int mn, int workers, int kblocks);
+
 #ifdef __cplusplus
 }
 #endif

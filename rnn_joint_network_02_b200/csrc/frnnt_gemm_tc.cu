@@ -921,36 +921,6 @@ int sm_count() {
   return n;
 }
 
-// K slices of a split-K GEMM with mn output tiles on `workers` persistent CTAs
-// (or CTA pairs), each taking units workers apart.  The launch lasts about
-// rounds x (k blocks per unit + a unit's fixed cost: pipeline fill and the
-// atomic epilogue), so the slice count minimising that is taken, the fewest on
-// a tie.  A round that only a few workers reach costs as much as a full one:
-// 12 tiles x 13 slices = 156 units on 74 pairs keep 8 pairs busy for a third
-// round, where 6 slices fit one.  The fixed cost is taken as 64 k blocks, which
-// favours fewer slices (fewer atomic epilogues) where the fill is about equal:
-// on 40000 k blocks, 6 slices (one round) and 37 (six) measured the same.
-int auto_splits(int mn, int workers, int kblocks) {
-  if (mn <= 0 || workers <= 0 || kblocks <= 1) return 1;
-  constexpr long long kUnitCost = 64;
-  int best = 1;
-  long long best_cost = -1;
-  for (int s = 1; s <= kblocks; ++s) {
-    const int per = (kblocks + s - 1) / s;
-    const int real = (kblocks + per - 1) / per;   // slices after rounding each to whole k blocks
-    if (real != s) continue;
-    const long long units = (long long)mn * real;
-    const long long rounds = (units + workers - 1) / workers;
-    const long long cost = rounds * (per + kUnitCost);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = real;
-    }
-    if (rounds > 16) break;   // more slices only add rounds
-  }
-  return best;
-}
-
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EW = 8>
 bool launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
@@ -984,6 +954,36 @@ bool launch2_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p
 }
 
 }  // namespace
+
+// K slices of a split-K GEMM with mn output tiles on `workers` persistent CTAs
+// (or CTA pairs), each taking units workers apart.  The launch lasts about
+// rounds x (k blocks per unit + a unit's fixed cost: pipeline fill and the
+// atomic epilogue), so the slice count minimising that is taken, the fewest on
+// a tie.  A round that only a few workers reach costs as much as a full one:
+// 12 tiles x 13 slices = 156 units on 74 pairs keep 8 pairs busy for a third
+// round, where 6 slices fit one.  The fixed cost is taken as 64 k blocks, which
+// favours fewer slices (fewer atomic epilogues) where the fill is about equal:
+// on 40000 k blocks, 6 slices (one round) and 37 (six) measured the same.
+int auto_splits(int mn, int workers, int kblocks) {
+  if (mn <= 0 || workers <= 0 || kblocks <= 1) return 1;
+  constexpr long long kUnitCost = 64;
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= kblocks; ++s) {
+    const int per = (kblocks + s - 1) / s;
+    const int real = (kblocks + per - 1) / per;   // slices after rounding each to whole k blocks
+    if (real != s) continue;
+    const long long units = (long long)mn * real;
+    const long long rounds = (units + workers - 1) / workers;
+    const long long cost = rounds * (per + kUnitCost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = real;
+    }
+    if (rounds > 16) break;   // more slices only add rounds
+  }
+  return best;
+}
 
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
                        uint32_t box_inner, uint32_t box_outer) {

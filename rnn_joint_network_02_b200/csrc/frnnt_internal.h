@@ -269,6 +269,9 @@ int gemm_tc(const GemmTcArgs& g, cudaStream_t st);
 // load (so a bounded wait expires and the status word gets FRNNT_STATUS_TIMEOUT);
 // returns the previous count.  Process-wide, not thread-safe.
 int lose_gemm_loads(int n);
+// K slices of a split-K GEMM (frnnt_gemm_tc.cu): mn output tiles on `workers`
+// persistent CTAs or CTA pairs, kblocks 64-wide K blocks.
+int auto_splits(int mn, int workers, int kblocks);
 
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_elems,
                        uint32_t box_inner, uint32_t box_outer);

@@ -32,3 +32,7 @@ extern "C" FRNNT_API int frnnt_test_gemm_bf16(int M, int N, int K, const void* A
 extern "C" FRNNT_API int frnnt_test_joint_variant(int variant) { return frnnt::set_joint_variant(variant); }
 
 extern "C" FRNNT_API int frnnt_test_lose_gemm_loads(int n) { return frnnt::lose_gemm_loads(n); }
+
+extern "C" FRNNT_API int frnnt_test_auto_splits(int mn, int workers, int kblocks) {
+  return frnnt::auto_splits(mn, workers, kblocks);
+}
